@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP4 MoE expert layer (libmxmoe, sm_100a).
+
+One step = one pass of the whole layer over one batch of tokens: router GEMM,
+top-k routing, grouping by expert, gate/up + SwiGLU, down projection, weighted
+combine, through the library's C ABI. Metric: layer tokens/s, with the
+expert-weight HBM GB/s and its fraction of the measured HBM peak alongside.
+
+Default workload: one DFlash verify block (8 tokens, the block size of the
+"MiMo-V2.5-Pro-FP4-DFlash" model card, section 3) through a layer of 384 MXFP4
+experts, top-8, hidden 6144, expert intermediate 2048. Inputs are synthetic
+(datagen); the touched experts' weights (~1.2 GB per step) exceed the 126 MB L2,
+and the batches rotate so consecutive steps touch different experts.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+Under torchrun each rank runs an independent replica on its own GPU (no
+collective on the data path; weak scaling); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import datagen  # noqa: E402
+
+METRIC = "MXFP4 MoE-layer tokens/s; expert-weight HBM GB/s as % of peak (1×B200)"
+UNIT = "tokens/s"
+KERNELS_PER_STEP = 7  # router_gemm, route, permute, act_convert, stage gate/up, stage down, combine
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--config", default="verify8", choices=[c.name for c in datagen.CONFIGS])
+    ap.add_argument("--batches", type=int, default=16, help="distinct rotating input batches")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def workload_config(cfg, world: int, batches: int):
+    return {
+        "workload": "%s: MXFP4 MoE layer, T=%d tokens, H=%d, E=%d experts, top-%d, I=%d, block 32"
+                    % (cfg.name, cfg.T, cfg.H, cfg.E, cfg.k, cfg.I),
+        "tokens_per_step": cfg.T,
+        "global_batch": cfg.T * world,
+        "hidden": cfg.H,
+        "experts": cfg.E,
+        "top_k": cfg.k,
+        "intermediate": cfg.I,
+        "router_bias_zipf": cfg.zipf_s,
+        "parallelism": "replicas x%d" % world,
+        "l2": "inputs larger than L2: each step streams the touched experts' MXFP4 weights (>1 GB) and "
+              "%d input batches rotate" % batches,
+    }
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in ("mxfp4_quantized_moe_router_b200/csrc/ffn.cu", "mxfp4_quantized_moe_router_b200/csrc/common.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the gate/up stage from a committed ncu summary,
+    only if the kernel source is unchanged since that capture."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        ent = d.get("ffn_gate_up", {}).get(workload)
+        if ent and ent.get("source_sha") == kernel_source_sha():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9 or not parts[0].endswith(self.uuid):
+                continue
+            try:
+                self.samples.append(dict(t=time.time(), sm=float(parts[1]), max=float(parts[2]),
+                                         hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                pass
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        win = [s for s in self.samples if t0 - 0.15 <= s["t"] <= t1 + 0.15] or self.samples[-3:]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        reasons = set()
+        for s in win:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if s[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s["sm"] for s in win), "sm_max_mhz": max(s["max"] for s in win),
+                "reasons": sorted(reasons), "samples": len(win)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_setup(cfg, seed, token_rows, x_bf16, bias):
+    """Route the sample tokens with the oracle and quantise (untimed) the experts
+    they touch. Returns the experts dict."""
+    import oracle
+    import torch
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wg = datagen.make_router_weight(cfg, seed, dev).cpu()
+    xs = x_bf16[token_rows].cpu()
+    logits = oracle.router_logits(xs, wg, bias)
+    ids, _ = oracle.route(logits, cfg.k)
+    experts = {}
+    for e in sorted(set(ids.ravel().tolist())):
+        w13 = datagen.make_w13(cfg, e, seed, dev).cpu()
+        w2 = datagen.make_w2(cfg, e, seed, dev).cpu()
+        p13, s13 = oracle.quantize(w13)
+        p2, s2 = oracle.quantize(w2)
+        experts[e] = (p13, s13, p2, s2)
+    return wg, xs, experts
+
+
+def oracle_layer_time(cfg, wg, xs, bias, experts):
+    import oracle
+
+    t = time.perf_counter()
+    oracle.moe_layer(xs, wg, bias, lambda e: experts[e], cfg.k, threads=1)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(cfg, seed, x_cpu, bias, n_tokens=2):
+    rows = list(range(min(n_tokens, cfg.T)))
+    wg, xs, experts = oracle_setup(cfg, seed, rows, x_cpu, bias)
+    dt = oracle_layer_time(cfg, wg, xs, bias, experts)
+    return {"value": len(rows) / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d token(s) of the %s workload through the float64 C oracle (router, routing, %d experts "
+                      "decoded and run, combine; experts quantised beforehand, untimed), one thread"
+                      % (len(rows), cfg.name, len(experts)),
+            "seconds": dt}
+
+
+def run_reference(args):
+    """--impl reference: the float64 CPU oracle as it stands, on host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    cfg = datagen.BY_NAME[args.config]
+    x = datagen.make_x(cfg, args.seed)
+    bias = datagen.make_router_bias(cfg, args.seed)
+    # one token per step (all of its k experts); a step is a bounded sample
+    tokens = list(range(min(cfg.T, max(1, args.warmup + args.steps))))
+    steps_tokens = [[tokens[i % len(tokens)]] for i in range(args.warmup + args.steps)]
+    need = sorted(set(t for s in steps_tokens for t in s))
+    wg, _, experts = oracle_setup(cfg, args.seed, need, x, bias)
+    times = []
+    for i, rows in enumerate(steps_tokens):
+        xs = x[rows]
+        dt = oracle_layer_time(cfg, wg, xs, bias, experts)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, 1, 1),
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": UNIT,
+                         "sample": "each step: 1 token of the %s workload through the float64 C oracle "
+                                   "(router, routing, its %d experts decoded and run, combine), one thread"
+                                   % (cfg.name, cfg.k)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_quantized_moe_router_b200 as mx
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = datagen.BY_NAME[args.config]
+    T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.k, cfg.I
+
+    # --- weights (same layer on every rank), quantised and prepacked on the device
+    wg = datagen.make_router_weight(cfg, args.seed, dev)
+    ew = mx.ExpertWeights(E, H, I, dev)
+    for e in range(E):
+        ew.quantize_expert(e, datagen.make_w13(cfg, e, args.seed, dev), datagen.make_w2(cfg, e, args.seed, dev))
+    ew.prepack()
+    torch.cuda.synchronize()
+    del ew.packed13, ew.sc13, ew.packed2, ew.sc2  # the kernels stream the prepacked blob only
+    torch.cuda.empty_cache()
+    prepacked = ew.prepacked
+    bias_np = datagen.make_router_bias(cfg, args.seed)
+    bias = torch.from_numpy(bias_np).to(dev) if bias_np is not None else None
+
+    # --- rotating input batches (per rank: its own tokens)
+    nb = max(1, args.batches)
+    xs = [datagen.make_x(cfg, args.seed + 1000 * rank + b, dev) for b in range(nb)]
+    logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    src_row = torch.empty(T * k, dtype=torch.int32, device=dev)
+    dst_of = torch.empty(T * k, dtype=torch.int32, device=dev)
+    fws = torch.empty(mx.mxmoe_ffn_workspace_size(T, k, E, H, I), dtype=torch.uint8, device=dev)
+    y_perm = torch.empty((T * k, H), dtype=torch.float32, device=dev)
+    y = torch.empty((T, H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    # raw C-ABI calls on one stream (the same kernels mxmoe_layer_forward chains)
+    L = mx.load()
+    P = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    fws_bytes = fws.numel()
+
+    def step(b, ev=None):
+        x = xs[b % nb]
+        rc = L.mxmoe_router_gemm(P(x), P(wg), P(bias), T, H, E, P(logits), sp)
+        rc |= L.mxmoe_route(P(logits), T, E, k, P(ids), P(w), sp)
+        rc |= L.mxmoe_permute(P(ids), T, k, E, P(offsets), P(src_row), P(dst_of), sp)
+        if ev is not None:
+            ev[0].record(stream)
+        rc |= L.mxmoe_ffn_gate_up(P(x), P(offsets), P(src_row), P(prepacked), T, k, E, H, I, P(fws), fws_bytes, sp)
+        if ev is not None:
+            ev[1].record(stream)
+        rc |= L.mxmoe_ffn_down(P(offsets), P(prepacked), T, k, E, H, I, P(y_perm), P(fws), fws_bytes, sp)
+        rc |= L.mxmoe_combine(P(y_perm), P(dst_of), P(w), T, k, H, P(y), sp)
+        if rc:
+            raise RuntimeError("libmxmoe call failed: " + mx.last_error())
+
+    # touched experts per batch (untimed), for the weight-byte accounting
+    touched = []
+    for b in range(nb):
+        step(b)
+        torch.cuda.synchronize()
+        touched.append(int(torch.unique(ids).numel()))
+    assert mx.mxmoe_read_status(fws) == mx.OK
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+
+    # --- device-resident timed region
+    for i in range(args.warmup):
+        step(i)
+    ev_unit = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, ev_unit[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    ms = start.elapsed_time(end)
+    ms_max = max_over_ranks(ms)
+    unit_ms = [a.elapsed_time(b) for a, b in ev_unit]
+    clk = clocks.summary(t0, t1)
+
+    # --- end to end through the public API with host buffers
+    import ctypes  # noqa: F401
+
+    x_host = [xb.cpu().pin_memory() for xb in xs]
+    y_host = torch.empty((T, H), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    lws = torch.empty(mx.mxmoe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
+    lws_bytes = lws.numel()
+
+    def e2e_step(b):
+        x_dev.copy_(x_host[b % nb], non_blocking=True)
+        rc = L.mxmoe_layer_forward(P(x_dev), P(wg), P(bias), P(prepacked), T, H, I, E, k, P(y), None, None, P(lws),
+                                   lws_bytes, sp)
+        if rc:
+            raise RuntimeError("mxmoe_layer_forward failed: " + mx.last_error())
+        y_host.copy_(y, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    barrier()
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for i in range(args.steps):
+        e2e_step(args.warmup + i)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(s2.elapsed_time(e2))
+    clocks.stop()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peak, peak_kind = load_peaks()
+    steps_batches = [(args.warmup + i) % nb for i in range(args.steps)]
+    mean_touched = float(np.mean([touched[b] for b in steps_batches]))
+    tokens = T * args.steps * world
+    value = tokens / (ms_max / 1e3)
+    weight_bytes_step = mean_touched * cfg.expert_bytes
+    weight_gbs = weight_bytes_step * args.steps / (ms / 1e3) / 1e9
+    # dominant unit: mxmoe_ffn_gate_up (act_convert + gate/up stage); algorithmic
+    # bytes = gate/up MXFP4 bytes of the touched experts + x read + h written
+    w13_bytes = 2 * I * H * 17 // 32
+    unit_bytes = mean_touched * w13_bytes + T * H * 2 + T * k * I * 2
+    unit_ms_mean = float(np.mean(unit_ms))
+    achieved = unit_bytes / (unit_ms_mean / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e2m1xf16->f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
+                                          "W~N(0,0.02) quantised to MXFP4 by the library)",
+        "config": workload_config(cfg, world, nb),
+        "weight_gbs": weight_gbs,
+        "weight_frac_of_hbm_peak": weight_gbs / peak,
+        "touched_experts_per_step": mean_touched,
+        "roofline": {"kernel": "mxmoe_ffn_gate_up (act_convert_kernel + ffn_stage_kernel<gate_up>)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                     else "fallback 6.65 TB/s",
+                     "traffic": profiled_traffic(cfg.name), "unit_ms": unit_ms_mean,
+                     "algorithmic_bytes_per_launch": unit_bytes},
+        "clocks": clk,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
+                "d2h_bytes_per_step": T * H * 4, "api": "mxmoe_layer_forward with pinned host x/y copies"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.seed, xs[0].cpu(), bias_np)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,227 @@
+/*
+ * mxmoe.h -- C ABI of libmxmoe.so: the MXFP4 MoE expert layer of a
+ * decode/verify step on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (pages: "MiMo-V2.5-Pro-FP4-DFlash" model card, section 2 "FP4
+ * Quantization" -- MoE experts stored as MXFP4 with block size 32, the rest at
+ * higher precision; nxbn.cn MiMo-V2.5-Pro-FP4-DFlash article, architecture
+ * section -- 384 experts, 8 activated per token, hidden size 6144):
+ *
+ *   logits = x Wg^T (+ bias)               mxmoe_router_gemm
+ *   ids, w = top-k of softmax(logits)      mxmoe_route
+ *   group (token, slot) pairs by expert    mxmoe_permute
+ *   h = silu(W_gate x) * (W_up x)          mxmoe_ffn_gate_up (stage 1)
+ *   y_e = W_down h                         mxmoe_ffn_down (stage 2)
+ *   (both stages)                          mxmoe_expert_ffn
+ *   y = sum_j w_j y_{e_j}                  mxmoe_combine
+ *   all of the above in one call           mxmoe_layer_forward
+ * plus the weight-format entry points mxmoe_quantize / mxmoe_dequantize and
+ * the kernel-layout re-tiling mxmoe_prepack_experts.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named as device memory must be device (or managed) memory that
+ *    the caller owns and keeps alive until the stream work finishes. No entry
+ *    point allocates device memory; scratch comes from a caller-provided
+ *    workspace sized by the matching *_workspace_size query.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream). Nothing synchronises the host except
+ *    mxmoe_read_status.
+ *  - Every call returns an mxmoe_status. Argument problems are detected on the
+ *    host before anything is enqueued. On failure mxmoe_last_error() returns a
+ *    message for the calling thread.
+ *  - bf16 tensors are passed as raw 16-bit words (const void*), row-major.
+ *  - Entry points are thread-safe: they keep no host state besides the
+ *    per-thread error message.
+ */
+#ifndef MXMOE_H
+#define MXMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MXMOE_API __attribute__((visibility("default")))
+
+enum mxmoe_status {
+    MXMOE_OK = 0,
+    MXMOE_ERR_INVALID_SHAPE = 1, /* a size is out of range or not a required multiple */
+    MXMOE_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned (bulk copies need it) */
+    MXMOE_ERR_NULL = 3,          /* a required pointer is NULL */
+    MXMOE_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    MXMOE_ERR_TIMEOUT = 5,       /* device side: a bounded wait gave up (read via mxmoe_read_status) */
+    MXMOE_ERR_DEVICE = 6,        /* the current device is not compute capability 10.0 */
+    MXMOE_ERR_WORKSPACE = 7      /* workspace NULL or smaller than the size query returns */
+};
+
+/* Library version string, e.g. "mxmoe 0.1.0". Never fails. */
+MXMOE_API const char *mxmoe_version(void);
+
+/* Message describing the last failing call made by this thread ("" if none).
+ * The pointer stays valid until this thread's next failing call. */
+MXMOE_API const char *mxmoe_last_error(void);
+
+/* ------------------------------------------------------------------------ */
+/* Weight format                                                             */
+/* ------------------------------------------------------------------------ */
+
+/* MXFP4 quantiser (model card, section 2: MXFP4, block size 32; the pages fix
+ * no scale or rounding rule, so the OCP MX convention is used).
+ *   w       device, bf16 [rows, K] row-major.
+ *   packed  device, uint8 [rows, K/2]: element 2j of a row in the low nibble
+ *           of byte j, element 2j+1 in the high nibble. E2M1 codes: bit 3
+ *           sign, bits 2..1 exponent (bias 1), bit 0 mantissa.
+ *   scales  device, uint8 [rows, K/32], one E8M0 byte per 32-element block.
+ * Per block: e = floor(log2 max|x|) - 2 clamped to [-127, 127] (e = -127 for
+ * an all-zero block), scale byte e + 127, each element |x|/2^e rounded to
+ * nearest E2M1 with ties to the even mantissa and saturation at 6, sign bit
+ * copied. Non-finite inputs are outside the contract.
+ * Errors: K % 32 != 0 or rows/K <= 0 -> INVALID_SHAPE; NULL -> NULL;
+ * w not 16-byte aligned or K % 8 != 0 -> ALIGNMENT (only the alignment of w
+ * matters; packed and scales are written bytewise). */
+MXMOE_API int mxmoe_quantize(const void *w, int64_t rows, int64_t K, uint8_t *packed, uint8_t *scales,
+                             void *stream);
+
+/* Inverse of the format above: out[r, k] = E2M1(code) * 2^(S - 127) as float.
+ *   packed device uint8 [rows, K/2], scales device uint8 [rows, K/32],
+ *   out device float [rows, K]. Errors as for mxmoe_quantize. */
+MXMOE_API int mxmoe_dequantize(const uint8_t *packed, const uint8_t *scales, int64_t rows, int64_t K, float *out,
+                               void *stream);
+
+/* Bytes of the prepacked expert blob for E experts of hidden size H and
+ * intermediate size I (= E * 3 * H * I * 17/32, the same bytes as the packed
+ * codes plus scales). Returns -1 if H % 64 or I % 32 is non-zero or a size is
+ * not positive. */
+MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I);
+
+/* Re-tile canonical MXFP4 expert weights into the layout the FFN kernels
+ * stream (a pure byte permutation; nothing is re-rounded).
+ *   packed13 device uint8 [E, 2I, H/2], sc13 device uint8 [E, 2I, H/32]:
+ *            rows 0..I-1 of each expert are the gate projection, rows
+ *            I..2I-1 the up projection (each row a K = H vector).
+ *   packed2  device uint8 [E, H, I/2], sc2 device uint8 [E, H, I/32]: down
+ *            projection (each row a K = I vector).
+ *   prepacked device, mxmoe_prepacked_size(E, H, I) bytes, 16-byte aligned.
+ * Layout of the blob: all gate/up tiles, then all down tiles. A tile is 64
+ * weight rows (gate/up: 32 gate rows and the 32 matching up rows) split along
+ * K into chunks of up to 256 elements; a chunk holds the nibbles in the order
+ * the tensor-core fragments consume them, then the scale bytes.
+ * Errors: shapes as in mxmoe_prepacked_size -> INVALID_SHAPE; NULL -> NULL;
+ * prepacked not 16-byte aligned -> ALIGNMENT. */
+MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const uint8_t *sc13, const uint8_t *packed2,
+                                    const uint8_t *sc2, int E, int H, int I, void *prepacked, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Router                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Router logits in float32: logits[t, e] = sum_k x[t, k] * Wg[e, k] + bias[e]
+ * (products of bf16 values are exact in float32; the sum is float32).
+ *   x device bf16 [T, H]; wg device bf16 [E, H]; bias device float [E] or
+ *   NULL for no bias; logits device float [T, E].
+ * Errors: T < 0, E <= 0, H <= 0 or H % 32 != 0 -> INVALID_SHAPE; x, wg not
+ * 16-byte aligned -> ALIGNMENT. T == 0 is a no-op. */
+MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const float *bias, int T, int H, int E,
+                                float *logits, void *stream);
+
+/* Top-k routing (384 experts, 8 per token in the layer on the pages).
+ * For each token: the k largest logits, a tie going to the lower expert
+ * index, in descending order; weights w_j = exp(l_j - l_max) / sum over the
+ * selected k, which equals a softmax over all E renormalised over the k.
+ *   logits device float [T, E]; ids device int32 [T, k]; w device float [T, k].
+ * Errors: k < 1, k > E, k > 32, E > 4096 or T < 0 -> INVALID_SHAPE. */
+MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, void *stream);
+
+/* Group the T*k (token, slot) pairs by expert (stable).
+ *   ids device int32 [T, k], every id in [0, E).
+ *   offsets device int32 [E+1]: pairs routed to experts < e.
+ *   src_row device int32 [T*k]: pair index t*k + j at each grouped position;
+ *           experts ascending, within an expert (t, j) ascending.
+ *   dst_of  device int32 [T*k]: grouped position of pair t*k + j.
+ * Errors: T*k > 2^24 or E > 4096 -> INVALID_SHAPE. Ids outside [0, E) are
+ * outside the contract (they are clamped into range, not reported). */
+MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
+                            int32_t *dst_of, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Experts                                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes needed by mxmoe_expert_ffn for these sizes (-1 on bad
+ * sizes). */
+MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I);
+
+/* Grouped SwiGLU expert FFN over MXFP4 weights (W4A16), fp32 accumulation.
+ * For every grouped position r (pair p = src_row[r] = t*k + j, routed to the
+ * expert e with offsets[e] <= r < offsets[e+1]):
+ *   g = W_gate[e] x_t, u = W_up[e] x_t, h = silu(g) * u, y_perm[r] = W_down[e] h.
+ *   x device bf16 [T, H]; offsets, src_row as produced by mxmoe_permute;
+ *   prepacked device blob from mxmoe_prepack_experts; y_perm device float
+ *   [T*k, H]; workspace device, >= mxmoe_ffn_workspace_size bytes, 256-byte
+ *   aligned. Its first 16 bytes hold the device status word of the call.
+ * Activations are carried into the tensor cores as f16 with one power-of-two
+ * scale per 32-element block (exact for bf16 x; h keeps 11 significant bits).
+ * Errors: H % 64, I % 32 != 0, k > 32, E > 1024 -> INVALID_SHAPE; workspace
+ * too small -> WORKSPACE; x, prepacked, y_perm not 16-byte aligned ->
+ * ALIGNMENT. Device-side wait timeouts -> mxmoe_read_status. */
+MXMOE_API int mxmoe_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked,
+                               int T, int k, int E, int H, int I, float *y_perm, void *workspace,
+                               int64_t workspace_bytes, void *stream);
+
+/* Stage 1 of mxmoe_expert_ffn on its own: for every grouped position r,
+ * h[r] = silu(W_gate[e] x_t) * (W_up[e] x_t), written into the workspace (as
+ * f16 values with one power-of-two factor per 32-value block) for
+ * mxmoe_ffn_down. Arguments, layout and errors as for mxmoe_expert_ffn
+ * (workspace from mxmoe_ffn_workspace_size, 256-byte aligned). */
+MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked,
+                                int T, int k, int E, int H, int I, void *workspace, int64_t workspace_bytes,
+                                void *stream);
+
+/* Stage 2 of mxmoe_expert_ffn on its own: y_perm[r] = W_down[e] h[r] for every
+ * grouped position r, reading the h that mxmoe_ffn_gate_up left in the same
+ * workspace (call it first, on the same stream). y_perm device float
+ * [T*k, H], 16-byte aligned. Errors as for mxmoe_expert_ffn. */
+MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, int E, int H, int I,
+                             float *y_perm, void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Weighted combine: y[t, c] = sum over j = 0..k-1 (in order) of
+ * w[t, j] * y_perm[dst_of[t*k + j], c], float32.
+ *   y_perm device float [T*k, H]; dst_of device int32 [T*k]; w device float
+ *   [T, k]; y device float [T, H].
+ * Errors: H % 4 != 0 -> INVALID_SHAPE; y_perm, y not 16-byte aligned ->
+ * ALIGNMENT. */
+MXMOE_API int mxmoe_combine(const float *y_perm, const int32_t *dst_of, const float *w, int T, int k, int H,
+                            float *y, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Whole layer                                                               */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes needed by mxmoe_layer_forward (-1 on bad sizes). */
+MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, int k);
+
+/* The whole MoE expert layer for T tokens: router GEMM, route, permute,
+ * expert FFN, combine, in stream order, with no host synchronisation.
+ *   x device bf16 [T, H]; wg device bf16 [E, H]; bias device float [E] or
+ *   NULL; prepacked device blob (mxmoe_prepack_experts); y device float
+ *   [T, H]; ids_out device int32 [T, k] or NULL; w_out device float [T, k]
+ *   or NULL; workspace device, >= mxmoe_workspace_size bytes, 256-byte
+ *   aligned (its first 16 bytes hold the device status word).
+ * Errors: the union of the steps' errors. */
+MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, const float *bias, const void *prepacked, int T,
+                                  int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out,
+                                  void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Synchronise `stream`, then read the device status word that the last
+ * mxmoe_expert_ffn / mxmoe_layer_forward call on this workspace left:
+ * MXMOE_OK, or MXMOE_ERR_TIMEOUT if a bounded device-side wait gave up.
+ *   workspace device (as passed to the call); *status host int. */
+MXMOE_API int mxmoe_read_status(const void *workspace, int *status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXMOE_H */

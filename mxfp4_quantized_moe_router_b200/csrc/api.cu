@@ -1,0 +1,169 @@
+// api.cu -- error reporting, device checks, workspace sizing, the
+// whole-layer entry point and the status read-back of libmxmoe.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "common.cuh"
+
+namespace mxmoe {
+
+static thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int check_launch(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(MXMOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return MXMOE_OK;
+}
+
+int check_device()
+{
+    static thread_local int cached_dev = -2, cached_ok = 0;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail(MXMOE_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev != cached_dev) {
+        int major = 0;
+        e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e != cudaSuccess)
+            return fail(MXMOE_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+        cached_ok = (major == 10);
+        cached_dev = dev;
+    }
+    if (!cached_ok)
+        return fail(MXMOE_ERR_DEVICE, "device %d is not compute capability 10.x (sm_100a build)", dev);
+    return MXMOE_OK;
+}
+
+// defined in ffn.cu
+int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
+                   int k, int E, int H, int I, float *y_perm, void *workspace, cudaStream_t st);
+int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int T, int k, int H, float *y,
+                cudaStream_t st);
+int64_t ffn_workspace_bytes(int T, int k, int H, int I);
+int validate_ffn_shapes(int T, int k, int E, int H, int I);
+
+namespace {
+
+// Layer workspace: the FFN workspace first (so the status word sits at offset
+// 0), then logits, routing and grouping arrays and the per-pair outputs.
+struct LayerWs {
+    void *ffn;
+    float *logits;
+    int32_t *ids;
+    float *w;
+    int32_t *offsets, *src_row, *dst_of;
+    float *y_perm;
+};
+
+int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *base)
+{
+    int64_t off = 0;
+    auto take = [&](int64_t bytes) {
+        int64_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    const int64_t n = (int64_t)T * k;
+    const int64_t o_ffn = take(ffn_workspace_bytes(T, k, H, I));
+    const int64_t o_logits = take((int64_t)T * E * 4);
+    const int64_t o_ids = take(n * 4);
+    const int64_t o_w = take(n * 4);
+    const int64_t o_off = take((int64_t)(E + 1) * 4);
+    const int64_t o_src = take(n * 4);
+    const int64_t o_dst = take(n * 4);
+    const int64_t o_yp = take(n * H * 4);
+    if (ws && base) {
+        uint8_t *b = static_cast<uint8_t *>(base);
+        ws->ffn = b + o_ffn;
+        ws->logits = reinterpret_cast<float *>(b + o_logits);
+        ws->ids = reinterpret_cast<int32_t *>(b + o_ids);
+        ws->w = reinterpret_cast<float *>(b + o_w);
+        ws->offsets = reinterpret_cast<int32_t *>(b + o_off);
+        ws->src_row = reinterpret_cast<int32_t *>(b + o_src);
+        ws->dst_of = reinterpret_cast<int32_t *>(b + o_dst);
+        ws->y_perm = reinterpret_cast<float *>(b + o_yp);
+    }
+    return off;
+}
+
+}  // namespace
+}  // namespace mxmoe
+
+using namespace mxmoe;
+
+extern "C" MXMOE_API const char *mxmoe_version(void) { return "mxmoe 0.1.0 (sm_100a)"; }
+
+extern "C" MXMOE_API const char *mxmoe_last_error(void) { return g_err; }
+
+extern "C" MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, int k)
+{
+    if (T < 0 || k < 1 || k > 32 || k > E || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 64 || I % 32)
+        return -1;
+    return layer_ws_layout(T, H, I, E, k, nullptr, nullptr);
+}
+
+extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, const float *bias, const void *prepacked,
+                                             int T, int H, int I, int E, int k, float *y, int32_t *ids_out,
+                                             float *w_out, void *workspace, int64_t workspace_bytes, void *stream)
+{
+    if (k > E)
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_layer_forward: k=%d > E=%d", k, E);
+    if (int rc = validate_ffn_shapes(T, k, E, H, I))
+        return rc;
+    const int64_t need = layer_ws_layout(T, H, I, E, k, nullptr, nullptr);
+    if (!workspace || workspace_bytes < need)
+        return fail(MXMOE_ERR_WORKSPACE, "mxmoe_layer_forward: workspace of %lld bytes, need %lld",
+                    (long long)workspace_bytes, (long long)need);
+    if (T == 0)
+        return MXMOE_OK;
+    if (!x || !wg || !prepacked || !y)
+        return fail(MXMOE_ERR_NULL, "mxmoe_layer_forward: NULL pointer");
+    if (!aligned16(x) || !aligned16(wg) || !aligned16(prepacked) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return fail(MXMOE_ERR_ALIGNMENT,
+                    "mxmoe_layer_forward: x, wg, prepacked, y need 16-byte and workspace 256-byte alignment");
+    if (int rc = check_device())
+        return rc;
+    LayerWs ws;
+    layer_ws_layout(T, H, I, E, k, &ws, workspace);
+    int32_t *ids = ids_out ? ids_out : ws.ids;
+    float *w = w_out ? w_out : ws.w;
+    if (int rc = mxmoe_router_gemm(x, wg, bias, T, H, E, ws.logits, stream))
+        return rc;
+    if (int rc = mxmoe_route(ws.logits, T, E, k, ids, w, stream))
+        return rc;
+    if (int rc = mxmoe_permute(ids, T, k, E, ws.offsets, ws.src_row, ws.dst_of, stream))
+        return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (int rc = run_expert_ffn(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn, st))
+        return rc;
+    return run_combine(ws.y_perm, ws.dst_of, w, T, k, H, y, st);
+}
+
+extern "C" MXMOE_API int mxmoe_read_status(const void *workspace, int *status, void *stream)
+{
+    if (!workspace || !status)
+        return fail(MXMOE_ERR_NULL, "mxmoe_read_status: NULL pointer");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess)
+        return fail(MXMOE_ERR_CUDA, "mxmoe_read_status: %s", cudaGetErrorString(e));
+    int v = 0;
+    e = cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess)
+        return fail(MXMOE_ERR_CUDA, "mxmoe_read_status: %s", cudaGetErrorString(e));
+    *status = v;
+    return MXMOE_OK;
+}

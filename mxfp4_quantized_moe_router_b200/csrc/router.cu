@@ -1,0 +1,313 @@
+// router.cu -- router GEMM (float32 logits), top-k routing, and the stable
+// grouping of (token, slot) pairs by expert.
+//
+// Pages: nxbn.cn MiMo-V2.5-Pro-FP4-DFlash article, architecture section: 384
+// experts, 8 activated per token, hidden size 6144. The router function is not
+// on the pages; it is read as the usual MoE gate: softmax over all expert
+// logits, the top k kept (a tie going to the lower expert index) and their
+// weights renormalised to sum 1.
+#include <float.h>
+
+#include "common.cuh"
+
+namespace mxmoe {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Router GEMM: logits[t, e] = sum_k x[t, k] Wg[e, k] + bias[e].
+// CTA tile: 16 experts x 32 tokens; 8 warps split K (warp w takes k32 blocks
+// w, w+8, ...), partial sums reduced in shared memory in a fixed order.
+// Tensor cores with bf16 operands and fp32 accumulation: every bf16 product is
+// exact in fp32. A and B fragments are loaded straight from global memory
+// with the K order permuted identically on both operands (lane t holds 8
+// consecutive k), which leaves the dot products unchanged.
+// ---------------------------------------------------------------------------
+constexpr int kRgExperts = 16, kRgTokens = 32, kRgWarps = 8, kRgUnroll = 4;
+
+__global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__restrict__ x,
+                                                          const uint16_t *__restrict__ wg,
+                                                          const float *__restrict__ bias, int T, int H, int E,
+                                                          float *__restrict__ logits)
+{
+    __shared__ float red[kRgWarps][kRgExperts][kRgTokens + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int e0 = blockIdx.x * kRgExperts, t0 = blockIdx.y * kRgTokens;
+    const int nkb = H / 32;
+    float acc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            acc[j][i] = 0.f;
+    const bool ra = e0 + g < E, rb = e0 + g + 8 < E;
+    const uint16_t *wa = wg + (int64_t)(e0 + g) * H + 8 * t;
+    const uint16_t *wb = wg + (int64_t)(e0 + g + 8) * H + 8 * t;
+    for (int kb0 = warp; kb0 < nkb; kb0 += kRgWarps * kRgUnroll) {
+        uint4 A[kRgUnroll][2];
+        uint4 B[kRgUnroll][4];
+#pragma unroll
+        for (int u = 0; u < kRgUnroll; ++u) {
+            const int kb = kb0 + u * kRgWarps;
+            const bool kv = kb < nkb;
+            A[u][0] = (kv && ra) ? __ldg(reinterpret_cast<const uint4 *>(wa + kb * 32)) : make_uint4(0, 0, 0, 0);
+            A[u][1] = (kv && rb) ? __ldg(reinterpret_cast<const uint4 *>(wb + kb * 32)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int tok = t0 + 8 * j + g;
+                B[u][j] = (kv && tok < T)
+                              ? __ldg(reinterpret_cast<const uint4 *>(x + (int64_t)tok * H + kb * 32 + 8 * t))
+                              : make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRgUnroll; ++u) {
+            const uint32_t a0[4] = {A[u][0].x, A[u][1].x, A[u][0].y, A[u][1].y};
+            const uint32_t a1[4] = {A[u][0].z, A[u][1].z, A[u][0].w, A[u][1].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                mma_bf16_16816(acc[j], a0, B[u][j].x, B[u][j].y, acc[j]);
+                mma_bf16_16816(acc[j], a1, B[u][j].z, B[u][j].w, acc[j]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        red[warp][g][8 * j + 2 * t] = acc[j][0];
+        red[warp][g][8 * j + 2 * t + 1] = acc[j][1];
+        red[warp][g + 8][8 * j + 2 * t] = acc[j][2];
+        red[warp][g + 8][8 * j + 2 * t + 1] = acc[j][3];
+    }
+    __syncthreads();
+    for (int o = threadIdx.x; o < kRgExperts * kRgTokens; o += blockDim.x) {
+        const int er = o % kRgExperts, tc = o / kRgExperts;
+        const int e = e0 + er, tok = t0 + tc;
+        if (e < E && tok < T) {
+            float s = 0.f;
+#pragma unroll
+            for (int w = 0; w < kRgWarps; ++w)
+                s += red[w][er][tc];
+            if (bias)
+                s += bias[e];
+            logits[(int64_t)tok * E + e] = s;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Top-k routing: one warp per token. Lane l holds logits l, l+32, ...; k
+// rounds of a warp arg-max (larger value first, then lower index).
+// ---------------------------------------------------------------------------
+constexpr int kRouteMaxPerLane = 128;  // E <= 4096
+
+template <int V>
+__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
+                                                    int32_t *__restrict__ ids, float *__restrict__ w)
+{
+    const int lane = threadIdx.x & 31;
+    const int tok = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (tok >= T)
+        return;
+    const float *l = logits + (int64_t)tok * E;
+    float v[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? l[e] : -FLT_MAX;
+    }
+    uint32_t taken[(V + 31) / 32];
+#pragma unroll
+    for (int i = 0; i < (V + 31) / 32; ++i)
+        taken[i] = 0;
+    float sel_v = 0.f, top = 0.f;
+    int sel_i = 0;
+    for (int j = 0; j < k; ++j) {
+        float bv = -FLT_MAX;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            const bool free = e < E && !((taken[i / 32] >> (i % 32)) & 1u);
+            if (free && (v[i] > bv || bi == 0x7FFFFFFF)) {
+                bv = v[i];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+            if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) {
+            const int slot = bi >> 5;
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                if (i == slot)
+                    taken[i / 32] |= 1u << (i % 32);
+        }
+        if (j == 0)
+            top = bv;
+        if (lane == j) {
+            sel_v = bv;
+            sel_i = bi;
+        }
+    }
+    // weights: exp(l_j - l_max) / sum over the selected, summed in slot order
+    const float ex = (lane < k) ? expf(sel_v - top) : 0.f;
+    float s = 0.f;
+    for (int j = 0; j < k; ++j)
+        s += __shfl_sync(0xFFFFFFFFu, ex, j);
+    if (lane < k) {
+        ids[(int64_t)tok * k + lane] = sel_i;
+        w[(int64_t)tok * k + lane] = ex / s;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Stable grouping by expert: one CTA of 1024 threads. Counts -> exclusive scan
+// -> offsets; then pairs are placed chunk by chunk (1024 pairs in index order),
+// each pair's rank = earlier chunks' count for its expert + count among lower
+// warps of the chunk + count among lower lanes of its warp.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict__ ids, int n, int E,
+                                                       int32_t *__restrict__ offsets, int32_t *__restrict__ src_row,
+                                                       int32_t *__restrict__ dst_of)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *cursor = sm;            // [E]
+    int32_t *wcnt = sm + E;          // [32][E]
+    int32_t *total = sm + 33 * E;    // [E]: pairs of the current chunk per expert
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = tid; e < E; e += blockDim.x)
+        cursor[e] = 0;
+    __syncthreads();
+    for (int p = tid; p < n; p += blockDim.x)
+        atomicAdd(&cursor[min(max(ids[p], 0), E - 1)], 1);
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of counts by one warp
+        int carry = 0;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            const int c = e < E ? cursor[e] : 0;
+            int incl = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                if (lane >= off)
+                    incl += o;
+            }
+            if (e < E) {
+                cursor[e] = carry + incl - c;
+                offsets[e] = carry + incl - c;
+            }
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0)
+            offsets[E] = carry;
+    }
+    __syncthreads();
+    for (int base = 0; base < n; base += blockDim.x) {
+        for (int i = tid; i < 32 * E; i += blockDim.x)
+            wcnt[i] = 0;
+        __syncthreads();
+        const int p = base + tid;
+        const bool valid = p < n;
+        const int e = valid ? min(max(ids[p], 0), E - 1) : -1;
+        const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid);
+        const uint32_t same = __match_any_sync(0xFFFFFFFFu, e) & vmask;
+        const int in_warp = __popc(same & ((1u << lane) - 1u));
+        if (valid && in_warp == 0)
+            wcnt[warp * E + e] = __popc(same);
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += blockDim.x) {  // exclusive scan over warps, per expert
+            int run = 0;
+            for (int w = 0; w < 32; ++w) {
+                const int c = wcnt[w * E + ee];
+                wcnt[w * E + ee] = run;
+                run += c;
+            }
+            total[ee] = run;
+        }
+        __syncthreads();
+        if (valid) {
+            const int pos = cursor[e] + wcnt[warp * E + e] + in_warp;
+            src_row[pos] = p;
+            dst_of[p] = pos;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += blockDim.x)
+            cursor[ee] += total[ee];
+        __syncthreads();
+    }
+}
+
+}  // namespace
+}  // namespace mxmoe
+
+using namespace mxmoe;
+
+extern "C" MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const float *bias, int T, int H, int E,
+                                           float *logits, void *stream)
+{
+    if (T < 0 || E <= 0 || H <= 0 || H % 32)
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_router_gemm: T=%d H=%d E=%d (H must be a positive multiple of 32)",
+                    T, H, E);
+    if (T == 0)
+        return MXMOE_OK;
+    if (!x || !wg || !logits)
+        return fail(MXMOE_ERR_NULL, "mxmoe_router_gemm: NULL pointer");
+    if (!aligned16(x) || !aligned16(wg))
+        return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_router_gemm: x and wg must be 16-byte aligned");
+    if (int rc = check_device())
+        return rc;
+    dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens);
+    router_gemm_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(static_cast<const uint16_t *>(x),
+                                                              static_cast<const uint16_t *>(wg), bias, T, H, E,
+                                                              logits);
+    return check_launch("router_gemm_kernel");
+}
+
+extern "C" MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, void *stream)
+{
+    if (T < 0 || E <= 0 || E > 4096 || k < 1 || k > E || k > 32)
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_route: T=%d E=%d k=%d (need 1 <= k <= min(E, 32), E <= 4096)", T,
+                    E, k);
+    if (T == 0)
+        return MXMOE_OK;
+    if (!logits || !ids || !w)
+        return fail(MXMOE_ERR_NULL, "mxmoe_route: NULL pointer");
+    if (int rc = check_device())
+        return rc;
+    const int blocks = (T + 7) / 8;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (E <= 32 * 16)
+        route_kernel<16><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w);
+    else
+        route_kernel<kRouteMaxPerLane><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w);
+    return check_launch("route_kernel");
+}
+
+extern "C" MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
+                                       int32_t *dst_of, void *stream)
+{
+    if (T < 0 || k < 1 || E <= 0 || E > 4096 || (int64_t)T * k > (1 << 24))
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_permute: T=%d k=%d E=%d", T, k, E);
+    if (!offsets || (T > 0 && (!ids || !src_row || !dst_of)))
+        return fail(MXMOE_ERR_NULL, "mxmoe_permute: NULL pointer");
+    if (int rc = check_device())
+        return rc;
+    const size_t smem = (size_t)(E + 32 * E + E) * sizeof(int32_t);
+    static thread_local int configured_E = -1;
+    if (smem > 48 * 1024 && configured_E < E) {
+        if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return fail(MXMOE_ERR_CUDA, "mxmoe_permute: cannot reserve %zu bytes of shared memory", smem);
+        configured_E = E;
+    }
+    permute_kernel<<<1, 1024, smem, (cudaStream_t)stream>>>(ids, T * k, E, offsets, src_row, dst_of);
+    return check_launch("permute_kernel");
+}

@@ -71,15 +71,16 @@ double mxo_bf16_to_double(uint16_t b) { return bf16_to_double(b); }
 
 /* Round a non-negative, exactly scaled magnitude q to an E2M1 magnitude code
  * (0..7): the nearest representable value; on a tie, the code whose mantissa
- * bit is 0; anything at or above 6 saturates to 6 (code 7). */
-static int e2m1_round_magnitude(double q)
+ * bit is 0; anything at or above 6 saturates to 6 (code 7). grid[c] is the
+ * value of magnitude code c. */
+static int e2m1_round_magnitude(double q, const double grid[8])
 {
     if (q >= 6.0)
         return 7;
     int best = 0;
-    double bestd = fabs(q - mxo_e2m1_value(0));
+    double bestd = fabs(q - grid[0]);
     for (int c = 1; c < 8; ++c) {
-        double d = fabs(q - mxo_e2m1_value(c));
+        double d = fabs(q - grid[c]);
         if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
             best = c;
             bestd = d;
@@ -88,7 +89,18 @@ static int e2m1_round_magnitude(double q)
     return best;
 }
 
-int mxo_e2m1_round(double q) { return e2m1_round_magnitude(q); }
+static void e2m1_grid(double grid[8])
+{
+    for (int c = 0; c < 8; ++c)
+        grid[c] = mxo_e2m1_value(c);
+}
+
+int mxo_e2m1_round(double q)
+{
+    double grid[8];
+    e2m1_grid(grid);
+    return e2m1_round_magnitude(q, grid);
+}
 
 /* ------------------------------------------------------------------------ */
 /* Quantise / dequantise                                                     */
@@ -110,6 +122,8 @@ int mxo_e2m1_round(double q) { return e2m1_round_magnitude(q); }
 void mxo_quantize(const uint16_t *w, int64_t rows, int64_t K, uint8_t *packed, uint8_t *scales)
 {
     int64_t nblk = K / MXO_BLOCK;
+    double grid[8];
+    e2m1_grid(grid);
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < nblk; ++b) {
             double v[MXO_BLOCK];
@@ -134,7 +148,7 @@ void mxo_quantize(const uint16_t *w, int64_t rows, int64_t K, uint8_t *packed, u
             scales[r * nblk + b] = (uint8_t)(e + 127);
             for (int i = 0; i < MXO_BLOCK; ++i) {
                 double q = ldexp(fabs(v[i]), -e);
-                int code = e2m1_round_magnitude(q) | (signbit(v[i]) ? 8 : 0);
+                int code = e2m1_round_magnitude(q, grid) | (signbit(v[i]) ? 8 : 0);
                 int64_t k = b * MXO_BLOCK + i;
                 uint8_t *byte = &packed[r * (K / 2) + k / 2];
                 if ((k & 1) == 0)
@@ -151,12 +165,17 @@ void mxo_quantize(const uint16_t *w, int64_t rows, int64_t K, uint8_t *packed, u
 void mxo_dequantize(const uint8_t *packed, const uint8_t *scales, int64_t rows, int64_t K, double *out)
 {
     int64_t nblk = K / MXO_BLOCK;
+    double value[16];
+    for (int c = 0; c < 16; ++c)
+        value[c] = mxo_e2m1_value(c);
     for (int64_t r = 0; r < rows; ++r) {
-        for (int64_t k = 0; k < K; ++k) {
-            uint8_t byte = packed[r * (K / 2) + k / 2];
-            int code = (k & 1) ? (byte >> 4) : (byte & 0x0F);
-            double s = mxo_e8m0_value(scales[r * nblk + k / MXO_BLOCK]);
-            out[r * K + k] = mxo_e2m1_value(code) * s;
+        for (int64_t b = 0; b < nblk; ++b) {
+            double s = mxo_e8m0_value(scales[r * nblk + b]);
+            for (int64_t k = b * MXO_BLOCK; k < (b + 1) * MXO_BLOCK; ++k) {
+                uint8_t byte = packed[r * (K / 2) + k / 2];
+                int code = (k & 1) ? (byte >> 4) : (byte & 0x0F);
+                out[r * K + k] = value[code] * s;
+            }
         }
     }
 }

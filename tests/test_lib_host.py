@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/mxmoe.h declares, and rejects bad arguments on the
+host (before anything would be enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxmoe.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"MXMOE_API\s+[\w\s\*]+?\b(mxmoe_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_symbols())
+    for n in ("mxmoe_quantize", "mxmoe_dequantize", "mxmoe_prepack_experts", "mxmoe_router_gemm", "mxmoe_route",
+              "mxmoe_permute", "mxmoe_expert_ffn", "mxmoe_combine", "mxmoe_layer_forward", "mxmoe_workspace_size",
+              "mxmoe_read_status", "mxmoe_last_error", "mxmoe_version"):
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol(mx):
+    lib = ctypes.CDLL(mx.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_binding_names_match_header(mx):
+    for name in declared_symbols():
+        if name in ("mxmoe_version", "mxmoe_last_error"):
+            continue
+        assert hasattr(mx, name), name
+
+
+def test_version(mx):
+    assert mx.version().startswith("mxmoe")
+
+
+def test_prepacked_size_is_format_bytes(mx):
+    # same bytes as the canonical codes + scales: 3*H*I*E*(1/2 + 1/32)
+    for E, H, I in [(384, 6144, 2048), (16, 256, 128), (3, 320, 96)]:
+        assert mx.mxmoe_prepacked_size(E, H, I) == E * 3 * H * I * 17 // 32
+    assert mx.mxmoe_prepacked_size(384, 6144, 2048) == 384 * 20_054_016
+    assert mx.mxmoe_prepacked_size(4, 96, 64) == -1  # H % 64
+    assert mx.mxmoe_prepacked_size(4, 128, 48) == -1  # I % 32
+
+
+def test_workspace_queries(mx):
+    assert mx.mxmoe_workspace_size(8, 6144, 2048, 384, 8) > 0
+    assert mx.mxmoe_workspace_size(8, 6144, 2048, 384, 400) == -1
+    assert mx.mxmoe_ffn_workspace_size(8, 8, 384, 6144, 2048) > 0
+    assert mx.mxmoe_ffn_workspace_size(8, 8, 384, 6100, 2048) == -1
+    # grows with T
+    assert mx.mxmoe_workspace_size(256, 6144, 2048, 384, 8) > mx.mxmoe_workspace_size(8, 6144, 2048, 384, 8)
+
+
+def _lib(mx):
+    return mx.lib
+
+
+def test_quantize_rejects_on_host(mx):
+    lib = _lib(mx)
+    buf = ctypes.create_string_buffer(4096 + 16)
+    base = (ctypes.addressof(buf) + 15) & ~15
+    assert lib.mxmoe_quantize(base, 4, 33, base, base, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_quantize(base, 0, 32, base, base, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_quantize(None, 4, 32, base, base, None) == mx.ERR_NULL
+    assert lib.mxmoe_quantize(base + 2, 4, 32, base, base, None) == mx.ERR_ALIGNMENT
+    assert "multiple of 32" in mx.last_error() or mx.last_error()
+
+
+def test_route_and_permute_reject_on_host(mx):
+    lib = _lib(mx)
+    assert lib.mxmoe_route(None, 4, 16, 0, None, None, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_route(None, 4, 16, 17, None, None, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_route(None, 4, 16, 2, None, None, None) == mx.ERR_NULL
+    assert lib.mxmoe_route(None, 0, 16, 2, None, None, None) == mx.OK  # empty input is a no-op
+    assert lib.mxmoe_permute(None, 4, 2, 5000, None, None, None, None) == mx.ERR_INVALID_SHAPE
+
+
+def test_ffn_and_layer_reject_on_host(mx):
+    lib = _lib(mx)
+    assert lib.mxmoe_expert_ffn(None, None, None, None, 8, 8, 384, 6100, 2048, None, None, 0, None) == \
+        mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_expert_ffn(None, None, None, None, 8, 8, 384, 6144, 2048, None, None, 0, None) == \
+        mx.ERR_WORKSPACE
+    need = mx.mxmoe_workspace_size(8, 6144, 2048, 384, 8)
+    assert lib.mxmoe_layer_forward(None, None, None, None, 8, 6144, 2048, 384, 8, None, None, None, None, need - 1,
+                                   None) == mx.ERR_WORKSPACE
+    assert lib.mxmoe_layer_forward(None, None, None, None, 8, 6144, 2048, 384, 8, None, None, None, 256, need,
+                                   None) == mx.ERR_NULL
+    assert lib.mxmoe_layer_forward(None, None, None, None, 8, 6144, 2048, 384, 9, None, None, None, 256, need,
+                                   None) != mx.OK
+
+
+def test_combine_rejects_on_host(mx):
+    lib = _lib(mx)
+    assert lib.mxmoe_combine(None, None, None, 4, 2, 6, None, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_combine(None, None, None, 4, 2, 8, None, None) == mx.ERR_NULL
+
+
+def test_cpu_only_box_reports_no_device(mx):
+    """Without a GPU an otherwise valid call fails with a CUDA or device error,
+    never silently succeeds (there is no CPU fallback)."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    lib = _lib(mx)
+    buf = ctypes.create_string_buffer(4096 + 16)
+    base = (ctypes.addressof(buf) + 15) & ~15
+    rc = lib.mxmoe_quantize(base, 4, 32, base, base, None)
+    assert rc in (mx.ERR_CUDA, mx.ERR_DEVICE)
