@@ -45,13 +45,15 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--config", default="verify8", choices=[c.name for c in datagen.CONFIGS])
     ap.add_argument("--batches", type=int, default=16, help="distinct rotating input batches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling only: shrink the layer to this many experts (0 = the workload's)")
     return ap.parse_args()
 
 
@@ -257,6 +259,10 @@ def run_native(args):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", torch.cuda.current_device())
     cfg = datagen.BY_NAME[args.config]
+    if args.experts:
+        import dataclasses
+
+        cfg = dataclasses.replace(cfg, name=cfg.name + "-E%d" % args.experts, E=args.experts)
     T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.k, cfg.I
 
     # --- weights (same layer on every rank), quantised and prepacked on the device
@@ -287,21 +293,30 @@ def run_native(args):
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
 
-    # raw C-ABI calls on one stream (the same kernels mxmoe_layer_forward chains)
+    # raw C-ABI calls on one stream
     L = mx.load()
     P = lambda t: None if t is None else t.data_ptr()  # noqa: E731
     fws_bytes = fws.numel()
+    lws = torch.empty(mx.mxmoe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
+    lws_bytes = lws.numel()
 
-    def step(b, ev=None):
+    def layer_step(b, x=None):
+        x = xs[b % nb] if x is None else x
+        rc = L.mxmoe_layer_forward(P(x), P(wg), P(bias), P(prepacked), T, H, I, E, k, P(y), P(ids), P(w), P(lws),
+                                   lws_bytes, sp)
+        if rc:
+            raise RuntimeError("mxmoe_layer_forward failed: " + mx.last_error())
+
+    def split_step(b, ev):
+        """The same layer through the per-step entry points, with events around
+        the gate/up stage (the kernel that streams 2/3 of the weight bytes)."""
         x = xs[b % nb]
         rc = L.mxmoe_router_gemm(P(x), P(wg), P(bias), T, H, E, P(logits), sp)
         rc |= L.mxmoe_route(P(logits), T, E, k, P(ids), P(w), sp)
         rc |= L.mxmoe_permute(P(ids), T, k, E, P(offsets), P(src_row), P(dst_of), sp)
-        if ev is not None:
-            ev[0].record(stream)
+        ev[0].record(stream)
         rc |= L.mxmoe_ffn_gate_up(P(x), P(offsets), P(src_row), P(prepacked), T, k, E, H, I, P(fws), fws_bytes, sp)
-        if ev is not None:
-            ev[1].record(stream)
+        ev[1].record(stream)
         rc |= L.mxmoe_ffn_down(P(offsets), P(prepacked), T, k, E, H, I, P(y_perm), P(fws), fws_bytes, sp)
         rc |= L.mxmoe_combine(P(y_perm), P(dst_of), P(w), T, k, H, P(y), sp)
         if rc:
@@ -310,10 +325,10 @@ def run_native(args):
     # touched experts per batch (untimed), for the weight-byte accounting
     touched = []
     for b in range(nb):
-        step(b)
+        layer_step(b)
         torch.cuda.synchronize()
         touched.append(int(torch.unique(ids).numel()))
-    assert mx.mxmoe_read_status(fws) == mx.OK
+    assert mx.mxmoe_read_status(lws) == mx.OK
 
     def barrier():
         if world > 1:
@@ -331,41 +346,45 @@ def run_native(args):
     clocks.start()
     time.sleep(0.3)
 
-    # --- device-resident timed region
+    # --- device-resident timed region: the whole layer per step
     for i in range(args.warmup):
-        step(i)
-    ev_unit = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        layer_step(i)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     t0 = time.time()
     start.record(stream)
     for i in range(args.steps):
-        step(args.warmup + i, ev_unit[i])
+        layer_step(args.warmup + i)
     end.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
     barrier()
     ms = start.elapsed_time(end)
     ms_max = max_over_ranks(ms)
-    unit_ms = [a.elapsed_time(b) for a, b in ev_unit]
     clk = clocks.summary(t0, t1)
 
-    # --- end to end through the public API with host buffers
-    import ctypes  # noqa: F401
+    # --- roofline region: same steps through the per-step entry points, with
+    # CUDA events on the launching stream around the gate/up stage
+    for i in range(args.warmup):
+        split_step(i, (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+    ev_unit = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        split_step(args.warmup + i, ev_unit[i])
+    torch.cuda.synchronize()
+    barrier()
+    unit_ms = [a.elapsed_time(b) for a, b in ev_unit]
 
+    # --- end to end through the public API with host buffers
     x_host = [xb.cpu().pin_memory() for xb in xs]
     y_host = torch.empty((T, H), dtype=torch.float32).pin_memory()
     x_dev = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    lws = torch.empty(mx.mxmoe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
-    lws_bytes = lws.numel()
 
     def e2e_step(b):
         x_dev.copy_(x_host[b % nb], non_blocking=True)
-        rc = L.mxmoe_layer_forward(P(x_dev), P(wg), P(bias), P(prepacked), T, H, I, E, k, P(y), None, None, P(lws),
-                                   lws_bytes, sp)
-        if rc:
-            raise RuntimeError("mxmoe_layer_forward failed: " + mx.last_error())
+        layer_step(b, x_dev)
         y_host.copy_(y, non_blocking=True)
 
     for i in range(args.warmup):

@@ -53,6 +53,9 @@ int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int 
                 cudaStream_t st);
 int64_t ffn_workspace_bytes(int T, int k, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
+int router_splits(int T, int H, int E);
+int run_router_and_route(const void *x, const void *wg, const float *bias, int T, int H, int E, int k,
+                         float *partials, int nsplit, int32_t *ids, float *w, cudaStream_t st);
 
 namespace {
 
@@ -77,7 +80,7 @@ int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *ba
     };
     const int64_t n = (int64_t)T * k;
     const int64_t o_ffn = take(ffn_workspace_bytes(T, k, H, I));
-    const int64_t o_logits = take((int64_t)T * E * 4);
+    const int64_t o_logits = take((int64_t)router_splits(T, H, E) * T * E * 4);
     const int64_t o_ids = take(n * 4);
     const int64_t o_w = take(n * 4);
     const int64_t o_off = take((int64_t)(E + 1) * 4);
@@ -140,13 +143,11 @@ extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, cons
     layer_ws_layout(T, H, I, E, k, &ws, workspace);
     int32_t *ids = ids_out ? ids_out : ws.ids;
     float *w = w_out ? w_out : ws.w;
-    if (int rc = mxmoe_router_gemm(x, wg, bias, T, H, E, ws.logits, stream))
-        return rc;
-    if (int rc = mxmoe_route(ws.logits, T, E, k, ids, w, stream))
+    cudaStream_t st = (cudaStream_t)stream;
+    if (int rc = run_router_and_route(x, wg, bias, T, H, E, k, ws.logits, router_splits(T, H, E), ids, w, st))
         return rc;
     if (int rc = mxmoe_permute(ids, T, k, E, ws.offsets, ws.src_row, ws.dst_of, stream))
         return rc;
-    cudaStream_t st = (cudaStream_t)stream;
     if (int rc = run_expert_ffn(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn, st))
         return rc;
     return run_combine(ws.y_perm, ws.dst_of, w, T, k, H, y, st);

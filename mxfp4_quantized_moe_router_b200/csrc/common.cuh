@@ -27,21 +27,28 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Layout constants shared by the prepack and FFN kernels
 // ---------------------------------------------------------------------------
 constexpr int kBlock = 32;       // MXFP4 block: elements per E8M0 scale
-constexpr int kChunkK = 256;     // K elements per streamed chunk (8 k32 blocks)
+constexpr int kChunkK = 512;     // K elements per streamed chunk (16 k32 blocks)
 constexpr int kTileRows = 64;    // weight rows per tile (4 slabs of 16)
 constexpr int kConsumerWarps = 8;
 
-// Bytes of one weight chunk covering kw (multiple of 32, <= 256) K elements:
-// nibbles 64 rows * kw/2 = 32*kw, then scales 64 rows * kw/32 = 2*kw.
+// Bytes of one weight chunk covering kw (multiple of 32, <= kChunkK) K
+// elements: nibbles 64 rows * kw/2 = 32*kw, then scales 64 rows * kw/32 = 2*kw.
+// Inside a chunk, k32 block b owns nibble bytes [1024 b, 1024 b + 1024) and
+// scale bytes [32 kw + 64 b, 32 kw + 64 b + 64).
 __host__ __device__ constexpr int64_t wchunk_bytes(int kw) { return 34LL * kw; }
 __host__ __device__ constexpr int64_t wchunk_nibble_bytes(int kw) { return 32LL * kw; }
 // Bytes of a whole weight tile covering K (multiple of 32): 34*K.
 __host__ __device__ constexpr int64_t wtile_bytes(int64_t K) { return 34LL * K; }
 
-// Activation row format ("act16"): a row of K values (K multiple of 32) is
-// stored chunk by chunk (chunks of up to 256 values); a chunk of kw values is
-// kw f16 values (each pre-multiplied by its block's power-of-two factor) then
-// kw/32 float inverse factors, padded to a multiple of 16 bytes.
+// Activation row formats.
+//  * "x16" (gate/up input): a row of K values is K f16 values, each the bf16
+//    input times one power-of-two factor per row; the inverse factors are
+//    kept in a separate float array.
+//  * "h16" (down input): a row of K values (K multiple of 32) is stored chunk
+//    by chunk (chunks of up to kChunkK values); a chunk of kw values is kw
+//    f16 values, each pre-multiplied by its 32-value block's power-of-two
+//    factor, then kw/32 float inverse factors, padded to a multiple of 16
+//    bytes.
 __host__ __device__ constexpr int act_scale_bytes(int kw) { return ((kw / 32) * 4 + 15) & ~15; }
 __host__ __device__ constexpr int act_chunk_bytes(int kw) { return kw * 2 + act_scale_bytes(kw); }
 __host__ __device__ inline int64_t act_row_bytes(int64_t K)
@@ -220,6 +227,17 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t
 __device__ __forceinline__ float e8m0_to_float(uint32_t s)
 {
     return __uint_as_float(s ? (s << 23) : 0x00400000u);
+}
+
+// The four E8M0 bytes of a word as floats 2^(S-127), byte 0 first. Two
+// instructions per scale; a zero byte (2^-127) reads as 0.0, a difference of
+// at most 6 * 2^-127 per weight.
+__device__ __forceinline__ void e8m0x4_to_float(uint32_t w, float &f0, float &f1, float &f2, float &f3)
+{
+    f0 = __uint_as_float((w << 23) & 0x7F800000u);
+    f1 = __uint_as_float((w << 15) & 0x7F800000u);
+    f2 = __uint_as_float((w << 7) & 0x7F800000u);
+    f3 = __uint_as_float((w >> 1) & 0x7F800000u);
 }
 
 // Power-of-two factor that maps a block maximum m (> 0, finite) into

@@ -39,19 +39,22 @@ namespace mxmoe {
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
-constexpr int kActStride = act_chunk_bytes(kChunkK) + 16;  // smem row stride of an act16 chunk (560 B)
+// Shared-memory row stride of one token's activation chunk: 1088 bytes of h16
+// chunk (or 1024 of x16) plus 16 so that ldmatrix rows hit distinct banks.
+constexpr int kActStride = act_chunk_bytes(kChunkK) + 16;
 
 struct StageParams {
     const uint8_t *wblob;     // first tile of this matrix in the prepacked blob
     int tiles_per_expert;     // I/32 (gate/up) or H/64 (down)
     int K;                    // reduction length
-    const uint8_t *act;       // act16 rows
+    const uint8_t *act;       // x16 rows (gate/up) or h16 rows (down)
     int64_t act_row_bytes;
+    const float *act_inv;     // gate/up: per-token inverse factor of x16
     const int32_t *offsets;   // [E+1]
     const int32_t *src_row;   // gate/up: token = src_row[r] / k; down: row r itself
     int k;
     int E;
-    uint8_t *h_out;           // gate/up: act16 rows of h [T*k]
+    uint8_t *h_out;           // gate/up: h16 rows [T*k]
     int64_t h_row_bytes;
     int I;
     float *y_out;             // down: [T*k, H]
@@ -62,13 +65,14 @@ struct StageParams {
 template <int NT>
 struct StageCfg {
     static constexpr int kNTiles = NT / 8;
-    static constexpr int kStages = NT <= 8 ? 6 : (NT <= 16 ? 4 : 4);
-    static constexpr int kWBytes = (int)wchunk_bytes(kChunkK);  // 8704
+    static constexpr int kStages = 3;
+    static constexpr int kWBytes = (int)wchunk_bytes(kChunkK);  // 17408
     static constexpr int kStageBytes = kWBytes + NT * kActStride;
-    static constexpr int kRedFloats = kConsumerWarps * 4 * 16 * NT;
-    static constexpr int kItemCap = 1025;  // item prefix for E <= 1024
+    static constexpr int kRedFloats = 4 * 4 * 16 * NT;  // half the consumer warps' partials
+    static constexpr int kItemCap = 1025;                // item prefix for E <= 1024
     static constexpr size_t kSmem = (size_t)kStages * kStageBytes + (size_t)kRedFloats * 4 +
                                     (size_t)kItemCap * 4 + 2 * kStages * 8 + 64 + 128;
+    static constexpr int kMinBlocks = NT <= 8 ? 2 : 1;
 };
 
 struct Item {
@@ -100,19 +104,74 @@ __device__ __forceinline__ Item decode_item(int64_t idx, const int *item_start, 
     return it;
 }
 
-// GATE_UP = true: stage 1 (SwiGLU epilogue writing act16 h);
-// GATE_UP = false: stage 2 (float output rows).
+// One k32 block of one chunk for one consumer warp: 4 slabs x 16 rows x 32 K of
+// weights against NT activation columns. The E2M1 codes of each slab become
+// f16 A fragments in registers (exact); two m16n8k16 MMAs give the block's
+// partial sums, which are scaled by the weight row's E8M0 scale (and, for the
+// h16 input, by the activation block's inverse factor) into the accumulators.
+template <int NT, bool ACT_BLOCK_SCALES>
+__device__ __forceinline__ void consume_block(const uint8_t *sb, int kw, int b, int lane,
+                                              float (&acc)[4][NT / 8][4])
+{
+    constexpr int NTL = NT / 8;
+    const int g = lane >> 2, t = lane & 3;
+    const uint4 a01 = *reinterpret_cast<const uint4 *>(sb + b * 1024 + lane * 16);
+    const uint4 a23 = *reinterpret_cast<const uint4 *>(sb + b * 1024 + 512 + lane * 16);
+    const uint2 scw = *reinterpret_cast<const uint2 *>(sb + wchunk_nibble_bytes(kw) + b * 64 + g * 8);
+    const uint8_t *act = sb + StageCfg<NT>::kWBytes;
+    uint32_t bf[NTL][4];
+    float sb0[NTL], sb1[NTL];
+#pragma unroll
+    for (int j = 0; j < NTL; ++j) {
+        const uint32_t addr = smem_u32(act + (8 * j + (lane & 7)) * kActStride + (b * 32 + (lane >> 3) * 8) * 2);
+        ldmatrix_x4(bf[j][0], bf[j][1], bf[j][2], bf[j][3], addr);
+        if (ACT_BLOCK_SCALES) {
+            sb0[j] = *reinterpret_cast<const float *>(act + (8 * j + 2 * t) * kActStride + kw * 2 + b * 4);
+            sb1[j] = *reinterpret_cast<const float *>(act + (8 * j + 2 * t + 1) * kActStride + kw * 2 + b * 4);
+        }
+    }
+    float sc[8];  // slab s: rows g -> sc[2s], g+8 -> sc[2s+1]
+    e8m0x4_to_float(scw.x, sc[0], sc[1], sc[2], sc[3]);
+    e8m0x4_to_float(scw.y, sc[4], sc[5], sc[6], sc[7]);
+    const uint32_t words[8] = {a01.x, a01.y, a01.z, a01.w, a23.x, a23.y, a23.z, a23.w};
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        uint32_t A0[4], A1[4];
+        e2m1x4_to_f16x2x4(words[2 * s], A0[0], A0[1], A0[2], A0[3]);
+        e2m1x4_to_f16x2x4(words[2 * s + 1], A1[0], A1[1], A1[2], A1[3]);
+#pragma unroll
+        for (int j = 0; j < NTL; ++j) {
+            float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_f16_16816(tmp, A0, bf[j][0], bf[j][1], tmp);
+            mma_f16_16816(tmp, A1, bf[j][2], bf[j][3], tmp);
+            if (ACT_BLOCK_SCALES) {
+                acc[s][j][0] = fmaf(tmp[0], sc[2 * s] * sb0[j], acc[s][j][0]);
+                acc[s][j][1] = fmaf(tmp[1], sc[2 * s] * sb1[j], acc[s][j][1]);
+                acc[s][j][2] = fmaf(tmp[2], sc[2 * s + 1] * sb0[j], acc[s][j][2]);
+                acc[s][j][3] = fmaf(tmp[3], sc[2 * s + 1] * sb1[j], acc[s][j][3]);
+            } else {
+                acc[s][j][0] = fmaf(tmp[0], sc[2 * s], acc[s][j][0]);
+                acc[s][j][1] = fmaf(tmp[1], sc[2 * s], acc[s][j][1]);
+                acc[s][j][2] = fmaf(tmp[2], sc[2 * s + 1], acc[s][j][2]);
+                acc[s][j][3] = fmaf(tmp[3], sc[2 * s + 1], acc[s][j][3]);
+            }
+        }
+    }
+}
+
+// GATE_UP = true: stage 1 (x16 input, SwiGLU epilogue writing h16);
+// GATE_UP = false: stage 2 (h16 input, float output rows).
 template <int NT, bool GATE_UP>
-__global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const StageParams p)
+__global__ void __launch_bounds__(288, StageCfg<NT>::kMinBlocks) ffn_stage_kernel(const StageParams p)
 {
     using C = StageCfg<NT>;
+    constexpr bool kBlockScales = !GATE_UP;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint8_t *stages = smem;
     float *red = reinterpret_cast<float *>(smem + (size_t)C::kStages * C::kStageBytes);
     int *item_start = reinterpret_cast<int *>(red + C::kRedFloats);
     uint64_t *full = reinterpret_cast<uint64_t *>(item_start + C::kItemCap + 1);
-    // keep the barriers 8-byte aligned
     full = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(full) + 7) & ~uintptr_t(7));
     uint64_t *empty = full + C::kStages;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + C::kStages);
@@ -168,10 +227,10 @@ __global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const 
         for (int64_t idx = i_begin; idx < i_end && ok; ++idx) {
             const Item it = decode_item<NT>(idx, item_start, p.offsets, E, p.tiles_per_expert);
             const uint8_t *wsrc = p.wblob + ((int64_t)it.e * p.tiles_per_expert + it.tile) * tile_bytes;
-            int64_t arow = 0;
+            const uint8_t *arow = p.act;
             if (lane < it.nt) {
                 const int r = it.r0 + lane;
-                arow = GATE_UP ? (int64_t)(p.src_row[r] / p.k) : (int64_t)r;
+                arow += (GATE_UP ? (int64_t)(p.src_row[r] / p.k) : (int64_t)r) * p.act_row_bytes;
             }
             for (int c = 0; c < nchunk; ++c) {
                 const int kw = min(kChunkK, p.K - c * kChunkK);
@@ -183,17 +242,17 @@ __global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const 
                     ok = false;
                     break;
                 }
-                uint8_t *sb = stages + (size_t)stage * C::kStageBytes;
-                const uint32_t abytes = (uint32_t)act_chunk_bytes(kw);
+                uint8_t *sbuf = stages + (size_t)stage * C::kStageBytes;
+                const uint32_t abytes = (uint32_t)(kBlockScales ? act_chunk_bytes(kw) : kw * 2);
+                const int64_t aoff = (int64_t)c * (kBlockScales ? act_chunk_bytes(kChunkK) : kChunkK * 2);
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[stage], (uint32_t)wchunk_bytes(kw) + (uint32_t)it.nt * abytes);
-                    bulk_g2s_hint(sb, wsrc + (int64_t)c * C::kWBytes, (uint32_t)wchunk_bytes(kw), &full[stage], pol_w);
+                    bulk_g2s_hint(sbuf, wsrc + (int64_t)c * C::kWBytes, (uint32_t)wchunk_bytes(kw), &full[stage],
+                                  pol_w);
                 }
                 __syncwarp();
                 if (lane < it.nt)
-                    bulk_g2s_hint(sb + C::kWBytes + lane * kActStride,
-                                  p.act + arow * p.act_row_bytes + (int64_t)c * act_chunk_bytes(kChunkK), abytes,
-                                  &full[stage], pol_a);
+                    bulk_g2s_hint(sbuf + C::kWBytes + lane * kActStride, arow + aoff, abytes, &full[stage], pol_a);
                 ++issued;
                 if (++stage == C::kStages) {
                     stage = 0;
@@ -244,43 +303,13 @@ __global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const 
                 }
                 aborted = true;
             }
-            const uint8_t *sb = stages + (size_t)stage * C::kStageBytes;
-            if (!aborted && warp * 32 < kw) {
-                const uint4 a01 = *reinterpret_cast<const uint4 *>(sb + warp * 1024 + lane * 16);
-                const uint4 a23 = *reinterpret_cast<const uint4 *>(sb + warp * 1024 + 512 + lane * 16);
-                const uint2 scw = *reinterpret_cast<const uint2 *>(sb + wchunk_nibble_bytes(kw) + warp * 64 + g * 8);
-                const uint8_t *act = sb + C::kWBytes;
-                uint32_t b[C::kNTiles][4];
-                float sb0[C::kNTiles], sb1[C::kNTiles];
-#pragma unroll
-                for (int j = 0; j < C::kNTiles; ++j) {
-                    const uint32_t addr =
-                        smem_u32(act + (8 * j + (lane & 7)) * kActStride + (warp * 32 + (lane >> 3) * 8) * 2);
-                    ldmatrix_x4(b[j][0], b[j][1], b[j][2], b[j][3], addr);
-                    sb0[j] = *reinterpret_cast<const float *>(act + (8 * j + 2 * t) * kActStride + kw * 2 + warp * 4);
-                    sb1[j] =
-                        *reinterpret_cast<const float *>(act + (8 * j + 2 * t + 1) * kActStride + kw * 2 + warp * 4);
-                }
-                const uint32_t words[8] = {a01.x, a01.y, a01.z, a01.w, a23.x, a23.y, a23.z, a23.w};
-                const uint32_t scb[8] = {scw.x & 0xFF, (scw.x >> 8) & 0xFF, (scw.x >> 16) & 0xFF, scw.x >> 24,
-                                         scw.y & 0xFF, (scw.y >> 8) & 0xFF, (scw.y >> 16) & 0xFF, scw.y >> 24};
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    uint32_t A0[4], A1[4];
-                    e2m1x4_to_f16x2x4(words[2 * s], A0[0], A0[1], A0[2], A0[3]);
-                    e2m1x4_to_f16x2x4(words[2 * s + 1], A1[0], A1[1], A1[2], A1[3]);
-                    const float sg = e8m0_to_float(scb[2 * s]), sg8 = e8m0_to_float(scb[2 * s + 1]);
-#pragma unroll
-                    for (int j = 0; j < C::kNTiles; ++j) {
-                        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_f16_16816(tmp, A0, b[j][0], b[j][1], tmp);
-                        mma_f16_16816(tmp, A1, b[j][2], b[j][3], tmp);
-                        acc[s][j][0] = fmaf(tmp[0], sg * sb0[j], acc[s][j][0]);
-                        acc[s][j][1] = fmaf(tmp[1], sg * sb1[j], acc[s][j][1]);
-                        acc[s][j][2] = fmaf(tmp[2], sg8 * sb0[j], acc[s][j][2]);
-                        acc[s][j][3] = fmaf(tmp[3], sg8 * sb1[j], acc[s][j][3]);
-                    }
-                }
+            const uint8_t *sbuf = stages + (size_t)stage * C::kStageBytes;
+            if (!aborted) {
+                // warp w takes k32 blocks 2w and 2w+1 of the chunk
+                if (2 * warp * 32 < kw)
+                    consume_block<NT, kBlockScales>(sbuf, kw, 2 * warp, lane, acc);
+                if ((2 * warp + 1) * 32 < kw)
+                    consume_block<NT, kBlockScales>(sbuf, kw, 2 * warp + 1, lane, acc);
             }
             __syncwarp();
             if (lane == 0)
@@ -291,18 +320,29 @@ __global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const 
             }
         }
         // ------------------------------------------------------------ epilogue
-        // red[((w*4 + s)*16 + row16)*NT + n]
+        // Two-level reduction over the 8 warps in a fixed order: warps 4..7
+        // store, warps 0..3 add their own partials, then the output threads add
+        // the four sums. red[((w*4 + s)*16 + row16)*NT + n], w < 4.
+        auto store_acc = [&](int w, bool add) {
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
+            for (int s = 0; s < 4; ++s)
 #pragma unroll
-            for (int j = 0; j < C::kNTiles; ++j) {
-                const int n0 = 8 * j + 2 * t;
-                float *rw = red + ((warp * 4 + s) * 16) * NT;
-                rw[g * NT + n0] = acc[s][j][0];
-                rw[g * NT + n0 + 1] = acc[s][j][1];
-                rw[(g + 8) * NT + n0] = acc[s][j][2];
-                rw[(g + 8) * NT + n0 + 1] = acc[s][j][3];
-            }
+                for (int j = 0; j < C::kNTiles; ++j) {
+                    const int n0 = 8 * j + 2 * t;
+                    float *rw = red + ((w * 4 + s) * 16) * NT;
+                    const float v[4] = {acc[s][j][0], acc[s][j][1], acc[s][j][2], acc[s][j][3]};
+                    float *d[4] = {&rw[g * NT + n0], &rw[g * NT + n0 + 1], &rw[(g + 8) * NT + n0],
+                                   &rw[(g + 8) * NT + n0 + 1]};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        *d[i] = add ? *d[i] + v[i] : v[i];
+                }
+        };
+        if (warp >= 4)
+            store_acc(warp - 4, false);
+        named_bar_sync(1, kConsumerWarps * 32);
+        if (warp < 4)
+            store_acc(warp, true);
         named_bar_sync(1, kConsumerWarps * 32);
         aborted = aborted || *abort_flag;
         if (aborted) {
@@ -316,10 +356,13 @@ __global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const 
             for (int n = warp; n < it.nt; n += kConsumerWarps) {
                 float gs = 0.f, us = 0.f;
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
+                for (int w = 0; w < 4; ++w) {
                     gs += red[((w * 4 + sg) * 16 + r16) * NT + n];
                     us += red[((w * 4 + 2 + sg) * 16 + r16) * NT + n];
                 }
+                const float xinv = p.act_inv[p.src_row[it.r0 + n] / p.k];
+                gs *= xinv;
+                us *= xinv;
                 const float h = gs / (1.f + expf(-gs)) * us;
                 float m = fabsf(h);
 #pragma unroll
@@ -341,7 +384,7 @@ __global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const 
                     const int rr = lane + 32 * half, s = rr >> 4, r16 = rr & 15;
                     float v = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w)
+                    for (int w = 0; w < 4; ++w)
                         v += red[((w * 4 + s) * 16 + r16) * NT + n];
                     yrow[rr] = v;
                 }
@@ -351,50 +394,55 @@ __global__ void __launch_bounds__(288, NT <= 16 ? 2 : 1) ffn_stage_kernel(const 
     }
 }
 
-// bf16 rows -> act16 rows. One warp per (row, 256-wide chunk); lane = (block
-// lane/4, part lane%4) converts 8 values. Block 0 also clears the status word.
+// bf16 rows -> x16 rows: one block per row; pass 1 finds max |x| of the row,
+// pass 2 writes x * 2^(14 - floor(log2 max)) as f16 and stores the inverse
+// factor. Block 0 also clears the status word.
 __global__ void __launch_bounds__(256) act_convert_kernel(const uint16_t *__restrict__ x, int64_t rows, int K,
-                                                          uint8_t *__restrict__ out, int64_t out_row_bytes,
+                                                          uint16_t *__restrict__ out, float *__restrict__ inv_out,
                                                           int *status)
 {
+    __shared__ float wmax[8];
     if (blockIdx.x == 0 && threadIdx.x == 0 && status)
         *status = 0;
-    const int lane = threadIdx.x & 31;
-    const int nchunk = (K + kChunkK - 1) / kChunkK;
-    const int64_t total = rows * nchunk;
-    for (int64_t item = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); item < total; item += (int64_t)gridDim.x * 8) {
-        const int64_t r = item / nchunk;
-        const int c = (int)(item % nchunk);
-        const int kw = min(kChunkK, K - c * kChunkK);
-        const int kk = (lane >> 2) * 32 + (lane & 3) * 8;
-        const bool valid = kk < kw;
-        float f[8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n16 = K / 8;  // 16-byte groups of 8 values
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + r * K);
         float m = 0.f;
-        if (valid) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + r * K + c * kChunkK + kk));
+        for (int i = threadIdx.x; i < n16; i += blockDim.x) {
+            const uint4 v = __ldg(src + i);
             const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                f[2 * i] = __uint_as_float(wv[i] << 16);
-                f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-                m = fmaxf(m, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
-            }
+            for (int q = 0; q < 4; ++q)
+                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[q] << 16)), fabsf(__uint_as_float(wv[q] & 0xFFFF0000u))));
         }
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        if (valid) {
-            float mul, inv;
-            act_block_factor(m, mul, inv);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+        if (lane == 0)
+            wmax[warp] = m;
+        __syncthreads();
+        m = wmax[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w)
+            m = fmaxf(m, wmax[w]);
+        float mul, inv;
+        act_block_factor(m, mul, inv);
+        uint4 *dst = reinterpret_cast<uint4 *>(out + r * K);
+        for (int i = threadIdx.x; i < n16; i += blockDim.x) {
+            const uint4 v = __ldg(src + i);
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
             uint32_t hv[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                hv[i] = (uint32_t)__half_as_ushort(__float2half_rn(f[2 * i] * mul)) |
-                        ((uint32_t)__half_as_ushort(__float2half_rn(f[2 * i + 1] * mul)) << 16);
-            uint8_t *dst = out + r * out_row_bytes + (int64_t)c * act_chunk_bytes(kChunkK);
-            *reinterpret_cast<uint4 *>(dst + kk * 2) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            if ((lane & 3) == 0)
-                reinterpret_cast<float *>(dst + kw * 2)[kk / 32] = inv;
+            for (int q = 0; q < 4; ++q)
+                hv[q] = (uint32_t)__half_as_ushort(__float2half_rn(__uint_as_float(wv[q] << 16) * mul)) |
+                        ((uint32_t)__half_as_ushort(__float2half_rn(__uint_as_float(wv[q] & 0xFFFF0000u) * mul))
+                         << 16);
+            dst[i] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
+        if (threadIdx.x == 0)
+            inv_out[r] = inv;
+        __syncthreads();  // wmax is reused by the next row
     }
 }
 
@@ -425,7 +473,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 // ---------------------------------------------------------------------------
 struct FfnWs {
     int *status;
-    uint8_t *x16;
+    uint16_t *x16;
+    float *xinv;
     uint8_t *h16;
 };
 
@@ -438,12 +487,14 @@ int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
         return o;
     };
     const int64_t o_status = take(16);
-    const int64_t o_x16 = take((int64_t)T * act_row_bytes(H));
+    const int64_t o_x16 = take((int64_t)T * H * 2);
+    const int64_t o_xinv = take((int64_t)T * 4);
     const int64_t o_h16 = take((int64_t)T * k * act_row_bytes(I));
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
         ws->status = reinterpret_cast<int *>(b + o_status);
-        ws->x16 = b + o_x16;
+        ws->x16 = reinterpret_cast<uint16_t *>(b + o_x16);
+        ws->xinv = reinterpret_cast<float *>(b + o_xinv);
         ws->h16 = b + o_h16;
     }
     return off;
@@ -487,8 +538,6 @@ int launch_stage_nt(int T, const StageParams &p, cudaStream_t st)
 {
     if (T <= 8)
         return launch_stage<8, GATE_UP>(p, st);
-    if (T <= 16)
-        return launch_stage<16, GATE_UP>(p, st);
     return launch_stage<32, GATE_UP>(p, st);
 }
 
@@ -509,12 +558,10 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
 {
     FfnWs ws;
     ffn_ws_layout(T, k, H, I, &ws, workspace);
-    const int64_t xrow = act_row_bytes(H), hrow = act_row_bytes(I);
     {
-        const int64_t items = (int64_t)T * ((H + kChunkK - 1) / kChunkK);
-        int blocks = (int)std::min<int64_t>((items + 7) / 8, (int64_t)num_sms() * 16);
+        int blocks = (int)std::min<int64_t>((int64_t)T, (int64_t)num_sms() * 8);
         act_convert_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), T, H, ws.x16,
-                                                                    xrow, ws.status);
+                                                                    ws.xinv, ws.status);
         if (int rc = check_launch("act_convert_kernel"))
             return rc;
     }
@@ -522,14 +569,15 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     p1.wblob = static_cast<const uint8_t *>(prepacked);
     p1.tiles_per_expert = I / 32;
     p1.K = H;
-    p1.act = ws.x16;
-    p1.act_row_bytes = xrow;
+    p1.act = reinterpret_cast<const uint8_t *>(ws.x16);
+    p1.act_row_bytes = (int64_t)H * 2;
+    p1.act_inv = ws.xinv;
     p1.offsets = offsets;
     p1.src_row = src_row;
     p1.k = k;
     p1.E = E;
     p1.h_out = ws.h16;
-    p1.h_row_bytes = hrow;
+    p1.h_row_bytes = act_row_bytes(I);
     p1.I = I;
     p1.y_out = nullptr;
     p1.H = H;
@@ -548,6 +596,7 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
     p2.K = I;
     p2.act = ws.h16;
     p2.act_row_bytes = act_row_bytes(I);
+    p2.act_inv = nullptr;
     p2.offsets = offsets;
     p2.src_row = nullptr;
     p2.k = k;

@@ -73,6 +73,15 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
     }
 }
 
+// Value of an E2M1 code from its fields: exponent e = bits 2..1, mantissa m =
+// bit 0, sign bit 3; e == 0 gives m * 0.5, otherwise 2^(e-1) * (1 + m/2).
+__device__ __forceinline__ float e2m1_decode(uint32_t c)
+{
+    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    const float mag = e ? __uint_as_float(((e + 126u) << 23) | (m << 22)) : 0.5f * (float)m;
+    return (c & 8u) ? -mag : mag;
+}
+
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restrict__ packed,
                                                          const uint8_t *__restrict__ scales, int64_t rows,
                                                          int64_t K, float *__restrict__ out)
@@ -82,10 +91,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = i / (K / 2), kk = (i % (K / 2)) * 2;
         const float s = e8m0_to_float(scales[r * (K / 32) + kk / 32]);
-        uint32_t h01, unused1, unused2, unused3;
-        e2m1x4_to_f16x2x4((uint32_t)packed[i], h01, unused1, unused2, unused3);
-        const float lo = __half2float(__ushort_as_half((unsigned short)(h01 & 0xFFFFu)));
-        const float hi = __half2float(__ushort_as_half((unsigned short)(h01 >> 16)));
+        const uint32_t byte = packed[i];
+        const float lo = e2m1_decode(byte & 0xF), hi = e2m1_decode(byte >> 4);
         *reinterpret_cast<float2 *>(out + r * K + kk) = make_float2(lo * s, hi * s);
     }
 }
@@ -106,15 +113,15 @@ __global__ void __launch_bounds__(256) prepack_kernel(const uint8_t *__restrict_
                                                       int K, int tiles_per_expert, bool gate_up, int I,
                                                       uint8_t *__restrict__ dst)
 {
-    const int nchunk = (K + 255) / 256;
+    const int nchunk = (K + kChunkK - 1) / kChunkK;
     const int64_t blk = blockIdx.x;
     const int c = (int)(blk % nchunk);
     const int tile = (int)((blk / nchunk) % tiles_per_expert);
     const int e = (int)(blk / ((int64_t)nchunk * tiles_per_expert));
-    const int k0 = c * 256;
-    const int kw = min(256, K - k0);
+    const int k0 = c * kChunkK;
+    const int kw = min(kChunkK, K - k0);
     const int64_t ebase = (int64_t)e * rows_per_expert;
-    uint8_t *out = dst + ((int64_t)e * tiles_per_expert + tile) * wtile_bytes(K) + (int64_t)c * wchunk_bytes(256);
+    uint8_t *out = dst + ((int64_t)e * tiles_per_expert + tile) * wtile_bytes(K) + (int64_t)c * wchunk_bytes(kChunkK);
     // nibble part: word index = ((w*2 + half)*32 + lane)*4 + jj
     const int nwords = (int)(wchunk_nibble_bytes(kw) / 4);
     for (int i = threadIdx.x; i < nwords; i += blockDim.x) {
@@ -210,12 +217,12 @@ extern "C" MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const ui
         return rc;
     uint8_t *dst = static_cast<uint8_t *>(prepacked);
     cudaStream_t st = (cudaStream_t)stream;
-    const int64_t blocks13 = (int64_t)E * (I / 32) * ((H + 255) / 256);
+    const int64_t blocks13 = (int64_t)E * (I / 32) * ((H + kChunkK - 1) / kChunkK);
     prepack_kernel<<<(unsigned)blocks13, 256, 0, st>>>(packed13, sc13, E, 2 * I, H, I / 32, true, I, dst);
     if (int rc = check_launch("prepack_kernel(gate/up)"))
         return rc;
     uint8_t *dst2 = dst + (int64_t)E * (I / 32) * wtile_bytes(H);
-    const int64_t blocks2 = (int64_t)E * (H / 64) * ((I + 255) / 256);
+    const int64_t blocks2 = (int64_t)E * (H / 64) * ((I + kChunkK - 1) / kChunkK);
     prepack_kernel<<<(unsigned)blocks2, 256, 0, st>>>(packed2, sc2, E, H, I, H / 64, false, I, dst2);
     return check_launch("prepack_kernel(down)");
 }

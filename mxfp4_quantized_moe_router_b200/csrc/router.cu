@@ -8,6 +8,8 @@
 // weights renormalised to sum 1.
 #include <float.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace mxmoe {
@@ -15,8 +17,11 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Router GEMM: logits[t, e] = sum_k x[t, k] Wg[e, k] + bias[e].
-// CTA tile: 16 experts x 32 tokens; 8 warps split K (warp w takes k32 blocks
-// w, w+8, ...), partial sums reduced in shared memory in a fixed order.
+// CTA tile: 16 experts x 32 tokens x (K / gridDim.z); 8 warps split the CTA's
+// K range (warp w takes its k32 blocks w, w+8, ...), partial sums reduced in
+// shared memory in a fixed order. With gridDim.z > 1 each CTA writes its
+// partial sums to out[z][t][e] (no bias) and the routing kernel adds the
+// splits in order.
 // Tensor cores with bf16 operands and fp32 accumulation: every bf16 product is
 // exact in fp32. A and B fragments are loaded straight from global memory
 // with the K order permuted identically on both operands (lane t holds 8
@@ -33,7 +38,10 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int e0 = blockIdx.x * kRgExperts, t0 = blockIdx.y * kRgTokens;
-    const int nkb = H / 32;
+    const int nkb_all = H / 32;
+    const int kb_lo = (int)((int64_t)nkb_all * blockIdx.z / gridDim.z);
+    const int kb_hi = (int)((int64_t)nkb_all * (blockIdx.z + 1) / gridDim.z);
+    logits += (int64_t)blockIdx.z * T * E;
     float acc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -43,13 +51,13 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
     const bool ra = e0 + g < E, rb = e0 + g + 8 < E;
     const uint16_t *wa = wg + (int64_t)(e0 + g) * H + 8 * t;
     const uint16_t *wb = wg + (int64_t)(e0 + g + 8) * H + 8 * t;
-    for (int kb0 = warp; kb0 < nkb; kb0 += kRgWarps * kRgUnroll) {
+    for (int kb0 = kb_lo + warp; kb0 < kb_hi; kb0 += kRgWarps * kRgUnroll) {
         uint4 A[kRgUnroll][2];
         uint4 B[kRgUnroll][4];
 #pragma unroll
         for (int u = 0; u < kRgUnroll; ++u) {
             const int kb = kb0 + u * kRgWarps;
-            const bool kv = kb < nkb;
+            const bool kv = kb < kb_hi;
             A[u][0] = (kv && ra) ? __ldg(reinterpret_cast<const uint4 *>(wa + kb * 32)) : make_uint4(0, 0, 0, 0);
             A[u][1] = (kv && rb) ? __ldg(reinterpret_cast<const uint4 *>(wb + kb * 32)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -87,7 +95,7 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
 #pragma unroll
             for (int w = 0; w < kRgWarps; ++w)
                 s += red[w][er][tc];
-            if (bias)
+            if (bias && gridDim.z == 1)
                 s += bias[e];
             logits[(int64_t)tok * E + e] = s;
         }
@@ -100,8 +108,11 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
 // ---------------------------------------------------------------------------
 constexpr int kRouteMaxPerLane = 128;  // E <= 4096
 
+// With nsplit > 1 the logits are the sum, in split order, of nsplit partial
+// [T, E] arrays plus bias (the split router GEMM's output).
 template <int V>
-__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int nsplit,
+                                                    const float *__restrict__ bias, int T, int E, int k,
                                                     int32_t *__restrict__ ids, float *__restrict__ w)
 {
     const int lane = threadIdx.x & 31;
@@ -114,6 +125,27 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
     for (int i = 0; i < V; ++i) {
         const int e = lane + 32 * i;
         v[i] = e < E ? l[e] : -FLT_MAX;
+    }
+    // add the other splits in split order; each split's loads are independent
+    for (int z = 1; z < nsplit; ++z) {
+        const float *lz = l + (int64_t)z * T * E;
+        float pz[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            pz[i] = e < E ? lz[e] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+            v[i] += pz[i];
+    }
+    if (bias) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E)
+                v[i] += bias[e];
+        }
     }
     uint32_t taken[(V + 31) / 32];
 #pragma unroll
@@ -264,12 +296,46 @@ extern "C" MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const 
         return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_router_gemm: x and wg must be 16-byte aligned");
     if (int rc = check_device())
         return rc;
-    dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens);
+    dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens, 1);
     router_gemm_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(static_cast<const uint16_t *>(x),
                                                               static_cast<const uint16_t *>(wg), bias, T, H, E,
                                                               logits);
     return check_launch("router_gemm_kernel");
 }
+
+namespace mxmoe {
+
+// K splits for the layer's router GEMM: enough CTAs to cover the GPU at
+// decode sizes, each split at least 8 k32 blocks (one per warp).
+int router_splits(int T, int H, int E)
+{
+    const int64_t base = (int64_t)((E + kRgExperts - 1) / kRgExperts) * ((T + kRgTokens - 1) / kRgTokens);
+    int z = (int)((2 * 148 + base / 2) / std::max<int64_t>(base, 1));
+    z = std::max(1, std::min(z, 8));
+    z = std::min(z, std::max(1, (H / 32) / 8));
+    return z;
+}
+
+// Router GEMM into nsplit partial arrays plus routing that sums them (the
+// layer path). partials: float [nsplit, T, E].
+int run_router_and_route(const void *x, const void *wg, const float *bias, int T, int H, int E, int k,
+                         float *partials, int nsplit, int32_t *ids, float *w, cudaStream_t st)
+{
+    dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens, nsplit);
+    router_gemm_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(wg),
+                                             bias, T, H, E, partials);
+    if (int rc = check_launch("router_gemm_kernel"))
+        return rc;
+    const int blocks = (T + 7) / 8;
+    if (E <= 32 * 16)
+        route_kernel<16><<<blocks, 256, 0, st>>>(partials, nsplit, nsplit > 1 ? bias : nullptr, T, E, k, ids, w);
+    else
+        route_kernel<kRouteMaxPerLane><<<blocks, 256, 0, st>>>(partials, nsplit, nsplit > 1 ? bias : nullptr, T,
+                                                               E, k, ids, w);
+    return check_launch("route_kernel");
+}
+
+}  // namespace mxmoe
 
 extern "C" MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, void *stream)
 {
@@ -285,9 +351,9 @@ extern "C" MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, i
     const int blocks = (T + 7) / 8;
     cudaStream_t st = (cudaStream_t)stream;
     if (E <= 32 * 16)
-        route_kernel<16><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w);
+        route_kernel<16><<<blocks, 256, 0, st>>>(logits, 1, nullptr, T, E, k, ids, w);
     else
-        route_kernel<kRouteMaxPerLane><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w);
+        route_kernel<kRouteMaxPerLane><<<blocks, 256, 0, st>>>(logits, 1, nullptr, T, E, k, ids, w);
     return check_launch("route_kernel");
 }
 
