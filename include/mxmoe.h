@@ -186,6 +186,30 @@ MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets, const int
 MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, int E, int H, int I,
                              float *y_perm, void *workspace, int64_t workspace_bytes, void *stream);
 
+/* Workspace-free variant of mxmoe_expert_ffn for callers that cannot
+ * allocate device memory: for example a process whose device memory is all
+ * reserved by another allocator's pool, or a latency-critical loop in which
+ * cudaMalloc (which may synchronise the device) is not allowed. There is no
+ * counterpart on the pages; it exists only for such callers.
+ * Arguments, layout and results are those of mxmoe_expert_ffn, minus the
+ * workspace. Scratch is a fixed 4 MiB static device array inside the library
+ * (held on every GPU where the library's device code is loaded, until the
+ * process exits); sizes whose mxmoe_ffn_workspace_size exceeds 4 MiB are
+ * rejected with MXMOE_ERR_WORKSPACE before anything is enqueued (the
+ * 6144/2048/top-8 layer fits up to 64 tokens).
+ *   status  device int or NULL: when given, receives the call's device status
+ *           word (MXMOE_OK or MXMOE_ERR_TIMEOUT) in stream order.
+ * The first call on each device looks up the array's device address (once,
+ * under a lock); make that first call before any stream capture. The call
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * All calls share the one array and it keeps the last call's contents (the
+ * call itself clears what must start at zero), so calls whose work overlaps
+ * on the GPU (different streams, or several host threads) race: serialise
+ * them, for example on one stream. */
+MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *offsets, const int32_t *src_row,
+                                       const void *prepacked, int T, int k, int E, int H, int I, float *y_perm,
+                                       int *status, void *stream);
+
 /* Weighted combine: y[t, c] = sum over j = 0..k-1 (in order) of
  * w[t, j] * y_perm[dst_of[t*k + j], c], float32.
  *   y_perm device float [T*k, H]; dst_of device int32 [T*k]; w device float

@@ -46,6 +46,7 @@ _SIGS = {
     "mxmoe_expert_ffn": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I64, _P]),
     "mxmoe_ffn_gate_up": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
     "mxmoe_ffn_down": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _I64, _P]),
+    "mxmoe_expert_ffn_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "mxmoe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "mxmoe_workspace_size": (_I64, [_I, _I, _I, _I, _I]),
     "mxmoe_layer_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
@@ -264,6 +265,23 @@ def mxmoe_ffn_down(offsets, prepacked, T, k, E, H, I, y_perm, workspace, stream=
     _check("mxmoe_ffn_down",
            load().mxmoe_ffn_down(_ptr(offsets), _ptr(prepacked), T, k, E, H, I, _ptr(y_perm), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def mxmoe_expert_ffn_noalloc(x, offsets, src_row, prepacked, k, E, I, y_perm, status=None, stream=None):
+    """mxmoe_expert_ffn without a workspace (scratch in the library's fixed
+    4 MiB static device array); for callers that cannot allocate."""
+    import torch
+
+    T, H = x.shape
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(src_row, torch.int32, (T * k,), "src_row")
+    _need(y_perm, torch.float32, (T * k, H), "y_perm")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    _check("mxmoe_expert_ffn_noalloc",
+           load().mxmoe_expert_ffn_noalloc(_ptr(x), _ptr(offsets), _ptr(src_row), _ptr(prepacked), T, k, E, H, I,
+                                           _ptr(y_perm), _ptr(status), _stream(stream)))
 
 
 def mxmoe_combine(y_perm, dst_of, w, y, stream=None):
