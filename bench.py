@@ -91,15 +91,17 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the gate/up stage from a committed ncu summary,
-    only if the kernel source is unchanged since that capture."""
+def profiled_traffic(workload: str, touched: float):
+    """DRAM bytes (read + write) per launch of the gate/up stage, from the
+    committed ncu capture of the same kernel source (null once the source has
+    changed). The capture's bytes per touched expert are scaled to this run's
+    mean number of touched experts per launch."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
         ent = d.get("ffn_gate_up", {}).get(workload)
         if ent and ent.get("source_sha") == kernel_source_sha():
-            return float(ent["dram_bytes_per_launch"])
+            return float(ent["dram_bytes_per_touched_expert"]) * touched
     except Exception:
         pass
     return None
@@ -432,7 +434,7 @@ def run_native(args):
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
                      else "fallback 6.65 TB/s",
-                     "traffic": profiled_traffic(cfg.name), "unit_ms": unit_ms_mean,
+                     "traffic": profiled_traffic(cfg.name, mean_touched), "unit_ms": unit_ms_mean,
                      "algorithmic_bytes_per_launch": unit_bytes},
         "clocks": clk,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
