@@ -38,7 +38,7 @@ import datagen  # noqa: E402
 
 METRIC = "MXFP4 MoE-layer tokens/s; expert-weight HBM GB/s as % of peak (1×B200)"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 7  # router_gemm, route, permute, act_convert, stage gate/up, stage down, combine
+KERNELS_PER_STEP = 7  # router_gemm, route, permute, x_terms, ffn gate/up, ffn down, combine
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -85,7 +85,8 @@ def load_peaks():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for rel in ("mxfp4_quantized_moe_router_b200/csrc/ffn.cu", "mxfp4_quantized_moe_router_b200/csrc/common.cuh"):
+    for rel in ("mxfp4_quantized_moe_router_b200/csrc/ffn.cu", "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
+                "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -415,7 +416,7 @@ def run_native(args):
     value = tokens / (ms_max / 1e3)
     weight_bytes_step = mean_touched * cfg.expert_bytes
     weight_gbs = weight_bytes_step * args.steps / (ms / 1e3) / 1e9
-    # dominant unit: mxmoe_ffn_gate_up (act_convert + gate/up stage); algorithmic
+    # dominant unit: mxmoe_ffn_gate_up (x_terms + gate/up stage); algorithmic
     # bytes = gate/up MXFP4 bytes of the touched experts + x read + h written
     w13_bytes = 2 * I * H * 17 // 32
     unit_bytes = mean_touched * w13_bytes + T * H * 2 + T * k * I * 2
@@ -424,13 +425,13 @@ def run_native(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e2m1xf16->f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
+        "dtype": "e2m1 x e4m3 terms -> f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
                                           "W~N(0,0.02) quantised to MXFP4 by the library)",
         "config": workload_config(cfg, world, nb),
         "weight_gbs": weight_gbs,
         "weight_frac_of_hbm_peak": weight_gbs / peak,
         "touched_experts_per_step": mean_touched,
-        "roofline": {"kernel": "mxmoe_ffn_gate_up (act_convert_kernel + ffn_stage_kernel<gate_up>)",
+        "roofline": {"kernel": "mxmoe_ffn_gate_up (x_terms_kernel + ffn_tc_kernel<gate_up>)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
                      else "fallback 6.65 TB/s",

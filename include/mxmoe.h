@@ -92,24 +92,29 @@ MXMOE_API int mxmoe_dequantize(const uint8_t *packed, const uint8_t *scales, int
 
 /* Bytes of the prepacked expert blob for E experts of hidden size H and
  * intermediate size I (= E * 3 * H * I * 17/32, the same bytes as the packed
- * codes plus scales). Returns -1 if H % 64 or I % 32 is non-zero or a size is
- * not positive. */
+ * codes plus scales). Returns -1 unless H and I are positive multiples of 128.
+ */
 MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I);
 
-/* Re-tile canonical MXFP4 expert weights into the layout the FFN kernels
- * stream (a pure byte permutation; nothing is re-rounded).
+/* Re-tile canonical MXFP4 expert weights into the layout the tensor-core FFN
+ * streams (a pure byte permutation; nothing is re-rounded).
  *   packed13 device uint8 [E, 2I, H/2], sc13 device uint8 [E, 2I, H/32]:
  *            rows 0..I-1 of each expert are the gate projection, rows
  *            I..2I-1 the up projection (each row a K = H vector).
  *   packed2  device uint8 [E, H, I/2], sc2 device uint8 [E, H, I/32]: down
  *            projection (each row a K = I vector).
- *   prepacked device, mxmoe_prepacked_size(E, H, I) bytes, 16-byte aligned.
- * Layout of the blob: all gate/up tiles, then all down tiles. A tile is 64
- * weight rows (gate/up: 32 gate rows and the 32 matching up rows) split along
- * K into chunks of up to 256 elements; a chunk holds the nibbles in the order
- * the tensor-core fragments consume them, then the scale bytes.
+ *   prepacked device, mxmoe_prepacked_size(E, H, I) bytes, 32-byte aligned.
+ * Layout of the blob: [gate/up code boxes][down code boxes][gate/up scale
+ * images][down scale images]. A code box is a 128-row tile by 128 values of
+ * K: 128 rows of 64 bytes, contiguous, boxes ordered by (expert, tile, K
+ * chunk). Within each gate/up tile t, tile row 32q + w is gate column
+ * 64t + 16q + w for w < 16 and up column 64t + 16q + w - 16 otherwise (down
+ * rows keep their order). A scale image covers the same tile and K chunk:
+ * byte (m % 32) * 16 + (m / 32) * 4 + kb is the scale of tile row m, 32-block
+ * kb.
  * Errors: shapes as in mxmoe_prepacked_size -> INVALID_SHAPE; NULL -> NULL;
- * prepacked not 16-byte aligned -> ALIGNMENT. */
+ * prepacked not 32-byte or packed13/packed2 not 16-byte aligned -> ALIGNMENT.
+ */
 MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const uint8_t *sc13, const uint8_t *packed2,
                                     const uint8_t *sc2, int E, int H, int I, void *prepacked, void *stream);
 
@@ -161,19 +166,21 @@ MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I);
  *   prepacked device blob from mxmoe_prepack_experts; y_perm device float
  *   [T*k, H]; workspace device, >= mxmoe_ffn_workspace_size bytes, 256-byte
  *   aligned. Its first 16 bytes hold the device status word of the call.
- * Activations are carried into the tensor cores as f16 with one power-of-two
- * scale per 32-element block (exact for bf16 x; h keeps 11 significant bits).
- * Errors: H % 64, I % 32 != 0, k > 32, E > 1024 -> INVALID_SHAPE; workspace
- * too small -> WORKSPACE; x, prepacked, y_perm not 16-byte aligned ->
- * ALIGNMENT. Device-side wait timeouts -> mxmoe_read_status. */
+ * The products run on tcgen05 block-scaled tensor cores (E2M1 weights x E4M3
+ * activation terms, UE8M0 scales per 32, fp32 accumulation): x enters as two
+ * E4M3 terms per 32-value block (exact for bf16), h as three (about 12
+ * significant bits).
+ * Errors: H or I not a multiple of 128 or above 32768, k > 32, E > 1024,
+ * T*k > 2^22 -> INVALID_SHAPE; workspace
+ * too small -> WORKSPACE; x, y_perm not 16-byte or prepacked not 32-byte
+ * aligned -> ALIGNMENT. Device-side wait timeouts -> mxmoe_read_status. */
 MXMOE_API int mxmoe_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked,
                                int T, int k, int E, int H, int I, float *y_perm, void *workspace,
                                int64_t workspace_bytes, void *stream);
 
 /* Stage 1 of mxmoe_expert_ffn on its own: for every grouped position r,
  * h[r] = silu(W_gate[e] x_t) * (W_up[e] x_t), written into the workspace (as
- * f16 values with one power-of-two factor per 32-value block) for
- * mxmoe_ffn_down. Arguments, layout and errors as for mxmoe_expert_ffn
+ * three E4M3 terms with one scale per 32 values) for mxmoe_ffn_down. Arguments, layout and errors as for mxmoe_expert_ffn
  * (workspace from mxmoe_ffn_workspace_size, 256-byte aligned). */
 MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked,
                                 int T, int k, int E, int H, int I, void *workspace, int64_t workspace_bytes,
@@ -192,11 +199,11 @@ MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prepacked, int 
  * cudaMalloc (which may synchronise the device) is not allowed. There is no
  * counterpart on the pages; it exists only for such callers.
  * Arguments, layout and results are those of mxmoe_expert_ffn, minus the
- * workspace. Scratch is a fixed 4 MiB static device array inside the library
+ * workspace. Scratch is a fixed 8 MiB static device array inside the library
  * (held on every GPU where the library's device code is loaded, until the
- * process exits); sizes whose mxmoe_ffn_workspace_size exceeds 4 MiB are
+ * process exits); sizes whose mxmoe_ffn_workspace_size exceeds 8 MiB are
  * rejected with MXMOE_ERR_WORKSPACE before anything is enqueued (the
- * 6144/2048/top-8 layer fits up to 64 tokens).
+ * 6144/2048/top-8 layer fits up to 50 tokens).
  *   status  device int or NULL: when given, receives the call's device status
  *           word (MXMOE_OK or MXMOE_ERR_TIMEOUT) in stream order.
  * The first call on each device looks up the array's device address (once,

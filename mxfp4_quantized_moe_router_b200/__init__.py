@@ -269,7 +269,7 @@ def mxmoe_ffn_down(offsets, prepacked, T, k, E, H, I, y_perm, workspace, stream=
 
 def mxmoe_expert_ffn_noalloc(x, offsets, src_row, prepacked, k, E, I, y_perm, status=None, stream=None):
     """mxmoe_expert_ffn without a workspace (scratch in the library's fixed
-    4 MiB static device array); for callers that cannot allocate."""
+    8 MiB static device array); for callers that cannot allocate."""
     import torch
 
     T, H = x.shape

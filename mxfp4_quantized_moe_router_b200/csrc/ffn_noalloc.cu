@@ -20,11 +20,11 @@ int validate_ffn_shapes(int T, int k, int E, int H, int I);
 
 namespace {
 
-constexpr int64_t kStaticScratchBytes = 4LL << 20;  // 4 MiB per device
+constexpr int64_t kStaticScratchBytes = 8LL << 20;  // 8 MiB per device
 constexpr int kMaxDevices = 64;
 
 // The shared scratch. Every GPU on which the library's device code is loaded
-// holds these 4 MiB until the process exits. In host code this name is only a
+// holds these 8 MiB until the process exits. In host code this name is only a
 // host-side stand-in: its device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_ffn_scratch[kStaticScratchBytes];
 
@@ -72,8 +72,9 @@ extern "C" MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *
         return MXMOE_OK;
     if (!x || !offsets || !src_row || !prepacked || !y_perm)
         return fail(MXMOE_ERR_NULL, "mxmoe_expert_ffn_noalloc: NULL pointer");
-    if (!aligned16(x) || !aligned16(prepacked) || !aligned16(y_perm))
-        return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_expert_ffn_noalloc: x, prepacked, y_perm need 16-byte alignment");
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(prepacked) & 31) || !aligned16(y_perm))
+        return fail(MXMOE_ERR_ALIGNMENT,
+                    "mxmoe_expert_ffn_noalloc: x and y_perm need 16-byte, prepacked 32-byte alignment");
     if (int rc = check_device())
         return rc;
     void *scratch = nullptr;
@@ -81,8 +82,8 @@ extern "C" MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *
         return rc;
     cudaStream_t st = (cudaStream_t)stream;
     // The first kernel of the chain clears the status word at the start of the
-    // scratch; every other scratch byte that is read was written earlier in
-    // the same call, so nothing else needs clearing between calls.
+    // scratch; every other scratch byte that can reach the outputs is written
+    // earlier in the same call, so nothing else needs clearing between calls.
     if (int rc = run_expert_ffn(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, scratch, st))
         return rc;
     if (status) {

@@ -97,55 +97,62 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
     }
 }
 
-// Canonical expert row of slab s (0..3), row r16 (0..15) of tile `tile`.
-// Gate/up part: tile = 32 intermediate columns; slabs 0,1 are gate rows,
-// slabs 2,3 the matching up rows (offset I). Down part: 64 consecutive rows.
-__device__ __forceinline__ int64_t tile_row(bool gate_up, int tile, int s, int r16, int I)
+// Prepacked blob for the tensor-core FFN (a byte permutation of the canonical
+// format, same size):
+//   [gate/up code boxes][down code boxes][gate/up scale images][down scale images]
+// A code box is one 128-row tile by 128 values of K: 128 rows of 64 bytes,
+// contiguous (8 KB), boxes ordered by (expert, tile, K chunk). Gate/up rows are
+// reordered per tile t so that tile row lr = 32q + w holds gate column
+// 64t + 16q + w (w < 16) or up column 64t + 16q + (w - 16) (w >= 16); down
+// rows keep their order. A scale image covers the same tile and K chunk:
+// byte (m % 32) * 16 + (m / 32) * 4 + kb holds the scale of tile row m,
+// k32 block kb.
+__device__ __forceinline__ int64_t tile_src_row(bool gate_up, int64_t lr_all, int I)
 {
-    if (gate_up)
-        return (int64_t)(s >= 2 ? I : 0) + tile * 32 + (s & 1) * 16 + r16;
-    return (int64_t)tile * 64 + s * 16 + r16;
+    if (!gate_up)
+        return lr_all;
+    const int64_t t = lr_all >> 7;
+    const int lr = (int)(lr_all & 127), q = lr >> 5, w = lr & 31;
+    return (w < 16) ? 64 * t + 16 * q + w : (int64_t)I + 64 * t + 16 * q + (w - 16);
 }
 
-// One block per (expert, tile, chunk) of one matrix (gate/up or down).
-__global__ void __launch_bounds__(256) prepack_kernel(const uint8_t *__restrict__ packed,
-                                                      const uint8_t *__restrict__ sc, int E, int rows_per_expert,
-                                                      int K, int tiles_per_expert, bool gate_up, int I,
-                                                      uint8_t *__restrict__ dst)
+// One thread per 16 bytes of the code boxes.
+__global__ void __launch_bounds__(256) prepack_rows_kernel(const uint8_t *__restrict__ packed, int E,
+                                                           int64_t rows_per_expert, int K, bool gate_up, int I,
+                                                           uint8_t *__restrict__ dst)
 {
-    const int nchunk = (K + kChunkK - 1) / kChunkK;
-    const int64_t blk = blockIdx.x;
-    const int c = (int)(blk % nchunk);
-    const int tile = (int)((blk / nchunk) % tiles_per_expert);
-    const int e = (int)(blk / ((int64_t)nchunk * tiles_per_expert));
-    const int k0 = c * kChunkK;
-    const int kw = min(kChunkK, K - k0);
-    const int64_t ebase = (int64_t)e * rows_per_expert;
-    uint8_t *out = dst + ((int64_t)e * tiles_per_expert + tile) * wtile_bytes(K) + (int64_t)c * wchunk_bytes(kChunkK);
-    // nibble part: word index = ((w*2 + half)*32 + lane)*4 + jj
-    const int nwords = (int)(wchunk_nibble_bytes(kw) / 4);
-    for (int i = threadIdx.x; i < nwords; i += blockDim.x) {
-        const int jj = i & 3, lane = (i >> 2) & 31, half = (i >> 7) & 1, w = i >> 8;
-        const int g = lane >> 2, t = lane & 3;
-        const int s = 2 * half + (jj >> 1), step = jj & 1;
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int r16 = (b & 1) ? g + 8 : g;
-            const int kk = k0 + 32 * w + 16 * step + 2 * t + ((b & 2) ? 8 : 0);
-            const int64_t row = ebase + tile_row(gate_up, tile, s, r16, I);
-            word |= (uint32_t)packed[row * (K / 2) + kk / 2] << (8 * b);
-        }
-        reinterpret_cast<uint32_t *>(out)[i] = word;
+    const int nchunk = K / 128;
+    const int64_t tiles = rows_per_expert / 128;
+    const int64_t total = (int64_t)E * rows_per_expert * (K / 32);  // 16-byte units
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
+        const int part = (int)(u & 3);          // 16-byte part of a 64-byte box row
+        const int lr = (int)((u >> 2) & 127);   // box row
+        const int64_t box = u >> 9;             // (e * tiles + t) * nchunk + c
+        const int c = (int)(box % nchunk);
+        const int64_t tile_id = box / nchunk;
+        const int64_t e = tile_id / tiles, t = tile_id % tiles;
+        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 128 + lr, I);
+        reinterpret_cast<uint4 *>(dst)[u] =
+            __ldg(reinterpret_cast<const uint4 *>(packed + src * (K / 2) + (int64_t)c * 64) + part);
     }
-    // scale part: byte index = ((w*8 + g)*4 + s)*2 + r2
-    uint8_t *osc = out + wchunk_nibble_bytes(kw);
-    const int nsc = 2 * kw;
-    for (int i = threadIdx.x; i < nsc; i += blockDim.x) {
-        const int r2 = i & 1, s = (i >> 1) & 3, g = (i >> 3) & 7, w = i >> 6;
-        const int r16 = r2 ? g + 8 : g;
-        const int64_t row = ebase + tile_row(gate_up, tile, s, r16, I);
-        osc[i] = sc[row * (K / 32) + (k0 + 32 * w) / 32];
+}
+
+__global__ void __launch_bounds__(256) prepack_sf_kernel(const uint8_t *__restrict__ sc, int E,
+                                                         int64_t rows_per_expert, int K, bool gate_up, int I,
+                                                         uint8_t *__restrict__ dst)
+{
+    const int nchunk = K / 128;
+    const int64_t tiles = rows_per_expert / 128;
+    const int64_t total = (int64_t)E * tiles * nchunk * 512;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int b = (int)(i & 511);
+        const int64_t img = i >> 9;
+        const int c = (int)(img % nchunk);
+        const int64_t tile_id = img / nchunk;
+        const int64_t e = tile_id / tiles, t = tile_id % tiles;
+        const int m = (b >> 4) + 32 * ((b & 15) >> 2), kb = b & 3;
+        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 128 + m, I);
+        dst[i] = sc[src * (K / 32) + 4 * c + kb];
     }
 }
 
@@ -197,9 +204,9 @@ extern "C" MXMOE_API int mxmoe_dequantize(const uint8_t *packed, const uint8_t *
 
 extern "C" MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I)
 {
-    if (E <= 0 || H <= 0 || I <= 0 || H % 64 || I % 32)
+    if (E <= 0 || H <= 0 || I <= 0 || H % 128 || I % 128)
         return -1;
-    return (int64_t)E * ((int64_t)(I / 32) * wtile_bytes(H) + (int64_t)(H / 64) * wtile_bytes(I));
+    return (int64_t)E * 3 * H * I / 2 + (int64_t)E * 3 * H * I / 32;
 }
 
 extern "C" MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const uint8_t *sc13, const uint8_t *packed2,
@@ -207,22 +214,31 @@ extern "C" MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const ui
                                                void *stream)
 {
     if (mxmoe_prepacked_size(E, H, I) < 0)
-        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_prepack_experts: E=%d H=%d I=%d (need H %% 64 == 0, I %% 32 == 0)",
-                    E, H, I);
+        return fail(MXMOE_ERR_INVALID_SHAPE,
+                    "mxmoe_prepack_experts: E=%d H=%d I=%d (need H %% 128 == 0, I %% 128 == 0)", E, H, I);
     if (!packed13 || !sc13 || !packed2 || !sc2 || !prepacked)
         return fail(MXMOE_ERR_NULL, "mxmoe_prepack_experts: NULL pointer");
-    if (!aligned16(prepacked))
-        return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_prepack_experts: prepacked must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(prepacked) & 31) || !aligned16(packed13) || !aligned16(packed2))
+        return fail(MXMOE_ERR_ALIGNMENT,
+                    "mxmoe_prepack_experts: prepacked needs 32-byte, packed13/packed2 16-byte alignment");
     if (int rc = check_device())
         return rc;
-    uint8_t *dst = static_cast<uint8_t *>(prepacked);
+    uint8_t *w13 = static_cast<uint8_t *>(prepacked);
+    uint8_t *w2 = w13 + (int64_t)E * 2 * I * (H / 2);
+    uint8_t *sf13 = w2 + (int64_t)E * H * (I / 2);
+    uint8_t *sf2 = sf13 + (int64_t)E * 2 * I * (H / 32);
     cudaStream_t st = (cudaStream_t)stream;
-    const int64_t blocks13 = (int64_t)E * (I / 32) * ((H + kChunkK - 1) / kChunkK);
-    prepack_kernel<<<(unsigned)blocks13, 256, 0, st>>>(packed13, sc13, E, 2 * I, H, I / 32, true, I, dst);
-    if (int rc = check_launch("prepack_kernel(gate/up)"))
+    prepack_rows_kernel<<<grid_for((int64_t)E * 2 * I * (H / 32), 256), 256, 0, st>>>(packed13, E, 2 * I, H, true,
+                                                                                       I, w13);
+    if (int rc = check_launch("prepack_rows_kernel(gate/up)"))
         return rc;
-    uint8_t *dst2 = dst + (int64_t)E * (I / 32) * wtile_bytes(H);
-    const int64_t blocks2 = (int64_t)E * (H / 64) * ((I + kChunkK - 1) / kChunkK);
-    prepack_kernel<<<(unsigned)blocks2, 256, 0, st>>>(packed2, sc2, E, H, I, H / 64, false, I, dst2);
-    return check_launch("prepack_kernel(down)");
+    prepack_rows_kernel<<<grid_for((int64_t)E * H * (I / 32), 256), 256, 0, st>>>(packed2, E, H, I, false, I, w2);
+    if (int rc = check_launch("prepack_rows_kernel(down)"))
+        return rc;
+    prepack_sf_kernel<<<grid_for((int64_t)E * 2 * I * (H / 32), 256), 256, 0, st>>>(sc13, E, 2 * I, H, true, I,
+                                                                                      sf13);
+    if (int rc = check_launch("prepack_sf_kernel(gate/up)"))
+        return rc;
+    prepack_sf_kernel<<<grid_for((int64_t)E * H * (I / 32), 256), 256, 0, st>>>(sc2, E, H, I, false, I, sf2);
+    return check_launch("prepack_sf_kernel(down)");
 }

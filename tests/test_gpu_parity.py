@@ -141,12 +141,14 @@ def test_permute_skewed(mx):
 # Expert FFN (grouped), element by element against the oracle
 # ---------------------------------------------------------------------------
 FFN_CASES = [
-    # H, I, E, k, T : tiles along I and H, partial K chunks, ragged token passes
+    # H, I, E, k, T : several tiles along I and H, several K steps, ragged
+    # token passes (8-token tiles for T <= 8, 32-token tiles otherwise)
     (256, 128, 16, 2, 4),
-    (320, 96, 6, 2, 37),
+    (384, 256, 6, 2, 37),
     (512, 256, 8, 2, 9),
-    (384, 160, 3, 1, 80),     # n_e up to ~40: several 32-token passes
-    (640, 288, 5, 3, 150),
+    (256, 384, 3, 1, 80),     # n_e up to ~40: several 32-token passes
+    (640, 384, 5, 3, 150),
+    (1024, 128, 2, 2, 1),     # one token, 8 of its tile rows padded
 ]
 
 
@@ -239,7 +241,7 @@ def test_layer_tiny(mx):
 
 @pytest.mark.parametrize("T", [1, 3, 64, 200])
 def test_layer_small_ragged(mx, T):
-    cfg = datagen.LayerConfig("small", 512, 24, 4, 96, T)
+    cfg = datagen.LayerConfig("small", 512, 24, 4, 128, T)
     layer = GpuLayer(mx, cfg, 1)
     x = datagen.make_x(cfg, 1)
     bias = (np.linspace(-0.5, 0.5, cfg.E)).astype(np.float32)
