@@ -92,7 +92,7 @@ MXMOE_API int mxmoe_dequantize(const uint8_t *packed, const uint8_t *scales, int
 
 /* Bytes of the prepacked expert blob for E experts of hidden size H and
  * intermediate size I (= E * 3 * H * I * 17/32, the same bytes as the packed
- * codes plus scales). Returns -1 unless H and I are positive multiples of 128.
+ * codes plus scales). Returns -1 unless H and I are positive multiples of 256.
  */
 MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I);
 
@@ -105,13 +105,13 @@ MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I);
  *            projection (each row a K = I vector).
  *   prepacked device, mxmoe_prepacked_size(E, H, I) bytes, 32-byte aligned.
  * Layout of the blob: [gate/up code boxes][down code boxes][gate/up scale
- * images][down scale images]. A code box is a 128-row tile by 128 values of
- * K: 128 rows of 64 bytes, contiguous, boxes ordered by (expert, tile, K
- * chunk). Within each gate/up tile t, tile row 32q + w is gate column
- * 64t + 16q + w for w < 16 and up column 64t + 16q + w - 16 otherwise (down
- * rows keep their order). A scale image covers the same tile and K chunk:
- * byte (m % 32) * 16 + (m / 32) * 4 + kb is the scale of tile row m, 32-block
- * kb.
+ * images][down scale images]. A code box is a 256-row tile by 256 values of
+ * K: 256 rows of 128 bytes (32 KB), contiguous, boxes ordered by (expert,
+ * tile, K chunk). Gate/up tile t holds gate rows 128t .. 128t+127 and then the
+ * matching up rows I + 128t .. I + 128t+127; down rows keep their order. The
+ * scale images of a box are four 512-byte images ordered (K half h, row half
+ * g): byte (r % 32) * 16 + (r / 32) * 4 + kb is the scale of tile row
+ * 128g + r, 32-block 4h + kb of the box.
  * Errors: shapes as in mxmoe_prepacked_size -> INVALID_SHAPE; NULL -> NULL;
  * prepacked not 32-byte or packed13/packed2 not 16-byte aligned -> ALIGNMENT.
  */
@@ -166,12 +166,12 @@ MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I);
  *   prepacked device blob from mxmoe_prepack_experts; y_perm device float
  *   [T*k, H]; workspace device, >= mxmoe_ffn_workspace_size bytes, 256-byte
  *   aligned. Its first 16 bytes hold the device status word of the call.
- * The products run on tcgen05 block-scaled tensor cores (E2M1 weights x E4M3
- * activation terms, UE8M0 scales per 32, fp32 accumulation): x enters as two
- * E4M3 terms per 32-value block (exact for bf16), h as three (about 12
- * significant bits).
- * Errors: H or I not a multiple of 128 or above 32768, k > 32, E > 1024,
- * T*k > 2^22 -> INVALID_SHAPE; workspace
+ * The products run on tcgen05 block-scaled tensor cores (E2M1 weights x E2M1
+ * activation terms, UE8M0 scales per 32, fp32 accumulation): x and h each
+ * enter as eight E2M1 terms per value, every term with its own scale per 32
+ * values, together within 3^-8 of the 32-block's largest magnitude.
+ * Errors: H or I not a multiple of 256 or above 32768, k > 32, E > 1024,
+ * T*k > 2^22, E*I*H >= 2^38 -> INVALID_SHAPE; workspace
  * too small -> WORKSPACE; x, y_perm not 16-byte or prepacked not 32-byte
  * aligned -> ALIGNMENT. Device-side wait timeouts -> mxmoe_read_status. */
 MXMOE_API int mxmoe_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked,
@@ -203,7 +203,7 @@ MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prepacked, int 
  * (held on every GPU where the library's device code is loaded, until the
  * process exits); sizes whose mxmoe_ffn_workspace_size exceeds 8 MiB are
  * rejected with MXMOE_ERR_WORKSPACE before anything is enqueued (the
- * 6144/2048/top-8 layer fits up to 50 tokens).
+ * 6144/2048/top-8 layer fits up to 15 tokens).
  *   status  device int or NULL: when given, receives the call's device status
  *           word (MXMOE_OK or MXMOE_ERR_TIMEOUT) in stream order.
  * The first call on each device looks up the array's device address (once,

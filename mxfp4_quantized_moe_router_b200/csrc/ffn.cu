@@ -11,35 +11,35 @@
 //
 // Design (one B200, sm_100a):
 //  * The weights stay MXFP4 all the way into the tensor core:
-//    tcgen05.mma.kind::mxf8f6f4.block_scale multiplies E2M1 weight codes by
-//    E4M3 activation codes and applies both operands' UE8M0 scales per 32
-//    elements of K in hardware, accumulating in fp32 in tensor memory. No
+//    tcgen05.mma.kind::mxf4.block_scale multiplies packed E2M1 weight codes by
+//    packed E2M1 activation codes, applies both operands' UE8M0 scales per 32
+//    elements of K in hardware and accumulates in fp32 in tensor memory. No
 //    instruction touches a weight element.
-//  * Weight tiles (128 rows x 128 K, one contiguous 8 KB box of the
-//    prepacked blob) arrive by TMA with the fp4 unpack (16U4_ALIGN16B), their
-//    scale images (512 B) by a bulk copy, and the scale images move into
-//    tensor memory by tcgen05.cp.
-//  * Activations are exact sums of E4M3 terms with one power-of-two scale per
-//    32 values: x (bf16) = 2 terms, exact for every element within 2^-14 of
-//    its block maximum; h (fp32) = 3 terms, about 12 significant bits. The
-//    terms are stacked along N (term t of token n is B row t*NT + n), so one
-//    MMA per 32 values of K covers all of them and the epilogue adds the term
-//    columns.
-//  * Activations are stored in grouped (expert-sorted) row order, so a token
-//    pass of an expert is a contiguous row range: one 3-D TMA box per K step
-//    brings all of its terms.
-//  * Warp roles per CTA: a producer warp (TMA and bulk copies into an S-stage
-//    ring), an MMA warp (tcgen05.cp of the scale images, the MMAs, commits),
-//    four epilogue warps reading the fp32 accumulators from tensor memory
-//    (two accumulator buffers, so item i's epilogue overlaps item i+1's MMAs;
-//    within an item the k32 blocks rotate over independent accumulators so
-//    the short MMAs of decode-sized N do not serialise on one accumulator).
-//  * Stage 1 (gate/up): a 128-row tile is 64 gate rows and the 64 matching up
-//    rows, interleaved by 16 so gate and up of one column meet in one warp;
-//    SwiGLU and the 3-term encoding of h are fused into the epilogue.
-//    Stage 2 (down): a tile is 128 output rows.
-//  * Work items (expert, tile, token pass) are split contiguously over a
-//    persistent grid of one CTA per SM.
+//  * A block-scaled MMA costs about the same issue time at any N, so the
+//    weights are the N operand, 256 rows per MMA, and each MMA covers 8 KB of
+//    weight codes (256 rows x 64 values of K): enough that the weight stream,
+//    not the MMA issue, sets the pace.
+//  * Activations become kT = 8 E2M1 terms per value: term t is the E2M1
+//    rounding of what terms 0..t-1 left over, with its own UE8M0 scale per 32
+//    values chosen so the block's largest remainder fits E2M1's range. Each
+//    term removes at least a factor 3 of the block's largest remainder, so 8
+//    terms reproduce a value to within 3^-8 of its block maximum. The terms
+//    of a token are consecutive MMA rows (row = token * kT + term; M = 128 rows
+//    = 16 tokens); the epilogue adds them.
+//  * Weight boxes (256 rows x 256 K, 32 KB, contiguous in the prepacked blob)
+//    and their scale images (2 KB) stream through a 5-deep ring; activation
+//    terms (one 4-D TMA box per chunk) and their scale images (written by the
+//    producing kernel directly in tensor-memory image order, one per token
+//    pass and 128 columns) through a 3-deep ring. tcgen05.cp moves the scale
+//    images into tensor memory.
+//  * Warp roles per CTA: a producer warp, an MMA warp and four epilogue warps.
+//    The epilogue sums a token's terms with a 3-round butterfly that leaves
+//    each lane 8 finished columns of every 64, then releases the accumulator.
+//  * Stage 1 (gate/up): a 256-row tile is 128 gate rows and the matching 128
+//    up rows; SwiGLU and the term encoding of h (with its scale images) are
+//    fused into the epilogue. Stage 2 (down): a tile is 256 output rows.
+//  * Work items (expert, tile, token pass of up to NT tokens) are split
+//    contiguously over a persistent grid of one CTA per SM.
 #include <float.h>
 
 #include <algorithm>
@@ -54,108 +54,101 @@ namespace mxmoe {
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
-constexpr int kKC = 128;            // K per chunk (one 128 x 128 fp4 box of the prepacked blob)
-constexpr int kChunkSmem = 16384;   // shared-memory bytes of an unpacked chunk box
-constexpr int kChunkTx = 8192;      // TMA transaction bytes of a chunk box (its packed size)
-constexpr int kSFImg = 512;         // scale image: 32 lanes x 16 bytes
-constexpr int kThreads = 192;       // producer, MMA, 4 epilogue warps
+constexpr int kT = 8;            // E2M1 terms per activation value
+constexpr int kKC = 256;         // K per chunk (one weight box)
+constexpr int kWBox = 32768;     // bytes of a weight box: 256 rows x 128 bytes
+constexpr int kWSf = 2048;       // its scale images: (K half, row half) x 512 bytes
+constexpr int kAStage = 16384;   // shared bytes the MMA reads for A: 128 rows x 128 bytes
+constexpr int kSFImg = 512;      // scale image: 32 lanes x 16 bytes
+constexpr int kThreads = 192;    // producer, MMA, 4 epilogue warps
+constexpr int kMaxE = 1024;
 
 struct FfnParams {
-    int tiles_per_expert;     // 2I/128 (gate/up) or H/128 (down)
-    int K;                    // reduction length (H or I)
-    int rows_act;             // rows of the activation term tensors (T*k)
-    const uint8_t *sfa;       // weight scale images [E*tiles][K/128][512]
-    const int32_t *offsets;   // [E+1]
+    int tiles;                  // 256-row tiles per expert: I/128 (gate/up) or H/256 (down)
+    int K;                      // reduction length (H or I)
+    int rows;                   // activation rows (T*k)
+    const uint8_t *wsf;         // weight scale images [E*tiles][K/256][2048]
+    const uint8_t *asf;         // activation scale images [pass][K/128][512]
+    const int32_t *offsets;     // [E+1]
+    const int32_t *pass_start;  // [E+1]: first token pass of each expert
     int E;
-    uint8_t *h_terms;         // gate/up output: terms of h (term_offset layout)
-    uint8_t *h_rec;           // gate/up output: their scale records (rec_offset layout)
+    uint8_t *h_terms;           // gate/up output: terms of h (term_offset layout)
+    uint8_t *h_sf;              // gate/up output: their scale images
     int I;
-    float *y_out;             // down output: [rows, H]
+    float *y_out;               // down output: [rows, H]
     int H;
     int *status;
 };
 
-// Byte offset of term t of activation row r, column k, in a term tensor laid
-// out [K/128][nterms][rows][128]: the terms of one 128-column chunk of a token
-// pass are nterms runs of consecutive 128-byte rows.
-__host__ __device__ __forceinline__ int64_t term_offset(int nterms, int64_t rows, int t, int64_t r, int k)
+// Byte offset of the E2M1 code byte holding columns k, k+1 (k even) of term t
+// of activation row r, in a term tensor laid out [K/256][rows][kT][128]: the
+// terms of one 256-column chunk of a token pass are consecutive 128-byte rows.
+__host__ __device__ __forceinline__ int64_t term_offset(int64_t rows, int t, int64_t r, int k)
 {
-    return (((int64_t)(k >> 7) * nterms + t) * rows + r) * 128 + (k & 127);
+    return (((int64_t)(k >> 8) * rows + r) * kT + t) * 128 + ((k & 255) >> 1);
 }
 
-// Byte offset of the UE8M0 scale of term t, row r, for the 32-block holding
-// column k, in a scale-record array of 16-byte records. With 8-token passes
-// (per_term) a record holds one term of one chunk (byte = k32 block), planes
-// chunk * nterms + t: the records of a pass and chunk then form that chunk's
-// B scale image, image row t * 8 + n. With 32-token passes a record holds all
-// terms of one chunk (byte 4t + k32 block), planes = chunks: image row n then
-// serves the stacked rows t * 32 + n through its t-th 32-bit column.
-__host__ __device__ __forceinline__ int64_t rec_offset(bool per_term, int nterms, int64_t rows, int t, int64_t r,
-                                                       int k)
+// Byte offset, within the scale images of one token pass and 128-column half
+// (512 bytes), of the scale of term t of pass row n for 32-block kb of the
+// half: MMA row m = n * kT + t sits in tensor-memory lane m % 32, column m / 32.
+__host__ __device__ __forceinline__ int image_byte(int n, int t, int kb)
 {
-    const int c = k >> 7, kb = (k >> 5) & 3;
-    if (per_term)
-        return (((int64_t)c * nterms + t) * rows + r) * 16 + kb;
-    return ((int64_t)c * rows + r) * 16 + 4 * t + kb;
+    const int m = n * kT + t;
+    return (m & 31) * 16 + (m >> 5) * 4 + kb;
 }
 
-__host__ __device__ __forceinline__ int64_t rec_planes(bool per_term, int nterms, int K)
+// Upper bound on token passes: every pass holds at least one row, and there
+// are at most ceil(rows / 8) + (non-empty experts) of them.
+inline int64_t max_passes(int64_t rows)
 {
-    return per_term ? (int64_t)(K / kKC) * nterms : K / kKC;
+    return std::min<int64_t>(rows, (rows + 7) / 8 + std::min<int64_t>(kMaxE, rows));
 }
 
-template <int NT, int NTERMS>
+template <int NT>
 struct Cfg {
-    static constexpr bool kPerTerm = NT <= 8;
-    static constexpr int kCPS = NT <= 8 ? 4 : 2;  // chunks per stage (one weight TMA request)
-    // Weight ring (codes + scale images, from HBM) and activation ring (terms +
-    // scale records, L2-resident), advanced together once per stage.
-    static constexpr int kStagesA = NT <= 8 ? 3 : (NTERMS == 2 ? 5 : 4);
-    static constexpr int kStagesB = NT <= 8 ? 2 : 3;
-    static constexpr int kAStage = kCPS * kChunkSmem;
-    static constexpr int kATx = kCPS * kChunkTx;
-    static constexpr int kSfaStage = kCPS * kSFImg;
-    static constexpr int kBChunk = NTERMS * NT * 128;  // one chunk's terms, rows t*NT + n
-    static constexpr int kBStage = kCPS * kBChunk;
-    static constexpr int kSfbZ = kPerTerm ? NTERMS * kCPS : kCPS;  // record planes per stage
-    static constexpr int kSfbTx = 16 * NT * kSfbZ;
-    static constexpr int kSfbImg = kSfbTx / kCPS;  // one chunk's B scale image
-    // a 32-lane tcgen05.cp of the last image reads up to 512 bytes
-    static constexpr int kSfbStage = kSfbTx + (kSfbImg < kSFImg ? kSFImg - kSfbImg : 0);
-    static constexpr int kN = NTERMS * NT;  // MMA N: the stacked terms
-    static constexpr int kXchg = 8 * NT;    // [pair][parity][quarter][NT] block maxima
-    // shared memory: A stages | B stages | A scale images | B scale images | xchg | barriers | tslot, cursor
-    static constexpr size_t kOffB = (size_t)kStagesA * kAStage;
-    static constexpr size_t kOffSfa = kOffB + (size_t)kStagesB * kBStage;
-    static constexpr size_t kOffSfb = kOffSfa + (size_t)kStagesA * kSfaStage;
-    static constexpr size_t kOffXchg = kOffSfb + (size_t)kStagesB * kSfbStage;
-    static constexpr size_t kOffBar = (kOffXchg + kXchg * 4 + 127) & ~size_t(127);
-    static constexpr int kBars = 2 * kStagesA + 2 * kStagesB + 5;
+    static constexpr int kM = NT * kT;  // MMA rows in use
+    static constexpr int kATx = kM * 128;
+    static constexpr int kStagesW = 5, kStagesA = 3;
+    // shared memory: W stages | A stages | W scale images | A scale images | barriers | tslot, cursor
+    static constexpr size_t kOffA = (size_t)kStagesW * kWBox;
+    static constexpr size_t kOffSfw = kOffA + (size_t)kStagesA * kAStage;
+    static constexpr size_t kOffSfa = kOffSfw + (size_t)kStagesW * kWSf;
+    static constexpr size_t kOffBar = kOffSfa + (size_t)kStagesA * 2 * kSFImg;
+    static constexpr int kBars = 2 * kStagesW + 2 * kStagesA + 3;
     static constexpr size_t kOffMisc = (kOffBar + kBars * 8 + 15) & ~size_t(15);
     static constexpr size_t kSmem = 1024 + kOffMisc + 64;
-    // Tensor memory: two accumulator buffers (item i and i+1), each holding
-    // kChains independent accumulators of kN columns (32-column aligned): the
-    // k32 blocks of an item rotate over the chains so that consecutive small-N
-    // MMAs do not wait on each other. Then the scale columns: per stage and
-    // chunk one group of 4 for A and one for B. An MMA's scale address must be
-    // a group base (a multiple of 4 columns).
-    static constexpr int kChains = NT <= 8 ? 4 : 2;
+    // Tensor memory: the accumulator (128 lanes x 256 columns), then per weight
+    // stage two 8-column scale groups (K halves; 256 rows = 8 columns) and per
+    // activation stage two 4-column groups.
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kAccStride = (kN + 31) & ~31;
-    static constexpr uint32_t kBufCols = kChains * kAccStride;
-    static constexpr uint32_t kSfaCol0 = 2 * kBufCols;
-    static constexpr uint32_t kSfaCols = 4 * kCPS;
-    static constexpr uint32_t kSfbCol0 = kSfaCol0 + kStagesA * kSfaCols;
-    static constexpr uint32_t kSfbCols = 4 * kCPS;
-    static_assert(NT <= 32 && NTERMS <= 3 && kN <= 256 && kN % 8 == 0, "MMA shape");
-    static_assert(!kPerTerm || kN <= 32, "a per-term B scale image has at most 32 rows");
-    static_assert(kSfbStage % 128 == 0 && kSfbImg % 16 == 0, "scale image alignment");
-    static_assert(kSfbCol0 + kStagesB * kSfbCols <= kTmemCols, "tensor memory columns");
-    static_assert(kAStage % 1024 == 0 && kBChunk % 1024 == 0 && kOffB % 1024 == 0, "128-byte swizzle atoms");
+    static constexpr uint32_t kSfwCol0 = 256;
+    static constexpr uint32_t kSfaCol0 = kSfwCol0 + 16 * kStagesW;
+    static_assert(NT == 8 || NT == 16, "token pass");
+    static_assert(kSfaCol0 + 8 * kStagesA <= kTmemCols, "tensor memory columns");
     static_assert(kSmem <= 232448, "shared memory");
 };
 
-// Work items of one FFN stage: (expert, weight tile, token pass), expert-major,
+// Instruction descriptor of kind::mxf4.block_scale: A and B E2M1, UE8M0
+// scales, both K-major, M = 128, N = n, scale byte pair sf_id (0 or 2) of
+// each operand's scale column.
+__device__ __forceinline__ uint32_t idesc_mxf4(int n, uint32_t sf_id)
+{
+    return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | (8u << 24) |
+           (sf_id << 29);
+}
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Work items of one FFN stage: (expert, 256-row tile, token pass), expert-major,
 // then tile, then pass, so that the passes of one weight tile are adjacent
 // (the repeated weight boxes then come from L2). A CTA takes a contiguous
 // range of items and every role walks it with its own cursor.
@@ -202,54 +195,64 @@ struct ItemCursor {
     __device__ __forceinline__ int nt() const { return min(NT, n_e - pass * NT); }
 };
 
-// Activation value v (already divided by its block's 2^s, |v| < 256) as
-// NTERMS E4M3 codes c_t with v ~= sum_t c_t * 16^-t (exact for 8-bit v).
-template <int NTERMS>
-__device__ __forceinline__ void split_terms(float v, uint32_t (&code)[NTERMS])
+// UE8M0 exponent s of an activation term block whose largest magnitude is m:
+// the smallest s with m <= 6 * 2^s (E2M1's largest value), clamped to the
+// UE8M0 range; zero and subnormal maxima take the smallest scale.
+__device__ __forceinline__ int e2m1_block_exp(float m)
 {
-    float r = v;
-#pragma unroll
-    for (int t = 0; t < NTERMS; ++t) {
-        code[t] = tc::f32_to_e4m3(r);
-        r = (r - tc::e4m3_to_f32(code[t])) * 16.f;
-    }
+    const uint32_t b = __float_as_uint(m);
+    if (b < 0x00800000u)
+        return -127;
+    const int e = (int)(b >> 23) - 127;
+    const int s = e - 2 + ((b & 0x7FFFFFu) > 0x400000u ? 1 : 0);
+    return max(-127, min(s, 126));
 }
 
-// Scale exponent s of a 32-value activation block with maximum m: m / 2^s
-// lands in [128, 256); clamped so that every term's scale byte s - 4t + 127
-// stays in [0, 254].
-__device__ __forceinline__ int act_block_exp(float m)
+__device__ __forceinline__ float pow2f(int s)  // 2^s for s in [-127, 127]
 {
-    const int s = m > 0.f ? tc::floor_log2(m) - 7 : 0;
-    return max(-119, min(s, 127));
+    return s >= -126 ? __uint_as_float((uint32_t)(s + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// E2M1 code of y (|y| <= 6, round to nearest even) in the low nibble, and the
+// value that code stands for.
+__device__ __forceinline__ uint32_t e2m1_code(float y, float &q)
+{
+    uint32_t code, h2;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %3;\n\t"
+        "cvt.u32.u8 %0, t;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, t;\n\t}"
+        : "=r"(code), "=r"(h2)
+        : "f"(0.f), "f"(y));
+    q = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    return code & 0xFu;
 }
 
 // One FFN stage over all experts.
-// GATE_UP = true: stage 1 (x terms in; h terms and records out).
+// GATE_UP = true: stage 1 (x terms in; h terms and their scale images out).
 // GATE_UP = false: stage 2 (h terms in; float rows out).
-template <int NT, int NTERMS, bool GATE_UP>
+template <int NT, bool GATE_UP>
 __global__ void __launch_bounds__(kThreads, 1)
-    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmSfb, const FfnParams p)
+    ffn_mxf4_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
+                    const FfnParams p)
 {
-    using C = Cfg<NT, NTERMS>;
+    using C = Cfg<NT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem, *sB = smem + C::kOffB, *sSfa = smem + C::kOffSfa, *sSfb = smem + C::kOffSfb;
-    float *xchg = reinterpret_cast<float *>(smem + C::kOffXchg);
-    uint64_t *fullA = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint8_t *sW = smem, *sA = smem + C::kOffA, *sSfw = smem + C::kOffSfw, *sSfa = smem + C::kOffSfa;
+    uint64_t *fullW = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint64_t *emptyW = fullW + C::kStagesW;
+    uint64_t *fullA = emptyW + C::kStagesW;
     uint64_t *emptyA = fullA + C::kStagesA;
-    uint64_t *fullB = emptyA + C::kStagesA;
-    uint64_t *emptyB = fullB + C::kStagesB;
-    uint64_t *accfull = emptyB + C::kStagesB;  // [2]
-    uint64_t *accempty = accfull + 2;          // [2]
-    uint64_t *mma_done = accempty + 2;         // [1]
+    uint64_t *accfull = emptyA + C::kStagesA;
+    uint64_t *accempty = accfull + 1;
+    uint64_t *mma_done = accempty + 1;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     int *cur = reinterpret_cast<int *>(tslot + 2);  // [0] first expert, [1] first item within it, [2] item count
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int E = p.E, tiles = p.tiles_per_expert;
+    const int E = p.E, tiles = p.tiles;
 
     if (warp == 0) {
         // Items of expert e: tiles * ceil(n_e / NT). Pass 1 counts them all;
@@ -293,18 +296,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (tid == 32) {
+        for (int s = 0; s < C::kStagesW; ++s) {
+            mbar_init(&fullW[s], 1);
+            mbar_init(&emptyW[s], 1);
+        }
         for (int s = 0; s < C::kStagesA; ++s) {
             mbar_init(&fullA[s], 1);
             mbar_init(&emptyA[s], 1);
         }
-        for (int s = 0; s < C::kStagesB; ++s) {
-            mbar_init(&fullB[s], 1);
-            mbar_init(&emptyB[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&accfull[b], 1);
-            mbar_init(&accempty[b], 4);
-        }
+        mbar_init(accfull, 1);
+        mbar_init(accempty, 4);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -319,47 +320,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     ItemCursor<NT> it;
     it.start(p.offsets, E, tiles, cur[0], cur[1]);
     const int nchunk = p.K / kKC;
-    const int nstage = (nchunk + C::kCPS - 1) / C::kCPS;
+    const int khalves = p.K / 128;
 
     if (warp == 0) {
         // ----------------------------------------------------------- producer
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
-            int sa = 0, sb = 0;
-            uint32_t pha = 0, phb = 0;
-            int64_t issued_a = 0, issued_b = 0;
+            int sw = 0, sa = 0;
+            uint32_t phw = 0, pha = 0;
+            int64_t issued_w = 0, issued_a = 0;
             bool ok = true;
             for (int i = 0; i < n_items && ok; ++i, it.next()) {
                 const int64_t box0 = ((int64_t)it.e * tiles + it.tile) * nchunk;
+                const int64_t pass_id = (int64_t)p.pass_start[it.e] + it.pass;
                 const int r0 = it.r0();
-                for (int st = 0; st < nstage; ++st) {
-                    const int c0 = st * C::kCPS, nc = min(C::kCPS, nchunk - c0);
+                for (int c = 0; c < nchunk; ++c) {
+                    if (*abort_flag || !mbar_wait_bounded(&emptyW[sw], phw ^ 1u, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&fullW[sw], (uint32_t)(kWBox + kWSf));
+                    tc::tma_load_2d(sW + (size_t)sw * kWBox, &tmW, 0, (int)((box0 + c) * 256), &fullW[sw], pol_w);
+                    bulk_g2s_hint(sSfw + sw * kWSf, p.wsf + (box0 + c) * kWSf, kWSf, &fullW[sw], pol_w);
+                    ++issued_w;
                     if (*abort_flag || !mbar_wait_bounded(&emptyA[sa], pha ^ 1u, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&fullA[sa], (uint32_t)(C::kATx + nc * kSFImg));
-                    tc::tma_load_3d(sA + (size_t)sa * C::kAStage, &tmA, 0, 0, (int)(box0 + c0), &fullA[sa], pol_w);
-                    bulk_g2s_hint(sSfa + sa * C::kSfaStage, p.sfa + (box0 + c0) * kSFImg, (uint32_t)(nc * kSFImg),
-                                  &fullA[sa], pol_w);
+                    mbar_arrive_expect_tx(&fullA[sa], (uint32_t)(C::kATx + 2 * kSFImg));
+                    tc::tma_load_4d(sA + (size_t)sa * kAStage, &tmA, 0, 0, r0, c, &fullA[sa], pol_a);
+                    bulk_g2s_hint(sSfa + sa * 2 * kSFImg, p.asf + (pass_id * khalves + 2 * c) * kSFImg, 2 * kSFImg,
+                                  &fullA[sa], pol_a);
                     ++issued_a;
-                    if (*abort_flag || !mbar_wait_bounded(&emptyB[sb], phb ^ 1u, kWaitLimitNs)) {
-                        ok = false;
-                        break;
+                    if (++sw == C::kStagesW) {
+                        sw = 0;
+                        phw ^= 1u;
                     }
-                    mbar_arrive_expect_tx(&fullB[sb], (uint32_t)(C::kBStage + C::kSfbTx));
-                    tc::tma_load_4d(sB + (size_t)sb * C::kBStage, &tmB, 0, r0, 0, c0, &fullB[sb], pol_a);
-                    tc::tma_load_3d(sSfb + sb * C::kSfbStage, &tmSfb, 0, r0, C::kPerTerm ? c0 * NTERMS : c0,
-                                    &fullB[sb], pol_a);
-                    ++issued_b;
                     if (++sa == C::kStagesA) {
                         sa = 0;
                         pha ^= 1u;
-                    }
-                    if (++sb == C::kStagesB) {
-                        sb = 0;
-                        phb ^= 1u;
                     }
                 }
             }
@@ -368,13 +368,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *abort_flag = 1;
             }
             // Drain: no copy of ours may still be landing when the CTA ends.
-            for (int64_t f = issued_a > C::kStagesA ? issued_a - C::kStagesA : 0; f < issued_a; ++f)
-                if (!mbar_wait_bounded(&fullA[f % C::kStagesA], (uint32_t)((f / C::kStagesA) & 1), kWaitLimitNs)) {
+            for (int64_t f = issued_w > C::kStagesW ? issued_w - C::kStagesW : 0; f < issued_w; ++f)
+                if (!mbar_wait_bounded(&fullW[f % C::kStagesW], (uint32_t)((f / C::kStagesW) & 1), kWaitLimitNs)) {
                     set_status(p.status, MXMOE_ERR_TIMEOUT);
                     break;
                 }
-            for (int64_t f = issued_b > C::kStagesB ? issued_b - C::kStagesB : 0; f < issued_b; ++f)
-                if (!mbar_wait_bounded(&fullB[f % C::kStagesB], (uint32_t)((f / C::kStagesB) & 1), kWaitLimitNs)) {
+            for (int64_t f = issued_a > C::kStagesA ? issued_a - C::kStagesA : 0; f < issued_a; ++f)
+                if (!mbar_wait_bounded(&fullA[f % C::kStagesA], (uint32_t)((f / C::kStagesA) & 1), kWaitLimitNs)) {
                     set_status(p.status, MXMOE_ERR_TIMEOUT);
                     break;
                 }
@@ -382,66 +382,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
-            int sa = 0, sb = 0;
-            uint32_t pha = 0, phb = 0;
+            int sw = 0, sa = 0;
+            uint32_t phw = 0, pha = 0;
             bool ok = true, any = false;
             for (int i = 0; i < n_items && ok; ++i) {
-                const int buf = i & 1;
-                const uint32_t use = (uint32_t)(i >> 1);
-                if (*abort_flag || !mbar_wait_bounded(&accempty[buf], (use & 1u) ^ 1u, kWaitLimitNs)) {
+                if (*abort_flag || !mbar_wait_bounded(accempty, ((uint32_t)i & 1u) ^ 1u, kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
                 tc::fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)buf * C::kBufCols;
-                for (int st = 0; st < nstage; ++st) {
-                    const int nc = min(C::kCPS, nchunk - st * C::kCPS);
-                    if (*abort_flag || !mbar_wait_bounded(&fullA[sa], pha, kWaitLimitNs) ||
-                        !mbar_wait_bounded(&fullB[sb], phb, kWaitLimitNs)) {
+                for (int c = 0; c < nchunk; ++c) {
+                    if (*abort_flag || !mbar_wait_bounded(&fullW[sw], phw, kWaitLimitNs) ||
+                        !mbar_wait_bounded(&fullA[sa], pha, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc::fence_after();
-                    const uint32_t sfa_t = tmem + C::kSfaCol0 + C::kSfaCols * sa;
-                    const uint32_t sfb_t = tmem + C::kSfbCol0 + C::kSfbCols * sb;
-                    const uint32_t a_base = smem_u32(sA + (size_t)sa * C::kAStage);
-                    const uint32_t b_base = smem_u32(sB + (size_t)sb * C::kBStage);
-                    const uint32_t sfa_s = smem_u32(sSfa + sa * C::kSfaStage);
-                    const uint32_t sfb_s = smem_u32(sSfb + sb * C::kSfbStage);
-                    for (int j = 0; j < nc; ++j)
-                        tc::cp_32x128b_warpx4(sfa_t + 4 * j, tc::smem_desc(sfa_s + j * kSFImg, 16, 128, 0));
-                    for (int j = 0; j < nc; ++j)
-                        tc::cp_32x128b_warpx4(sfb_t + 4 * j, tc::smem_desc(sfb_s + j * C::kSfbImg, 16, 128, 0));
-                    for (int j = 0; j < nc; ++j) {
-                        const uint32_t sfa_j = sfa_t + 4 * j;
-                        const uint32_t sfb_j = sfb_t + 4 * j;
+                    const uint32_t sfw_t = tmem + C::kSfwCol0 + 16 * sw;  // + 8 per K half, + 4 per row half
+                    const uint32_t sfa_t = tmem + C::kSfaCol0 + 8 * sa;   // + 4 per K half
+                    const uint32_t sfw_s = smem_u32(sSfw + sw * kWSf);
+                    const uint32_t sfa_s = smem_u32(sSfa + sa * 2 * kSFImg);
 #pragma unroll
-                        for (int kb = 0; kb < 4; ++kb) {
-                            const uint64_t adesc =
-                                tc::smem_desc(a_base + j * kChunkSmem + kb * 32, 16, 1024, 2);
-                            const uint64_t bdesc = tc::smem_desc(b_base + j * C::kBChunk + kb * 32, 16, 1024, 2);
-                            const uint32_t idesc = tc::idesc_e2m1_e4m3(C::kN, (uint32_t)kb);
-                            const int step = 4 * j + kb;
-                            const int chain = step % C::kChains;
-                            tc::mma_mxf8f6f4(d_tmem + (uint32_t)chain * C::kAccStride, adesc, bdesc, idesc,
-                                             (st > 0 || step >= C::kChains) ? 1u : 0u, sfa_j | ((uint32_t)kb << 30),
-                                             sfb_j | ((uint32_t)kb << 30));
-                        }
+                    for (int img = 0; img < 4; ++img)
+                        tc::cp_32x128b_warpx4(sfw_t + 4 * img, tc::smem_desc(sfw_s + img * kSFImg, 16, 128, 0));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tc::cp_32x128b_warpx4(sfa_t + 4 * h, tc::smem_desc(sfa_s + h * kSFImg, 16, 128, 0));
+                    const uint32_t a_base = smem_u32(sA + (size_t)sa * kAStage);
+                    const uint32_t w_base = smem_u32(sW + (size_t)sw * kWBox);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {  // 64 values of K per MMA
+                        const uint32_t h = (uint32_t)(k >> 1), id = 2u * (uint32_t)(k & 1);
+                        mma_mxf4(tmem, tc::smem_desc(a_base + k * 32, 16, 1024, 2),
+                                 tc::smem_desc(w_base + k * 32, 16, 1024, 2), idesc_mxf4(256, id),
+                                 (c > 0 || k > 0) ? 1u : 0u, (sfa_t + 4 * h) | (id << 30),
+                                 (sfw_t + 8 * h) | (id << 30));
                     }
-                    tc::commit(&emptyA[sa]);  // frees both stages once these MMAs are done
-                    tc::commit(&emptyB[sb]);
+                    tc::commit(&emptyW[sw]);  // frees both stages once these MMAs are done
+                    tc::commit(&emptyA[sa]);
                     any = true;
+                    if (++sw == C::kStagesW) {
+                        sw = 0;
+                        phw ^= 1u;
+                    }
                     if (++sa == C::kStagesA) {
                         sa = 0;
                         pha ^= 1u;
                     }
-                    if (++sb == C::kStagesB) {
-                        sb = 0;
-                        phb ^= 1u;
-                    }
                 }
                 if (ok)
-                    tc::commit(&accfull[buf]);
+                    tc::commit(accfull);
             }
             if (!ok) {
                 set_status(p.status, MXMOE_ERR_TIMEOUT);
@@ -456,95 +446,109 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ----------------------------------------------------------- epilogue
-        // A warp that gives up on a wait stops reading tensor memory and writing
-        // outputs but keeps taking part in the pair barriers.
-        const int q = warp & 3;  // tensor-memory lane quarter: rows 32q .. 32q+31
-        const int pair = q >> 1;
+        // Warp quarter q reads accumulator lanes 32q .. 32q+31: tokens 4q .. 4q+3
+        // of the pass, term tl = lane % 8 in each. A warp that gives up on a wait
+        // stops reading tensor memory and writing outputs.
+        const int q = warp & 3;
+        const int tl = lane & 7;
+        const int n = 4 * q + (lane >> 3);  // token within the pass
+        const bool has_rows = 4 * q < NT;   // this quarter holds MMA rows in use
         bool aborted = false;
         for (int i = 0; i < n_items; ++i, it.next()) {
-            const int buf = i & 1;
-            const uint32_t use = (uint32_t)(i >> 1);
-            const int r0 = it.r0(), ntile = it.nt();
-            if (!aborted && (*abort_flag || !mbar_wait_bounded(&accfull[buf], use & 1u, kWaitLimitNs))) {
-                if (lane == 0) {
+            if (!aborted) {  // lane 0 waits; the warp follows its verdict
+                int ok = 1;
+                if (lane == 0 && (*abort_flag || !mbar_wait_bounded(accfull, (uint32_t)i & 1u, kWaitLimitNs))) {
                     set_status(p.status, MXMOE_ERR_TIMEOUT);
                     *abort_flag = 1;
+                    ok = 0;
                 }
-                aborted = true;
+                aborted = !__shfl_sync(0xFFFFFFFFu, ok, 0);
             }
             tc::fence_after();
-            float acc[NT];
+            // v[b][j]: column 64b + 8tl + j of the token's term sum
+            float v[4][8];
 #pragma unroll
-            for (int j0 = 0; j0 < NT; j0 += 8) {
-                float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                if (!aborted && j0 < ntile) {
-                    // chains, then term columns t*NT + n, added in that order
+            for (int b = 0; b < 4; ++b)
 #pragma unroll
-                    for (int a = 0; a < C::kChains; ++a)
+                for (int j = 0; j < 8; ++j)
+                    v[b][j] = 0.f;
+            if (!aborted && has_rows) {
 #pragma unroll
-                        for (int t = 0; t < NTERMS; ++t) {
-                            float w8[8];
-                            tc::ld_32x32b_x8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)buf * C::kBufCols +
-                                                 (uint32_t)(a * C::kAccStride + t * NT + j0),
-                                             w8);
+                for (int b = 0; b < 4; ++b) {
+                    float x[64];
+                    tc::ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * b), x);
+                    tc::ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * b + 32), x + 32);
+                    // reduce-scatter over the 8 term lanes of each token
 #pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                v8[k] = (a | t) ? v8[k] + w8[k] : w8[k];
+                    for (int round = 0; round < 3; ++round) {
+                        const int half = 32 >> round, mask = 4 >> round;
+                        const bool up = (tl & mask) != 0;
+#pragma unroll
+                        for (int j = 0; j < half; ++j) {
+                            const float send = up ? x[j] : x[j + half];
+                            const float keep = up ? x[j + half] : x[j];
+                            x[j] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, mask);
                         }
-                }
+                    }
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    acc[j0 + k] = v8[k];
+                    for (int j = 0; j < 8; ++j)
+                        v[b][j] = x[j];
+                }
             }
             tc::fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&accempty[buf]);
+                mbar_arrive(accempty);
+            const int ntile = it.nt();
+            const bool valid = !aborted && has_rows && n < ntile;
             if (GATE_UP) {
-                // lanes 0..15 hold gate column col, lanes 16..31 the up column col
-                const int col = 64 * it.tile + 16 * q + (lane & 15);
-                float *xb = xchg + (pair * 2 + (i & 1)) * 2 * NT;
+                // h columns 64b + 8tl + j of the tile (b = 0, 1): gate = v[b], up = v[b + 2]
+                float hv[2][8];
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const float g = acc[n];
-                    const float u = __shfl_down_sync(0xFFFFFFFFu, g, 16);
-                    const float h = (n < ntile) ? g / (1.f + expf(-g)) * u : 0.f;
-                    float m = (lane < 16) ? fabsf(h) : 0.f;
+                for (int b = 0; b < 2; ++b)
 #pragma unroll
-                    for (int off = 8; off > 0; off >>= 1)
-                        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-                    acc[n] = h;
-                    if (lane == 0)
-                        xb[(q & 1) * NT + n] = m;  // this quarter's half-block maximum
-                }
-                named_bar_sync(2 + pair, 64);
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    if (aborted || n >= ntile)
-                        continue;
-                    const float bm = fmaxf(xb[n], xb[NT + n]);
-                    const int s = act_block_exp(bm);
-                    const float inv = __uint_as_float((uint32_t)(127 - s) << 23);  // 2^-s
-                    const int r = r0 + n;
-                    if (lane < 16) {
-                        uint32_t code[3];
-                        split_terms<3>(acc[n] * inv, code);
-#pragma unroll
-                        for (int t = 0; t < 3; ++t)
-                            p.h_terms[term_offset(3, p.rows_act, t, r, col)] = (uint8_t)code[t];
+                    for (int j = 0; j < 8; ++j) {
+                        const float g = v[b][j];
+                        hv[b][j] = valid ? g / (1.f + expf(-g)) * v[b + 2][j] : 0.f;
                     }
-                    if (lane == 0 && !(q & 1)) {
+                const int r = it.r0() + n;
+                const int64_t img = ((int64_t)p.pass_start[it.e] + it.pass) * (p.I / 128) + it.tile;
 #pragma unroll
-                        for (int t = 0; t < 3; ++t)
-                            p.h_rec[rec_offset(C::kPerTerm, 3, p.rows_act, t, r, col)] = (uint8_t)(s - 4 * t + 127);
+                for (int t = 0; t < kT; ++t) {
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        // the 32-block of these 8 columns spans the lanes tl ^ {0..3}
+                        float m = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            m = fmaxf(m, fabsf(hv[b][j]));
+                        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                        const int s = e2m1_block_exp(m);
+                        const float inv = pow2f(-s), pw = pow2f(s);
+                        uint32_t word = 0;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            float qv;
+                            word |= e2m1_code(hv[b][j] * inv, qv) << (4 * j);
+                            hv[b][j] -= qv * pw;
+                        }
+                        if (valid) {
+                            const int col = 128 * it.tile + 64 * b + 8 * tl;
+                            *reinterpret_cast<uint32_t *>(p.h_terms + term_offset(p.rows, t, r, col)) = word;
+                            if ((tl & 3) == 0)
+                                p.h_sf[img * kSFImg + image_byte(n, t, 2 * b + (tl >> 2))] = (uint8_t)(s + 127);
+                        }
                     }
                 }
-            } else if (!aborted) {
-                float *yrow = p.y_out + (int64_t)r0 * p.H + 128 * it.tile + 32 * q + lane;
+            } else if (valid) {
+                float *yrow = p.y_out + (int64_t)(it.r0() + n) * p.H + 256 * it.tile + 8 * tl;
 #pragma unroll
-                for (int n = 0; n < NT; ++n)
-                    if (n < ntile)
-                        yrow[(int64_t)n * p.H] = acc[n];
+                for (int b = 0; b < 4; ++b) {
+                    float4 *dst = reinterpret_cast<float4 *>(yrow + 64 * b);
+                    dst[0] = make_float4(v[b][0], v[b][1], v[b][2], v[b][3]);
+                    dst[1] = make_float4(v[b][4], v[b][5], v[b][6], v[b][7]);
+                }
             }
         }
     }
@@ -556,37 +560,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// x rows (bf16) -> 2 E4M3 terms per value in grouped row order (row r holds
-// token src_row[r] / k), in the term_offset layout, and their UE8M0 scales per
-// 32-value block in the rec_offset layout. One warp per 32-value block.
-// Block 0 also clears the status word.
-__global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ src_row,
-                                                      int k, int rows, int H, uint8_t *__restrict__ terms,
-                                                      uint8_t *__restrict__ rec, bool per_term, int *status)
+// Token passes of each expert: pass_start[e] = sum over e' < e of
+// ceil(n_e' / nt), for one block's warp 0 (E <= kMaxE).
+__device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
 {
-    if (blockIdx.x == 0 && threadIdx.x == 0 && status)
-        *status = 0;
     const int lane = threadIdx.x & 31;
+    int carry = 0;
+    for (int b = 0; b <= E; b += 32) {
+        const int e = b + lane;
+        const int c = e < E ? (offsets[e + 1] - offsets[e] + nt - 1) / nt : 0;
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off)
+                incl += o;
+        }
+        if (e <= E)
+            out[e] = carry + incl - c;
+        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+}
+
+// x rows (bf16) -> kT E2M1 terms per value in grouped row order (row r holds
+// token src_row[r] / k), in the term_offset layout, with their scale images
+// (one per token pass and 128 columns). One warp per 32-value block. Block 0
+// also writes pass_start for the FFN stages and clears the status word.
+__global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ src_row,
+                                                      const int32_t *__restrict__ offsets, int E, int k, int rows,
+                                                      int H, int nt, uint8_t *__restrict__ terms,
+                                                      uint8_t *__restrict__ sf, int32_t *__restrict__ pass_start_out,
+                                                      int *status)
+{
+    __shared__ int32_t s_off[kMaxE + 1], s_pass[kMaxE + 1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp == 0)
+        pass_prefix(offsets, E, nt, s_pass);
+    for (int e = threadIdx.x; e <= E; e += blockDim.x)
+        s_off[e] = offsets[e];
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x)
+            pass_start_out[e] = s_pass[e];
+        if (threadIdx.x == 0 && status)
+            *status = 0;
+    }
     const int nkb = H / 32;
     const int64_t total = (int64_t)rows * nkb;
-    for (int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); w < total; w += (int64_t)gridDim.x * 8) {
+    for (int64_t w = (int64_t)blockIdx.x * 8 + warp; w < total; w += (int64_t)gridDim.x * 8) {
         const int r = (int)(w / nkb), kb = (int)(w % nkb);
+        int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_off[mid] <= r)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int local = r - s_off[lo];
+        const int64_t img = ((int64_t)s_pass[lo] + local / nt) * (H / 128) + kb / 4;
+        const int n = local % nt;
         const int tok = src_row[r] / k;
         const int col = kb * 32 + lane;
-        const float v = __uint_as_float((uint32_t)x[(int64_t)tok * H + col] << 16);
-        float m = fabsf(v);
+        float res = __uint_as_float((uint32_t)x[(int64_t)tok * H + col] << 16);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-        const int s = act_block_exp(m);
-        const float inv = __uint_as_float((uint32_t)(127 - s) << 23);
-        uint32_t code[2];
-        split_terms<2>(v * inv, code);
-        terms[term_offset(2, rows, 0, r, col)] = (uint8_t)code[0];
-        terms[term_offset(2, rows, 1, r, col)] = (uint8_t)code[1];
-        if (lane == 0) {
-            rec[rec_offset(per_term, 2, rows, 0, r, col)] = (uint8_t)(s + 127);
-            rec[rec_offset(per_term, 2, rows, 1, r, col)] = (uint8_t)(s - 4 + 127);
+        for (int t = 0; t < kT; ++t) {
+            float m = fabsf(res);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+            const int s = e2m1_block_exp(m);
+            float qv;
+            const uint32_t code = e2m1_code(res * pow2f(-s), qv);
+            res -= qv * pow2f(s);
+            const uint32_t hi_code = __shfl_down_sync(0xFFFFFFFFu, code, 1);
+            if (!(lane & 1))
+                terms[term_offset(rows, t, r, col)] = (uint8_t)(code | (hi_code << 4));
+            if (lane == 0)
+                sf[img * kSFImg + image_byte(n, t, kb & 3)] = (uint8_t)(s + 127);
         }
     }
 }
@@ -618,10 +669,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 // ---------------------------------------------------------------------------
 struct FfnWs {
     int *status;
-    uint8_t *x_terms;  // [H/128][2][rows][128]
-    uint8_t *x_rec;    // records (rec_offset layout)
-    uint8_t *h_terms;  // [I/128][3][rows][128]
-    uint8_t *h_rec;    // records (rec_offset layout)
+    int32_t *pass_start;  // [kMaxE + 1]
+    uint8_t *x_terms;     // term_offset layout, K = H
+    uint8_t *x_sf;        // scale images [pass][H/128][512]
+    uint8_t *h_terms;     // term_offset layout, K = I
+    uint8_t *h_sf;        // scale images [pass][I/128][512]
 };
 
 int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
@@ -633,21 +685,21 @@ int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
         return o;
     };
     const int64_t rows = (int64_t)T * k;
-    // record planes for either record layout
-    const int64_t xr_planes = std::max(rec_planes(true, 2, H), rec_planes(false, 2, H));
-    const int64_t hr_planes = std::max(rec_planes(true, 3, I), rec_planes(false, 3, I));
+    const int64_t passes = max_passes(rows);
     const int64_t o_status = take(16);
-    const int64_t o_xt = take(2 * rows * H);
-    const int64_t o_xr = take(xr_planes * rows * 16);
-    const int64_t o_ht = take(3 * rows * I);
-    const int64_t o_hr = take(hr_planes * rows * 16);
+    const int64_t o_ps = take((kMaxE + 1) * 4);
+    const int64_t o_xt = take(rows * kT * H / 2);
+    const int64_t o_xs = take(passes * (H / 128) * kSFImg);
+    const int64_t o_ht = take(rows * kT * I / 2);
+    const int64_t o_hs = take(passes * (I / 128) * kSFImg);
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
         ws->status = reinterpret_cast<int *>(b + o_status);
+        ws->pass_start = reinterpret_cast<int32_t *>(b + o_ps);
         ws->x_terms = b + o_xt;
-        ws->x_rec = b + o_xr;
+        ws->x_sf = b + o_xs;
         ws->h_terms = b + o_ht;
-        ws->h_rec = b + o_hr;
+        ws->h_sf = b + o_hs;
     }
     return off;
 }
@@ -678,93 +730,75 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-int encode(CUtensorMap *m, CUtensorMapDataType type, int rank, const void *base, const cuuint64_t *dims,
-           const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle swizzle, CUtensorMapL2promotion promo,
-           const char *what)
+int encode(CUtensorMap *m, int rank, const void *base, const cuuint64_t *dims, const cuuint64_t *strides,
+           const cuuint32_t *box, CUtensorMapL2promotion promo, const char *what)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    CUresult r = enc(m, type, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
+                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (%s) failed: %d", what, (int)r);
     return MXMOE_OK;
 }
 
-// The code boxes of one weight matrix (all experts): n_boxes boxes of 128
-// rows x 128 fp4 codes (64 bytes a row, 8 KB a box), read `cps` consecutive
-// boxes per request, each unpacked into one 16-byte slot per 16 codes with the
-// 128-byte swizzle. Boxes past the end read as zero.
-int encode_weights(CUtensorMap *m, const void *base, int64_t n_boxes, int cps)
+// The code boxes of one weight matrix (all experts) as rows of 128 bytes; a
+// request brings one box (256 rows), with the 128-byte swizzle.
+int encode_weights(CUtensorMap *m, const void *base, int64_t n_boxes)
 {
-    const cuuint64_t dims[3] = {128, 128, (cuuint64_t)n_boxes};
-    const cuuint64_t strides[2] = {64, kChunkTx};
-    const cuuint32_t box[3] = {128, 128, (cuuint32_t)cps};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, "weights");
+    const cuuint64_t dims[2] = {128, (cuuint64_t)(n_boxes * 256)};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, 256};
+    return encode(m, 2, base, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, "weights");
 }
 
-// Activation terms in the term_offset layout, dims {128, rows, nterms,
-// chunks}; a request brings nt rows x all terms x cps chunks. Rows and chunks
-// past the end read as zero.
-int encode_terms(CUtensorMap *m, const void *base, int64_t rows, int K, int nterms, int nt, int cps)
+// Activation terms (term_offset layout), dims {128, kT, rows, K/256}; a
+// request brings all terms of nt rows of one chunk. Rows past the end read as
+// zero.
+int encode_terms(CUtensorMap *m, const void *base, int64_t rows, int K, int nt)
 {
-    const cuuint64_t dims[4] = {128, (cuuint64_t)rows, (cuuint64_t)nterms, (cuuint64_t)(K / kKC)};
-    const cuuint64_t strides[3] = {128, (cuuint64_t)(rows * 128), (cuuint64_t)(rows * 128 * nterms)};
-    const cuuint32_t box[4] = {128, (cuuint32_t)nt, (cuuint32_t)nterms, (cuuint32_t)cps};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, "activation terms");
+    const cuuint64_t dims[4] = {128, (cuuint64_t)kT, (cuuint64_t)rows, (cuuint64_t)(K / kKC)};
+    const cuuint64_t strides[3] = {128, (cuuint64_t)(kT * 128), (cuuint64_t)(rows * kT * 128)};
+    const cuuint32_t box[4] = {128, (cuuint32_t)kT, (cuuint32_t)nt, 1};
+    return encode(m, 4, base, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, "activation terms");
 }
 
-// Scale records (rec_offset layout), dims {16, rows, planes}; a request brings
-// nt rows x z planes.
-int encode_records(CUtensorMap *m, const void *base, int64_t rows, int64_t planes, int nt, int z)
+template <int NT, bool GATE_UP>
+int launch_ffn(const void *codes, const uint8_t *act_terms, const FfnParams &p, cudaStream_t st)
 {
-    const cuuint64_t dims[3] = {16, (cuuint64_t)rows, (cuuint64_t)planes};
-    const cuuint64_t strides[2] = {16, (cuuint64_t)(rows * 16)};
-    const cuuint32_t box[3] = {16, (cuuint32_t)nt, (cuuint32_t)z};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_NONE, "activation scale records");
-}
-
-template <int NT, int NTERMS, bool GATE_UP>
-int launch_ffn(const void *codes, const uint8_t *act_terms, const uint8_t *act_rec, FfnParams p, cudaStream_t st)
-{
-    using C = Cfg<NT, NTERMS>;
+    using C = Cfg<NT>;
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(ffn_tc_kernel<NT, NTERMS, GATE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(ffn_mxf4_kernel<NT, GATE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)C::kSmem) != cudaSuccess)
-            return fail(MXMOE_ERR_CUDA, "ffn_tc_kernel: cannot reserve %zu bytes of shared memory", C::kSmem);
+            return fail(MXMOE_ERR_CUDA, "ffn_mxf4_kernel: cannot reserve %zu bytes of shared memory", C::kSmem);
         configured_dev = dev;
     }
-    const int64_t n_boxes = (int64_t)p.E * p.tiles_per_expert * (p.K / kKC);
-    CUtensorMap tmA, tmB, tmSfb;
-    if (int rc = encode_weights(&tmA, codes, n_boxes, C::kCPS))
+    CUtensorMap tmW, tmA;
+    if (int rc = encode_weights(&tmW, codes, (int64_t)p.E * p.tiles * (p.K / kKC)))
         return rc;
-    if (int rc = encode_terms(&tmB, act_terms, p.rows_act, p.K, NTERMS, NT, C::kCPS))
+    if (int rc = encode_terms(&tmA, act_terms, p.rows, p.K, NT))
         return rc;
-    if (int rc = encode_records(&tmSfb, act_rec, p.rows_act, rec_planes(C::kPerTerm, NTERMS, p.K), NT, C::kSfbZ))
-        return rc;
-    ffn_tc_kernel<NT, NTERMS, GATE_UP><<<num_sms(), kThreads, C::kSmem, st>>>(tmA, tmB, tmSfb, p);
-    return check_launch(GATE_UP ? "ffn_tc_kernel<gate_up>" : "ffn_tc_kernel<down>");
+    ffn_mxf4_kernel<NT, GATE_UP><<<num_sms(), kThreads, C::kSmem, st>>>(tmW, tmA, p);
+    return check_launch(GATE_UP ? "ffn_mxf4_kernel<gate_up>" : "ffn_mxf4_kernel<down>");
 }
 
-// Token rows per pass: 8 while the mean rows per expert is at most 8 (decode
-// and verify blocks), else 32.
-int token_tile(int T, int k, int E) { return (int64_t)T * k <= 8LL * E ? 8 : 32; }
+// Token rows per pass: 8 up to 8 tokens (an expert then never sees more than
+// 8 rows), else 16.
+int token_tile(int T) { return T <= 8 ? 8 : 16; }
 
 int validate_ffn(int T, int k, int E, int H, int I)
 {
-    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 128 || I % 128 || H > 32768 ||
-        I > 32768 || (int64_t)T * k > (1 << 22))
+    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > kMaxE || H <= 0 || I <= 0 || H % 256 || I % 256 || H > 32768 ||
+        I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31))
         return fail(MXMOE_ERR_INVALID_SHAPE,
-                    "expert FFN: T=%d k=%d E=%d H=%d I=%d (need H, I multiples of 128 up to 32768, 1 <= k <= 32, "
-                    "E <= 1024, T*k <= 2^22)",
+                    "expert FFN: T=%d k=%d E=%d H=%d I=%d (need H, I multiples of 256 up to 32768, 1 <= k <= 32, "
+                    "E <= 1024, T*k <= 2^22, E*I*H < 2^38)",
                     T, k, E, H, I);
     return MXMOE_OK;
 }
@@ -793,32 +827,35 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     FfnWs ws;
     ffn_ws_layout(T, k, H, I, &ws, workspace);
     const int rows = T * k;
-    const int nt = token_tile(T, k, E);
+    const int nt = token_tile(T);
     {
         const int64_t warps = (int64_t)rows * (H / 32);
-        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 16);
-        x_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, k, rows,
-                                                                 H, ws.x_terms, ws.x_rec, nt <= 8, ws.status);
+        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 8);
+        x_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
+                                                                 k, rows, H, nt, ws.x_terms, ws.x_sf, ws.pass_start,
+                                                                 ws.status);
         if (int rc = check_launch("x_terms_kernel"))
             return rc;
     }
     const Blob bl = blob_parts(prepacked, E, H, I);
     FfnParams p{};
-    p.tiles_per_expert = 2 * I / 128;
+    p.tiles = I / 128;
     p.K = H;
-    p.rows_act = rows;
-    p.sfa = bl.sf13;
+    p.rows = rows;
+    p.wsf = bl.sf13;
+    p.asf = ws.x_sf;
     p.offsets = offsets;
+    p.pass_start = ws.pass_start;
     p.E = E;
     p.h_terms = ws.h_terms;
-    p.h_rec = ws.h_rec;
+    p.h_sf = ws.h_sf;
     p.I = I;
     p.y_out = nullptr;
     p.H = H;
     p.status = ws.status;
     if (nt == 8)
-        return launch_ffn<8, 2, true>(bl.w13, ws.x_terms, ws.x_rec, p, st);
-    return launch_ffn<32, 2, true>(bl.w13, ws.x_terms, ws.x_rec, p, st);
+        return launch_ffn<8, true>(bl.w13, ws.x_terms, p, st);
+    return launch_ffn<16, true>(bl.w13, ws.x_terms, p, st);
 }
 
 int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, int E, int H, int I, float *y_perm,
@@ -827,24 +864,26 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
     FfnWs ws;
     ffn_ws_layout(T, k, H, I, &ws, workspace);
     const int rows = T * k;
-    const int nt = token_tile(T, k, E);
+    const int nt = token_tile(T);
     const Blob bl = blob_parts(prepacked, E, H, I);
     FfnParams p{};
-    p.tiles_per_expert = H / 128;
+    p.tiles = H / 256;
     p.K = I;
-    p.rows_act = rows;
-    p.sfa = bl.sf2;
+    p.rows = rows;
+    p.wsf = bl.sf2;
+    p.asf = ws.h_sf;
     p.offsets = offsets;
+    p.pass_start = ws.pass_start;
     p.E = E;
     p.h_terms = nullptr;
-    p.h_rec = nullptr;
+    p.h_sf = nullptr;
     p.I = I;
     p.y_out = y_perm;
     p.H = H;
     p.status = ws.status;
     if (nt == 8)
-        return launch_ffn<8, 3, false>(bl.w2, ws.h_terms, ws.h_rec, p, st);
-    return launch_ffn<32, 3, false>(bl.w2, ws.h_terms, ws.h_rec, p, st);
+        return launch_ffn<8, false>(bl.w2, ws.h_terms, p, st);
+    return launch_ffn<16, false>(bl.w2, ws.h_terms, p, st);
 }
 
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
@@ -873,8 +912,8 @@ using namespace mxmoe;
 
 extern "C" MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I)
 {
-    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 128 || I % 128 || H > 32768 ||
-        I > 32768 || (int64_t)T * k > (1 << 22))
+    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 256 || I % 256 || H > 32768 ||
+        I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31))
         return -1;
     return ffn_workspace_bytes(T, k, H, I);
 }

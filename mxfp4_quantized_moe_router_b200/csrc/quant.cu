@@ -100,20 +100,20 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
 // Prepacked blob for the tensor-core FFN (a byte permutation of the canonical
 // format, same size):
 //   [gate/up code boxes][down code boxes][gate/up scale images][down scale images]
-// A code box is one 128-row tile by 128 values of K: 128 rows of 64 bytes,
-// contiguous (8 KB), boxes ordered by (expert, tile, K chunk). Gate/up rows are
-// reordered per tile t so that tile row lr = 32q + w holds gate column
-// 64t + 16q + w (w < 16) or up column 64t + 16q + (w - 16) (w >= 16); down
-// rows keep their order. A scale image covers the same tile and K chunk:
-// byte (m % 32) * 16 + (m / 32) * 4 + kb holds the scale of tile row m,
-// k32 block kb.
+// A code box is one 256-row wide tile by 256 values of K: 256 rows of 128
+// bytes (32 KB, contiguous), boxes ordered by (expert, tile, K chunk). Gate/up
+// tile t holds gate rows 128t .. 128t+127 (tile rows 0..127) and then the
+// matching up rows (tile rows 128..255); down rows keep their order. The
+// scale images of a box are four 512-byte images ordered (K half h, row half
+// g): byte (r % 32) * 16 + (r / 32) * 4 + kb holds the scale of tile row
+// 128g + r, k32 block 4h + kb of the box.
 __device__ __forceinline__ int64_t tile_src_row(bool gate_up, int64_t lr_all, int I)
 {
     if (!gate_up)
         return lr_all;
-    const int64_t t = lr_all >> 7;
-    const int lr = (int)(lr_all & 127), q = lr >> 5, w = lr & 31;
-    return (w < 16) ? 64 * t + 16 * q + w : (int64_t)I + 64 * t + 16 * q + (w - 16);
+    const int64_t t = lr_all >> 8;
+    const int lr = (int)(lr_all & 255);
+    return lr < 128 ? 128 * t + lr : (int64_t)I + 128 * t + (lr - 128);
 }
 
 // One thread per 16 bytes of the code boxes.
@@ -121,40 +121,43 @@ __global__ void __launch_bounds__(256) prepack_rows_kernel(const uint8_t *__rest
                                                            int64_t rows_per_expert, int K, bool gate_up, int I,
                                                            uint8_t *__restrict__ dst)
 {
-    const int nchunk = K / 128;
-    const int64_t tiles = rows_per_expert / 128;
+    const int nchunk = K / 256;
+    const int64_t tiles = rows_per_expert / 256;
     const int64_t total = (int64_t)E * rows_per_expert * (K / 32);  // 16-byte units
     for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
-        const int part = (int)(u & 3);          // 16-byte part of a 64-byte box row
-        const int lr = (int)((u >> 2) & 127);   // box row
-        const int64_t box = u >> 9;             // (e * tiles + t) * nchunk + c
+        const int part = (int)(u & 7);          // 16-byte part of a 128-byte box row
+        const int lr = (int)((u >> 3) & 255);   // box row
+        const int64_t box = u >> 11;            // (e * tiles + t) * nchunk + c
         const int c = (int)(box % nchunk);
         const int64_t tile_id = box / nchunk;
         const int64_t e = tile_id / tiles, t = tile_id % tiles;
-        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 128 + lr, I);
+        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 256 + lr, I);
         reinterpret_cast<uint4 *>(dst)[u] =
-            __ldg(reinterpret_cast<const uint4 *>(packed + src * (K / 2) + (int64_t)c * 64) + part);
+            __ldg(reinterpret_cast<const uint4 *>(packed + src * (K / 2) + (int64_t)c * 128) + part);
     }
 }
 
+// One thread per byte of the scale images.
 __global__ void __launch_bounds__(256) prepack_sf_kernel(const uint8_t *__restrict__ sc, int E,
                                                          int64_t rows_per_expert, int K, bool gate_up, int I,
                                                          uint8_t *__restrict__ dst)
 {
-    const int nchunk = K / 128;
-    const int64_t tiles = rows_per_expert / 128;
-    const int64_t total = (int64_t)E * tiles * nchunk * 512;
+    const int nchunk = K / 256;
+    const int64_t tiles = rows_per_expert / 256;
+    const int64_t total = (int64_t)E * tiles * nchunk * 2048;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         const int b = (int)(i & 511);
-        const int64_t img = i >> 9;
-        const int c = (int)(img % nchunk);
-        const int64_t tile_id = img / nchunk;
+        const int g = (int)((i >> 9) & 1), h = (int)((i >> 10) & 1);
+        const int64_t box = i >> 11;
+        const int c = (int)(box % nchunk);
+        const int64_t tile_id = box / nchunk;
         const int64_t e = tile_id / tiles, t = tile_id % tiles;
         const int m = (b >> 4) + 32 * ((b & 15) >> 2), kb = b & 3;
-        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 128 + m, I);
-        dst[i] = sc[src * (K / 32) + 4 * c + kb];
+        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 256 + 128 * g + m, I);
+        dst[i] = sc[src * (K / 32) + 8 * c + 4 * h + kb];
     }
 }
+
 
 int grid_for(int64_t work, int per_block)
 {
@@ -204,7 +207,7 @@ extern "C" MXMOE_API int mxmoe_dequantize(const uint8_t *packed, const uint8_t *
 
 extern "C" MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I)
 {
-    if (E <= 0 || H <= 0 || I <= 0 || H % 128 || I % 128)
+    if (E <= 0 || H <= 0 || I <= 0 || H % 256 || I % 256)
         return -1;
     return (int64_t)E * 3 * H * I / 2 + (int64_t)E * 3 * H * I / 32;
 }
@@ -215,7 +218,7 @@ extern "C" MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const ui
 {
     if (mxmoe_prepacked_size(E, H, I) < 0)
         return fail(MXMOE_ERR_INVALID_SHAPE,
-                    "mxmoe_prepack_experts: E=%d H=%d I=%d (need H %% 128 == 0, I %% 128 == 0)", E, H, I);
+                    "mxmoe_prepack_experts: E=%d H=%d I=%d (need H %% 256 == 0, I %% 256 == 0)", E, H, I);
     if (!packed13 || !sc13 || !packed2 || !sc2 || !prepacked)
         return fail(MXMOE_ERR_NULL, "mxmoe_prepack_experts: NULL pointer");
     if ((reinterpret_cast<uintptr_t>(prepacked) & 31) || !aligned16(packed13) || !aligned16(packed2))

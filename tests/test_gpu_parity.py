@@ -141,14 +141,15 @@ def test_permute_skewed(mx):
 # Expert FFN (grouped), element by element against the oracle
 # ---------------------------------------------------------------------------
 FFN_CASES = [
-    # H, I, E, k, T : several tiles along I and H, several K steps, ragged
-    # token passes (8-token tiles for T <= 8, 32-token tiles otherwise)
-    (256, 128, 16, 2, 4),
-    (384, 256, 6, 2, 37),
-    (512, 256, 8, 2, 9),
-    (256, 384, 3, 1, 80),     # n_e up to ~40: several 32-token passes
-    (640, 384, 5, 3, 150),
-    (1024, 128, 2, 2, 1),     # one token, 8 of its tile rows padded
+    # H, I, E, k, T : several 256-row tiles along I and H, several K chunks,
+    # ragged token passes (8-token passes for T <= 8, 16-token passes
+    # otherwise)
+    (256, 256, 16, 2, 4),
+    (512, 256, 6, 2, 37),     # n_e up to ~20: two 16-token passes
+    (512, 512, 8, 2, 9),
+    (256, 768, 3, 1, 80),     # n_e up to ~40: several passes, 3 tiles along I
+    (768, 512, 5, 3, 150),
+    (1024, 256, 2, 2, 1),     # one token: 7 of the 8 pass rows unused
 ]
 
 
@@ -241,7 +242,7 @@ def test_layer_tiny(mx):
 
 @pytest.mark.parametrize("T", [1, 3, 64, 200])
 def test_layer_small_ragged(mx, T):
-    cfg = datagen.LayerConfig("small", 512, 24, 4, 128, T)
+    cfg = datagen.LayerConfig("small", 512, 24, 4, 256, T)
     layer = GpuLayer(mx, cfg, 1)
     x = datagen.make_x(cfg, 1)
     bias = (np.linspace(-0.5, 0.5, cfg.E)).astype(np.float32)

@@ -45,9 +45,9 @@ def test_noalloc_matches_workspace_ffn_twice(mx):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(mx):
-    # 6144/2048/top-8 needs more than the fixed 8 MiB beyond 50 tokens
-    assert mx.mxmoe_ffn_workspace_size(50, 8, 384, 6144, 2048) <= 8 << 20
-    assert mx.mxmoe_ffn_workspace_size(51, 8, 384, 6144, 2048) > 8 << 20
-    rc = mx.load().mxmoe_expert_ffn_noalloc(None, None, None, None, 51, 8, 384, 6144, 2048, None, None, None)
+    # 6144/2048/top-8 needs more than the fixed 8 MiB beyond 15 tokens
+    assert mx.mxmoe_ffn_workspace_size(15, 8, 384, 6144, 2048) <= 8 << 20
+    assert mx.mxmoe_ffn_workspace_size(16, 8, 384, 6144, 2048) > 8 << 20
+    rc = mx.load().mxmoe_expert_ffn_noalloc(None, None, None, None, 16, 8, 384, 6144, 2048, None, None, None)
     assert rc == mx.ERR_WORKSPACE
     assert "8388608" in mx.last_error()
