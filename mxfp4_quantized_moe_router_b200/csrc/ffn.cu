@@ -19,13 +19,13 @@
 //    weights are the N operand, 256 rows per MMA, and each MMA covers 8 KB of
 //    weight codes (256 rows x 64 values of K): enough that the weight stream,
 //    not the MMA issue, sets the pace.
-//  * Activations become kT = 8 E2M1 terms per value: term t is the E2M1
-//    rounding of what terms 0..t-1 left over, with its own UE8M0 scale per 32
-//    values chosen so the block's largest remainder fits E2M1's range. Each
-//    term removes at least a factor 3 of the block's largest remainder, so 8
-//    terms reproduce a value to within 3^-8 of its block maximum. The terms
-//    of a token are consecutive MMA rows (row = token * kT + term; M = 128 rows
-//    = 16 tokens); the epilogue adds them.
+//  * Activations become kT = 8 E2M1 terms per value: the balanced base-8
+//    digits (each in -4..4, all exact E2M1 values) of the value on the grid
+//    2^(E-22), E the exponent of its 32-value block's largest magnitude; term
+//    t carries scale 2^(E-1-3t). That is exact for every bf16 x within 2^-15
+//    of its block maximum and keeps h to within 2^-23 of its block maximum.
+//    The terms of a token are consecutive MMA rows (row = token * kT + term;
+//    M = 128 rows = 16 tokens); the epilogue adds them.
 //  * Weight boxes (256 rows x 256 K, 32 KB, contiguous in the prepacked blob)
 //    and their scale images (2 KB) stream through a 5-deep ring; activation
 //    terms (one 4-D TMA box per chunk) and their scale images (written by the
@@ -195,37 +195,43 @@ struct ItemCursor {
     __device__ __forceinline__ int nt() const { return min(NT, n_e - pass * NT); }
 };
 
-// UE8M0 exponent s of an activation term block whose largest magnitude is m:
-// the smallest s with m <= 6 * 2^s (E2M1's largest value), clamped to the
-// UE8M0 range; zero and subnormal maxima take the smallest scale.
-__device__ __forceinline__ int e2m1_block_exp(float m)
+__device__ __forceinline__ float pow2f(int s)  // 2^s for s in [-126, 127]
+{
+    return __uint_as_float((uint32_t)(s + 127) << 23);
+}
+
+// Exponent E of a 32-value activation block whose largest magnitude is m:
+// floor(log2 m), raised to -104 for tiny or zero blocks so that every term's
+// scale 2^(E - 1 - 3t) stays a normal UE8M0 value.
+__device__ __forceinline__ int act_block_exp(float m)
 {
     const uint32_t b = __float_as_uint(m);
-    if (b < 0x00800000u)
-        return -127;
-    const int e = (int)(b >> 23) - 127;
-    const int s = e - 2 + ((b & 0x7FFFFFu) > 0x400000u ? 1 : 0);
-    return max(-127, min(s, 126));
+    return max((int)(b >> 23) - 127, -104);
 }
 
-__device__ __forceinline__ float pow2f(int s)  // 2^s for s in [-127, 127]
+// The kT balanced base-8 digits of an activation value v in a block of
+// exponent E, as E2M1 codes: v ~= sum_t d_t * 2^(E - 1 - 3t), d_t in
+// {-4..4} (all exact E2M1 values), t = 0 most significant. The digits are
+// exact for any v that is a multiple of 2^(E - 22) -- every bf16 value within
+// 2^-15 of its block maximum -- and otherwise represent v rounded to that
+// grid (within 2^-23 of the block maximum).
+__device__ __forceinline__ uint32_t e2m1_digit_code(int d)  // d in [-4, 4]
 {
-    return s >= -126 ? __uint_as_float((uint32_t)(s + 127) << 23) : __uint_as_float(0x00400000u);
+    const int mag = d < 0 ? -d : d;
+    // E2M1 codes of 0, 1, 2, 3, 4 are 0x0, 0x2, 0x4, 0x5, 0x6; bit 3 is the sign
+    return ((0x65420u >> (4 * mag)) & 0xFu) | (d < 0 ? 8u : 0u);
 }
 
-// E2M1 code of y (|y| <= 6, round to nearest even) in the low nibble, and the
-// value that code stands for.
-__device__ __forceinline__ uint32_t e2m1_code(float y, float &q)
+__device__ __forceinline__ void act_digits(float v, int E, uint32_t (&code)[kT])
 {
-    uint32_t code, h2;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %3;\n\t"
-        "cvt.u32.u8 %0, t;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, t;\n\t}"
-        : "=r"(code), "=r"(h2)
-        : "f"(0.f), "f"(y));
-    q = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    return code & 0xFu;
+    int iv = (int)rintf(v * pow2f(22 - E));  // |iv| <= 2^23
+#pragma unroll
+    for (int t = kT - 1; t > 0; --t) {
+        const int d = ((iv + 4) & 7) - 4;  // balanced residue in [-4, 3]
+        iv = (iv - d) >> 3;                // exact: iv - d is a multiple of 8
+        code[t] = e2m1_digit_code(d);
+    }
+    code[0] = e2m1_digit_code(iv);  // |iv| <= 4 after kT - 1 such steps
 }
 
 // One FFN stage over all experts.
@@ -514,30 +520,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int r = it.r0() + n;
                 const int64_t img = ((int64_t)p.pass_start[it.e] + it.pass) * (p.I / 128) + it.tile;
 #pragma unroll
-                for (int t = 0; t < kT; ++t) {
+                for (int b = 0; b < 2; ++b) {
+                    // the 32-block of these 8 columns spans the lanes tl ^ {0..3}
+                    float m = 0.f;
 #pragma unroll
-                    for (int b = 0; b < 2; ++b) {
-                        // the 32-block of these 8 columns spans the lanes tl ^ {0..3}
-                        float m = 0.f;
+                    for (int j = 0; j < 8; ++j)
+                        m = fmaxf(m, fabsf(hv[b][j]));
+                    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                    const int E_blk = act_block_exp(m);
+                    uint32_t word[kT];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            m = fmaxf(m, fabsf(hv[b][j]));
-                        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-                        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-                        const int s = e2m1_block_exp(m);
-                        const float inv = pow2f(-s), pw = pow2f(s);
-                        uint32_t word = 0;
+                    for (int t = 0; t < kT; ++t)
+                        word[t] = 0;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            float qv;
-                            word |= e2m1_code(hv[b][j] * inv, qv) << (4 * j);
-                            hv[b][j] -= qv * pw;
-                        }
-                        if (valid) {
-                            const int col = 128 * it.tile + 64 * b + 8 * tl;
-                            *reinterpret_cast<uint32_t *>(p.h_terms + term_offset(p.rows, t, r, col)) = word;
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t code[kT];
+                        act_digits(hv[b][j], E_blk, code);
+#pragma unroll
+                        for (int t = 0; t < kT; ++t)
+                            word[t] |= code[t] << (4 * j);
+                    }
+                    if (valid) {
+                        const int col = 128 * it.tile + 64 * b + 8 * tl;
+#pragma unroll
+                        for (int t = 0; t < kT; ++t) {
+                            *reinterpret_cast<uint32_t *>(p.h_terms + term_offset(p.rows, t, r, col)) = word[t];
                             if ((tl & 3) == 0)
-                                p.h_sf[img * kSFImg + image_byte(n, t, 2 * b + (tl >> 2))] = (uint8_t)(s + 127);
+                                p.h_sf[img * kSFImg + image_byte(n, t, 2 * b + (tl >> 2))] =
+                                    (uint8_t)(E_blk - 1 - 3 * t + 127);
                         }
                     }
                 }
@@ -622,22 +633,21 @@ __global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict
         const int n = local % nt;
         const int tok = src_row[r] / k;
         const int col = kb * 32 + lane;
-        float res = __uint_as_float((uint32_t)x[(int64_t)tok * H + col] << 16);
+        const float v = __uint_as_float((uint32_t)x[(int64_t)tok * H + col] << 16);
+        float m = fabsf(v);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+        const int E_blk = act_block_exp(m);
+        uint32_t code[kT];
+        act_digits(v, E_blk, code);
 #pragma unroll
         for (int t = 0; t < kT; ++t) {
-            float m = fabsf(res);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-            const int s = e2m1_block_exp(m);
-            float qv;
-            const uint32_t code = e2m1_code(res * pow2f(-s), qv);
-            res -= qv * pow2f(s);
-            const uint32_t hi_code = __shfl_down_sync(0xFFFFFFFFu, code, 1);
+            const uint32_t hi_code = __shfl_down_sync(0xFFFFFFFFu, code[t], 1);
             if (!(lane & 1))
-                terms[term_offset(rows, t, r, col)] = (uint8_t)(code | (hi_code << 4));
+                terms[term_offset(rows, t, r, col)] = (uint8_t)(code[t] | (hi_code << 4));
             if (lane == 0)
-                sf[img * kSFImg + image_byte(n, t, kb & 3)] = (uint8_t)(s + 127);
+                sf[img * kSFImg + image_byte(n, t, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * t + 127);
         }
     }
 }
