@@ -109,6 +109,37 @@ def profiled_traffic(workload: str, touched: float):
 
 
 # ---------------------------------------------------------------------------
+# replicas (one process per GPU under torchrun; no collective on the data path)
+# ---------------------------------------------------------------------------
+def dist_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_input_seed(seed: int, rank: int, batch: int) -> int:
+    """Seed of input batch `batch` on rank `rank`: every replica runs its own tokens."""
+    return seed + 1000 * rank + batch
+
+
+def max_over_ranks(v: float, world: int, device="cpu") -> float:
+    """Largest v over all ranks (every rank must call it, in the same order)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_step_per_rank * steps * world / (ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -253,9 +284,7 @@ def run_native(args):
 
     import mxfp4_quantized_moe_router_b200 as mx
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -283,7 +312,7 @@ def run_native(args):
 
     # --- rotating input batches (per rank: its own tokens)
     nb = max(1, args.batches)
-    xs = [datagen.make_x(cfg, args.seed + 1000 * rank + b, dev) for b in range(nb)]
+    xs = [datagen.make_x(cfg, replica_input_seed(args.seed, rank, b), dev) for b in range(nb)]
     logits = torch.empty((T, E), dtype=torch.float32, device=dev)
     ids = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
@@ -337,12 +366,8 @@ def run_native(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(v: float) -> float:
+        return max_over_ranks(v, world, dev)
 
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     clocks = ClockSampler(uuid)
@@ -364,7 +389,7 @@ def run_native(args):
     t1 = time.time()
     barrier()
     ms = start.elapsed_time(end)
-    ms_max = max_over_ranks(ms)
+    ms_max = rank_max(ms)
     clk = clocks.summary(t0, t1)
 
     # --- roofline region: same steps through the per-step entry points, with
@@ -401,7 +426,7 @@ def run_native(args):
     e2.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = max_over_ranks(s2.elapsed_time(e2))
+    ms_e2e = rank_max(s2.elapsed_time(e2))
     clocks.stop()
 
     if rank != 0:
@@ -413,7 +438,7 @@ def run_native(args):
     steps_batches = [(args.warmup + i) % nb for i in range(args.steps)]
     mean_touched = float(np.mean([touched[b] for b in steps_batches]))
     tokens = T * args.steps * world
-    value = tokens / (ms_max / 1e3)
+    value = whole_job_rate(T, args.steps, world, ms_max)
     weight_bytes_step = mean_touched * cfg.expert_bytes
     weight_gbs = weight_bytes_step * args.steps / (ms / 1e3) / 1e9
     # dominant unit: mxmoe_ffn_gate_up (x_terms + gate/up stage); algorithmic
@@ -425,13 +450,13 @@ def run_native(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e2m1 x e4m3 terms -> f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
+        "dtype": "e2m1 x e2m1 digit terms -> f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
                                           "W~N(0,0.02) quantised to MXFP4 by the library)",
         "config": workload_config(cfg, world, nb),
         "weight_gbs": weight_gbs,
         "weight_frac_of_hbm_peak": weight_gbs / peak,
         "touched_experts_per_step": mean_touched,
-        "roofline": {"kernel": "mxmoe_ffn_gate_up (x_terms_kernel + ffn_tc_kernel<gate_up>)",
+        "roofline": {"kernel": "mxmoe_ffn_gate_up (x_terms_kernel + ffn_mxf4_kernel<gate_up>)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
                      else "fallback 6.65 TB/s",

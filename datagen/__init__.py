@@ -11,7 +11,7 @@ section; the verify block of 8 tokens from the model card's section 3 and its
 size 2048 is a synthetic choice that is consistent with "1.02T" total
 parameters in the model summary, 384 * 3 * 6144 * 2048 * 70 layers = 1.015T):
 
-* ``tiny``        H 256,  E 16,  k 2, I 256,  T 4
+* ``tiny``        H 256,  E 16,  k 2, I 128,  T 4
 * ``verify8``     H 6144, E 384, k 8, I 2048, T 8      (one verify block)
 * ``verify256``   same layer, T 256 (32 sequences x 8-token blocks)
 * ``zipf1024``    same layer, T 1024, per-expert router bias so that expert
@@ -49,7 +49,7 @@ class LayerConfig:
 
 
 CONFIGS = [
-    LayerConfig("tiny", 256, 16, 2, 256, 4),
+    LayerConfig("tiny", 256, 16, 2, 128, 4),
     LayerConfig("verify8", 6144, 384, 8, 2048, 8),
     LayerConfig("verify256", 6144, 384, 8, 2048, 256),
     LayerConfig("zipf1024", 6144, 384, 8, 2048, 1024, zipf_s=1.2),

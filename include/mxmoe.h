@@ -91,8 +91,11 @@ MXMOE_API int mxmoe_dequantize(const uint8_t *packed, const uint8_t *scales, int
                                void *stream);
 
 /* Bytes of the prepacked expert blob for E experts of hidden size H and
- * intermediate size I (= E * 3 * H * I * 17/32, the same bytes as the packed
- * codes plus scales). Returns -1 unless H and I are positive multiples of 256.
+ * intermediate size I: E * (2*I*Hp + Hp*Ip) * 17/32 with Hp, Ip = H, I rounded
+ * up to multiples of 256, i.e. the bytes of the packed codes plus scales
+ * (E * 3 * H * I * 17/32) when H and I are multiples of 256, and those bytes
+ * padded with zero codes and zero scale bytes otherwise. Returns -1 unless H and I are positive
+ * multiples of 128.
  */
 MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I);
 
@@ -111,7 +114,9 @@ MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I);
  * matching up rows I + 128t .. I + 128t+127; down rows keep their order. The
  * scale images of a box are four 512-byte images ordered (K half h, row half
  * g): byte (r % 32) * 16 + (r / 32) * 4 + kb is the scale of tile row
- * 128g + r, 32-block 4h + kb of the box.
+ * 128g + r, 32-block 4h + kb of the box. K, and the down rows, are padded to
+ * multiples of 256 with zero codes and zero scale bytes (no padding when H and
+ * I are multiples of 256: the blob is then a byte permutation of the inputs).
  * Errors: shapes as in mxmoe_prepacked_size -> INVALID_SHAPE; NULL -> NULL;
  * prepacked not 32-byte or packed13/packed2 not 16-byte aligned -> ALIGNMENT.
  */
@@ -170,7 +175,7 @@ MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I);
  * activation terms, UE8M0 scales per 32, fp32 accumulation): x and h each
  * enter as eight E2M1 terms per value, every term with its own scale per 32
  * values, together within 3^-8 of the 32-block's largest magnitude.
- * Errors: H or I not a multiple of 256 or above 32768, k > 32, E > 1024,
+ * Errors: H or I not a multiple of 128 or above 32768, k > 32, E > 1024,
  * T*k > 2^22, E*I*H >= 2^38 -> INVALID_SHAPE; workspace
  * too small -> WORKSPACE; x, y_perm not 16-byte or prepacked not 32-byte
  * aligned -> ALIGNMENT. Device-side wait timeouts -> mxmoe_read_status. */

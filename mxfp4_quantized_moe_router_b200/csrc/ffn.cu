@@ -80,6 +80,8 @@ struct FfnParams {
     int *status;
 };
 
+__host__ __device__ __forceinline__ int64_t pad256(int64_t v) { return (v + 255) & ~int64_t(255); }
+
 // Byte offset of the E2M1 code byte holding columns k, k+1 (k even) of term t
 // of activation row r, in a term tensor laid out [K/256][rows][kT][128]: the
 // terms of one 256-column chunk of a token pass are consecutive 128-byte rows.
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_items = cur[2];
     ItemCursor<NT> it;
     it.start(p.offsets, E, tiles, cur[0], cur[1]);
-    const int nchunk = p.K / kKC;
+    const int nchunk = (p.K + kKC - 1) / kKC;  // the last chunk may hold one 128-column half
     const int khalves = p.K / 128;
 
     if (warp == 0) {
@@ -354,10 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&fullA[sa], (uint32_t)(C::kATx + 2 * kSFImg));
+                    const int nh = min(2, khalves - 2 * c);  // K halves in this chunk
+                    mbar_arrive_expect_tx(&fullA[sa], (uint32_t)(C::kATx + nh * kSFImg));
                     tc::tma_load_4d(sA + (size_t)sa * kAStage, &tmA, 0, 0, r0, c, &fullA[sa], pol_a);
-                    bulk_g2s_hint(sSfa + sa * 2 * kSFImg, p.asf + (pass_id * khalves + 2 * c) * kSFImg, 2 * kSFImg,
-                                  &fullA[sa], pol_a);
+                    bulk_g2s_hint(sSfa + sa * 2 * kSFImg, p.asf + (pass_id * khalves + 2 * c) * kSFImg,
+                                  (uint32_t)(nh * kSFImg), &fullA[sa], pol_a);
                     ++issued_a;
                     if (++sw == C::kStagesW) {
                         sw = 0;
@@ -411,13 +414,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int img = 0; img < 4; ++img)
                         tc::cp_32x128b_warpx4(sfw_t + 4 * img, tc::smem_desc(sfw_s + img * kSFImg, 16, 128, 0));
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                    for (int h = 0; h < min(2, khalves - 2 * c); ++h)
                         tc::cp_32x128b_warpx4(sfa_t + 4 * h, tc::smem_desc(sfa_s + h * kSFImg, 16, 128, 0));
                     const uint32_t a_base = smem_u32(sA + (size_t)sa * kAStage);
                     const uint32_t w_base = smem_u32(sW + (size_t)sw * kWBox);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {  // 64 values of K per MMA
+                    const int nk = 2 * min(2, khalves - 2 * c);  // a half chunk takes two MMAs
+                    for (int k = 0; k < nk; ++k) {  // 64 values of K per MMA
                         const uint32_t h = (uint32_t)(k >> 1), id = 2u * (uint32_t)(k & 1);
                         mma_mxf4(tmem, tc::smem_desc(a_base + k * 32, 16, 1024, 2),
                                  tc::smem_desc(w_base + k * 32, 16, 1024, 2), idesc_mxf4(256, id),
@@ -554,8 +556,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else if (valid) {
                 float *yrow = p.y_out + (int64_t)(it.r0() + n) * p.H + 256 * it.tile + 8 * tl;
+                const int ncols = min(256, p.H - 256 * it.tile);  // 128 in a padded last tile
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
+                    if (64 * b >= ncols)
+                        break;
                     float4 *dst = reinterpret_cast<float4 *>(yrow + 64 * b);
                     dst[0] = make_float4(v[b][0], v[b][1], v[b][2], v[b][3]);
                     dst[1] = make_float4(v[b][4], v[b][5], v[b][6], v[b][7]);
@@ -698,9 +703,9 @@ int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
     const int64_t passes = max_passes(rows);
     const int64_t o_status = take(16);
     const int64_t o_ps = take((kMaxE + 1) * 4);
-    const int64_t o_xt = take(rows * kT * H / 2);
+    const int64_t o_xt = take(rows * kT * pad256(H) / 2);
     const int64_t o_xs = take(passes * (H / 128) * kSFImg);
-    const int64_t o_ht = take(rows * kT * I / 2);
+    const int64_t o_ht = take(rows * kT * pad256(I) / 2);
     const int64_t o_hs = take(passes * (I / 128) * kSFImg);
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
@@ -770,7 +775,7 @@ int encode_weights(CUtensorMap *m, const void *base, int64_t n_boxes)
 // zero.
 int encode_terms(CUtensorMap *m, const void *base, int64_t rows, int K, int nt)
 {
-    const cuuint64_t dims[4] = {128, (cuuint64_t)kT, (cuuint64_t)rows, (cuuint64_t)(K / kKC)};
+    const cuuint64_t dims[4] = {128, (cuuint64_t)kT, (cuuint64_t)rows, (cuuint64_t)((K + kKC - 1) / kKC)};
     const cuuint64_t strides[3] = {128, (cuuint64_t)(kT * 128), (cuuint64_t)(rows * kT * 128)};
     const cuuint32_t box[4] = {128, (cuuint32_t)kT, (cuuint32_t)nt, 1};
     return encode(m, 4, base, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, "activation terms");
@@ -790,7 +795,7 @@ int launch_ffn(const void *codes, const uint8_t *act_terms, const FfnParams &p, 
         configured_dev = dev;
     }
     CUtensorMap tmW, tmA;
-    if (int rc = encode_weights(&tmW, codes, (int64_t)p.E * p.tiles * (p.K / kKC)))
+    if (int rc = encode_weights(&tmW, codes, (int64_t)p.E * p.tiles * ((p.K + kKC - 1) / kKC)))
         return rc;
     if (int rc = encode_terms(&tmA, act_terms, p.rows, p.K, NT))
         return rc;
@@ -804,10 +809,10 @@ int token_tile(int T) { return T <= 8 ? 8 : 16; }
 
 int validate_ffn(int T, int k, int E, int H, int I)
 {
-    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > kMaxE || H <= 0 || I <= 0 || H % 256 || I % 256 || H > 32768 ||
+    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > kMaxE || H <= 0 || I <= 0 || H % 128 || I % 128 || H > 32768 ||
         I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31))
         return fail(MXMOE_ERR_INVALID_SHAPE,
-                    "expert FFN: T=%d k=%d E=%d H=%d I=%d (need H, I multiples of 256 up to 32768, 1 <= k <= 32, "
+                    "expert FFN: T=%d k=%d E=%d H=%d I=%d (need H, I multiples of 128 up to 32768, 1 <= k <= 32, "
                     "E <= 1024, T*k <= 2^22, E*I*H < 2^38)",
                     T, k, E, H, I);
     return MXMOE_OK;
@@ -823,9 +828,10 @@ Blob blob_parts(const void *prepacked, int E, int H, int I)
     const uint8_t *b = static_cast<const uint8_t *>(prepacked);
     Blob o;
     o.w13 = b;
-    o.w2 = o.w13 + (int64_t)E * 2 * I * (H / 2);
-    o.sf13 = o.w2 + (int64_t)E * H * (I / 2);
-    o.sf2 = o.sf13 + (int64_t)E * 2 * I * (H / 32);
+    const int64_t Hp = pad256(H), Ip = pad256(I);
+    o.w2 = o.w13 + (int64_t)E * 2 * I * (Hp / 2);
+    o.sf13 = o.w2 + (int64_t)E * Hp * (Ip / 2);
+    o.sf2 = o.sf13 + (int64_t)E * 2 * I * (Hp / 32);
     return o;
 }
 
@@ -877,7 +883,7 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
     const int nt = token_tile(T);
     const Blob bl = blob_parts(prepacked, E, H, I);
     FfnParams p{};
-    p.tiles = H / 256;
+    p.tiles = (int)(pad256(H) / 256);
     p.K = I;
     p.rows = rows;
     p.wsf = bl.sf2;
@@ -922,7 +928,7 @@ using namespace mxmoe;
 
 extern "C" MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I)
 {
-    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 256 || I % 256 || H > 32768 ||
+    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 128 || I % 128 || H > 32768 ||
         I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31))
         return -1;
     return ffn_workspace_bytes(T, k, H, I);

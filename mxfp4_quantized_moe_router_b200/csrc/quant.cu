@@ -97,8 +97,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
     }
 }
 
-// Prepacked blob for the tensor-core FFN (a byte permutation of the canonical
-// format, same size):
+// Prepacked blob for the tensor-core FFN:
 //   [gate/up code boxes][down code boxes][gate/up scale images][down scale images]
 // A code box is one 256-row wide tile by 256 values of K: 256 rows of 128
 // bytes (32 KB, contiguous), boxes ordered by (expert, tile, K chunk). Gate/up
@@ -106,7 +105,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t *__restri
 // matching up rows (tile rows 128..255); down rows keep their order. The
 // scale images of a box are four 512-byte images ordered (K half h, row half
 // g): byte (r % 32) * 16 + (r / 32) * 4 + kb holds the scale of tile row
-// 128g + r, k32 block 4h + kb of the box.
+// 128g + r, k32 block 4h + kb of the box. K is padded to a multiple of 256 and
+// the down rows to a multiple of 256 with zero codes and zero scale bytes; at
+// H, I multiples of 256 the blob is a byte permutation of the canonical format.
 __device__ __forceinline__ int64_t tile_src_row(bool gate_up, int64_t lr_all, int I)
 {
     if (!gate_up)
@@ -116,14 +117,15 @@ __device__ __forceinline__ int64_t tile_src_row(bool gate_up, int64_t lr_all, in
     return lr < 128 ? 128 * t + lr : (int64_t)I + 128 * t + (lr - 128);
 }
 
-// One thread per 16 bytes of the code boxes.
-__global__ void __launch_bounds__(256) prepack_rows_kernel(const uint8_t *__restrict__ packed, int E,
-                                                           int64_t rows_per_expert, int K, bool gate_up, int I,
+// One thread per 16 bytes of the code boxes. rows: real rows per expert;
+// rows_pad: padded (multiple of 256); K real, K padded to a multiple of 256.
+__global__ void __launch_bounds__(256) prepack_rows_kernel(const uint8_t *__restrict__ packed, int E, int64_t rows,
+                                                           int64_t rows_pad, int K, bool gate_up, int I,
                                                            uint8_t *__restrict__ dst)
 {
-    const int nchunk = K / 256;
-    const int64_t tiles = rows_per_expert / 256;
-    const int64_t total = (int64_t)E * rows_per_expert * (K / 32);  // 16-byte units
+    const int nchunk = (K + 255) / 256;
+    const int64_t tiles = rows_pad / 256;
+    const int64_t total = (int64_t)E * rows_pad * nchunk * 8;  // 16-byte units
     for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
         const int part = (int)(u & 7);          // 16-byte part of a 128-byte box row
         const int lr = (int)((u >> 3) & 255);   // box row
@@ -131,19 +133,22 @@ __global__ void __launch_bounds__(256) prepack_rows_kernel(const uint8_t *__rest
         const int c = (int)(box % nchunk);
         const int64_t tile_id = box / nchunk;
         const int64_t e = tile_id / tiles, t = tile_id % tiles;
-        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 256 + lr, I);
-        reinterpret_cast<uint4 *>(dst)[u] =
-            __ldg(reinterpret_cast<const uint4 *>(packed + src * (K / 2) + (int64_t)c * 128) + part);
+        const int64_t row = tile_src_row(gate_up, t * 256 + lr, I);
+        const int64_t byte = (int64_t)c * 128 + part * 16;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < rows && byte < K / 2)
+            v = __ldg(reinterpret_cast<const uint4 *>(packed + (e * rows + row) * (K / 2) + byte));
+        reinterpret_cast<uint4 *>(dst)[u] = v;
     }
 }
 
 // One thread per byte of the scale images.
-__global__ void __launch_bounds__(256) prepack_sf_kernel(const uint8_t *__restrict__ sc, int E,
-                                                         int64_t rows_per_expert, int K, bool gate_up, int I,
+__global__ void __launch_bounds__(256) prepack_sf_kernel(const uint8_t *__restrict__ sc, int E, int64_t rows,
+                                                         int64_t rows_pad, int K, bool gate_up, int I,
                                                          uint8_t *__restrict__ dst)
 {
-    const int nchunk = K / 256;
-    const int64_t tiles = rows_per_expert / 256;
+    const int nchunk = (K + 255) / 256;
+    const int64_t tiles = rows_pad / 256;
     const int64_t total = (int64_t)E * tiles * nchunk * 2048;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         const int b = (int)(i & 511);
@@ -153,11 +158,11 @@ __global__ void __launch_bounds__(256) prepack_sf_kernel(const uint8_t *__restri
         const int64_t tile_id = box / nchunk;
         const int64_t e = tile_id / tiles, t = tile_id % tiles;
         const int m = (b >> 4) + 32 * ((b & 15) >> 2), kb = b & 3;
-        const int64_t src = e * rows_per_expert + tile_src_row(gate_up, t * 256 + 128 * g + m, I);
-        dst[i] = sc[src * (K / 32) + 8 * c + 4 * h + kb];
+        const int64_t row = tile_src_row(gate_up, t * 256 + 128 * g + m, I);
+        const int blk = 8 * c + 4 * h + kb;
+        dst[i] = (row < rows && blk < K / 32) ? sc[(e * rows + row) * (K / 32) + blk] : (uint8_t)0;
     }
 }
-
 
 int grid_for(int64_t work, int per_block)
 {
@@ -205,11 +210,14 @@ extern "C" MXMOE_API int mxmoe_dequantize(const uint8_t *packed, const uint8_t *
     return check_launch("dequantize_kernel");
 }
 
+static int64_t pad256(int64_t v) { return (v + 255) & ~int64_t(255); }
+
 extern "C" MXMOE_API int64_t mxmoe_prepacked_size(int E, int H, int I)
 {
-    if (E <= 0 || H <= 0 || I <= 0 || H % 256 || I % 256)
+    if (E <= 0 || H <= 0 || I <= 0 || H % 128 || I % 128)
         return -1;
-    return (int64_t)E * 3 * H * I / 2 + (int64_t)E * 3 * H * I / 32;
+    const int64_t Hp = pad256(H), Ip = pad256(I);
+    return (int64_t)E * (2 * (int64_t)I * Hp + Hp * Ip) * 17 / 32;
 }
 
 extern "C" MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const uint8_t *sc13, const uint8_t *packed2,
@@ -218,7 +226,7 @@ extern "C" MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const ui
 {
     if (mxmoe_prepacked_size(E, H, I) < 0)
         return fail(MXMOE_ERR_INVALID_SHAPE,
-                    "mxmoe_prepack_experts: E=%d H=%d I=%d (need H %% 256 == 0, I %% 256 == 0)", E, H, I);
+                    "mxmoe_prepack_experts: E=%d H=%d I=%d (need H %% 128 == 0, I %% 128 == 0)", E, H, I);
     if (!packed13 || !sc13 || !packed2 || !sc2 || !prepacked)
         return fail(MXMOE_ERR_NULL, "mxmoe_prepack_experts: NULL pointer");
     if ((reinterpret_cast<uintptr_t>(prepacked) & 31) || !aligned16(packed13) || !aligned16(packed2))
@@ -226,22 +234,24 @@ extern "C" MXMOE_API int mxmoe_prepack_experts(const uint8_t *packed13, const ui
                     "mxmoe_prepack_experts: prepacked needs 32-byte, packed13/packed2 16-byte alignment");
     if (int rc = check_device())
         return rc;
+    const int64_t Hp = pad256(H), Ip = pad256(I);
     uint8_t *w13 = static_cast<uint8_t *>(prepacked);
-    uint8_t *w2 = w13 + (int64_t)E * 2 * I * (H / 2);
-    uint8_t *sf13 = w2 + (int64_t)E * H * (I / 2);
-    uint8_t *sf2 = sf13 + (int64_t)E * 2 * I * (H / 32);
+    uint8_t *w2 = w13 + (int64_t)E * 2 * I * (Hp / 2);
+    uint8_t *sf13 = w2 + (int64_t)E * Hp * (Ip / 2);
+    uint8_t *sf2 = sf13 + (int64_t)E * 2 * I * (Hp / 32);
     cudaStream_t st = (cudaStream_t)stream;
-    prepack_rows_kernel<<<grid_for((int64_t)E * 2 * I * (H / 32), 256), 256, 0, st>>>(packed13, E, 2 * I, H, true,
-                                                                                       I, w13);
+    prepack_rows_kernel<<<grid_for((int64_t)E * 2 * I * (Hp / 32), 256), 256, 0, st>>>(packed13, E, 2 * I, 2 * I, H,
+                                                                                        true, I, w13);
     if (int rc = check_launch("prepack_rows_kernel(gate/up)"))
         return rc;
-    prepack_rows_kernel<<<grid_for((int64_t)E * H * (I / 32), 256), 256, 0, st>>>(packed2, E, H, I, false, I, w2);
+    prepack_rows_kernel<<<grid_for((int64_t)E * Hp * (Ip / 32), 256), 256, 0, st>>>(packed2, E, H, Hp, I, false, I,
+                                                                                    w2);
     if (int rc = check_launch("prepack_rows_kernel(down)"))
         return rc;
-    prepack_sf_kernel<<<grid_for((int64_t)E * 2 * I * (H / 32), 256), 256, 0, st>>>(sc13, E, 2 * I, H, true, I,
-                                                                                      sf13);
+    prepack_sf_kernel<<<grid_for((int64_t)E * 2 * I * (Hp / 32), 256), 256, 0, st>>>(sc13, E, 2 * I, 2 * I, H, true,
+                                                                                      I, sf13);
     if (int rc = check_launch("prepack_sf_kernel(gate/up)"))
         return rc;
-    prepack_sf_kernel<<<grid_for((int64_t)E * H * (I / 32), 256), 256, 0, st>>>(sc2, E, H, I, false, I, sf2);
+    prepack_sf_kernel<<<grid_for((int64_t)E * Hp * (Ip / 32), 256), 256, 0, st>>>(sc2, E, H, Hp, I, false, I, sf2);
     return check_launch("prepack_sf_kernel(down)");
 }

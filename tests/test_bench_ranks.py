@@ -1,0 +1,88 @@
+"""The multi-rank plumbing of bench.py on CPU: two gloo ranks run the same
+helpers bench.py's timed path uses under torchrun (max over ranks, whole-job
+rate, per-replica inputs), and the reference arm does no work off rank 0."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_env_defaults(monkeypatch):
+    for v in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(v, raising=False)
+    assert bench.dist_env() == (1, 0, 0)
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    monkeypatch.setenv("RANK", "3")
+    monkeypatch.setenv("LOCAL_RANK", "3")
+    assert bench.dist_env() == (4, 3, 3)
+
+
+def test_whole_job_rate_counts_every_rank_over_the_slowest():
+    # 8 tokens per step per rank, 100 steps, 2 ranks, slowest rank 50 ms -> 32000 tokens/s
+    assert bench.whole_job_rate(8, 100, 2, 50.0) == pytest.approx(32000.0)
+    assert bench.whole_job_rate(8, 100, 1, 50.0) == pytest.approx(16000.0)
+
+
+def test_replicas_draw_distinct_inputs():
+    seeds = {bench.replica_input_seed(0, r, b) for r in range(8) for b in range(16)}
+    assert len(seeds) == 8 * 16
+
+
+def test_single_rank_max_is_identity():
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+_WORKER = r"""
+import json, os, sys
+sys.path.insert(0, sys.argv[1])
+import torch.distributed as dist
+import bench
+world, rank, _ = bench.dist_env()
+dist.init_process_group("gloo", init_method="env://", world_size=world, rank=rank)
+ms = 10.0 + 5.0 * rank           # rank 1 is the slower one
+ms_max = bench.max_over_ranks(ms, world)
+dist.barrier()
+rate = bench.whole_job_rate(8, 100, world, ms_max)
+dist.destroy_process_group()
+print(json.dumps({"rank": rank, "ms_max": ms_max, "rate": rate}))
+"""
+
+
+def test_two_gloo_ranks_agree_on_the_max(tmp_path):
+    port = _free_port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, WORLD_SIZE="2", RANK=str(r), LOCAL_RANK=str(r), MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, "-c", _WORKER, ROOT], env=env, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    outs = []
+    for p in procs:
+        out, err = p.communicate(timeout=120)
+        assert p.returncode == 0, err
+        outs.append(json.loads(out.strip().splitlines()[-1]))
+    for o in outs:
+        assert o["ms_max"] == 15.0
+        assert o["rate"] == pytest.approx(8 * 100 * 2 / 0.015)
+
+
+def test_reference_arm_does_no_work_off_rank_zero():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "3",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
+    assert p.returncode == 0, p.stderr
+    assert p.stdout.strip() == ""

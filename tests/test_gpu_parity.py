@@ -143,13 +143,14 @@ def test_permute_skewed(mx):
 FFN_CASES = [
     # H, I, E, k, T : several 256-row tiles along I and H, several K chunks,
     # ragged token passes (8-token passes for T <= 8, 16-token passes
-    # otherwise)
-    (256, 256, 16, 2, 4),
-    (512, 256, 6, 2, 37),     # n_e up to ~20: two 16-token passes
+    # otherwise); H or I = 128 mod 256 gives a trailing half K chunk and, for
+    # H, a down tile of 128 real rows
+    (256, 128, 16, 2, 4),
+    (384, 256, 6, 2, 37),     # n_e up to ~20: two 16-token passes
     (512, 512, 8, 2, 9),
-    (256, 768, 3, 1, 80),     # n_e up to ~40: several passes, 3 tiles along I
-    (768, 512, 5, 3, 150),
-    (1024, 256, 2, 2, 1),     # one token: 7 of the 8 pass rows unused
+    (256, 384, 3, 1, 80),     # n_e up to ~40: several passes, 3 tiles along I
+    (640, 384, 5, 3, 150),
+    (1024, 128, 2, 2, 1),     # one token: 7 of the 8 pass rows unused
 ]
 
 
@@ -242,7 +243,7 @@ def test_layer_tiny(mx):
 
 @pytest.mark.parametrize("T", [1, 3, 64, 200])
 def test_layer_small_ragged(mx, T):
-    cfg = datagen.LayerConfig("small", 512, 24, 4, 256, T)
+    cfg = datagen.LayerConfig("small", 512, 24, 4, 128, T)
     layer = GpuLayer(mx, cfg, 1)
     x = datagen.make_x(cfg, 1)
     bias = (np.linspace(-0.5, 0.5, cfg.E)).astype(np.float32)

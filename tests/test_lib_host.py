@@ -42,12 +42,15 @@ def test_version(mx):
 
 
 def test_prepacked_size_is_format_bytes(mx):
-    # same bytes as the canonical codes + scales: 3*H*I*E*(1/2 + 1/32)
-    for E, H, I in [(384, 6144, 2048), (16, 256, 256), (3, 512, 768)]:
-        assert mx.mxmoe_prepacked_size(E, H, I) == E * 3 * H * I * 17 // 32
-    assert mx.mxmoe_prepacked_size(384, 6144, 2048) == 384 * 20_054_016
-    assert mx.mxmoe_prepacked_size(4, 384, 256) == -1  # H % 256
-    assert mx.mxmoe_prepacked_size(4, 256, 128) == -1  # I % 256
+    # codes + scales, 3*H*I*E*(1/2 + 1/32), with H and I padded to multiples of 256
+    def pad(v):
+        return (v + 255) // 256 * 256
+    for E, H, I in [(384, 6144, 2048), (16, 256, 256), (3, 512, 768), (16, 256, 128), (5, 640, 384)]:
+        Hp, Ip = pad(H), pad(I)
+        assert mx.mxmoe_prepacked_size(E, H, I) == E * (2 * I * Hp + Hp * Ip) * 17 // 32
+    assert mx.mxmoe_prepacked_size(384, 6144, 2048) == 384 * 20_054_016  # no padding at the layer's shape
+    assert mx.mxmoe_prepacked_size(4, 192, 128) == -1  # H % 128
+    assert mx.mxmoe_prepacked_size(4, 256, 64) == -1  # I % 128
 
 
 def test_workspace_queries(mx):
@@ -56,7 +59,7 @@ def test_workspace_queries(mx):
     assert mx.mxmoe_ffn_workspace_size(8, 8, 384, 6144, 2048) > 0
     assert mx.mxmoe_ffn_workspace_size(8, 8, 384, 6100, 2048) == -1
     assert mx.mxmoe_ffn_workspace_size(8, 8, 384, 6144, 32768 + 256) == -1
-    assert mx.mxmoe_ffn_workspace_size(8, 8, 384, 6144, 2048 + 128) == -1  # I % 256
+    assert mx.mxmoe_ffn_workspace_size(8, 8, 384, 6144, 2048 + 64) == -1  # I % 128
     assert mx.mxmoe_ffn_workspace_size((1 << 22) // 8 + 1, 8, 384, 6144, 2048) == -1
     # grows with T
     assert mx.mxmoe_workspace_size(256, 6144, 2048, 384, 8) > mx.mxmoe_workspace_size(8, 6144, 2048, 384, 8)
