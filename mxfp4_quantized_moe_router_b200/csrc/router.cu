@@ -126,8 +126,27 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
         const int e = lane + 32 * i;
         v[i] = e < E ? l[e] : -FLT_MAX;
     }
-    // add the other splits in split order; each split's loads are independent
-    for (int z = 1; z < nsplit; ++z) {
+    // add the other splits in split order, loading four splits at a time (up to
+    // 512 experts) so their loads overlap; the sums keep the split order
+    int z = 1;
+    for (; V <= 16 && z + 3 < nsplit; z += 4) {
+        float pz[4][V];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const float *lz = l + (int64_t)(z + g) * T * E;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int e = lane + 32 * i;
+                pz[g][i] = e < E ? lz[e] : 0.f;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                v[i] += pz[g][i];
+    }
+    for (; z < nsplit; ++z) {
         const float *lz = l + (int64_t)z * T * E;
         float pz[V];
 #pragma unroll
