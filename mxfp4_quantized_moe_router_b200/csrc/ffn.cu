@@ -577,7 +577,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Token passes of each expert: pass_start[e] = sum over e' < e of
-// ceil(n_e' / nt), for one block's warp 0 (E <= kMaxE).
+// ceil(n_e' / nt), from the block's copy of the offsets, for one block's warp
+// 0 (E <= kMaxE).
 __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
 {
     const int lane = threadIdx.x & 31;
@@ -610,10 +611,11 @@ __global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict
 {
     __shared__ int32_t s_off[kMaxE + 1], s_pass[kMaxE + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (warp == 0)
-        pass_prefix(offsets, E, nt, s_pass);
     for (int e = threadIdx.x; e <= E; e += blockDim.x)
         s_off[e] = offsets[e];
+    __syncthreads();
+    if (warp == 0)
+        pass_prefix(s_off, E, nt, s_pass);
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int e = threadIdx.x; e <= E; e += blockDim.x)
@@ -621,22 +623,31 @@ __global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict
         if (threadIdx.x == 0 && status)
             *status = 0;
     }
+    // Each warp takes a contiguous run of (row, 32-block) units, so the row's
+    // expert, pass and token are looked up once per row.
     const int nkb = H / 32;
     const int64_t total = (int64_t)rows * nkb;
-    for (int64_t w = (int64_t)blockIdx.x * 8 + warp; w < total; w += (int64_t)gridDim.x * 8) {
+    const int64_t nwarps = (int64_t)gridDim.x * 8, gw = (int64_t)blockIdx.x * 8 + warp;
+    const int64_t w_begin = total * gw / nwarps, w_end = total * (gw + 1) / nwarps;
+    int r_cur = -1, n = 0, tok = 0;
+    int64_t img_row = 0;
+    for (int64_t w = w_begin; w < w_end; ++w) {
         const int r = (int)(w / nkb), kb = (int)(w % nkb);
-        int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (s_off[mid] <= r)
-                lo = mid;
-            else
-                hi = mid;
+        if (r != r_cur) {
+            r_cur = r;
+            int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (s_off[mid] <= r)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            const int local = r - s_off[lo];
+            img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
+            n = local % nt;
+            tok = src_row[r] / k;
         }
-        const int local = r - s_off[lo];
-        const int64_t img = ((int64_t)s_pass[lo] + local / nt) * (H / 128) + kb / 4;
-        const int n = local % nt;
-        const int tok = src_row[r] / k;
         const int col = kb * 32 + lane;
         const float v = __uint_as_float((uint32_t)x[(int64_t)tok * H + col] << 16);
         float m = fabsf(v);
@@ -646,13 +657,17 @@ __global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict
         const int E_blk = act_block_exp(m);
         uint32_t code[kT];
         act_digits(v, E_blk, code);
+        // term t sits 128 bytes after term t-1; its scale 16 bytes after (the
+        // image rows n*kT + t of one pass row are consecutive lanes)
+        uint8_t *tp = terms + term_offset(rows, 0, r, col);
+        uint8_t *sp = sf + (img_row + kb / 4) * kSFImg + image_byte(n, 0, kb & 3);
 #pragma unroll
         for (int t = 0; t < kT; ++t) {
             const uint32_t hi_code = __shfl_down_sync(0xFFFFFFFFu, code[t], 1);
             if (!(lane & 1))
-                terms[term_offset(rows, t, r, col)] = (uint8_t)(code[t] | (hi_code << 4));
+                tp[128 * t] = (uint8_t)(code[t] | (hi_code << 4));
             if (lane == 0)
-                sf[img * kSFImg + image_byte(n, t, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * t + 127);
+                sp[16 * t] = (uint8_t)(E_blk - 1 - 3 * t + 127);
         }
     }
 }
@@ -846,7 +861,7 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     const int nt = token_tile(T);
     {
         const int64_t warps = (int64_t)rows * (H / 32);
-        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 8);
+        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 2);
         x_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
                                                                  k, rows, H, nt, ws.x_terms, ws.x_sf, ws.pass_start,
                                                                  ws.status);

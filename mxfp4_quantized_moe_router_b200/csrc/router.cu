@@ -103,40 +103,50 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
 }
 
 // ---------------------------------------------------------------------------
-// Top-k routing: one warp per token. Lane l holds logits l, l+32, ...; k
-// rounds of a warp arg-max (larger value first, then lower index).
+// Top-k routing: one 128-thread block per token. Thread i holds logits i,
+// i+128, ...; k rounds of a block arg-max (larger value first, then lower
+// index): thread, warp (shuffles), then the four warp winners in shared
+// memory, combined in the same order by every thread.
 // ---------------------------------------------------------------------------
-constexpr int kRouteMaxPerLane = 128;  // E <= 4096
+constexpr int kRouteThreads = 128;
+
+__device__ __forceinline__ bool route_better(float ov, int oi, float bv, int bi)
+{
+    return oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi));
+}
 
 // With nsplit > 1 the logits are the sum, in split order, of nsplit partial
-// [T, E] arrays plus bias (the split router GEMM's output).
+// [T, E] arrays plus bias (the split router GEMM's output). E <= 128 * V.
 template <int V>
-__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int nsplit,
-                                                    const float *__restrict__ bias, int T, int E, int k,
-                                                    int32_t *__restrict__ ids, float *__restrict__ w)
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__restrict__ logits, int nsplit,
+                                                              const float *__restrict__ bias, int T, int E, int k,
+                                                              int32_t *__restrict__ ids, float *__restrict__ w)
 {
-    const int lane = threadIdx.x & 31;
-    const int tok = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    __shared__ float s_bv[kRouteThreads / 32];
+    __shared__ int s_bi[kRouteThreads / 32];
+    __shared__ float s_sel_v[32];
+    __shared__ int s_sel_i[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tok = blockIdx.x;
     if (tok >= T)
         return;
     const float *l = logits + (int64_t)tok * E;
     float v[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-        const int e = lane + 32 * i;
+        const int e = tid + kRouteThreads * i;
         v[i] = e < E ? l[e] : -FLT_MAX;
     }
-    // add the other splits in split order, loading four splits at a time (up to
-    // 512 experts) so their loads overlap; the sums keep the split order
+    // add the other splits in split order, four splits' loads at a time
     int z = 1;
-    for (; V <= 16 && z + 3 < nsplit; z += 4) {
+    for (; z + 3 < nsplit; z += 4) {
         float pz[4][V];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             const float *lz = l + (int64_t)(z + g) * T * E;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int e = lane + 32 * i;
+                const int e = tid + kRouteThreads * i;
                 pz[g][i] = e < E ? lz[e] : 0.f;
             }
         }
@@ -148,38 +158,28 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
     }
     for (; z < nsplit; ++z) {
         const float *lz = l + (int64_t)z * T * E;
-        float pz[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int e = lane + 32 * i;
-            pz[i] = e < E ? lz[e] : 0.f;
+            const int e = tid + kRouteThreads * i;
+            v[i] += e < E ? lz[e] : 0.f;
         }
-#pragma unroll
-        for (int i = 0; i < V; ++i)
-            v[i] += pz[i];
     }
     if (bias) {
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int e = lane + 32 * i;
+            const int e = tid + kRouteThreads * i;
             if (e < E)
                 v[i] += bias[e];
         }
     }
-    uint32_t taken[(V + 31) / 32];
-#pragma unroll
-    for (int i = 0; i < (V + 31) / 32; ++i)
-        taken[i] = 0;
-    float sel_v = 0.f, top = 0.f;
-    int sel_i = 0;
+    uint32_t taken = 0;
     for (int j = 0; j < k; ++j) {
         float bv = -FLT_MAX;
         int bi = 0x7FFFFFFF;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int e = lane + 32 * i;
-            const bool free = e < E && !((taken[i / 32] >> (i % 32)) & 1u);
-            if (free && (v[i] > bv || bi == 0x7FFFFFFF)) {
+            const int e = tid + kRouteThreads * i;
+            if (e < E && !((taken >> i) & 1u) && route_better(v[i], e, bv, bi)) {
                 bv = v[i];
                 bi = e;
             }
@@ -188,33 +188,42 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
         for (int off = 16; off > 0; off >>= 1) {
             const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
             const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-            if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
+            if (route_better(ov, oi, bv, bi)) {
                 bv = ov;
                 bi = oi;
             }
         }
-        if ((bi & 31) == lane) {
-            const int slot = bi >> 5;
+        if (lane == 0) {
+            s_bv[warp] = bv;
+            s_bi[warp] = bi;
+        }
+        __syncthreads();
+        bv = s_bv[0];
+        bi = s_bi[0];
 #pragma unroll
-            for (int i = 0; i < V; ++i)
-                if (i == slot)
-                    taken[i / 32] |= 1u << (i % 32);
+        for (int q = 1; q < kRouteThreads / 32; ++q)
+            if (route_better(s_bv[q], s_bi[q], bv, bi)) {
+                bv = s_bv[q];
+                bi = s_bi[q];
+            }
+        if (bi != 0x7FFFFFFF && bi % kRouteThreads == tid)
+            taken |= 1u << (bi / kRouteThreads);
+        if (tid == 0) {
+            s_sel_v[j] = bv;
+            s_sel_i[j] = bi;
         }
-        if (j == 0)
-            top = bv;
-        if (lane == j) {
-            sel_v = bv;
-            sel_i = bi;
-        }
+        __syncthreads();
     }
     // weights: exp(l_j - l_max) / sum over the selected, summed in slot order
-    const float ex = (lane < k) ? expf(sel_v - top) : 0.f;
-    float s = 0.f;
-    for (int j = 0; j < k; ++j)
-        s += __shfl_sync(0xFFFFFFFFu, ex, j);
-    if (lane < k) {
-        ids[(int64_t)tok * k + lane] = sel_i;
-        w[(int64_t)tok * k + lane] = ex / s;
+    if (warp == 0) {
+        const float ex = (lane < k) ? expf(s_sel_v[lane < k ? lane : 0] - s_sel_v[0]) : 0.f;
+        float s = 0.f;
+        for (int j = 0; j < k; ++j)
+            s += __shfl_sync(0xFFFFFFFFu, ex, j);
+        if (lane < k) {
+            ids[(int64_t)tok * k + lane] = s_sel_i[lane];
+            w[(int64_t)tok * k + lane] = ex / s;
+        }
     }
 }
 
@@ -326,6 +335,16 @@ namespace mxmoe {
 
 // K splits for the layer's router GEMM: enough CTAs to cover the GPU at
 // decode sizes, each split at least 8 k32 blocks (one per warp).
+int launch_route(const float *logits, int nsplit, const float *bias, int T, int E, int k, int32_t *ids, float *w,
+                 cudaStream_t st)
+{
+    if (E <= kRouteThreads * 4)
+        route_kernel<4><<<T, kRouteThreads, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+    else
+        route_kernel<32><<<T, kRouteThreads, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+    return check_launch("route_kernel");
+}
+
 int router_splits(int T, int H, int E)
 {
     const int64_t base = (int64_t)((E + kRgExperts - 1) / kRgExperts) * ((T + kRgTokens - 1) / kRgTokens);
@@ -345,13 +364,7 @@ int run_router_and_route(const void *x, const void *wg, const float *bias, int T
                                              bias, T, H, E, partials);
     if (int rc = check_launch("router_gemm_kernel"))
         return rc;
-    const int blocks = (T + 7) / 8;
-    if (E <= 32 * 16)
-        route_kernel<16><<<blocks, 256, 0, st>>>(partials, nsplit, nsplit > 1 ? bias : nullptr, T, E, k, ids, w);
-    else
-        route_kernel<kRouteMaxPerLane><<<blocks, 256, 0, st>>>(partials, nsplit, nsplit > 1 ? bias : nullptr, T,
-                                                               E, k, ids, w);
-    return check_launch("route_kernel");
+    return launch_route(partials, nsplit, nsplit > 1 ? bias : nullptr, T, E, k, ids, w, st);
 }
 
 }  // namespace mxmoe
@@ -367,13 +380,7 @@ extern "C" MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, i
         return fail(MXMOE_ERR_NULL, "mxmoe_route: NULL pointer");
     if (int rc = check_device())
         return rc;
-    const int blocks = (T + 7) / 8;
-    cudaStream_t st = (cudaStream_t)stream;
-    if (E <= 32 * 16)
-        route_kernel<16><<<blocks, 256, 0, st>>>(logits, 1, nullptr, T, E, k, ids, w);
-    else
-        route_kernel<kRouteMaxPerLane><<<blocks, 256, 0, st>>>(logits, 1, nullptr, T, E, k, ids, w);
-    return check_launch("route_kernel");
+    return launch_route(logits, 1, nullptr, T, E, k, ids, w, (cudaStream_t)stream);
 }
 
 extern "C" MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
