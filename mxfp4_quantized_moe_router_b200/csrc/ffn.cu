@@ -60,7 +60,7 @@ constexpr int kWBox = 32768;     // bytes of a weight box: 256 rows x 128 bytes
 constexpr int kWSf = 2048;       // its scale images: (K half, row half) x 512 bytes
 constexpr int kAStage = 16384;   // shared bytes the MMA reads for A: 128 rows x 128 bytes
 constexpr int kSFImg = 512;      // scale image: 32 lanes x 16 bytes
-constexpr int kThreads = 192;    // producer, MMA, 4 epilogue warps
+constexpr int kThreads = 224;    // producer, MMA, 4 epilogue warps, scale-copy warp
 constexpr int kMaxE = 1024;
 
 struct FfnParams {
@@ -116,7 +116,7 @@ struct Cfg {
     static constexpr size_t kOffSfw = kOffA + (size_t)kStagesA * kAStage;
     static constexpr size_t kOffSfa = kOffSfw + (size_t)kStagesW * kWSf;
     static constexpr size_t kOffBar = kOffSfa + (size_t)kStagesA * 2 * kSFImg;
-    static constexpr int kBars = 2 * kStagesW + 2 * kStagesA + 3;
+    static constexpr int kBars = 2 * kStagesW + 2 * kStagesA + 3 + kStagesA + 1;
     static constexpr size_t kOffMisc = (kOffBar + kBars * 8 + 15) & ~size_t(15);
     static constexpr size_t kSmem = 1024 + kOffMisc + 64;
     // Tensor memory: the accumulator (128 lanes x 256 columns), then per weight
@@ -255,6 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *accfull = emptyA + C::kStagesA;
     uint64_t *accempty = accfull + 1;
     uint64_t *mma_done = accempty + 1;
+    uint64_t *sfready = mma_done + 1;        // [kStagesA]: a chunk's scale images are in tensor memory
+    uint64_t *cp_done = sfready + C::kStagesA;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     int *cur = reinterpret_cast<int *>(tslot + 2);  // [0] first expert, [1] first item within it, [2] item count
@@ -315,6 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(accfull, 1);
         mbar_init(accempty, 4);
         mbar_init(mma_done, 1);
+        for (int s = 0; s < C::kStagesA; ++s)
+            mbar_init(&sfready[s], 1);
+        mbar_init(cp_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -402,20 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_after();
                 for (int c = 0; c < nchunk; ++c) {
                     if (*abort_flag || !mbar_wait_bounded(&fullW[sw], phw, kWaitLimitNs) ||
-                        !mbar_wait_bounded(&fullA[sa], pha, kWaitLimitNs)) {
+                        !mbar_wait_bounded(&fullA[sa], pha, kWaitLimitNs) ||
+                        !mbar_wait_bounded(&sfready[sa], pha, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc::fence_after();
                     const uint32_t sfw_t = tmem + C::kSfwCol0 + 16 * sw;  // + 8 per K half, + 4 per row half
                     const uint32_t sfa_t = tmem + C::kSfaCol0 + 8 * sa;   // + 4 per K half
-                    const uint32_t sfw_s = smem_u32(sSfw + sw * kWSf);
-                    const uint32_t sfa_s = smem_u32(sSfa + sa * 2 * kSFImg);
-#pragma unroll
-                    for (int img = 0; img < 4; ++img)
-                        tc::cp_32x128b_warpx4(sfw_t + 4 * img, tc::smem_desc(sfw_s + img * kSFImg, 16, 128, 0));
-                    for (int h = 0; h < min(2, khalves - 2 * c); ++h)
-                        tc::cp_32x128b_warpx4(sfa_t + 4 * h, tc::smem_desc(sfa_s + h * kSFImg, 16, 128, 0));
                     const uint32_t a_base = smem_u32(sA + (size_t)sa * kAStage);
                     const uint32_t w_base = smem_u32(sW + (size_t)sw * kWBox);
                     const int nk = 2 * min(2, khalves - 2 * c);  // a half chunk takes two MMAs
@@ -449,6 +448,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (any) {
                 tc::commit(mma_done);
                 if (!mbar_wait_bounded(mma_done, 0, kWaitLimitNs))
+                    set_status(p.status, MXMOE_ERR_TIMEOUT);
+            }
+        }
+    } else if (warp == 6) {
+        // ---------------------------------------------------- scale images
+        // Moves each chunk's scale images from shared into tensor memory and
+        // signals sfready, so the MMA warp issues nothing but MMAs. A slot's
+        // columns are rewritten only after its full barrier fired again, i.e.
+        // after the MMAs that read them completed.
+        if (lane == 0) {
+            int sw = 0, sa = 0;
+            uint32_t phw = 0, pha = 0;
+            bool ok = true, any = false;
+            const int64_t total = (int64_t)n_items * nchunk;
+            for (int64_t j = 0; j < total; ++j) {
+                const int c = (int)(j % nchunk);
+                if (*abort_flag || !mbar_wait_bounded(&fullW[sw], phw, kWaitLimitNs) ||
+                    !mbar_wait_bounded(&fullA[sa], pha, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after();
+                const uint32_t sfw_t = tmem + C::kSfwCol0 + 16 * sw;
+                const uint32_t sfa_t = tmem + C::kSfaCol0 + 8 * sa;
+                const uint32_t sfw_s = smem_u32(sSfw + sw * kWSf);
+                const uint32_t sfa_s = smem_u32(sSfa + sa * 2 * kSFImg);
+#pragma unroll
+                for (int img = 0; img < 4; ++img)
+                    tc::cp_32x128b_warpx4(sfw_t + 4 * img, tc::smem_desc(sfw_s + img * kSFImg, 16, 128, 0));
+                for (int h = 0; h < min(2, khalves - 2 * c); ++h)
+                    tc::cp_32x128b_warpx4(sfa_t + 4 * h, tc::smem_desc(sfa_s + h * kSFImg, 16, 128, 0));
+                tc::commit(&sfready[sa]);
+                any = true;
+                if (++sw == C::kStagesW) {
+                    sw = 0;
+                    phw ^= 1u;
+                }
+                if (++sa == C::kStagesA) {
+                    sa = 0;
+                    pha ^= 1u;
+                }
+            }
+            if (!ok) {
+                set_status(p.status, MXMOE_ERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            // Every copy of ours completes before tensor memory is released.
+            if (any) {
+                tc::commit(cp_done);
+                if (!mbar_wait_bounded(cp_done, 0, kWaitLimitNs))
                     set_status(p.status, MXMOE_ERR_TIMEOUT);
             }
         }

@@ -142,7 +142,7 @@ def test_permute_skewed(mx):
 # ---------------------------------------------------------------------------
 FFN_CASES = [
     # H, I, E, k, T : several 256-row tiles along I and H, several K chunks,
-    # whole and half items (up to 148 items every CTA gets half items only),
+    # more work items than SMs, with the leftover items split along K,
     # ragged token passes (8-token passes for T <= 8, 16-token passes
     # otherwise); H or I = 128 mod 256 gives a trailing half K chunk and, for
     # H, a down tile of 128 real rows
@@ -152,7 +152,8 @@ FFN_CASES = [
     (256, 384, 3, 1, 80),     # n_e up to ~40: several passes, 3 tiles along I
     (640, 384, 5, 3, 150),
     (1024, 128, 2, 2, 1),     # one token: 7 of the 8 pass rows unused
-    (1024, 1024, 64, 4, 64),  # more items than SMs: whole items, then half items, in both stages
+    (1024, 1024, 64, 4, 64),  # more items than SMs in both stages
+    (1024, 512, 64, 8, 8),    # ~180 items: the leftover items split along K (4 pieces gate/up, 2 down)
 ]
 
 
