@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: shrink the layer to this many experts (0 = the workload's)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling only: this many tokens per step (0 = the workload's)")
     return ap.parse_args()
 
 
@@ -295,6 +297,10 @@ def run_native(args):
         import dataclasses
 
         cfg = dataclasses.replace(cfg, name=cfg.name + "-E%d" % args.experts, E=args.experts)
+    if args.tokens:
+        import dataclasses
+
+        cfg = dataclasses.replace(cfg, name=cfg.name + "-T%d" % args.tokens, T=args.tokens)
     T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.k, cfg.I
 
     # --- weights (same layer on every rank), quantised and prepacked on the device

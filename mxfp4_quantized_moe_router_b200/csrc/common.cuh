@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include "../../include/mxmoe.h"
@@ -15,6 +16,11 @@
 namespace mxmoe {
 
 // ---------------------------------------------------------------------------
+// SM count of the current device and the driver's cuTensorMapEncodeTiled
+// (defined in api.cu)
+int num_sms();
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
 // Host-side error reporting (defined in api.cu)
 // ---------------------------------------------------------------------------
 int fail(int code, const char *fmt, ...);

@@ -51,6 +51,9 @@
 #include "tcgen05.cuh"
 
 namespace mxmoe {
+int run_bf16_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row, const uint8_t *w13,
+                     const uint8_t *sf13, int T, int k, int E, int H, int I, uint16_t *x_perm, float *h, int *status,
+                     cudaStream_t st);
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
@@ -648,11 +651,15 @@ __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
     }
 }
 
-// x rows (bf16) -> kT E2M1 terms per value in grouped row order (row r holds
-// token src_row[r] / k), in the term_offset layout, with their scale images
-// (one per token pass and 128 columns). One warp per 32-value block. Block 0
-// also writes pass_start for the FFN stages and clears the status word.
-__global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ src_row,
+// Activation rows -> kT E2M1 terms per value in grouped row order, in the
+// term_offset layout, with their scale images (one per token pass and 128
+// columns). GROUPED_F32 = false: x rows (bf16), row r holding token
+// src_row[r] / k; true: rows already grouped, fp32 (h of the gate/up stage
+// when it ran on bf16 tensor cores; src_row and k unused). One warp per
+// 32-value block. Block 0 also writes pass_start for the FFN stages and clears
+// the status word.
+template <bool GROUPED_F32>
+__global__ void __launch_bounds__(256) act_terms_kernel(const void *__restrict__ act, const int32_t *__restrict__ src_row,
                                                       const int32_t *__restrict__ offsets, int E, int k, int rows,
                                                       int H, int nt, uint8_t *__restrict__ terms,
                                                       uint8_t *__restrict__ sf, int32_t *__restrict__ pass_start_out,
@@ -695,10 +702,12 @@ __global__ void __launch_bounds__(256) x_terms_kernel(const uint16_t *__restrict
             const int local = r - s_off[lo];
             img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
             n = local % nt;
-            tok = src_row[r] / k;
+            tok = GROUPED_F32 ? r : src_row[r] / k;
         }
         const int col = kb * 32 + lane;
-        const float v = __uint_as_float((uint32_t)x[(int64_t)tok * H + col] << 16);
+        const float v = GROUPED_F32 ? static_cast<const float *>(act)[(int64_t)tok * H + col]
+                                    : __uint_as_float((uint32_t)static_cast<const uint16_t *>(act)[(int64_t)tok * H + col]
+                                                      << 16);
         float m = fabsf(v);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
@@ -753,7 +762,16 @@ struct FfnWs {
     uint8_t *x_sf;        // scale images [pass][H/128][512]
     uint8_t *h_terms;     // term_offset layout, K = I
     uint8_t *h_sf;        // scale images [pass][I/128][512]
+    uint16_t *x_perm;     // bf16 gate/up path only: x rows in grouped order [rows][H]
+    float *h_f32;         // bf16 gate/up path only: h [rows][I]
 };
+
+// Token counts at which the gate/up stage runs on bf16 tensor cores (weights
+// dequantised in shared memory, x as is) instead of the E2M1-term MMAs: from
+// 16384 grouped rows (2048 tokens at top-8), where experts see hundreds of
+// tokens and the stage is bound by the tensor cores.
+constexpr int64_t kBf16GateUpRows = 16384;
+bool use_bf16_gate_up(int T, int k) { return (int64_t)T * k >= kBf16GateUpRows; }
 
 int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
 {
@@ -767,10 +785,13 @@ int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
     const int64_t passes = max_passes(rows);
     const int64_t o_status = take(16);
     const int64_t o_ps = take((kMaxE + 1) * 4);
-    const int64_t o_xt = take(rows * kT * pad256(H) / 2);
-    const int64_t o_xs = take(passes * (H / 128) * kSFImg);
+    const bool bf16 = use_bf16_gate_up(T, k);  // x goes to the tensor cores as bf16: no x terms
+    const int64_t o_xt = take(bf16 ? 0 : rows * kT * pad256(H) / 2);
+    const int64_t o_xs = take(bf16 ? 0 : passes * (H / 128) * kSFImg);
     const int64_t o_ht = take(rows * kT * pad256(I) / 2);
     const int64_t o_hs = take(passes * (I / 128) * kSFImg);
+    const int64_t o_xp = bf16 ? take(rows * H * 2) : 0;
+    const int64_t o_hf = bf16 ? take(rows * I * 4) : 0;
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
         ws->status = reinterpret_cast<int *>(b + o_status);
@@ -779,35 +800,12 @@ int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
         ws->x_sf = b + o_xs;
         ws->h_terms = b + o_ht;
         ws->h_sf = b + o_hs;
+        ws->x_perm = bf16 ? reinterpret_cast<uint16_t *>(b + o_xp) : nullptr;
+        ws->h_f32 = bf16 ? reinterpret_cast<float *>(b + o_hf) : nullptr;
     }
     return off;
 }
 
-int num_sms()
-{
-    static thread_local int cached_dev = -1, cached = 0;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev != cached_dev) {
-        cudaDeviceGetAttribute(&cached, cudaDevAttrMultiProcessorCount, dev);
-        cached_dev = dev;
-    }
-    return cached > 0 ? cached : 148;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
-{
-    static std::once_flag once;
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    std::call_once(once, [] {
-        cudaDriverEntryPointQueryResult q;
-        void *ptr = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
 
 int encode(CUtensorMap *m, int rank, const void *base, const cuuint64_t *dims, const cuuint64_t *strides,
            const cuuint32_t *box, CUtensorMapL2promotion promo, const char *what)
@@ -908,13 +906,26 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     ffn_ws_layout(T, k, H, I, &ws, workspace);
     const int rows = T * k;
     const int nt = token_tile(T);
+    if (use_bf16_gate_up(T, k)) {
+        // h on bf16 tensor cores, then its E2M1 digit terms for the down stage
+        const Blob bl = blob_parts(prepacked, E, H, I);
+        if (int rc = run_bf16_gate_up(x, offsets, src_row, bl.w13, bl.sf13, T, k, E, H, I, ws.x_perm, ws.h_f32,
+                                      ws.status, st))
+            return rc;
+        const int64_t warps = (int64_t)rows * (I / 32);
+        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 2);
+        act_terms_kernel<true><<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(ws.h_f32, nullptr, offsets, E, 1, rows, I,
+                                                                        nt, ws.h_terms, ws.h_sf, ws.pass_start,
+                                                                        nullptr);
+        return check_launch("act_terms_kernel<h>");
+    }
     {
         const int64_t warps = (int64_t)rows * (H / 32);
         const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 2);
-        x_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
+        act_terms_kernel<false><<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(x, src_row, offsets, E,
                                                                  k, rows, H, nt, ws.x_terms, ws.x_sf, ws.pass_start,
                                                                  ws.status);
-        if (int rc = check_launch("x_terms_kernel"))
+        if (int rc = check_launch("act_terms_kernel<x>"))
             return rc;
     }
     const Blob bl = blob_parts(prepacked, E, H, I);
