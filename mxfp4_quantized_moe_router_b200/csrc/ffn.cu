@@ -121,7 +121,8 @@ struct Cfg {
     static constexpr size_t kOffBar = kOffSfa + (size_t)kStagesA * 2 * kSFImg;
     static constexpr int kBars = 2 * kStagesW + 2 * kStagesA + 3 + kStagesA + 1;
     static constexpr size_t kOffMisc = (kOffBar + kBars * 8 + 15) & ~size_t(15);
-    static constexpr size_t kSmem = 1024 + kOffMisc + 64;
+    static constexpr size_t kOffItems = kOffMisc + 64;  // items before each expert [kMaxE + 1]
+    static constexpr size_t kSmem = 1024 + kOffItems + (kMaxE + 1) * 4;
     // Tensor memory: the accumulator (128 lanes x 256 columns), then per weight
     // stage two 8-column scale groups (K halves; 256 rows = 8 columns) and per
     // activation stage two 4-column groups.
@@ -154,51 +155,37 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64
 }
 
 // Work items of one FFN stage: (expert, 256-row tile, token pass), expert-major,
-// then tile, then pass, so that the passes of one weight tile are adjacent
-// (the repeated weight boxes then come from L2). A CTA takes a contiguous
-// range of items and every role walks it with its own cursor.
-template <int NT>
-struct ItemCursor {
-    const int32_t *offsets;
-    int E, tiles;
-    int e, tile, pass, npass, base, n_e;
-
-    __device__ __forceinline__ void load_expert()
-    {
-        base = offsets[e];
-        n_e = offsets[e + 1] - base;
-        npass = (n_e + NT - 1) / NT;
-    }
-    __device__ __forceinline__ void start(const int32_t *off, int E_, int tiles_, int e0, int local)
-    {
-        offsets = off;
-        E = E_;
-        tiles = tiles_;
-        e = e0;
-        if (e >= E)
-            return;
-        load_expert();
-        tile = npass ? local / npass : 0;
-        pass = npass ? local % npass : 0;
-    }
-    __device__ __forceinline__ void next()
-    {
-        if (++pass < npass)
-            return;
-        pass = 0;
-        if (++tile < tiles)
-            return;
-        tile = 0;
-        do {
-            ++e;
-            if (e >= E)
-                return;
-            load_expert();
-        } while (npass == 0);
-    }
-    __device__ __forceinline__ int r0() const { return base + pass * NT; }
-    __device__ __forceinline__ int nt() const { return min(NT, n_e - pass * NT); }
+// then tile, then pass. CTA b takes items b, b + G, b + 2G, ... (G CTAs), so
+// the passes of one weight tile run on neighbouring CTAs at about the same
+// time and all but the first read its boxes from L2. Every role decodes the
+// same items.
+struct Item {
+    int e, tile, pass, r0, nt;
 };
+
+template <int NT>
+__device__ __forceinline__ Item decode_item(int64_t idx, const int32_t *items, const int32_t *offsets, int E,
+                                            int tiles)
+{
+    int lo = 0, hi = E;  // largest e with items[e] <= idx
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (items[mid] <= idx)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    const int base = offsets[lo], n_e = offsets[lo + 1] - base;
+    const int npass = (n_e + NT - 1) / NT;
+    const int local = (int)(idx - items[lo]);
+    Item it;
+    it.e = lo;
+    it.tile = local / npass;
+    it.pass = local % npass;
+    it.r0 = base + it.pass * NT;
+    it.nt = min(NT, n_e - it.pass * NT);
+    return it;
+}
 
 __device__ __forceinline__ float pow2f(int s)  // 2^s for s in [-126, 127]
 {
@@ -262,49 +249,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *cp_done = sfready + C::kStagesA;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
-    int *cur = reinterpret_cast<int *>(tslot + 2);  // [0] first expert, [1] first item within it, [2] item count
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = p.E, tiles = p.tiles;
 
-    if (warp == 0) {
-        // Items of expert e: tiles * ceil(n_e / NT). Pass 1 counts them all;
-        // pass 2 finds the expert holding this CTA's first item.
-        int64_t total = 0;
-        for (int b = 0; b < E; b += 32) {
+    int32_t *s_items = reinterpret_cast<int32_t *>(smem + C::kOffItems);
+    for (int e = tid; e < E; e += kThreads)  // items of expert e: tiles * ceil(n_e / NT)
+        s_items[e] = tiles * ((p.offsets[e + 1] - p.offsets[e] + NT - 1) / NT);
+    __syncthreads();
+    if (warp == 0) {  // exclusive prefix, in place; s_items[E] = all items
+        int carry = 0;
+        for (int b = 0; b <= E; b += 32) {
             const int e = b + lane;
-            const int n_e = e < E ? p.offsets[e + 1] - p.offsets[e] : 0;
-            int64_t c = (int64_t)tiles * ((n_e + NT - 1) / NT);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                c += __shfl_xor_sync(0xFFFFFFFFu, c, off);
-            total += c;
-        }
-        const int64_t i_begin = total * blockIdx.x / gridDim.x;
-        const int64_t i_end = total * (blockIdx.x + 1) / gridDim.x;
-        if (lane == 0) {
-            cur[0] = E;
-            cur[1] = 0;
-            cur[2] = (int)(i_end - i_begin);
-        }
-        __syncwarp();
-        int64_t carry = 0;
-        for (int b = 0; b < E && i_end > i_begin; b += 32) {
-            const int e = b + lane;
-            const int n_e = e < E ? p.offsets[e + 1] - p.offsets[e] : 0;
-            const int64_t c = (int64_t)tiles * ((n_e + NT - 1) / NT);
-            int64_t incl = c;
+            const int c = e < E ? s_items[e] : 0;
+            int incl = c;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
                 if (lane >= off)
                     incl += o;
             }
-            const int64_t excl = carry + incl - c;
-            if (c > 0 && excl <= i_begin && i_begin < excl + c) {
-                cur[0] = e;
-                cur[1] = (int)(i_begin - excl);
-            }
+            __syncwarp();
+            if (e <= E)
+                s_items[e] = carry + incl - c;
             carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
     }
@@ -332,9 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = *tslot;
-    const int n_items = cur[2];
-    ItemCursor<NT> it;
-    it.start(p.offsets, E, tiles, cur[0], cur[1]);
+    const int64_t G = gridDim.x, total = s_items[E];
+    const int n_items = (int)(total > blockIdx.x ? (total - blockIdx.x + G - 1) / G : 0);
+#define ITEM(i) decode_item<NT>(blockIdx.x + (int64_t)(i) * G, s_items, p.offsets, E, tiles)
     const int nchunk = (p.K + kKC - 1) / kKC;  // the last chunk may hold one 128-column half
     const int khalves = p.K / 128;
 
@@ -347,10 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phw = 0, pha = 0;
             int64_t issued_w = 0, issued_a = 0;
             bool ok = true;
-            for (int i = 0; i < n_items && ok; ++i, it.next()) {
+            for (int i = 0; i < n_items && ok; ++i) {
+                const Item it = ITEM(i);
                 const int64_t box0 = ((int64_t)it.e * tiles + it.tile) * nchunk;
                 const int64_t pass_id = (int64_t)p.pass_start[it.e] + it.pass;
-                const int r0 = it.r0();
+                const int r0 = it.r0;
                 for (int c = 0; c < nchunk; ++c) {
                     if (*abort_flag || !mbar_wait_bounded(&emptyW[sw], phw ^ 1u, kWaitLimitNs)) {
                         ok = false;
@@ -514,7 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = 4 * q + (lane >> 3);  // token within the pass
         const bool has_rows = 4 * q < NT;   // this quarter holds MMA rows in use
         bool aborted = false;
-        for (int i = 0; i < n_items; ++i, it.next()) {
+        for (int i = 0; i < n_items; ++i) {
+            const Item it = ITEM(i);
             if (!aborted) {  // lane 0 waits; the warp follows its verdict
                 int ok = 1;
                 if (lane == 0 && (*abort_flag || !mbar_wait_bounded(accfull, (uint32_t)i & 1u, kWaitLimitNs))) {
@@ -559,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(accempty);
-            const int ntile = it.nt();
+            const int ntile = it.nt;
             const bool valid = !aborted && has_rows && n < ntile;
             if (GATE_UP) {
                 // h columns 64b + 8tl + j of the tile (b = 0, 1): gate = v[b], up = v[b + 2]
@@ -571,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float g = v[b][j];
                         hv[b][j] = valid ? g / (1.f + expf(-g)) * v[b + 2][j] : 0.f;
                     }
-                const int r = it.r0() + n;
+                const int r = it.r0 + n;
                 const int64_t img = ((int64_t)p.pass_start[it.e] + it.pass) * (p.I / 128) + it.tile;
 #pragma unroll
                 for (int b = 0; b < 2; ++b) {
@@ -607,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else if (valid) {
-                float *yrow = p.y_out + (int64_t)(it.r0() + n) * p.H + 256 * it.tile + 8 * tl;
+                float *yrow = p.y_out + (int64_t)(it.r0 + n) * p.H + 256 * it.tile + 8 * tl;
                 const int ncols = min(256, p.H - 256 * it.tile);  // 128 in a padded last tile
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
@@ -626,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_after();
         tc::dealloc(tmem, C::kTmemCols);
     }
+#undef ITEM
 }
 
 // Token passes of each expert: pass_start[e] = sum over e' < e of
