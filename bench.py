@@ -38,7 +38,14 @@ import datagen  # noqa: E402
 
 METRIC = "MXFP4 MoE-layer tokens/s; expert-weight HBM GB/s as % of peak (1×B200)"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 7  # router_gemm, route, permute, x_terms, ffn gate/up, ffn down, combine
+BF16_PATH_ROWS = 16384  # grouped rows (tokens x top-k) from which both FFN stages run on bf16 tensor cores
+
+
+def kernels_per_step(rows: int) -> int:
+    """Launches of one layer step: router_gemm, route, permute, then x_terms +
+    the two E2M1-term FFN stages, or (bf16 path) passes + x_tile + the two bf16
+    stages, then combine."""
+    return 8 if rows >= BF16_PATH_ROWS else 7
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -77,12 +84,14 @@ def workload_config(cfg, world: int, batches: int):
 
 
 def load_peaks():
+    """(HBM GB/s, sustained bf16 TFLOP/s, source): the machine's measured copy
+    bandwidth and cuBLAS bf16 GEMM rate under the power cap, else the fallback."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, 1400.0, "fallback"
 
 
 def kernel_source_sha() -> str:
@@ -440,36 +449,50 @@ def run_native(args):
             dist.destroy_process_group()
         return
 
-    peak, peak_kind = load_peaks()
+    peak, peak_tf, peak_kind = load_peaks()
     steps_batches = [(args.warmup + i) % nb for i in range(args.steps)]
     mean_touched = float(np.mean([touched[b] for b in steps_batches]))
     tokens = T * args.steps * world
     value = whole_job_rate(T, args.steps, world, ms_max)
     weight_bytes_step = mean_touched * cfg.expert_bytes
     weight_gbs = weight_bytes_step * args.steps / (ms / 1e3) / 1e9
-    # dominant unit: mxmoe_ffn_gate_up (x_terms + gate/up stage); algorithmic
-    # bytes = gate/up MXFP4 bytes of the touched experts + x read + h written
-    w13_bytes = 2 * I * H * 17 // 32
-    unit_bytes = mean_touched * w13_bytes + T * H * 2 + T * k * I * 2
     unit_ms_mean = float(np.mean(unit_ms))
-    achieved = unit_bytes / (unit_ms_mean / 1e3) / 1e9
+    if T * k >= BF16_PATH_ROWS:
+        # dominant unit: mxmoe_ffn_gate_up on bf16 tensor cores (x_gather +
+        # ffn_bf16_kernel<gate_up>); algorithmic work = the dense gate/up
+        # contraction of every grouped row: 2 * rows * 2I * H flops
+        unit_flops = 2.0 * T * k * 2 * I * H
+        achieved = unit_flops / (unit_ms_mean / 1e3) / 1e12
+        roofline = {"kernel": "mxmoe_ffn_gate_up (x_gather_kernel + ffn_bf16_kernel<gate_up>)", "bound": "tensor",
+                    "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops_sustained)" % peak_kind
+                    if peak_kind == "measured" else "fallback 1.4 PFLOP/s sustained",
+                    "traffic": None, "unit_ms": unit_ms_mean, "algorithmic_flops_per_launch": unit_flops}
+    else:
+        # dominant unit: mxmoe_ffn_gate_up (x_terms + gate/up stage); algorithmic
+        # bytes = gate/up MXFP4 bytes of the touched experts + x read + h written
+        w13_bytes = 2 * I * H * 17 // 32
+        unit_bytes = mean_touched * w13_bytes + T * H * 2 + T * k * I * 2
+        achieved = unit_bytes / (unit_ms_mean / 1e3) / 1e9
+        roofline = {"kernel": "mxmoe_ffn_gate_up (x_terms_kernel + ffn_mxf4_kernel<gate_up>)",
+                    "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                    else "fallback 6.65 TB/s",
+                    "traffic": profiled_traffic(cfg.name, mean_touched), "unit_ms": unit_ms_mean,
+                    "algorithmic_bytes_per_launch": unit_bytes}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e2m1 x e2m1 digit terms -> f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
+        "dtype": "bf16 x dequantised e2m1 -> f32" if T * k >= BF16_PATH_ROWS
+        else "e2m1 x e2m1 digit terms -> f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
                                           "W~N(0,0.02) quantised to MXFP4 by the library)",
         "config": workload_config(cfg, world, nb),
         "weight_gbs": weight_gbs,
         "weight_frac_of_hbm_peak": weight_gbs / peak,
         "touched_experts_per_step": mean_touched,
-        "roofline": {"kernel": "mxmoe_ffn_gate_up (x_terms_kernel + ffn_mxf4_kernel<gate_up>)",
-                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
-                     else "fallback 6.65 TB/s",
-                     "traffic": profiled_traffic(cfg.name, mean_touched), "unit_ms": unit_ms_mean,
-                     "algorithmic_bytes_per_launch": unit_bytes},
+        "roofline": roofline,
         "clocks": clk,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(T * k) * args.steps,
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
                 "d2h_bytes_per_step": T * H * 4, "api": "mxmoe_layer_forward with pinned host x/y copies"},
     }

@@ -82,7 +82,7 @@ int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row
                    int k, int E, int H, int I, float *y_perm, void *workspace, cudaStream_t st);
 int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int T, int k, int H, float *y,
                 cudaStream_t st);
-int64_t ffn_workspace_bytes(int T, int k, int H, int I);
+int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
 int router_splits(int T, int H, int E);
 int run_router_and_route(const void *x, const void *wg, const float *bias, int T, int H, int E, int k,
@@ -110,7 +110,7 @@ int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *ba
         return o;
     };
     const int64_t n = (int64_t)T * k;
-    const int64_t o_ffn = take(ffn_workspace_bytes(T, k, H, I));
+    const int64_t o_ffn = take(ffn_workspace_bytes(T, k, E, H, I));
     const int64_t o_logits = take((int64_t)router_splits(T, H, E) * T * E * 4);
     const int64_t o_ids = take(n * 4);
     const int64_t o_w = take(n * 4);

@@ -51,9 +51,12 @@
 #include "tcgen05.cuh"
 
 namespace mxmoe {
-int run_bf16_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row, const uint8_t *w13,
-                     const uint8_t *sf13, int T, int k, int E, int H, int I, uint16_t *x_perm, float *h, int *status,
-                     cudaStream_t st);
+int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
+                  int32_t *pass_start, uint8_t *x_tiled, int *status, cudaStream_t st);
+int run_bf16_stage(bool gate_up, const uint8_t *act_tiled, const int32_t *offsets, const int32_t *pass_start,
+                   const uint8_t *w, const uint8_t *sf, int rows, int E, int H, int I, uint8_t *h_tiled, float *y,
+                   int *status, cudaStream_t st);
+int64_t bf16_max_passes(int64_t rows, int E);
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
@@ -623,13 +626,10 @@ __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
 
 // Activation rows -> kT E2M1 terms per value in grouped row order, in the
 // term_offset layout, with their scale images (one per token pass and 128
-// columns). GROUPED_F32 = false: x rows (bf16), row r holding token
-// src_row[r] / k; true: rows already grouped, fp32 (h of the gate/up stage
-// when it ran on bf16 tensor cores; src_row and k unused). One warp per
-// 32-value block. Block 0 also writes pass_start for the FFN stages and clears
+// columns), from x rows (bf16), row r holding token src_row[r] / k. One warp
+// per 32-value block. Block 0 also writes pass_start for the FFN stages and clears
 // the status word.
-template <bool GROUPED_F32>
-__global__ void __launch_bounds__(256) act_terms_kernel(const void *__restrict__ act, const int32_t *__restrict__ src_row,
+__global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restrict__ act, const int32_t *__restrict__ src_row,
                                                       const int32_t *__restrict__ offsets, int E, int k, int rows,
                                                       int H, int nt, uint8_t *__restrict__ terms,
                                                       uint8_t *__restrict__ sf, int32_t *__restrict__ pass_start_out,
@@ -672,12 +672,10 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const void *__restrict__
             const int local = r - s_off[lo];
             img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
             n = local % nt;
-            tok = GROUPED_F32 ? r : src_row[r] / k;
+            tok = src_row[r] / k;
         }
         const int col = kb * 32 + lane;
-        const float v = GROUPED_F32 ? static_cast<const float *>(act)[(int64_t)tok * H + col]
-                                    : __uint_as_float((uint32_t)static_cast<const uint16_t *>(act)[(int64_t)tok * H + col]
-                                                      << 16);
+        const float v = __uint_as_float((uint32_t)act[(int64_t)tok * H + col] << 16);
         float m = fabsf(v);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
@@ -727,23 +725,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 // ---------------------------------------------------------------------------
 struct FfnWs {
     int *status;
-    int32_t *pass_start;  // [kMaxE + 1]
+    int32_t *pass_start;  // [kMaxE + 1]: token passes before each expert
     uint8_t *x_terms;     // term_offset layout, K = H
     uint8_t *x_sf;        // scale images [pass][H/128][512]
     uint8_t *h_terms;     // term_offset layout, K = I
     uint8_t *h_sf;        // scale images [pass][I/128][512]
-    uint16_t *x_perm;     // bf16 gate/up path only: x rows in grouped order [rows][H]
-    float *h_f32;         // bf16 gate/up path only: h [rows][I]
+    uint8_t *x_tiled;     // bf16 path only: x per (pass, K step) as the shared-memory image
+    uint8_t *h_tiled;     // bf16 path only: h hi, lo per (pass, K step, term) likewise
 };
 
-// Token counts at which the gate/up stage runs on bf16 tensor cores (weights
-// dequantised in shared memory, x as is) instead of the E2M1-term MMAs: from
-// 16384 grouped rows (2048 tokens at top-8), where experts see hundreds of
-// tokens and the stage is bound by the tensor cores.
-constexpr int64_t kBf16GateUpRows = 16384;
-bool use_bf16_gate_up(int T, int k) { return (int64_t)T * k >= kBf16GateUpRows; }
+// Token counts at which both FFN stages run on bf16 tensor cores (weights
+// dequantised in shared memory; x as is, h as two bf16 terms) instead of the
+// E2M1-term MMAs: from 16384 grouped rows (2048 tokens at top-8), where experts
+// see hundreds of tokens and the stages are bound by the tensor cores.
+constexpr int64_t kBf16Rows = 16384;
+bool use_bf16_path(int T, int k) { return (int64_t)T * k >= kBf16Rows; }
 
-int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
+int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
 {
     int64_t off = 0;
     auto take = [&](int64_t bytes) {
@@ -755,13 +753,14 @@ int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
     const int64_t passes = max_passes(rows);
     const int64_t o_status = take(16);
     const int64_t o_ps = take((kMaxE + 1) * 4);
-    const bool bf16 = use_bf16_gate_up(T, k);  // x goes to the tensor cores as bf16: no x terms
+    const bool bf16 = use_bf16_path(T, k);  // x and h go to the tensor cores as bf16: no digit terms
     const int64_t o_xt = take(bf16 ? 0 : rows * kT * pad256(H) / 2);
     const int64_t o_xs = take(bf16 ? 0 : passes * (H / 128) * kSFImg);
-    const int64_t o_ht = take(rows * kT * pad256(I) / 2);
-    const int64_t o_hs = take(passes * (I / 128) * kSFImg);
-    const int64_t o_xp = bf16 ? take(rows * H * 2) : 0;
-    const int64_t o_hf = bf16 ? take(rows * I * 4) : 0;
+    const int64_t o_ht = take(bf16 ? 0 : rows * kT * pad256(I) / 2);
+    const int64_t o_hs = take(bf16 ? 0 : passes * (I / 128) * kSFImg);
+    const int64_t bp = bf16 ? bf16_max_passes(rows, E) : 0;  // 256-token passes, at most
+    const int64_t o_xp = bf16 ? take(bp * 256 * H * 2) : 0;
+    const int64_t o_h2 = bf16 ? take(bp * 256 * I * 4) : 0;
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
         ws->status = reinterpret_cast<int *>(b + o_status);
@@ -770,8 +769,8 @@ int64_t ffn_ws_layout(int T, int k, int H, int I, FfnWs *ws, void *base)
         ws->x_sf = b + o_xs;
         ws->h_terms = b + o_ht;
         ws->h_sf = b + o_hs;
-        ws->x_perm = bf16 ? reinterpret_cast<uint16_t *>(b + o_xp) : nullptr;
-        ws->h_f32 = bf16 ? reinterpret_cast<float *>(b + o_hf) : nullptr;
+        ws->x_tiled = bf16 ? b + o_xp : nullptr;
+        ws->h_tiled = bf16 ? b + o_h2 : nullptr;
     }
     return off;
 }
@@ -873,29 +872,23 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
                     int k, int E, int H, int I, void *workspace, cudaStream_t st)
 {
     FfnWs ws;
-    ffn_ws_layout(T, k, H, I, &ws, workspace);
+    ffn_ws_layout(T, k, E, H, I, &ws, workspace);
     const int rows = T * k;
     const int nt = token_tile(T);
-    if (use_bf16_gate_up(T, k)) {
-        // h on bf16 tensor cores, then its E2M1 digit terms for the down stage
+    if (use_bf16_path(T, k)) {  // h on bf16 tensor cores, leaving as bf16 hi, lo terms
         const Blob bl = blob_parts(prepacked, E, H, I);
-        if (int rc = run_bf16_gate_up(x, offsets, src_row, bl.w13, bl.sf13, T, k, E, H, I, ws.x_perm, ws.h_f32,
-                                      ws.status, st))
+        if (int rc = run_bf16_prep(x, offsets, src_row, k, rows, E, H, ws.pass_start, ws.x_tiled, ws.status, st))
             return rc;
-        const int64_t warps = (int64_t)rows * (I / 32);
-        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 2);
-        act_terms_kernel<true><<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(ws.h_f32, nullptr, offsets, E, 1, rows, I,
-                                                                        nt, ws.h_terms, ws.h_sf, ws.pass_start,
-                                                                        nullptr);
-        return check_launch("act_terms_kernel<h>");
+        return run_bf16_stage(true, ws.x_tiled, offsets, ws.pass_start, bl.w13, bl.sf13, rows, E, H, I, ws.h_tiled,
+                              nullptr, ws.status, st);
     }
     {
         const int64_t warps = (int64_t)rows * (H / 32);
         const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 2);
-        act_terms_kernel<false><<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(x, src_row, offsets, E,
+        act_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
                                                                  k, rows, H, nt, ws.x_terms, ws.x_sf, ws.pass_start,
                                                                  ws.status);
-        if (int rc = check_launch("act_terms_kernel<x>"))
+        if (int rc = check_launch("act_terms_kernel"))
             return rc;
     }
     const Blob bl = blob_parts(prepacked, E, H, I);
@@ -923,10 +916,13 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
                  void *workspace, cudaStream_t st)
 {
     FfnWs ws;
-    ffn_ws_layout(T, k, H, I, &ws, workspace);
+    ffn_ws_layout(T, k, E, H, I, &ws, workspace);
     const int rows = T * k;
     const int nt = token_tile(T);
     const Blob bl = blob_parts(prepacked, E, H, I);
+    if (use_bf16_path(T, k))
+        return run_bf16_stage(false, ws.h_tiled, offsets, ws.pass_start, bl.w2, bl.sf2, rows, E, H, I, nullptr,
+                              y_perm, ws.status, st);
     FfnParams p{};
     p.tiles = (int)(pad256(H) / 256);
     p.K = I;
@@ -963,7 +959,10 @@ int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int 
     return check_launch("combine_kernel");
 }
 
-int64_t ffn_workspace_bytes(int T, int k, int H, int I) { return ffn_ws_layout(T, k, H, I, nullptr, nullptr); }
+int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I)
+{
+    return ffn_ws_layout(T, k, E, H, I, nullptr, nullptr);
+}
 
 int validate_ffn_shapes(int T, int k, int E, int H, int I) { return validate_ffn(T, k, E, H, I); }
 
@@ -976,16 +975,16 @@ extern "C" MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H
     if (T < 0 || k < 1 || k > 32 || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 128 || I % 128 || H > 32768 ||
         I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31))
         return -1;
-    return ffn_workspace_bytes(T, k, H, I);
+    return ffn_workspace_bytes(T, k, E, H, I);
 }
 
 static int check_ffn_args(const char *fn, int T, int k, int E, int H, int I, void *workspace, int64_t workspace_bytes)
 {
     if (int rc = validate_ffn_shapes(T, k, E, H, I))
         return rc;
-    if (!workspace || workspace_bytes < ffn_workspace_bytes(T, k, H, I))
+    if (!workspace || workspace_bytes < ffn_workspace_bytes(T, k, E, H, I))
         return fail(MXMOE_ERR_WORKSPACE, "%s: workspace of %lld bytes, need %lld", fn, (long long)workspace_bytes,
-                    (long long)ffn_workspace_bytes(T, k, H, I));
+                    (long long)ffn_workspace_bytes(T, k, E, H, I));
     if (reinterpret_cast<uintptr_t>(workspace) & 255)
         return fail(MXMOE_ERR_ALIGNMENT, "%s: workspace needs 256-byte alignment", fn);
     return MXMOE_OK;

@@ -14,7 +14,7 @@
 namespace mxmoe {
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
                    int k, int E, int H, int I, float *y_perm, void *workspace, cudaStream_t st);
-int64_t ffn_workspace_bytes(int T, int k, int H, int I);
+int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
 }  // namespace mxmoe
 
@@ -62,7 +62,7 @@ extern "C" MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *
     using namespace mxmoe;
     if (int rc = validate_ffn_shapes(T, k, E, H, I))
         return rc;
-    const int64_t need = ffn_workspace_bytes(T, k, H, I);
+    const int64_t need = ffn_workspace_bytes(T, k, E, H, I);
     if (need > kStaticScratchBytes)
         return fail(MXMOE_ERR_WORKSPACE,
                     "mxmoe_expert_ffn_noalloc: these sizes need %lld bytes of scratch, more than the fixed %lld "
