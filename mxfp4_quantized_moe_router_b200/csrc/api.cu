@@ -79,14 +79,14 @@ int check_device()
 
 // defined in ffn.cu
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
-                   int k, int E, int H, int I, float *y_perm, void *workspace, cudaStream_t st);
+                   int k, int E, int H, int I, float *y_perm, void *workspace, bool clear_status, cudaStream_t st);
 int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int T, int k, int H, float *y,
                 cudaStream_t st);
 int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
 int router_splits(int T, int H, int E);
 int run_router_and_route(const void *x, const void *wg, const float *bias, int T, int H, int E, int k,
-                         float *partials, int nsplit, int32_t *ids, float *w, cudaStream_t st);
+                         float *partials, int nsplit, int32_t *ids, float *w, int *status, cudaStream_t st);
 
 namespace {
 
@@ -175,11 +175,17 @@ extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, cons
     int32_t *ids = ids_out ? ids_out : ws.ids;
     float *w = w_out ? w_out : ws.w;
     cudaStream_t st = (cudaStream_t)stream;
-    if (int rc = run_router_and_route(x, wg, bias, T, H, E, k, ws.logits, router_splits(T, H, E), ids, w, st))
+    // one status record for the whole layer (the FFN workspace's first word): cleared here, so that a timeout
+    // of the router kernel survives to mxmoe_read_status
+    int *status = static_cast<int *>(ws.ffn);
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess)
+        return fail(MXMOE_ERR_CUDA, "mxmoe_layer_forward: cannot clear the status word");
+    if (int rc = run_router_and_route(x, wg, bias, T, H, E, k, ws.logits, router_splits(T, H, E), ids, w, status,
+                                      st))
         return rc;
     if (int rc = mxmoe_permute(ids, T, k, E, ws.offsets, ws.src_row, ws.dst_of, stream))
         return rc;
-    if (int rc = run_expert_ffn(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn, st))
+    if (int rc = run_expert_ffn(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn, false, st))
         return rc;
     return run_combine(ws.y_perm, ws.dst_of, w, T, k, H, y, st);
 }

@@ -868,16 +868,19 @@ Blob blob_parts(const void *prepacked, int E, int H, int I)
 
 }  // namespace
 
+// clear_status: whether this call starts a new status record (the layer
+// clears it itself before the router, which may record a timeout in it).
 int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
-                    int k, int E, int H, int I, void *workspace, cudaStream_t st)
+                    int k, int E, int H, int I, void *workspace, bool clear_status, cudaStream_t st)
 {
     FfnWs ws;
     ffn_ws_layout(T, k, E, H, I, &ws, workspace);
+    int *clear = clear_status ? ws.status : nullptr;
     const int rows = T * k;
     const int nt = token_tile(T);
     if (use_bf16_path(T, k)) {  // h on bf16 tensor cores, leaving as bf16 hi, lo terms
         const Blob bl = blob_parts(prepacked, E, H, I);
-        if (int rc = run_bf16_prep(x, offsets, src_row, k, rows, E, H, ws.pass_start, ws.x_tiled, ws.status, st))
+        if (int rc = run_bf16_prep(x, offsets, src_row, k, rows, E, H, ws.pass_start, ws.x_tiled, clear, st))
             return rc;
         return run_bf16_stage(true, ws.x_tiled, offsets, ws.pass_start, bl.w13, bl.sf13, rows, E, H, I, ws.h_tiled,
                               nullptr, ws.status, st);
@@ -887,7 +890,7 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
         const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 2);
         act_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
                                                                  k, rows, H, nt, ws.x_terms, ws.x_sf, ws.pass_start,
-                                                                 ws.status);
+                                                                 clear);
         if (int rc = check_launch("act_terms_kernel"))
             return rc;
     }
@@ -944,9 +947,9 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
 }
 
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
-                   int k, int E, int H, int I, float *y_perm, void *workspace, cudaStream_t st)
+                   int k, int E, int H, int I, float *y_perm, void *workspace, bool clear_status, cudaStream_t st)
 {
-    if (int rc = run_ffn_gate_up(x, offsets, src_row, prepacked, T, k, E, H, I, workspace, st))
+    if (int rc = run_ffn_gate_up(x, offsets, src_row, prepacked, T, k, E, H, I, workspace, clear_status, st))
         return rc;
     return run_ffn_down(offsets, prepacked, T, k, E, H, I, y_perm, workspace, st);
 }
@@ -1006,7 +1009,8 @@ extern "C" MXMOE_API int mxmoe_expert_ffn(const void *x, const int32_t *offsets,
         return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_expert_ffn: x and y_perm need 16-byte, prepacked 32-byte alignment");
     if (int rc = check_device())
         return rc;
-    return run_expert_ffn(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, workspace, (cudaStream_t)stream);
+    return run_expert_ffn(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, workspace, true,
+                          (cudaStream_t)stream);
 }
 
 extern "C" MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row,
@@ -1023,7 +1027,7 @@ extern "C" MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets
         return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_ffn_gate_up: x needs 16-byte, prepacked 32-byte alignment");
     if (int rc = check_device())
         return rc;
-    return run_ffn_gate_up(x, offsets, src_row, prepacked, T, k, E, H, I, workspace, (cudaStream_t)stream);
+    return run_ffn_gate_up(x, offsets, src_row, prepacked, T, k, E, H, I, workspace, true, (cudaStream_t)stream);
 }
 
 extern "C" MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, int E, int H,

@@ -13,7 +13,7 @@
 
 namespace mxmoe {
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
-                   int k, int E, int H, int I, float *y_perm, void *workspace, cudaStream_t st);
+                   int k, int E, int H, int I, float *y_perm, void *workspace, bool clear_status, cudaStream_t st);
 int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
 }  // namespace mxmoe
@@ -84,7 +84,7 @@ extern "C" MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *
     // The first kernel of the chain clears the status word at the start of the
     // scratch; every other scratch byte that can reach the outputs is written
     // earlier in the same call, so nothing else needs clearing between calls.
-    if (int rc = run_expert_ffn(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, scratch, st))
+    if (int rc = run_expert_ffn(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, scratch, true, st))
         return rc;
     if (status) {
         cudaError_t e = cudaMemcpyAsync(status, scratch, sizeof(int), cudaMemcpyDeviceToDevice, st);

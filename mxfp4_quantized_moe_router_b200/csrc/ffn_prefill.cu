@@ -188,21 +188,6 @@ __device__ __forceinline__ PItem decode_item(int64_t idx, const int32_t *__restr
     return it;
 }
 
-__device__ __forceinline__ uint32_t idesc_bf16(int n)  // kind::f16, bf16 x bf16 -> f32, K-major, M = 128
-{
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (8u << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
-        : "memory");
-}
-
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
     uint32_t d;
@@ -436,7 +421,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     break;
                 }
                 tc::fence_after();
-                const uint32_t idesc = idesc_bf16((it.nt + 15) & ~15);  // N: the pass's tokens, rounded up to 16
+                const uint32_t idesc = tc::idesc_bf16((it.nt + 15) & ~15);  // N: the pass's tokens, rounded up to 16
                 for (int ks = 0; ks < nks && ok; ++ks) {
                     if (*abort_flag || !mbar_wait_bounded(&aready[ra.slot], ra.phase, kPWaitNs)) {
                         ok = false;
@@ -452,7 +437,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         const uint32_t b_base = smem_u32(sB + (size_t)rb.slot * kPBBytes);
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4)  // 16 values of K per MMA
-                            mma_bf16(d_tmem, tc::smem_desc(a_base + 32 * k4, 16, 1024, 2),
+                            tc::mma_bf16(d_tmem, tc::smem_desc(a_base + 32 * k4, 16, 1024, 2),
                                      tc::smem_desc(b_base + 32 * k4, 16, 1024, 2), idesc,
                                      (ks > 0 || b > 0 || k4 > 0) ? 1u : 0u);
                         tc::commit(&empty_b[rb.slot]);

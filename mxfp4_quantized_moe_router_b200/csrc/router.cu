@@ -13,10 +13,15 @@
 #include "common.cuh"
 
 namespace mxmoe {
+bool use_router_tc(int T, int H);
+int router_tc_splits(int T, int H, int E);
+int run_router_gemm_tc(const void *x, const void *wg, const float *bias, int T, int H, int E, float *out, int nsplit,
+                       int *status, cudaStream_t st);
 namespace {
 
 // ---------------------------------------------------------------------------
-// Router GEMM: logits[t, e] = sum_k x[t, k] Wg[e, k] + bias[e].
+// Router GEMM (small T; from 512 tokens the tcgen05 kernel of router_tc.cu
+// runs instead): logits[t, e] = sum_k x[t, k] Wg[e, k] + bias[e].
 // CTA tile: 16 experts x 32 tokens x (K / gridDim.z); 8 warps split the CTA's
 // K range (warp w takes its k32 blocks w, w+8, ...), partial sums reduced in
 // shared memory in a fixed order. With gridDim.z > 1 each CTA writes its
@@ -324,6 +329,8 @@ extern "C" MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const 
         return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_router_gemm: x and wg must be 16-byte aligned");
     if (int rc = check_device())
         return rc;
+    if (use_router_tc(T, H))
+        return run_router_gemm_tc(x, wg, bias, T, H, E, logits, 1, nullptr, (cudaStream_t)stream);
     dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens, 1);
     router_gemm_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(static_cast<const uint16_t *>(x),
                                                               static_cast<const uint16_t *>(wg), bias, T, H, E,
@@ -347,6 +354,8 @@ int launch_route(const float *logits, int nsplit, const float *bias, int T, int 
 
 int router_splits(int T, int H, int E)
 {
+    if (use_router_tc(T, H))
+        return router_tc_splits(T, H, E);
     const int64_t base = (int64_t)((E + kRgExperts - 1) / kRgExperts) * ((T + kRgTokens - 1) / kRgTokens);
     int z = (int)((2 * 148 + base / 2) / std::max<int64_t>(base, 1));
     z = std::max(1, std::min(z, 8));
@@ -354,11 +363,17 @@ int router_splits(int T, int H, int E)
     return z;
 }
 
-// Router GEMM into nsplit partial arrays plus routing that sums them (the
-// layer path). partials: float [nsplit, T, E].
+// Router GEMM into nsplit partial arrays (nsplit = router_splits(T, H, E))
+// plus routing that sums them (the layer path). partials: float [nsplit, T, E].
+// status: where a timeout of the tcgen05 router is recorded.
 int run_router_and_route(const void *x, const void *wg, const float *bias, int T, int H, int E, int k,
-                         float *partials, int nsplit, int32_t *ids, float *w, cudaStream_t st)
+                         float *partials, int nsplit, int32_t *ids, float *w, int *status, cudaStream_t st)
 {
+    if (use_router_tc(T, H)) {
+        if (int rc = run_router_gemm_tc(x, wg, bias, T, H, E, partials, nsplit, status, st))
+            return rc;
+        return launch_route(partials, nsplit, nsplit > 1 ? bias : nullptr, T, E, k, ids, w, st);
+    }
     dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens, nsplit);
     router_gemm_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(wg),
                                              bias, T, H, E, partials);

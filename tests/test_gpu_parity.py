@@ -80,7 +80,10 @@ def test_dequantize_exact(mx):
 # ---------------------------------------------------------------------------
 # Router
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("T,H,E", [(1, 64, 16), (8, 6144, 384), (37, 256, 20), (300, 512, 64)])
+# From 512 tokens (H a multiple of 64) the router runs on tcgen05: ragged expert
+# and token tiles, one K step, and the full hidden size.
+@pytest.mark.parametrize("T,H,E", [(1, 64, 16), (8, 6144, 384), (37, 256, 20), (300, 512, 64), (700, 384, 200),
+                                   (513, 64, 8), (1024, 6144, 384)])
 def test_router_gemm(mx, T, H, E):
     cfg = datagen.LayerConfig("t", H, E, 2, 64, T)
     x = datagen.make_x(cfg, 3)
@@ -253,6 +256,15 @@ def test_layer_small_ragged(mx, T):
     x = datagen.make_x(cfg, 1)
     bias = (np.linspace(-0.5, 0.5, cfg.E)).astype(np.float32)
     check_layer(mx, layer, OracleExperts(cfg, 1), x, bias, np.arange(T))
+
+
+def test_layer_router_splits(mx):
+    # 600 tokens at H 2048: the tcgen05 router in 4 K splits, summed with the bias by the routing kernel
+    cfg = datagen.LayerConfig("small", 2048, 24, 4, 128, 600)
+    layer = GpuLayer(mx, cfg, 2)
+    x = datagen.make_x(cfg, 2)
+    bias = (np.linspace(-0.5, 0.5, cfg.E)).astype(np.float32)
+    check_layer(mx, layer, OracleExperts(cfg, 2), x, bias, np.arange(0, 600, 3))
 
 
 def test_layer_zero_tokens(mx):
