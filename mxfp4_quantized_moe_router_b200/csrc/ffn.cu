@@ -627,8 +627,10 @@ __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
 // Activation rows -> kT E2M1 terms per value in grouped row order, in the
 // term_offset layout, with their scale images (one per token pass and 128
 // columns), from x rows (bf16), row r holding token src_row[r] / k. One warp
-// per 32-value block. Block 0 also writes pass_start for the FFN stages and clears
-// the status word.
+// per (row, 256-value chunk): lane l holds values 8l .. 8l+7 of the chunk (one
+// 16-byte load), a 32-value block is four lanes, and each of the kT terms of
+// the chunk leaves as one 128-byte row of 32-bit stores. Block 0 also writes
+// pass_start for the FFN stages and clears the status word (when given).
 __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restrict__ act, const int32_t *__restrict__ src_row,
                                                       const int32_t *__restrict__ offsets, int E, int k, int rows,
                                                       int H, int nt, uint8_t *__restrict__ terms,
@@ -649,16 +651,17 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
         if (threadIdx.x == 0 && status)
             *status = 0;
     }
-    // Each warp takes a contiguous run of (row, 32-block) units, so the row's
+    // Each warp takes a contiguous run of (row, chunk) units, so the row's
     // expert, pass and token are looked up once per row.
-    const int nkb = H / 32;
-    const int64_t total = (int64_t)rows * nkb;
+    const int nch = (H + kKC - 1) / kKC;
+    const int64_t total = (int64_t)rows * nch;
     const int64_t nwarps = (int64_t)gridDim.x * 8, gw = (int64_t)blockIdx.x * 8 + warp;
-    const int64_t w_begin = total * gw / nwarps, w_end = total * (gw + 1) / nwarps;
+    const int64_t u_begin = total * gw / nwarps, u_end = total * (gw + 1) / nwarps;
+    const int kb = lane >> 2, q = lane & 3;  // the lane's 32-block within the chunk; its place in the block
     int r_cur = -1, n = 0, tok = 0;
     int64_t img_row = 0;
-    for (int64_t w = w_begin; w < w_end; ++w) {
-        const int r = (int)(w / nkb), kb = (int)(w % nkb);
+    for (int64_t u = u_begin; u < u_end; ++u) {
+        const int r = (int)(u / nch), c = (int)(u % nch);
         if (r != r_cur) {
             r_cur = r;
             int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
@@ -674,26 +677,50 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
             n = local % nt;
             tok = src_row[r] / k;
         }
-        const int col = kb * 32 + lane;
-        const float v = __uint_as_float((uint32_t)act[(int64_t)tok * H + col] << 16);
-        float m = fabsf(v);
+        const int col = c * kKC + 8 * lane;
+        const bool live = col < H;  // H % 128 == 0: in a half chunk lanes 0..15 are live
+        float v[8];
+        if (live) {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(act + (int64_t)tok * H + col));
+            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+            for (int j = 0; j < 4; ++j) {
+                v[2 * j] = __uint_as_float(w4[j] << 16);
+                v[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                v[j] = 0.f;
+        }
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            m = fmaxf(m, fabsf(v[j]));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
         const int E_blk = act_block_exp(m);
-        uint32_t code[kT];
-        act_digits(v, E_blk, code);
-        // term t sits 128 bytes after term t-1; its scale 16 bytes after (the
-        // image rows n*kT + t of one pass row are consecutive lanes)
-        uint8_t *tp = terms + term_offset(rows, 0, r, col);
-        uint8_t *sp = sf + (img_row + kb / 4) * kSFImg + image_byte(n, 0, kb & 3);
+        uint32_t word[kT];
 #pragma unroll
-        for (int t = 0; t < kT; ++t) {
-            const uint32_t hi_code = __shfl_down_sync(0xFFFFFFFFu, code[t], 1);
-            if (!(lane & 1))
-                tp[128 * t] = (uint8_t)(code[t] | (hi_code << 4));
-            if (lane == 0)
-                sp[16 * t] = (uint8_t)(E_blk - 1 - 3 * t + 127);
+        for (int t = 0; t < kT; ++t)
+            word[t] = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {  // value j of the lane: nibble j (element 2i in the low nibble of byte i)
+            uint32_t code[kT];
+            act_digits(v[j], E_blk, code);
+#pragma unroll
+            for (int t = 0; t < kT; ++t)
+                word[t] |= code[t] << (4 * j);
+        }
+        if (live) {
+            uint32_t *tp = reinterpret_cast<uint32_t *>(terms + term_offset(rows, 0, r, col));
+#pragma unroll
+            for (int t = 0; t < kT; ++t)  // term t sits 128 bytes after term t-1
+                tp[32 * t] = word[t];
+            // scales of the block: lane q of it writes terms q and q + 4
+            uint8_t *sp = sf + (img_row + 2 * c + (kb >> 2)) * kSFImg;
+            sp[image_byte(n, q, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * q + 127);
+            sp[image_byte(n, q + 4, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * (q + 4) + 127);
         }
     }
 }
@@ -886,8 +913,8 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
                               nullptr, ws.status, st);
     }
     {
-        const int64_t warps = (int64_t)rows * (H / 32);
-        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 2);
+        const int64_t warps = (int64_t)rows * ((H + kKC - 1) / kKC);
+        const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 8);
         act_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
                                                                  k, rows, H, nt, ws.x_terms, ws.x_sf, ws.pass_start,
                                                                  clear);
