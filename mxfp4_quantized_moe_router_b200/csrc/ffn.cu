@@ -41,6 +41,7 @@
 //  * Work items (expert, tile, token pass of up to NT tokens) are split
 //    contiguously over a persistent grid of one CTA per SM.
 #include <float.h>
+#include <limits.h>
 
 #include <algorithm>
 #include <mutex>
@@ -52,11 +53,11 @@
 
 namespace mxmoe {
 int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
-                  int32_t *pass_start, uint8_t *x_tiled, int *status, cudaStream_t st);
+                  int min_rows, int32_t *pass_start, uint8_t *x_tiled, int *status, cudaStream_t st);
 int run_bf16_stage(bool gate_up, const uint8_t *act_tiled, const int32_t *offsets, const int32_t *pass_start,
                    const uint8_t *w, const uint8_t *sf, int rows, int E, int H, int I, uint8_t *h_tiled, float *y,
                    int *status, cudaStream_t st);
-int64_t bf16_max_passes(int64_t rows, int E);
+int64_t bf16_max_passes(int64_t rows, int E, int min_rows);
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
@@ -83,6 +84,7 @@ struct FfnParams {
     int I;
     float *y_out;               // down output: [rows, H]
     int H;
+    int hot_rows;               // experts with at least this many rows are left to the bf16 kernel
     int *status;
 };
 
@@ -257,8 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int E = p.E, tiles = p.tiles;
 
     int32_t *s_items = reinterpret_cast<int32_t *>(smem + C::kOffItems);
-    for (int e = tid; e < E; e += kThreads)  // items of expert e: tiles * ceil(n_e / NT)
-        s_items[e] = tiles * ((p.offsets[e + 1] - p.offsets[e] + NT - 1) / NT);
+    for (int e = tid; e < E; e += kThreads) {  // items of expert e: tiles * ceil(n_e / NT), none if it is hot
+        const int n_e = p.offsets[e + 1] - p.offsets[e];
+        s_items[e] = n_e >= p.hot_rows ? 0 : tiles * ((n_e + NT - 1) / NT);
+    }
     __syncthreads();
     if (warp == 0) {  // exclusive prefix, in place; s_items[E] = all items
         int carry = 0;
@@ -629,11 +633,13 @@ __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
 // columns), from x rows (bf16), row r holding token src_row[r] / k. One warp
 // per (row, 256-value chunk): lane l holds values 8l .. 8l+7 of the chunk (one
 // 16-byte load), a 32-value block is four lanes, and each of the kT terms of
-// the chunk leaves as one 128-byte row of 32-bit stores. Block 0 also writes
-// pass_start for the FFN stages and clears the status word (when given).
+// the chunk leaves as one 128-byte row of 32-bit stores. Rows of experts with
+// at least hot_rows rows are skipped (the bf16 kernel takes those experts).
+// Block 0 also writes pass_start for the FFN stages and clears the status word
+// (when given).
 __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restrict__ act, const int32_t *__restrict__ src_row,
                                                       const int32_t *__restrict__ offsets, int E, int k, int rows,
-                                                      int H, int nt, uint8_t *__restrict__ terms,
+                                                      int H, int nt, int hot_rows, uint8_t *__restrict__ terms,
                                                       uint8_t *__restrict__ sf, int32_t *__restrict__ pass_start_out,
                                                       int *status)
 {
@@ -659,6 +665,7 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
     const int64_t u_begin = total * gw / nwarps, u_end = total * (gw + 1) / nwarps;
     const int kb = lane >> 2, q = lane & 3;  // the lane's 32-block within the chunk; its place in the block
     int r_cur = -1, n = 0, tok = 0;
+    bool hot = false;
     int64_t img_row = 0;
     for (int64_t u = u_begin; u < u_end; ++u) {
         const int r = (int)(u / nch), c = (int)(u % nch);
@@ -673,10 +680,13 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
                     hi = mid;
             }
             const int local = r - s_off[lo];
+            hot = s_off[lo + 1] - s_off[lo] >= hot_rows;
             img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
             n = local % nt;
             tok = src_row[r] / k;
         }
+        if (hot)
+            continue;
         const int col = c * kKC + 8 * lane;
         const bool live = col < H;  // H % 128 == 0: in a half chunk lanes 0..15 are live
         float v[8];
@@ -757,16 +767,27 @@ struct FfnWs {
     uint8_t *x_sf;        // scale images [pass][H/128][512]
     uint8_t *h_terms;     // term_offset layout, K = I
     uint8_t *h_sf;        // scale images [pass][I/128][512]
-    uint8_t *x_tiled;     // bf16 path only: x per (pass, K step) as the shared-memory image
-    uint8_t *h_tiled;     // bf16 path only: h hi, lo per (pass, K step, term) likewise
+    int32_t *bf_pass_start;  // bf16 kernel: its 256-token passes before each expert [kMaxE + 1]
+    uint8_t *x_tiled;     // bf16 kernel: x per (pass, K step) as the shared-memory image
+    uint8_t *h_tiled;     // bf16 kernel: h hi, lo per (pass, K step, term) likewise
 };
 
-// Token counts at which both FFN stages run on bf16 tensor cores (weights
-// dequantised in shared memory; x as is, h as two bf16 terms) instead of the
-// E2M1-term MMAs: from 16384 grouped rows (2048 tokens at top-8), where experts
-// see hundreds of tokens and the stages are bound by the tensor cores.
+// Token counts at which both FFN stages run on bf16 tensor cores for every
+// expert (weights dequantised in shared memory; x as is, h as two bf16 terms)
+// instead of the E2M1-term MMAs: from 16384 grouped rows (2048 tokens at
+// top-8), where experts see hundreds of tokens and the stages are bound by the
+// tensor cores.
 constexpr int64_t kBf16Rows = 16384;
 bool use_bf16_path(int T, int k) { return (int64_t)T * k >= kBf16Rows; }
+
+// Below that, experts with at least kHotRows rows (a skewed router) still go
+// to the bf16 kernel, the rest to the E2M1-term kernel: an E2M1-term pass of 16
+// tokens costs about as much MMA issue as 1/5 of a 256-token bf16 pass, so the
+// bf16 kernel wins from about a hundred tokens per expert. Only token counts
+// that can produce such an expert (T >= kHotRows) launch its kernels.
+constexpr int kHotRows = 128;
+bool use_hybrid(int T, int k) { return !use_bf16_path(T, k) && T >= kHotRows; }
+int bf16_min_rows(int T, int k) { return use_bf16_path(T, k) ? 0 : kHotRows; }
 
 int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
 {
@@ -780,14 +801,16 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
     const int64_t passes = max_passes(rows);
     const int64_t o_status = take(16);
     const int64_t o_ps = take((kMaxE + 1) * 4);
-    const bool bf16 = use_bf16_path(T, k);  // x and h go to the tensor cores as bf16: no digit terms
-    const int64_t o_xt = take(bf16 ? 0 : rows * kT * pad256(H) / 2);
-    const int64_t o_xs = take(bf16 ? 0 : passes * (H / 128) * kSFImg);
-    const int64_t o_ht = take(bf16 ? 0 : rows * kT * pad256(I) / 2);
-    const int64_t o_hs = take(bf16 ? 0 : passes * (I / 128) * kSFImg);
-    const int64_t bp = bf16 ? bf16_max_passes(rows, E) : 0;  // 256-token passes, at most
-    const int64_t o_xp = bf16 ? take(bp * 256 * H * 2) : 0;
-    const int64_t o_h2 = bf16 ? take(bp * 256 * I * 4) : 0;
+    const bool terms = !use_bf16_path(T, k);                 // the E2M1-term kernel runs
+    const bool bf16 = !terms || use_hybrid(T, k);           // the bf16 kernel runs
+    const int64_t o_xt = take(terms ? rows * kT * pad256(H) / 2 : 0);
+    const int64_t o_xs = take(terms ? passes * (H / 128) * kSFImg : 0);
+    const int64_t o_ht = take(terms ? rows * kT * pad256(I) / 2 : 0);
+    const int64_t o_hs = take(terms ? passes * (I / 128) * kSFImg : 0);
+    const int64_t o_bps = take(bf16 ? (kMaxE + 1) * 4 : 0);
+    const int64_t bp = bf16 ? bf16_max_passes(rows, E, bf16_min_rows(T, k)) : 0;  // 256-token passes, at most
+    const int64_t o_xp = take(bp * 256 * H * 2);
+    const int64_t o_h2 = take(bp * 256 * I * 4);
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
         ws->status = reinterpret_cast<int *>(b + o_status);
@@ -796,6 +819,7 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
         ws->x_sf = b + o_xs;
         ws->h_terms = b + o_ht;
         ws->h_sf = b + o_hs;
+        ws->bf_pass_start = bf16 ? reinterpret_cast<int32_t *>(b + o_bps) : nullptr;
         ws->x_tiled = bf16 ? b + o_xp : nullptr;
         ws->h_tiled = bf16 ? b + o_h2 : nullptr;
     }
@@ -905,41 +929,45 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     int *clear = clear_status ? ws.status : nullptr;
     const int rows = T * k;
     const int nt = token_tile(T);
-    if (use_bf16_path(T, k)) {  // h on bf16 tensor cores, leaving as bf16 hi, lo terms
-        const Blob bl = blob_parts(prepacked, E, H, I);
-        if (int rc = run_bf16_prep(x, offsets, src_row, k, rows, E, H, ws.pass_start, ws.x_tiled, clear, st))
-            return rc;
-        return run_bf16_stage(true, ws.x_tiled, offsets, ws.pass_start, bl.w13, bl.sf13, rows, E, H, I, ws.h_tiled,
-                              nullptr, ws.status, st);
-    }
-    {
+    const Blob bl = blob_parts(prepacked, E, H, I);
+    if (!use_bf16_path(T, k)) {  // E2M1-term kernel: every expert, or (hybrid) those below kHotRows rows
+        const int hot_rows = use_hybrid(T, k) ? kHotRows : INT_MAX;
         const int64_t warps = (int64_t)rows * ((H + kKC - 1) / kKC);
         const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 8);
         act_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
-                                                                 k, rows, H, nt, ws.x_terms, ws.x_sf, ws.pass_start,
-                                                                 clear);
+                                                                 k, rows, H, nt, hot_rows, ws.x_terms, ws.x_sf,
+                                                                 ws.pass_start, clear);
         if (int rc = check_launch("act_terms_kernel"))
             return rc;
+        clear = nullptr;  // cleared once, before anything could record a timeout
+        FfnParams p{};
+        p.tiles = I / 128;
+        p.K = H;
+        p.rows = rows;
+        p.wsf = bl.sf13;
+        p.asf = ws.x_sf;
+        p.offsets = offsets;
+        p.pass_start = ws.pass_start;
+        p.E = E;
+        p.h_terms = ws.h_terms;
+        p.h_sf = ws.h_sf;
+        p.I = I;
+        p.y_out = nullptr;
+        p.H = H;
+        p.hot_rows = hot_rows;
+        p.status = ws.status;
+        if (int rc = nt == 8 ? launch_ffn<8, true>(bl.w13, ws.x_terms, p, st)
+                             : launch_ffn<16, true>(bl.w13, ws.x_terms, p, st))
+            return rc;
+        if (!use_hybrid(T, k))
+            return MXMOE_OK;
     }
-    const Blob bl = blob_parts(prepacked, E, H, I);
-    FfnParams p{};
-    p.tiles = I / 128;
-    p.K = H;
-    p.rows = rows;
-    p.wsf = bl.sf13;
-    p.asf = ws.x_sf;
-    p.offsets = offsets;
-    p.pass_start = ws.pass_start;
-    p.E = E;
-    p.h_terms = ws.h_terms;
-    p.h_sf = ws.h_sf;
-    p.I = I;
-    p.y_out = nullptr;
-    p.H = H;
-    p.status = ws.status;
-    if (nt == 8)
-        return launch_ffn<8, true>(bl.w13, ws.x_terms, p, st);
-    return launch_ffn<16, true>(bl.w13, ws.x_terms, p, st);
+    // bf16 kernel: every expert, or (hybrid) those with at least kHotRows rows; h leaves as bf16 hi, lo terms
+    if (int rc = run_bf16_prep(x, offsets, src_row, k, rows, E, H, bf16_min_rows(T, k), ws.bf_pass_start,
+                               ws.x_tiled, clear, st))
+        return rc;
+    return run_bf16_stage(true, ws.x_tiled, offsets, ws.bf_pass_start, bl.w13, bl.sf13, rows, E, H, I, ws.h_tiled,
+                          nullptr, ws.status, st);
 }
 
 int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, int E, int H, int I, float *y_perm,
@@ -950,27 +978,31 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
     const int rows = T * k;
     const int nt = token_tile(T);
     const Blob bl = blob_parts(prepacked, E, H, I);
-    if (use_bf16_path(T, k))
-        return run_bf16_stage(false, ws.h_tiled, offsets, ws.pass_start, bl.w2, bl.sf2, rows, E, H, I, nullptr,
-                              y_perm, ws.status, st);
-    FfnParams p{};
-    p.tiles = (int)(pad256(H) / 256);
-    p.K = I;
-    p.rows = rows;
-    p.wsf = bl.sf2;
-    p.asf = ws.h_sf;
-    p.offsets = offsets;
-    p.pass_start = ws.pass_start;
-    p.E = E;
-    p.h_terms = nullptr;
-    p.h_sf = nullptr;
-    p.I = I;
-    p.y_out = y_perm;
-    p.H = H;
-    p.status = ws.status;
-    if (nt == 8)
-        return launch_ffn<8, false>(bl.w2, ws.h_terms, p, st);
-    return launch_ffn<16, false>(bl.w2, ws.h_terms, p, st);
+    if (!use_bf16_path(T, k)) {
+        FfnParams p{};
+        p.tiles = (int)(pad256(H) / 256);
+        p.K = I;
+        p.rows = rows;
+        p.wsf = bl.sf2;
+        p.asf = ws.h_sf;
+        p.offsets = offsets;
+        p.pass_start = ws.pass_start;
+        p.E = E;
+        p.h_terms = nullptr;
+        p.h_sf = nullptr;
+        p.I = I;
+        p.y_out = y_perm;
+        p.H = H;
+        p.hot_rows = use_hybrid(T, k) ? kHotRows : INT_MAX;
+        p.status = ws.status;
+        if (int rc = nt == 8 ? launch_ffn<8, false>(bl.w2, ws.h_terms, p, st)
+                             : launch_ffn<16, false>(bl.w2, ws.h_terms, p, st))
+            return rc;
+        if (!use_hybrid(T, k))
+            return MXMOE_OK;
+    }
+    return run_bf16_stage(false, ws.h_tiled, offsets, ws.bf_pass_start, bl.w2, bl.sf2, rows, E, H, I, nullptr, y_perm,
+                          ws.status, st);
 }
 
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,

@@ -86,14 +86,17 @@ constexpr size_t kPSmem = 1024 + kPOffMisc + 64;
 static_assert(kPSmem <= 232448, "shared memory");
 
 // Token passes of up to 256 rows before each expert: pass_start[e] = sum over
-// e' < e of ceil(n_e' / 256), e = 0 .. E (E <= 1024). One block of 1024
-// threads; also clears the status word.
+// e' < e of ceil(n_e' / 256), e = 0 .. E (E <= 1024), counting only experts
+// with at least min_rows rows (the others run on the E2M1-term kernel). One
+// block of 1024 threads; also clears the status word (when given).
 __global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__restrict__ offsets, int E,
-                                                              int32_t *__restrict__ pass_start, int *status)
+                                                              int min_rows, int32_t *__restrict__ pass_start,
+                                                              int *status)
 {
     __shared__ int32_t s_warp[32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
-    const int c = e < E ? (__ldg(offsets + e + 1) - __ldg(offsets + e) + kPTok - 1) / kPTok : 0;
+    const int n_e = e < E ? __ldg(offsets + e + 1) - __ldg(offsets + e) : 0;
+    const int c = n_e >= min_rows ? (n_e + kPTok - 1) / kPTok : 0;
     int incl = c;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -128,15 +131,18 @@ __global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__r
 // bulk copy brings a whole activation step. Row r of the grouped order (token
 // src_row[r] / k) is row r - offsets[e] - 256 p of pass p of its expert e;
 // rows past an expert's last token are left as they are (the FFN ignores
-// their columns). One warp per row.
+// their columns). Rows of experts with fewer than min_rows rows are skipped.
+// One warp per row.
 __global__ void __launch_bounds__(256) x_tile_kernel(const uint16_t *__restrict__ x,
                                                      const int32_t *__restrict__ src_row,
                                                      const int32_t *__restrict__ offsets,
-                                                     const int32_t *__restrict__ pass_start, int E, int k, int rows,
-                                                     int H, uint8_t *__restrict__ x_tiled)
+                                                     const int32_t *__restrict__ pass_start, int E, int min_rows,
+                                                     int k, int rows, int H, uint8_t *__restrict__ x_tiled)
 {
     const int lane = threadIdx.x & 31;
     const int nks = H / kPK;
+    if (__ldg(pass_start + E) == 0)  // no expert for the bf16 kernel
+        return;
     for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
         int lo = 0, hi = E;  // expert of row r: largest e with offsets[e] <= r
         while (hi - lo > 1) {
@@ -147,6 +153,8 @@ __global__ void __launch_bounds__(256) x_tile_kernel(const uint16_t *__restrict_
                 hi = mid;
         }
         const int local = r - __ldg(offsets + lo);
+        if (__ldg(offsets + lo + 1) - __ldg(offsets + lo) < min_rows)
+            continue;
         const int64_t pass = __ldg(pass_start + lo) + local / kPTok;
         const int m = local % kPTok;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(__ldg(src_row + r) / k) * H);
@@ -295,6 +303,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     ffn_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const PrefillParams p)
 {
     constexpr int NB = GATE_UP ? 1 : 2;  // activation steps per K step: x, or h's hi then lo
+    if (__ldg(p.pass_start + p.E) == 0)  // no expert for this kernel (the E2M1-term kernel took them all)
+        return;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem, *sA = smem + kPOffA, *sW = smem + kPOffW, *sSf = smem + kPOffSf;
@@ -627,23 +637,29 @@ int launch_bf16_stage(const CUtensorMap &tmW, const PrefillParams &p, cudaStream
 
 }  // namespace
 
-// Upper bound on the 256-token passes of `rows` grouped rows over E experts:
-// sum of ceil(n_e / 256) <= rows / 256 + E. Sizes the tiled activations.
-int64_t bf16_max_passes(int64_t rows, int E) { return (rows + kPTok - 1) / kPTok + E; }
-
-// Before the gate/up stage: the passes before each expert (pass_start, E + 1
-// ints), then x tiled per (pass, K step) into x_tiled
-// (bf16_max_passes(rows, E) * 256 * H * 2 bytes); clears the status word.
-// E <= 1024 (every accepted shape).
-int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
-                  int32_t *pass_start, uint8_t *x_tiled, int *status, cudaStream_t st)
+// Upper bound on the 256-token passes of `rows` grouped rows over E experts
+// when only experts with at least min_rows rows count: sum of ceil(n_e / 256)
+// <= rows / 256 + (number of such experts). Sizes the tiled activations.
+int64_t bf16_max_passes(int64_t rows, int E, int min_rows)
 {
-    prefill_passes_kernel<<<1, 1024, 0, st>>>(offsets, E, pass_start, status);
+    const int64_t experts = min_rows > 0 ? std::min<int64_t>(E, rows / min_rows) : E;
+    return (rows + kPTok - 1) / kPTok + experts;
+}
+
+// Before the gate/up stage: the passes before each expert with at least
+// min_rows rows (pass_start, E + 1 ints), then those experts' x rows tiled per
+// (pass, K step) into x_tiled (bf16_max_passes(rows, E, min_rows) * 256 * H *
+// 2 bytes); clears the status word when status is given. E <= 1024 (every
+// accepted shape).
+int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
+                  int min_rows, int32_t *pass_start, uint8_t *x_tiled, int *status, cudaStream_t st)
+{
+    prefill_passes_kernel<<<1, 1024, 0, st>>>(offsets, E, min_rows, pass_start, status);
     if (int rc = check_launch("prefill_passes_kernel"))
         return rc;
     const int blocks = (int)std::min<int64_t>(((int64_t)rows + 7) / 8, (int64_t)num_sms() * 8);
     x_tile_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets,
-                                                           pass_start, E, k, rows, H, x_tiled);
+                                                           pass_start, E, min_rows, k, rows, H, x_tiled);
     return check_launch("x_tile_kernel");
 }
 

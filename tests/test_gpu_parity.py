@@ -157,6 +157,8 @@ FFN_CASES = [
     (1024, 128, 2, 2, 1),     # one token: 7 of the 8 pass rows unused
     (1024, 1024, 64, 4, 64),  # more items than SMs in both stages
     (1024, 512, 64, 8, 8),    # ~180 items of one pass each
+    (256, 128, 12, 2, 800),   # ~133 rows per expert: hybrid, experts above 128 rows on the bf16 kernel
+    (640, 384, 10, 2, 640),   # hybrid with ragged H and I: ~128 rows per expert, either side of the cut
     (256, 128, 7, 2, 8192),   # 16384 grouped rows: both stages on bf16 tensor cores, ragged passes
     (640, 384, 5, 2, 8192),   # bf16 path with 3 gate/up boxes, a half-real down box and half K chunks
 ]
