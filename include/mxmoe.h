@@ -155,6 +155,19 @@ MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, int32_t *ids
 MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
                             int32_t *dst_of, void *stream);
 
+/* mxmoe_permute for many pairs, with caller scratch: the same outputs (bit for
+ * bit) from a multi-block grouping when T*k > 4096 and E <= 1024 (otherwise it
+ * runs mxmoe_permute's kernel and leaves the scratch alone).
+ *   scratch device, >= mxmoe_permute_scratch_size(T, k, E) bytes, 16-byte
+ *   aligned, contents not kept between calls.
+ * Errors: those of mxmoe_permute; scratch NULL or too small ->
+ * WORKSPACE. */
+MXMOE_API int mxmoe_permute_ws(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
+                               int32_t *dst_of, void *scratch, int64_t scratch_bytes, void *stream);
+
+/* Scratch bytes for mxmoe_permute_ws (-1 on bad sizes). */
+MXMOE_API int64_t mxmoe_permute_scratch_size(int T, int k, int E);
+
 /* ------------------------------------------------------------------------ */
 /* Experts                                                                   */
 /* ------------------------------------------------------------------------ */
@@ -184,9 +197,13 @@ MXMOE_API int mxmoe_expert_ffn(const void *x, const int32_t *offsets, const int3
                                int64_t workspace_bytes, void *stream);
 
 /* Stage 1 of mxmoe_expert_ffn on its own: for every grouped position r,
- * h[r] = silu(W_gate[e] x_t) * (W_up[e] x_t), written into the workspace (as
- * three E4M3 terms with one scale per 32 values) for mxmoe_ffn_down. Arguments, layout and errors as for mxmoe_expert_ffn
- * (workspace from mxmoe_ffn_workspace_size, 256-byte aligned). */
+ * h[r] = silu(W_gate[e] x_t) * (W_up[e] x_t), written into the workspace for
+ * mxmoe_ffn_down: as 8 E2M1 digit terms per value with their scale images,
+ * or, for experts that the bf16 tensor-core kernel takes (every expert from
+ * 16384 grouped rows; from 128 tokens, experts with at least 128 rows), as
+ * bf16 hi + lo (within 2^-15 of h) in the tiled layout that kernel reads.
+ * Arguments, layout and errors as for mxmoe_expert_ffn (workspace from
+ * mxmoe_ffn_workspace_size, 256-byte aligned). */
 MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked,
                                 int T, int k, int E, int H, int I, void *workspace, int64_t workspace_bytes,
                                 void *stream);
@@ -249,6 +266,16 @@ MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, int k);
 MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, const float *bias, const void *prepacked, int T,
                                   int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out,
                                   void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Test of the device-side timeout path (failure detection): one thread waits
+ * on a shared-memory mbarrier that nothing ever arrives on, through the same
+ * bounded wait that every wait of the FFN and router kernels uses, with a
+ * limit of limit_us microseconds, then writes MXMOE_ERR_TIMEOUT to *status
+ * (MXMOE_OK if the wait had completed) and the kernel returns normally, so the
+ * context stays usable. No counterpart on the pages.
+ *   status device int; limit_us 1 .. 1000000.
+ * Errors: status NULL -> NULL; limit_us out of range -> INVALID_SHAPE. */
+MXMOE_API int mxmoe_selftest_wait_timeout(int *status, int limit_us, void *stream);
 
 /* Synchronise `stream`, then read the device status word that the last
  * mxmoe_expert_ffn / mxmoe_layer_forward call on this workspace left:

@@ -51,6 +51,9 @@ _SIGS = {
     "mxmoe_workspace_size": (_I64, [_I, _I, _I, _I, _I]),
     "mxmoe_layer_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
     "mxmoe_read_status": (_I, [_P, _P, _P]),
+    "mxmoe_selftest_wait_timeout": (_I, [_P, _I, _P]),
+    "mxmoe_permute_ws": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
+    "mxmoe_permute_scratch_size": (_I64, [_I, _I, _I]),
 }
 
 _lib = None
@@ -324,6 +327,34 @@ def mxmoe_read_status(workspace, stream=None) -> int:
     st = ctypes.c_int(-1)
     _check("mxmoe_read_status", load().mxmoe_read_status(_ptr(workspace), ctypes.byref(st), _stream(stream)))
     return st.value
+
+
+def mxmoe_permute_scratch_size(T, k, E) -> int:
+    return int(load().mxmoe_permute_scratch_size(T, k, E))
+
+
+def mxmoe_permute_ws(ids, E, offsets, src_row, dst_of, scratch, stream=None):
+    """mxmoe_permute with caller scratch (the multi-block grouping for many pairs)."""
+    import torch
+
+    T, k = ids.shape
+    _need(ids, torch.int32, (T, k), "ids")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(src_row, torch.int32, (T * k,), "src_row")
+    _need(dst_of, torch.int32, (T * k,), "dst_of")
+    _check("mxmoe_permute_ws",
+           load().mxmoe_permute_ws(_ptr(ids), T, k, E, _ptr(offsets), _ptr(src_row), _ptr(dst_of), _ptr(scratch),
+                                   scratch.numel() * scratch.element_size(), _stream(stream)))
+
+
+def mxmoe_selftest_wait_timeout(status, limit_us: int, stream=None) -> None:
+    """Make one bounded device-side wait run out (nothing arrives on its
+    barrier); status (device int32 [1]) receives MXMOE_ERR_TIMEOUT."""
+    import torch
+
+    _need(status, torch.int32, (1,), "status")
+    _check("mxmoe_selftest_wait_timeout",
+           load().mxmoe_selftest_wait_timeout(_ptr(status), int(limit_us), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

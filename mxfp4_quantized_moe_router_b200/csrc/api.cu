@@ -85,6 +85,9 @@ int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int 
 int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
 int router_splits(int T, int H, int E);
+int64_t permute_scratch_ints(int n, int E);
+int run_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row, int32_t *dst_of,
+                int32_t *scratch, cudaStream_t st);
 int run_router_and_route(const void *x, const void *wg, const float *bias, int T, int H, int E, int k,
                          float *partials, int nsplit, int32_t *ids, float *w, int *status, cudaStream_t st);
 
@@ -98,6 +101,7 @@ struct LayerWs {
     int32_t *ids;
     float *w;
     int32_t *offsets, *src_row, *dst_of;
+    int32_t *permute_scratch;
     float *y_perm;
 };
 
@@ -117,6 +121,7 @@ int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *ba
     const int64_t o_off = take((int64_t)(E + 1) * 4);
     const int64_t o_src = take(n * 4);
     const int64_t o_dst = take(n * 4);
+    const int64_t o_pm = take(permute_scratch_ints((int)n, E) * 4);
     const int64_t o_yp = take(n * H * 4);
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
@@ -127,6 +132,7 @@ int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *ba
         ws->offsets = reinterpret_cast<int32_t *>(b + o_off);
         ws->src_row = reinterpret_cast<int32_t *>(b + o_src);
         ws->dst_of = reinterpret_cast<int32_t *>(b + o_dst);
+        ws->permute_scratch = reinterpret_cast<int32_t *>(b + o_pm);
         ws->y_perm = reinterpret_cast<float *>(b + o_yp);
     }
     return off;
@@ -183,11 +189,42 @@ extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, cons
     if (int rc = run_router_and_route(x, wg, bias, T, H, E, k, ws.logits, router_splits(T, H, E), ids, w, status,
                                       st))
         return rc;
-    if (int rc = mxmoe_permute(ids, T, k, E, ws.offsets, ws.src_row, ws.dst_of, stream))
+    if (int rc = run_permute(ids, T, k, E, ws.offsets, ws.src_row, ws.dst_of, ws.permute_scratch, st))
         return rc;
     if (int rc = run_expert_ffn(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn, false, st))
         return rc;
     return run_combine(ws.y_perm, ws.dst_of, w, T, k, H, y, st);
+}
+
+namespace mxmoe {
+namespace {
+// One thread waits on an mbarrier that nothing arrives on (phase 0 of a fresh
+// barrier with one expected arrival never completes) until the bounded wait
+// gives up.
+__global__ void wait_timeout_kernel(int *status, uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        *status = mbar_wait_bounded(&bar, 0, limit_ns) ? MXMOE_OK : MXMOE_ERR_TIMEOUT;
+}
+}  // namespace
+}  // namespace mxmoe
+
+extern "C" MXMOE_API int mxmoe_selftest_wait_timeout(int *status, int limit_us, void *stream)
+{
+    if (!status)
+        return fail(MXMOE_ERR_NULL, "mxmoe_selftest_wait_timeout: NULL status");
+    if (limit_us < 1 || limit_us > 1000000)
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_selftest_wait_timeout: limit_us=%d (1 .. 1000000)", limit_us);
+    if (int rc = check_device())
+        return rc;
+    wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(status, (uint64_t)limit_us * 1000ull);
+    return check_launch("wait_timeout_kernel");
 }
 
 extern "C" MXMOE_API int mxmoe_read_status(const void *workspace, int *status, void *stream)

@@ -310,6 +310,142 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict
     }
 }
 
+// ---------------------------------------------------------------------------
+// Multi-block stable grouping (many pairs; E <= 1024): the same result as
+// permute_kernel from three launches over blocks of 1024 pairs.
+//  1. permute_count_kernel: pairs of block b per expert -> counts[e][b].
+//  2. permute_scan_kernel: block e turns counts[e][.] into its exclusive
+//     prefix over blocks and writes the expert's total.
+//  3. permute_scatter_kernel: each block scans the totals into the expert
+//     offsets (block 0 writes them) and places its pairs: position =
+//     offset[e] + pairs of e in earlier blocks + earlier pairs of e in this
+//     block (warp match, then warps in order), so the order within an expert
+//     stays ascending.
+// ---------------------------------------------------------------------------
+constexpr int kPmBlock = 1024;
+
+__global__ void __launch_bounds__(kPmBlock) permute_count_kernel(const int32_t *__restrict__ ids, int n, int E,
+                                                                 int32_t *__restrict__ counts)
+{
+    extern __shared__ int32_t cnt[];  // [E]
+    const int tid = threadIdx.x, nb = gridDim.x;
+    for (int e = tid; e < E; e += kPmBlock)
+        cnt[e] = 0;
+    __syncthreads();
+    const int p = blockIdx.x * kPmBlock + tid;
+    if (p < n)
+        atomicAdd(&cnt[min(max(ids[p], 0), E - 1)], 1);
+    __syncthreads();
+    for (int e = tid; e < E; e += kPmBlock)
+        counts[(int64_t)e * nb + blockIdx.x] = cnt[e];
+}
+
+// Exclusive scan of v over the block's 1024 threads; returns the prefix and
+// puts the block total in *total (shared scratch s_warp[32]).
+__device__ __forceinline__ int block_excl_scan_1024(int v, int32_t *s_warp, int *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off)
+            incl += o;
+    }
+    if (lane == 31)
+        s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int w = s_warp[lane];
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xFFFFFFFFu, wi, off);
+            if (lane >= off)
+                wi += o;
+        }
+        s_warp[lane] = wi - w;
+        if (lane == 31)
+            s_warp[32] = wi;
+    }
+    __syncthreads();
+    const int r = s_warp[warp] + incl - v;
+    *total = s_warp[32];
+    __syncthreads();  // s_warp free again
+    return r;
+}
+
+__global__ void __launch_bounds__(kPmBlock) permute_scan_kernel(int32_t *__restrict__ counts, int nb,
+                                                                int32_t *__restrict__ totals)
+{
+    __shared__ int32_t s_warp[33];
+    int32_t *c = counts + (int64_t)blockIdx.x * nb;
+    int carry = 0;
+    for (int base = 0; base < nb; base += kPmBlock) {
+        const int i = base + threadIdx.x;
+        const int v = i < nb ? c[i] : 0;
+        int tot;
+        const int ex = block_excl_scan_1024(v, s_warp, &tot);
+        if (i < nb)
+            c[i] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0)
+        totals[blockIdx.x] = carry;
+}
+
+__global__ void __launch_bounds__(kPmBlock) permute_scatter_kernel(const int32_t *__restrict__ ids, int n, int E,
+                                                                   const int32_t *__restrict__ counts,
+                                                                   const int32_t *__restrict__ totals,
+                                                                   int32_t *__restrict__ offsets,
+                                                                   int32_t *__restrict__ src_row,
+                                                                   int32_t *__restrict__ dst_of)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *base_e = sm;      // [E]: first position of this block's pairs of expert e
+    int32_t *wcnt = sm + E;    // [32][E]: per warp, then exclusive over warps
+    __shared__ int32_t s_warp[33];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nb = gridDim.x;
+    {  // expert offsets: exclusive scan of the totals (E <= 1024: one expert per thread)
+        const int t = tid < E ? totals[tid] : 0;
+        int all;
+        const int off = block_excl_scan_1024(t, s_warp, &all);
+        if (tid < E) {
+            base_e[tid] = off + counts[(int64_t)tid * nb + blockIdx.x];
+            if (blockIdx.x == 0)
+                offsets[tid] = off;
+        }
+        if (blockIdx.x == 0 && tid == 0)
+            offsets[E] = all;
+    }
+    for (int i = tid; i < 32 * E; i += kPmBlock)
+        wcnt[i] = 0;
+    __syncthreads();
+    const int p = blockIdx.x * kPmBlock + tid;
+    const bool valid = p < n;
+    const int e = valid ? min(max(ids[p], 0), E - 1) : -1;
+    const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid);
+    const uint32_t same = __match_any_sync(0xFFFFFFFFu, e) & vmask;
+    const int in_warp = __popc(same & ((1u << lane) - 1u));
+    if (valid && in_warp == 0)
+        wcnt[warp * E + e] = __popc(same);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += kPmBlock) {  // exclusive over warps, per expert
+        int run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int c = wcnt[w * E + ee];
+            wcnt[w * E + ee] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    if (valid) {
+        const int pos = base_e[e] + wcnt[warp * E + e] + in_warp;
+        src_row[pos] = p;
+        dst_of[p] = pos;
+    }
+}
+
 }  // namespace
 }  // namespace mxmoe
 
@@ -398,6 +534,44 @@ extern "C" MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, i
     return launch_route(logits, 1, nullptr, T, E, k, ids, w, (cudaStream_t)stream);
 }
 
+namespace mxmoe {
+
+// Scratch ints of the multi-block grouping: counts [E][blocks] + totals [E].
+int64_t permute_scratch_ints(int n, int E) { return (int64_t)E * ((n + kPmBlock - 1) / kPmBlock) + E; }
+bool use_multiblock_permute(int n, int E) { return n > 4 * kPmBlock && E <= kPmBlock; }
+
+// The layer path's grouping: the multi-block kernels when use_multiblock_permute
+// (scratch: permute_scratch_ints(n, E) ints), else permute_kernel.
+int run_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row, int32_t *dst_of,
+                int32_t *scratch, cudaStream_t st)
+{
+    const int n = T * k;
+    if (!use_multiblock_permute(n, E) || !scratch)
+        return mxmoe_permute(ids, T, k, E, offsets, src_row, dst_of, st);
+    const int nb = (n + kPmBlock - 1) / kPmBlock;
+    int32_t *counts = scratch, *totals = scratch + (int64_t)E * nb;
+    const size_t smem_scatter = (size_t)33 * E * sizeof(int32_t);
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(33 * kPmBlock * sizeof(int32_t))) != cudaSuccess)
+            return fail(MXMOE_ERR_CUDA, "permute_scatter_kernel: cannot reserve shared memory");
+        configured_dev = dev;
+    }
+    permute_count_kernel<<<nb, kPmBlock, E * sizeof(int32_t), st>>>(ids, n, E, counts);
+    if (int rc = check_launch("permute_count_kernel"))
+        return rc;
+    permute_scan_kernel<<<E, kPmBlock, 0, st>>>(counts, nb, totals);
+    if (int rc = check_launch("permute_scan_kernel"))
+        return rc;
+    permute_scatter_kernel<<<nb, kPmBlock, smem_scatter, st>>>(ids, n, E, counts, totals, offsets, src_row, dst_of);
+    return check_launch("permute_scatter_kernel");
+}
+
+}  // namespace mxmoe
+
 extern "C" MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
                                        int32_t *dst_of, void *stream)
 {
@@ -417,4 +591,28 @@ extern "C" MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, 
     }
     permute_kernel<<<1, 1024, smem, (cudaStream_t)stream>>>(ids, T * k, E, offsets, src_row, dst_of);
     return check_launch("permute_kernel");
+}
+
+extern "C" MXMOE_API int64_t mxmoe_permute_scratch_size(int T, int k, int E)
+{
+    if (T < 0 || k < 1 || E <= 0 || E > 4096 || (int64_t)T * k > (1 << 24))
+        return -1;
+    return permute_scratch_ints(T * k, E) * (int64_t)sizeof(int32_t);
+}
+
+extern "C" MXMOE_API int mxmoe_permute_ws(const int32_t *ids, int T, int k, int E, int32_t *offsets,
+                                          int32_t *src_row, int32_t *dst_of, void *scratch, int64_t scratch_bytes,
+                                          void *stream)
+{
+    if (T < 0 || k < 1 || E <= 0 || E > 4096 || (int64_t)T * k > (1 << 24))
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_permute_ws: T=%d k=%d E=%d", T, k, E);
+    if (!scratch || scratch_bytes < mxmoe_permute_scratch_size(T, k, E))
+        return fail(MXMOE_ERR_WORKSPACE, "mxmoe_permute_ws: scratch of %lld bytes, need %lld",
+                    (long long)scratch_bytes, (long long)mxmoe_permute_scratch_size(T, k, E));
+    if (!offsets || (T > 0 && (!ids || !src_row || !dst_of)))
+        return fail(MXMOE_ERR_NULL, "mxmoe_permute_ws: NULL pointer");
+    if (int rc = check_device())
+        return rc;
+    return run_permute(ids, T, k, E, offsets, src_row, dst_of, static_cast<int32_t *>(scratch),
+                       (cudaStream_t)stream);
 }

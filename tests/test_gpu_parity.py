@@ -124,6 +124,28 @@ def test_permute_bitexact(mx, T, k, E):
     assert np.array_equal(dst.cpu().numpy(), dst_ref)
 
 
+@pytest.mark.parametrize("T,k,E,skew", [(1024, 8, 384, False), (8192, 8, 384, False), (3001, 7, 1000, False),
+                                        (4097, 1, 16, False), (6000, 8, 384, True)])
+def test_permute_ws_bitexact(mx, T, k, E, skew):
+    # the multi-block grouping (more than 4096 pairs), ragged last block, one-pair-per-token, hot experts
+    if skew:
+        rng = np.random.default_rng(5)
+        hot = rng.choice(E, 6, replace=False)
+        ids_np = np.stack([np.concatenate([hot[:3], rng.choice(np.setdiff1d(np.arange(E), hot[:3]), k - 3, False)])
+                           for _ in range(T)]).astype(np.int32)
+    else:
+        ids_np = datagen.make_ids(T, E, k, seed=T + 3)
+    off_ref, src_ref, dst_ref = oracle.permute(ids_np, E)
+    scratch = torch.empty(mx.mxmoe_permute_scratch_size(T, k, E), dtype=torch.uint8, device=DEV)
+    off = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    src = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    dst = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    mx.mxmoe_permute_ws(torch.from_numpy(ids_np).to(DEV), E, off, src, dst, scratch)
+    assert np.array_equal(off.cpu().numpy(), off_ref)
+    assert np.array_equal(src.cpu().numpy(), src_ref)
+    assert np.array_equal(dst.cpu().numpy(), dst_ref)
+
+
 def test_permute_skewed(mx):
     T, k, E = 1500, 8, 384
     rng = np.random.default_rng(1)

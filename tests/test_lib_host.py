@@ -122,3 +122,11 @@ def test_cpu_only_box_reports_no_device(mx):
     base = (ctypes.addressof(buf) + 15) & ~15
     rc = lib.mxmoe_quantize(base, 4, 32, base, base, None)
     assert rc in (mx.ERR_CUDA, mx.ERR_DEVICE)
+
+
+def test_timeout_selftest_rejects_on_host(mx):
+    lib = mx.load()
+    base = 1 << 20  # never dereferenced: rejected before anything is enqueued
+    assert lib.mxmoe_selftest_wait_timeout(None, 1000, None) == mx.ERR_NULL
+    assert lib.mxmoe_selftest_wait_timeout(base, 0, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_selftest_wait_timeout(base, 1000001, None) == mx.ERR_INVALID_SHAPE
