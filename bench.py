@@ -41,11 +41,24 @@ UNIT = "tokens/s"
 BF16_PATH_ROWS = 16384  # grouped rows (tokens x top-k) from which both FFN stages run on bf16 tensor cores
 
 
-def kernels_per_step(rows: int) -> int:
-    """Launches of one layer step: router_gemm, route, permute, then x_terms +
-    the two E2M1-term FFN stages, or (bf16 path) passes + x_tile + the two bf16
-    stages, then combine."""
-    return 8 if rows >= BF16_PATH_ROWS else 7
+def kernels_per_step(T: int, k: int, E: int, H: int) -> int:
+    """Kernels one layer step launches, following the library's dispatch:
+    router GEMM (one kernel either way), route, grouping (one kernel, or three
+    above 4096 pairs with E <= 1024), then the FFN -- E2M1-term path:
+    x_terms + two stages; bf16 path: passes + slot rows + x_tile + two stages;
+    both from 128 tokens below 16384 grouped rows -- then combine."""
+    rows = T * k
+    n = 3 if (rows > 4096 and E <= 1024) else 1
+    n += 2  # router GEMM, route
+    bf16_all = rows >= BF16_PATH_ROWS
+    hybrid = not bf16_all and T >= 128
+    if not bf16_all:
+        n += 3
+    if bf16_all or hybrid:
+        n += 5
+    return n + 1  # combine
+
+
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -492,7 +505,7 @@ def run_native(args):
         "touched_experts_per_step": mean_touched,
         "roofline": roofline,
         "clocks": clk,
-        "gpu_launches": kernels_per_step(T * k) * args.steps,
+        "gpu_launches": kernels_per_step(T, k, E, H) * args.steps,
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
                 "d2h_bytes_per_step": T * H * 4, "api": "mxmoe_layer_forward with pinned host x/y copies"},
     }

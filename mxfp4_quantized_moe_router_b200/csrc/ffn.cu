@@ -53,7 +53,8 @@
 
 namespace mxmoe {
 int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
-                  int min_rows, int32_t *pass_start, uint8_t *x_tiled, int *status, cudaStream_t st);
+                  int min_rows, int32_t *pass_start, int32_t *slot_row, uint8_t *x_tiled, int *status,
+                  cudaStream_t st);
 int run_bf16_stage(bool gate_up, const uint8_t *act_tiled, const int32_t *offsets, const int32_t *pass_start,
                    const uint8_t *w, const uint8_t *sf, int rows, int E, int H, int I, uint8_t *h_tiled, float *y,
                    int *status, cudaStream_t st);
@@ -768,6 +769,7 @@ struct FfnWs {
     uint8_t *h_terms;     // term_offset layout, K = I
     uint8_t *h_sf;        // scale images [pass][I/128][512]
     int32_t *bf_pass_start;  // bf16 kernel: its 256-token passes before each expert [kMaxE + 1]
+    int32_t *slot_row;    // bf16 kernel: grouped row of each (token, slot) [rows]
     uint8_t *x_tiled;     // bf16 kernel: x per (pass, K step) as the shared-memory image
     uint8_t *h_tiled;     // bf16 kernel: h hi, lo per (pass, K step, term) likewise
 };
@@ -808,6 +810,7 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
     const int64_t o_ht = take(terms ? rows * kT * pad256(I) / 2 : 0);
     const int64_t o_hs = take(terms ? passes * (I / 128) * kSFImg : 0);
     const int64_t o_bps = take(bf16 ? (kMaxE + 1) * 4 : 0);
+    const int64_t o_sr = take(bf16 ? rows * 4 : 0);
     const int64_t bp = bf16 ? bf16_max_passes(rows, E, bf16_min_rows(T, k)) : 0;  // 256-token passes, at most
     const int64_t o_xp = take(bp * 256 * H * 2);
     const int64_t o_h2 = take(bp * 256 * I * 4);
@@ -820,6 +823,7 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
         ws->h_terms = b + o_ht;
         ws->h_sf = b + o_hs;
         ws->bf_pass_start = bf16 ? reinterpret_cast<int32_t *>(b + o_bps) : nullptr;
+        ws->slot_row = bf16 ? reinterpret_cast<int32_t *>(b + o_sr) : nullptr;
         ws->x_tiled = bf16 ? b + o_xp : nullptr;
         ws->h_tiled = bf16 ? b + o_h2 : nullptr;
     }
@@ -964,7 +968,7 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     }
     // bf16 kernel: every expert, or (hybrid) those with at least kHotRows rows; h leaves as bf16 hi, lo terms
     if (int rc = run_bf16_prep(x, offsets, src_row, k, rows, E, H, bf16_min_rows(T, k), ws.bf_pass_start,
-                               ws.x_tiled, clear, st))
+                               ws.slot_row, ws.x_tiled, clear, st))
         return rc;
     return run_bf16_stage(true, ws.x_tiled, offsets, ws.bf_pass_start, bl.w13, bl.sf13, rows, E, H, I, ws.h_tiled,
                           nullptr, ws.status, st);

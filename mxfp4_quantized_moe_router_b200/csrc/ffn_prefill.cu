@@ -125,44 +125,71 @@ __global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__r
         *status = 0;
 }
 
+// slot_row[src_row[r]] = r: the grouped row of each (token, slot) pair.
+__global__ void __launch_bounds__(256) slot_rows_kernel(const int32_t *__restrict__ src_row, int rows,
+                                                        int32_t *__restrict__ slot_row)
+{
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x)
+        slot_row[__ldg(src_row + r)] = r;
+}
+
 // x rows in grouped order, tiled as the bf16 stage reads them: the block of
 // (pass, K step) holds the pass's 256 rows x 64 values in the 128-byte
 // swizzle (16-byte chunk c of row m at chunk c ^ (m % 8)), 32 KB, so that one
-// bulk copy brings a whole activation step. Row r of the grouped order (token
-// src_row[r] / k) is row r - offsets[e] - 256 p of pass p of its expert e;
-// rows past an expert's last token are left as they are (the FFN ignores
-// their columns). Rows of experts with fewer than min_rows rows are skipped.
-// One warp per row.
+// bulk copy brings a whole activation step. Grouped row r of expert e is row
+// r - offsets[e] - 256 p of pass p of e; rows past an expert's last token are
+// left as they are (the FFN ignores their columns), and rows of experts with
+// fewer than min_rows rows are skipped. One warp per token: lane j < k finds
+// where the token's slot j goes, then the warp reads x[t] once and writes it
+// to every such place.
+constexpr int kTileMaxK = 32;
+
 __global__ void __launch_bounds__(256) x_tile_kernel(const uint16_t *__restrict__ x,
-                                                     const int32_t *__restrict__ src_row,
+                                                     const int32_t *__restrict__ slot_row,
                                                      const int32_t *__restrict__ offsets,
                                                      const int32_t *__restrict__ pass_start, int E, int min_rows,
-                                                     int k, int rows, int H, uint8_t *__restrict__ x_tiled)
+                                                     int k, int T, int H, uint8_t *__restrict__ x_tiled)
 {
-    const int lane = threadIdx.x & 31;
+    __shared__ int64_t s_dst[8][kTileMaxK];  // per warp: byte offset of slot j's row in x_tiled, or -1
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int nks = H / kPK;
     if (__ldg(pass_start + E) == 0)  // no expert for the bf16 kernel
         return;
-    for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
-        int lo = 0, hi = E;  // expert of row r: largest e with offsets[e] <= r
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (__ldg(offsets + mid) <= r)
-                lo = mid;
-            else
-                hi = mid;
+    for (int t = blockIdx.x * 8 + wl; t < T; t += gridDim.x * 8) {
+        if (lane < k) {
+            const int r = __ldg(slot_row + (int64_t)t * k + lane);
+            int lo = 0, hi = E;  // expert of row r: largest e with offsets[e] <= r
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (__ldg(offsets + mid) <= r)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            const int local = r - __ldg(offsets + lo);
+            int64_t d = -1;
+            if (__ldg(offsets + lo + 1) - __ldg(offsets + lo) >= min_rows) {
+                const int64_t pass = __ldg(pass_start + lo) + local / kPTok;
+                const int m = local % kPTok;
+                d = (pass * nks * kPTok + m) * 128 + m % 8;  // m % 8 rides along for the swizzle
+            }
+            s_dst[wl][lane] = d;
         }
-        const int local = r - __ldg(offsets + lo);
-        if (__ldg(offsets + lo + 1) - __ldg(offsets + lo) < min_rows)
-            continue;
-        const int64_t pass = __ldg(pass_start + lo) + local / kPTok;
-        const int m = local % kPTok;
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(__ldg(src_row + r) / k) * H);
-        uint8_t *dst = x_tiled + (pass * nks * kPTok + m) * 128;
+        __syncwarp();
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)t * H);
         for (int c8 = lane; c8 < H / 8; c8 += 32) {  // 16-byte chunk c8: K step c8 / 8, chunk c8 % 8
+            const uint4 v = __ldg(src + c8);
             const int c = c8 & 7;
-            *reinterpret_cast<uint4 *>(dst + (int64_t)(c8 >> 3) * kPBBytes + ((c ^ (m & 7)) << 4)) = __ldg(src + c8);
+            const int64_t step = (int64_t)(c8 >> 3) * kPBBytes;
+            for (int j = 0; j < k; ++j) {
+                const int64_t d = s_dst[wl][j];
+                if (d >= 0) {
+                    const int64_t row = d & ~int64_t(7);
+                    *reinterpret_cast<uint4 *>(x_tiled + row + step + ((c ^ (int)(d & 7)) << 4)) = v;
+                }
+            }
         }
+        __syncwarp();
     }
 }
 
@@ -649,17 +676,26 @@ int64_t bf16_max_passes(int64_t rows, int E, int min_rows)
 // Before the gate/up stage: the passes before each expert with at least
 // min_rows rows (pass_start, E + 1 ints), then those experts' x rows tiled per
 // (pass, K step) into x_tiled (bf16_max_passes(rows, E, min_rows) * 256 * H *
-// 2 bytes); clears the status word when status is given. E <= 1024 (every
-// accepted shape).
+// 2 bytes), through slot_row (rows ints: the grouped row of each (token,
+// slot)); clears the status word when status is given. E <= 1024 and
+// k <= 32 (every accepted shape).
 int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
-                  int min_rows, int32_t *pass_start, uint8_t *x_tiled, int *status, cudaStream_t st)
+                  int min_rows, int32_t *pass_start, int32_t *slot_row, uint8_t *x_tiled, int *status,
+                  cudaStream_t st)
 {
     prefill_passes_kernel<<<1, 1024, 0, st>>>(offsets, E, min_rows, pass_start, status);
     if (int rc = check_launch("prefill_passes_kernel"))
         return rc;
-    const int blocks = (int)std::min<int64_t>(((int64_t)rows + 7) / 8, (int64_t)num_sms() * 8);
-    x_tile_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets,
-                                                           pass_start, E, min_rows, k, rows, H, x_tiled);
+    {
+        const int blocks = (int)std::min<int64_t>(((int64_t)rows + 255) / 256, (int64_t)num_sms() * 4);
+        slot_rows_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(src_row, rows, slot_row);
+        if (int rc = check_launch("slot_rows_kernel"))
+            return rc;
+    }
+    const int T = rows / k;
+    const int blocks = (int)std::min<int64_t>(((int64_t)T + 7) / 8, (int64_t)num_sms() * 8);
+    x_tile_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), slot_row, offsets,
+                                                           pass_start, E, min_rows, k, T, H, x_tiled);
     return check_launch("x_tile_kernel");
 }
 

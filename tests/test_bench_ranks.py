@@ -86,3 +86,16 @@ def test_reference_arm_does_no_work_off_rank_zero():
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
     assert p.returncode == 0, p.stderr
     assert p.stdout.strip() == ""
+
+
+def test_bench_parses_its_arguments():
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True, text=True,
+                       timeout=120)
+    assert p.returncode == 0, p.stderr
+    assert "--steps" in p.stdout
+
+
+def test_launch_count_follows_the_dispatch():
+    # verify8: one grouping kernel, E2M1-term FFN; verify256: hybrid; zipf1024: hybrid + multi-block grouping;
+    # prefill8192: bf16 FFN + multi-block grouping
+    assert [bench.kernels_per_step(T, 8, 384, 6144) for T in (8, 256, 1024, 8192)] == [7, 12, 14, 11]
