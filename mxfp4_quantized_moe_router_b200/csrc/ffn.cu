@@ -222,14 +222,17 @@ __device__ __forceinline__ uint32_t e2m1_digit_code(int d)  // d in [-4, 4]
 
 __device__ __forceinline__ void act_digits(float v, int E, uint32_t (&code)[kT])
 {
-    int iv = (int)rintf(v * pow2f(22 - E));  // |iv| <= 2^23
+    const int iv = (int)rintf(v * pow2f(22 - E));  // |iv| <= 2^23
+    // Balanced base-8 digits: the 7 low ones in [-4, 3], the top one in
+    // [-4, 4]. Adding 4 at each of the 7 low positions turns the low digits
+    // into plain base-8 digits d + 4 (no carries), and what is left above
+    // them (an arithmetic shift) is the top digit. Codes of d = -4 .. 3 by
+    // d + 4: 0xE, 0xD, 0xC, 0xA, 0x0, 0x2, 0x4, 0x5 (bit 3 the sign).
+    const int u = iv + 0x124924;  // 4 * (8^0 + 8^1 + ... + 8^6)
 #pragma unroll
-    for (int t = kT - 1; t > 0; --t) {
-        const int d = ((iv + 4) & 7) - 4;  // balanced residue in [-4, 3]
-        iv = (iv - d) >> 3;                // exact: iv - d is a multiple of 8
-        code[t] = e2m1_digit_code(d);
-    }
-    code[0] = e2m1_digit_code(iv);  // |iv| <= 4 after kT - 1 such steps
+    for (int t = kT - 1; t > 0; --t)  // term kT-1 holds the lowest digit
+        code[t] = (0x5420ACDEu >> (4 * ((u >> (3 * (kT - 1 - t))) & 7))) & 0xFu;
+    code[0] = e2m1_digit_code(u >> 21);
 }
 
 // One FFN stage over all experts.
@@ -658,36 +661,29 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
         if (threadIdx.x == 0 && status)
             *status = 0;
     }
-    // Each warp takes a contiguous run of (row, chunk) units, so the row's
-    // expert, pass and token are looked up once per row.
+    // Units (row, chunk) go round-robin over the warps (warp g: units g,
+    // g + W, ...), so that skipped rows of hot experts, which are contiguous,
+    // do not leave some warps idle while others carry double work.
     const int nch = (H + kKC - 1) / kKC;
     const int64_t total = (int64_t)rows * nch;
     const int64_t nwarps = (int64_t)gridDim.x * 8, gw = (int64_t)blockIdx.x * 8 + warp;
-    const int64_t u_begin = total * gw / nwarps, u_end = total * (gw + 1) / nwarps;
     const int kb = lane >> 2, q = lane & 3;  // the lane's 32-block within the chunk; its place in the block
-    int r_cur = -1, n = 0, tok = 0;
-    bool hot = false;
-    int64_t img_row = 0;
-    for (int64_t u = u_begin; u < u_end; ++u) {
+    for (int64_t u = gw; u < total; u += nwarps) {
         const int r = (int)(u / nch), c = (int)(u % nch);
-        if (r != r_cur) {
-            r_cur = r;
-            int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (s_off[mid] <= r)
-                    lo = mid;
-                else
-                    hi = mid;
-            }
-            const int local = r - s_off[lo];
-            hot = s_off[lo + 1] - s_off[lo] >= hot_rows;
-            img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
-            n = local % nt;
-            tok = src_row[r] / k;
+        int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_off[mid] <= r)
+                lo = mid;
+            else
+                hi = mid;
         }
-        if (hot)
+        if (s_off[lo + 1] - s_off[lo] >= hot_rows)  // the bf16 kernel takes this expert
             continue;
+        const int local = r - s_off[lo];
+        const int64_t img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
+        const int n = local % nt;
+        const int tok = __ldg(src_row + r) / k;
         const int col = c * kKC + 8 * lane;
         const bool live = col < H;  // H % 128 == 0: in a half chunk lanes 0..15 are live
         float v[8];
