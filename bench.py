@@ -65,8 +65,8 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--config", default="verify8", choices=[c.name for c in datagen.CONFIGS])
     ap.add_argument("--batches", type=int, default=16, help="distinct rotating input batches")
