@@ -471,12 +471,12 @@ def run_native(args):
     weight_gbs = weight_bytes_step * args.steps / (ms / 1e3) / 1e9
     unit_ms_mean = float(np.mean(unit_ms))
     if T * k >= BF16_PATH_ROWS:
-        # dominant unit: mxmoe_ffn_gate_up on bf16 tensor cores (x_gather +
+        # dominant unit: mxmoe_ffn_gate_up on bf16 tensor cores (passes, slot rows, x_tile +
         # ffn_bf16_kernel<gate_up>); algorithmic work = the dense gate/up
         # contraction of every grouped row: 2 * rows * 2I * H flops
         unit_flops = 2.0 * T * k * 2 * I * H
         achieved = unit_flops / (unit_ms_mean / 1e3) / 1e12
-        roofline = {"kernel": "mxmoe_ffn_gate_up (x_gather_kernel + ffn_bf16_kernel<gate_up>)", "bound": "tensor",
+        roofline = {"kernel": "mxmoe_ffn_gate_up (x_tile_kernel + ffn_bf16_kernel<gate_up>)", "bound": "tensor",
                     "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
                     "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops_sustained)" % peak_kind
                     if peak_kind == "measured" else "fallback 1.4 PFLOP/s sustained",
@@ -487,7 +487,7 @@ def run_native(args):
         w13_bytes = 2 * I * H * 17 // 32
         unit_bytes = mean_touched * w13_bytes + T * H * 2 + T * k * I * 2
         achieved = unit_bytes / (unit_ms_mean / 1e3) / 1e9
-        roofline = {"kernel": "mxmoe_ffn_gate_up (x_terms_kernel + ffn_mxf4_kernel<gate_up>)",
+        roofline = {"kernel": "mxmoe_ffn_gate_up (act_terms_kernel + ffn_mxf4_kernel<gate_up>)",
                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
                     else "fallback 6.65 TB/s",

@@ -150,13 +150,13 @@ MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, int32_t *ids
  *   src_row device int32 [T*k]: pair index t*k + j at each grouped position;
  *           experts ascending, within an expert (t, j) ascending.
  *   dst_of  device int32 [T*k]: grouped position of pair t*k + j.
- * Errors: T*k > 2^24 or E > 4096 -> INVALID_SHAPE. Ids outside [0, E) are
+ * Errors: T*k > 2^24 or E > 1024 -> INVALID_SHAPE. Ids outside [0, E) are
  * outside the contract (they are clamped into range, not reported). */
 MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
                             int32_t *dst_of, void *stream);
 
 /* mxmoe_permute for many pairs, with caller scratch: the same outputs (bit for
- * bit) from a multi-block grouping when T*k > 4096 and E <= 1024 (otherwise it
+ * bit) from a multi-block grouping when T*k > 4096 (otherwise it
  * runs mxmoe_permute's kernel and leaves the scratch alone).
  *   scratch device, >= mxmoe_permute_scratch_size(T, k, E) bytes, 16-byte
  *   aligned, contents not kept between calls.

@@ -323,6 +323,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict
 //     stays ascending.
 // ---------------------------------------------------------------------------
 constexpr int kPmBlock = 1024;
+constexpr int kPmMaxE = 1024;  // experts the grouping kernels take (shared memory: 34 ints per expert)
 
 __global__ void __launch_bounds__(kPmBlock) permute_count_kernel(const int32_t *__restrict__ ids, int n, int E,
                                                                  int32_t *__restrict__ counts)
@@ -538,7 +539,7 @@ namespace mxmoe {
 
 // Scratch ints of the multi-block grouping: counts [E][blocks] + totals [E].
 int64_t permute_scratch_ints(int n, int E) { return (int64_t)E * ((n + kPmBlock - 1) / kPmBlock) + E; }
-bool use_multiblock_permute(int n, int E) { return n > 4 * kPmBlock && E <= kPmBlock; }
+bool use_multiblock_permute(int n, int E) { return n > 4 * kPmBlock && E <= kPmMaxE; }
 
 // The layer path's grouping: the multi-block kernels when use_multiblock_permute
 // (scratch: permute_scratch_ints(n, E) ints), else permute_kernel.
@@ -575,19 +576,22 @@ int run_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32
 extern "C" MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row,
                                        int32_t *dst_of, void *stream)
 {
-    if (T < 0 || k < 1 || E <= 0 || E > 4096 || (int64_t)T * k > (1 << 24))
-        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_permute: T=%d k=%d E=%d", T, k, E);
+    if (T < 0 || k < 1 || E <= 0 || E > kPmMaxE || (int64_t)T * k > (1 << 24))
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_permute: T=%d k=%d E=%d (need E <= %d, T*k <= 2^24)", T, k, E,
+                    kPmMaxE);
     if (!offsets || (T > 0 && (!ids || !src_row || !dst_of)))
         return fail(MXMOE_ERR_NULL, "mxmoe_permute: NULL pointer");
     if (int rc = check_device())
         return rc;
-    const size_t smem = (size_t)(E + 32 * E + E) * sizeof(int32_t);
-    static thread_local int configured_E = -1;
-    if (smem > 48 * 1024 && configured_E < E) {
-        if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return fail(MXMOE_ERR_CUDA, "mxmoe_permute: cannot reserve %zu bytes of shared memory", smem);
-        configured_E = E;
+    const size_t smem = (size_t)(E + 32 * E + E) * sizeof(int32_t);  // <= 136 KB for E <= 1024
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(34 * kPmMaxE * sizeof(int32_t))) != cudaSuccess)
+            return fail(MXMOE_ERR_CUDA, "mxmoe_permute: cannot reserve shared memory");
+        configured_dev = dev;
     }
     permute_kernel<<<1, 1024, smem, (cudaStream_t)stream>>>(ids, T * k, E, offsets, src_row, dst_of);
     return check_launch("permute_kernel");
@@ -595,7 +599,7 @@ extern "C" MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, 
 
 extern "C" MXMOE_API int64_t mxmoe_permute_scratch_size(int T, int k, int E)
 {
-    if (T < 0 || k < 1 || E <= 0 || E > 4096 || (int64_t)T * k > (1 << 24))
+    if (T < 0 || k < 1 || E <= 0 || E > kPmMaxE || (int64_t)T * k > (1 << 24))
         return -1;
     return permute_scratch_ints(T * k, E) * (int64_t)sizeof(int32_t);
 }
@@ -604,7 +608,7 @@ extern "C" MXMOE_API int mxmoe_permute_ws(const int32_t *ids, int T, int k, int 
                                           int32_t *src_row, int32_t *dst_of, void *scratch, int64_t scratch_bytes,
                                           void *stream)
 {
-    if (T < 0 || k < 1 || E <= 0 || E > 4096 || (int64_t)T * k > (1 << 24))
+    if (T < 0 || k < 1 || E <= 0 || E > kPmMaxE || (int64_t)T * k > (1 << 24))
         return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_permute_ws: T=%d k=%d E=%d", T, k, E);
     if (!scratch || scratch_bytes < mxmoe_permute_scratch_size(T, k, E))
         return fail(MXMOE_ERR_WORKSPACE, "mxmoe_permute_ws: scratch of %lld bytes, need %lld",

@@ -130,3 +130,11 @@ def test_timeout_selftest_rejects_on_host(mx):
     assert lib.mxmoe_selftest_wait_timeout(None, 1000, None) == mx.ERR_NULL
     assert lib.mxmoe_selftest_wait_timeout(base, 0, None) == mx.ERR_INVALID_SHAPE
     assert lib.mxmoe_selftest_wait_timeout(base, 1000001, None) == mx.ERR_INVALID_SHAPE
+
+
+def test_grouping_expert_limit(mx):
+    lib = mx.load()
+    # the grouping kernels take up to 1024 experts (34 ints of shared memory each)
+    assert lib.mxmoe_permute(None, 4, 2, 2000, None, None, None, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_permute_scratch_size(4, 2, 1025) == -1
+    assert lib.mxmoe_permute_scratch_size(4, 2, 1024) > 0
