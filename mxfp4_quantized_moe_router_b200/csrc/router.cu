@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
 }
 
 // ---------------------------------------------------------------------------
-// Top-k routing: one 128-thread block per token. Thread i holds logits i,
+// Top-k routing for more than 1024 experts: one 128-thread block per token
+// (up to 4096 experts). Thread i holds logits i,
 // i+128, ...; k rounds of a block arg-max (larger value first, then lower
 // index): thread, warp (shuffles), then the four warp winners in shared
 // memory, combined in the same order by every thread.
@@ -310,6 +311,84 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict
     }
 }
 
+// One warp per token (E <= 32 * V): lane l holds the logits of experts
+// l, l + 32, ..., summed over the splits in split order plus the bias; k
+// rounds of a warp-wide arg-max (ties to the lower expert) pick the experts,
+// with no block-wide barrier, so that 8 tokens share a 256-thread block.
+template <int V>
+__global__ void __launch_bounds__(256) route_warp_kernel(const float *__restrict__ logits, int nsplit,
+                                                         const float *__restrict__ bias, int T, int E, int k,
+                                                         int32_t *__restrict__ ids, float *__restrict__ w)
+{
+    const int lane = threadIdx.x & 31;
+    const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (tok >= T)
+        return;
+    const float *l = logits + (int64_t)tok * E;
+    float v[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? __ldg(l + e) : -FLT_MAX;
+    }
+    for (int z = 1; z < nsplit; ++z) {  // the other splits, in split order
+        const float *lz = l + (int64_t)z * T * E;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            v[i] += e < E ? __ldg(lz + e) : 0.f;
+        }
+    }
+    if (bias) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E)
+                v[i] += __ldg(bias + e);
+        }
+    }
+    uint32_t taken = 0;
+    float sel_v = 0.f;  // lane j < k: the j-th pick
+    int sel_i = 0;
+    for (int j = 0; j < k; ++j) {
+        float bv = -FLT_MAX;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && route_better(v[i], e, bv, bi)) {
+                bv = v[i];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+            if (route_better(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if (bi != 0x7FFFFFFF && (bi & 31) == lane)
+            taken |= 1u << (bi >> 5);
+        if (lane == j) {
+            sel_v = bv;
+            sel_i = bi;
+        }
+    }
+    // weights: exp(l_j - l_max) / sum over the selected, summed in slot order
+    const float top = __shfl_sync(0xFFFFFFFFu, sel_v, 0);
+    const float ex = lane < k ? expf(sel_v - top) : 0.f;
+    float ssum = 0.f;
+    for (int j = 0; j < k; ++j)
+        ssum += __shfl_sync(0xFFFFFFFFu, ex, j);
+    if (lane < k) {
+        ids[(int64_t)tok * k + lane] = sel_i;
+        w[(int64_t)tok * k + lane] = ex / ssum;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Multi-block stable grouping (many pairs; E <= 1024): the same result as
 // permute_kernel from three launches over blocks of 1024 pairs.
@@ -477,18 +556,31 @@ extern "C" MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const 
 
 namespace mxmoe {
 
-// K splits for the layer's router GEMM: enough CTAs to cover the GPU at
-// decode sizes, each split at least 8 k32 blocks (one per warp).
+// Top-k routing of T tokens: a warp per token up to 1024 experts, else the
+// block-per-token kernel.
 int launch_route(const float *logits, int nsplit, const float *bias, int T, int E, int k, int32_t *ids, float *w,
                  cudaStream_t st)
 {
-    if (E <= kRouteThreads * 4)
-        route_kernel<4><<<T, kRouteThreads, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
-    else
-        route_kernel<32><<<T, kRouteThreads, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+    if (E <= 1024) {  // a warp per token
+        const int blocks = (T + 7) / 8;
+        if (E <= 128)
+            route_warp_kernel<4><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+        else if (E <= 256)
+            route_warp_kernel<8><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+        else if (E <= 384)
+            route_warp_kernel<12><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+        else if (E <= 512)
+            route_warp_kernel<16><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+        else
+            route_warp_kernel<32><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+        return check_launch("route_warp_kernel");
+    }
+    route_kernel<32><<<T, kRouteThreads, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
     return check_launch("route_kernel");
 }
 
+// K splits for the layer's router GEMM: enough CTAs to cover the GPU at
+// decode sizes, each split at least 8 k32 blocks (one per warp).
 int router_splits(int T, int H, int E)
 {
     if (use_router_tc(T, H))

@@ -97,9 +97,17 @@ def test_router_gemm(mx, T, H, E):
     assert np.all(np.abs(got - ref) <= 1e-5 * scale + 1e-6)
 
 
-@pytest.mark.parametrize("T,E,k", [(64, 384, 8), (37, 16, 2), (5, 1000, 32), (1, 8, 8), (200, 96, 1)])
-def test_route_bitexact(mx, T, E, k):
+# every expert-count bin of the warp-per-token kernel (128/256/384/512/1024),
+# the block kernel (E > 1024), and logits rounded to few levels (many ties,
+# which go to the lower expert index)
+@pytest.mark.parametrize("T,E,k,ties", [(64, 384, 8, False), (37, 16, 2, False), (5, 1000, 32, False),
+                                        (1, 8, 8, False), (200, 96, 1, False), (33, 256, 8, False),
+                                        (9, 512, 4, False), (17, 1024, 8, False), (3, 3000, 8, False),
+                                        (41, 384, 8, True), (7, 2500, 6, True)])
+def test_route_bitexact(mx, T, E, k, ties):
     l = datagen.make_logits(T, E, seed=T + E)
+    if ties:
+        l = np.round(l * 2.0).astype(np.float32) / np.float32(2.0)
     ids_ref, w_ref = oracle.route(l, k)
     ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
     w = torch.empty((T, k), dtype=torch.float32, device=DEV)
