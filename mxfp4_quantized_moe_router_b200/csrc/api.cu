@@ -49,6 +49,26 @@ int fail(int code, const char *fmt, ...)
     return code;
 }
 
+namespace {
+thread_local int t_chain_depth = 0;
+thread_local bool t_chain_started = false;
+}  // namespace
+
+ChainScope::ChainScope()
+{
+    if (t_chain_depth++ == 0)
+        t_chain_started = false;
+}
+
+ChainScope::~ChainScope() { --t_chain_depth; }
+
+bool chain_next()
+{
+    const bool chained = t_chain_depth > 0 && t_chain_started;
+    t_chain_started = true;
+    return chained;
+}
+
 int check_launch(const char *what)
 {
     cudaError_t e = cudaGetLastError();
@@ -186,6 +206,7 @@ extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, cons
     int *status = static_cast<int *>(ws.ffn);
     if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess)
         return fail(MXMOE_ERR_CUDA, "mxmoe_layer_forward: cannot clear the status word");
+    ChainScope chain;  // the router GEMM starts after the clear; every later kernel is chained
     if (int rc = run_router_and_route(x, wg, bias, T, H, E, k, ws.logits, router_splits(T, H, E), ids, w, status,
                                       st))
         return rc;

@@ -30,6 +30,52 @@ int check_device();  // MXMOE_ERR_DEVICE unless the current device is CC 10.x
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---------------------------------------------------------------------------
+// Launch chains (programmatic dependent launch). Inside a ChainScope -- one
+// per C entry point that launches kernels -- every kernel started through
+// launch_kernel after the first may begin while its predecessor on the stream
+// is still running. Every such kernel runs grid_dep_wait() in each thread that
+// touches its predecessor's results (and in each CTA before it exits), and
+// grid_dep_launch() only after that wait. So when a chained kernel begins,
+// every kernel before its predecessor has completed: what it reads before its
+// own wait (routing offsets, pass tables, weights) was written by those. The
+// first kernel of a scope is launched plainly, after all earlier work on the
+// stream, so a chain never overlaps the caller's own kernels.
+// ---------------------------------------------------------------------------
+struct ChainScope {
+    ChainScope();
+    ~ChainScope();
+    ChainScope(const ChainScope &) = delete;
+    ChainScope &operator=(const ChainScope &) = delete;
+};
+bool chain_next();  // whether the next launch may overlap its predecessor; marks the chain as started
+
+// Launches kernel<<<grid, block, smem, st>>>(args...) (chained when inside a
+// ChainScope after its first launch); MXMOE_OK or MXMOE_ERR_CUDA naming what.
+template <typename... P, typename... A>
+int launch_kernel(const char *what, void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                  A &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (chain_next()) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<A &&>(args)...);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MXMOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    }
+    return check_launch(what);
+}
+
+// ---------------------------------------------------------------------------
 // Layout constants shared by the prepack and FFN kernels
 // ---------------------------------------------------------------------------
 constexpr int kBlock = 32;       // MXFP4 block: elements per E8M0 scale
@@ -75,6 +121,13 @@ __device__ __forceinline__ void set_status(int *status, int code)
 }
 
 #if defined(__CUDACC__)
+
+// Programmatic dependent launch: grid_dep_wait() returns once the kernel this
+// one was chained after has completed and its writes are visible (at once
+// when it was launched plainly); grid_dep_launch() lets the next chained
+// kernel start its own prologue.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ uint64_t globaltimer_ns()
 {

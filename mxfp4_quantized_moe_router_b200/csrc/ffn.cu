@@ -315,6 +315,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #define ITEM(i) decode_item<NT>(blockIdx.x + (int64_t)(i) * G, s_items, p.offsets, E, tiles)
     const int nchunk = (p.K + kKC - 1) / kKC;  // the last chunk may hold one 128-column half
     const int khalves = p.K / 128;
+    // Chained launch: the producer fills the weight ring before waiting for
+    // the preceding kernel (weights and offsets are older than it; the
+    // activation terms, their scale images and the pass table are its
+    // results); every other thread waits here. The next kernel is let start
+    // only as this one's CTAs exit: triggered earlier, its CTAs sat resident
+    // and waiting beside these, which measured slower.
+    if (!(warp == 0 && lane == 0))
+        grid_dep_wait();
 
     if (warp == 0) {
         // ----------------------------------------------------------- producer
@@ -325,19 +333,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phw = 0, pha = 0;
             int64_t issued_w = 0, issued_a = 0;
             bool ok = true;
+            auto load_w = [&](int sl, int64_t box) {  // weight box and its scale images into slot sl
+                mbar_arrive_expect_tx(&fullW[sl], (uint32_t)(kWBox + kWSf));
+                tc::tma_load_2d(sW + (size_t)sl * kWBox, &tmW, 0, (int)(box * 256), &fullW[sl], pol_w);
+                bulk_g2s_hint(sSfw + sl * kWSf, p.wsf + box * kWSf, kWSf, &fullW[sl], pol_w);
+            };
+            int64_t pre_w = 0;  // weight boxes issued before the wait (slots 0 .. pre_w-1, first use)
+            for (int i = 0; i < n_items && pre_w < C::kStagesW; ++i) {
+                const Item it = ITEM(i);
+                const int64_t box0 = ((int64_t)it.e * tiles + it.tile) * nchunk;
+                for (int c = 0; c < nchunk && pre_w < C::kStagesW; ++c, ++pre_w)
+                    load_w((int)pre_w, box0 + c);
+            }
+            grid_dep_wait();
             for (int i = 0; i < n_items && ok; ++i) {
                 const Item it = ITEM(i);
                 const int64_t box0 = ((int64_t)it.e * tiles + it.tile) * nchunk;
                 const int64_t pass_id = (int64_t)p.pass_start[it.e] + it.pass;
                 const int r0 = it.r0;
                 for (int c = 0; c < nchunk; ++c) {
-                    if (*abort_flag || !mbar_wait_bounded(&emptyW[sw], phw ^ 1u, kWaitLimitNs)) {
-                        ok = false;
-                        break;
+                    if (issued_w >= pre_w) {
+                        if (*abort_flag || !mbar_wait_bounded(&emptyW[sw], phw ^ 1u, kWaitLimitNs)) {
+                            ok = false;
+                            break;
+                        }
+                        load_w(sw, box0 + c);
                     }
-                    mbar_arrive_expect_tx(&fullW[sw], (uint32_t)(kWBox + kWSf));
-                    tc::tma_load_2d(sW + (size_t)sw * kWBox, &tmW, 0, (int)((box0 + c) * 256), &fullW[sw], pol_w);
-                    bulk_g2s_hint(sSfw + sw * kWSf, p.wsf + (box0 + c) * kWSf, kWSf, &fullW[sw], pol_w);
                     ++issued_w;
                     if (*abort_flag || !mbar_wait_bounded(&emptyA[sa], pha ^ 1u, kWaitLimitNs)) {
                         ok = false;
@@ -647,6 +668,8 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
                                                       uint8_t *__restrict__ sf, int32_t *__restrict__ pass_start_out,
                                                       int *status)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     __shared__ int32_t s_off[kMaxE + 1], s_pass[kMaxE + 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int e = threadIdx.x; e <= E; e += blockDim.x)
@@ -738,6 +761,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
                                                       const float *__restrict__ w, int T, int k, int H,
                                                       float *__restrict__ y)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     const int t = blockIdx.y;
     const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= T || c4 * 4 >= H)
@@ -881,8 +906,8 @@ int launch_ffn(const void *codes, const uint8_t *act_terms, const FfnParams &p, 
         return rc;
     if (int rc = encode_terms(&tmA, act_terms, p.rows, p.K, NT))
         return rc;
-    ffn_mxf4_kernel<NT, GATE_UP><<<num_sms(), kThreads, C::kSmem, st>>>(tmW, tmA, p);
-    return check_launch(GATE_UP ? "ffn_mxf4_kernel<gate_up>" : "ffn_mxf4_kernel<down>");
+    return launch_kernel(GATE_UP ? "ffn_mxf4_kernel<gate_up>" : "ffn_mxf4_kernel<down>", ffn_mxf4_kernel<NT, GATE_UP>,
+                         num_sms(), kThreads, C::kSmem, st, tmW, tmA, p);
 }
 
 // Token rows per pass: 8 up to 8 tokens (an expert then never sees more than
@@ -934,10 +959,9 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
         const int hot_rows = use_hybrid(T, k) ? kHotRows : INT_MAX;
         const int64_t warps = (int64_t)rows * ((H + kKC - 1) / kKC);
         const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 8);
-        act_terms_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), src_row, offsets, E,
-                                                                 k, rows, H, nt, hot_rows, ws.x_terms, ws.x_sf,
-                                                                 ws.pass_start, clear);
-        if (int rc = check_launch("act_terms_kernel"))
+        if (int rc = launch_kernel("act_terms_kernel", act_terms_kernel, blocks < 1 ? 1 : blocks, 256, 0, st,
+                                   static_cast<const uint16_t *>(x), src_row, offsets, E, k, rows, H, nt, hot_rows,
+                                   ws.x_terms, ws.x_sf, ws.pass_start, clear))
             return rc;
         clear = nullptr;  // cleared once, before anything could record a timeout
         FfnParams p{};
@@ -1017,8 +1041,7 @@ int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int 
                 cudaStream_t st)
 {
     dim3 grid((H / 4 + 255) / 256, T);
-    combine_kernel<<<grid, 256, 0, st>>>(y_perm, dst_of, w, T, k, H, y);
-    return check_launch("combine_kernel");
+    return launch_kernel("combine_kernel", combine_kernel, grid, 256, 0, st, y_perm, dst_of, w, T, k, H, y);
 }
 
 int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I)
@@ -1068,6 +1091,7 @@ extern "C" MXMOE_API int mxmoe_expert_ffn(const void *x, const int32_t *offsets,
         return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_expert_ffn: x and y_perm need 16-byte, prepacked 32-byte alignment");
     if (int rc = check_device())
         return rc;
+    ChainScope chain;
     return run_expert_ffn(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, workspace, true,
                           (cudaStream_t)stream);
 }
@@ -1086,6 +1110,7 @@ extern "C" MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets
         return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_ffn_gate_up: x needs 16-byte, prepacked 32-byte alignment");
     if (int rc = check_device())
         return rc;
+    ChainScope chain;
     return run_ffn_gate_up(x, offsets, src_row, prepacked, T, k, E, H, I, workspace, true, (cudaStream_t)stream);
 }
 
@@ -1102,6 +1127,7 @@ extern "C" MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prep
         return fail(MXMOE_ERR_ALIGNMENT, "mxmoe_ffn_down: prepacked needs 32-byte, y_perm 16-byte alignment");
     if (int rc = check_device())
         return rc;
+    ChainScope chain;
     return run_ffn_down(offsets, prepacked, T, k, E, H, I, y_perm, workspace, (cudaStream_t)stream);
 }
 

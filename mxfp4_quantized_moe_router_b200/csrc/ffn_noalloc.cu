@@ -84,6 +84,7 @@ extern "C" MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *
     // The first kernel of the chain clears the status word at the start of the
     // scratch; every other scratch byte that can reach the outputs is written
     // earlier in the same call, so nothing else needs clearing between calls.
+    ChainScope chain;
     if (int rc = run_expert_ffn(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, scratch, true, st))
         return rc;
     if (status) {

@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__r
                                                               int min_rows, int32_t *__restrict__ pass_start,
                                                               int *status)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     __shared__ int32_t s_warp[32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     const int n_e = e < E ? __ldg(offsets + e + 1) - __ldg(offsets + e) : 0;
@@ -129,6 +131,8 @@ __global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__r
 __global__ void __launch_bounds__(256) slot_rows_kernel(const int32_t *__restrict__ src_row, int rows,
                                                         int32_t *__restrict__ slot_row)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x)
         slot_row[__ldg(src_row + r)] = r;
 }
@@ -150,6 +154,8 @@ __global__ void __launch_bounds__(256) x_tile_kernel(const uint16_t *__restrict_
                                                      const int32_t *__restrict__ pass_start, int E, int min_rows,
                                                      int k, int T, int H, uint8_t *__restrict__ x_tiled)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     __shared__ int64_t s_dst[8][kTileMaxK];  // per warp: byte offset of slot j's row in x_tiled, or -1
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int nks = H / kPK;
@@ -330,8 +336,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     ffn_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const PrefillParams p)
 {
     constexpr int NB = GATE_UP ? 1 : 2;  // activation steps per K step: x, or h's hi then lo
-    if (__ldg(p.pass_start + p.E) == 0)  // no expert for this kernel (the E2M1-term kernel took them all)
+    if (__ldg(p.pass_start + p.E) == 0) {  // no expert for this kernel (the E2M1-term kernel took them all)
+        grid_dep_wait();                    // a chained CTA ends after the preceding kernel
+        grid_dep_launch();
         return;
+    }
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem, *sA = smem + kPOffA, *sW = smem + kPOffW, *sSf = smem + kPOffSf;
@@ -381,6 +390,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int n_items = (int)(total > blockIdx.x ? (total - blockIdx.x + G - 1) / G : 0);
 #define ITEM(i) decode_item(blockIdx.x + (int64_t)(i) * G, p.pass_start, p.offsets, E, pairs)
     const int nks = p.K / kPK;  // K steps (even: K is a multiple of 128)
+    // Chained launch: the weight producer fills its ring before waiting for
+    // the preceding kernel (weights, offsets and the pass table are older than
+    // it); every other role waits here. The next kernel is let start only as
+    // this one's CTAs exit (an earlier trigger measured slower).
+    if (!((warp == kPWarpB || warp == kPWarpW) && lane == 0))
+        grid_dep_wait();
 
     if (warp == kPWarpB || warp == kPWarpW) {
         // ---------------------------------------------------------- producers
@@ -399,28 +414,41 @@ __global__ void __launch_bounds__(kPThreads, 1)
             uint32_t ph = 0;
             int64_t issued = 0;
             bool ok = true;
+            // packed weights and scale images of K steps ks, ks + 1 of a box into slot sl
+            auto load_w = [&](int sl, int64_t box, int ks) {
+                const int64_t chunk = box * p.nchunk + (ks >> 2);  // 256-K chunk of the box
+                mbar_arrive_expect_tx(&full[sl], (uint32_t)(kPWBytes + kPSfBytes));
+                tc::tma_load_2d(sW + (size_t)sl * kPWBytes, &tmW, 64 * ((ks & 3) >> 1), (int)(chunk * 256), &full[sl],
+                                pol);
+                bulk_g2s_hint(sSf + (size_t)sl * kPSfBytes, p.sf + chunk * 2048 + ((ks & 3) >> 1) * kPSfBytes,
+                              kPSfBytes, &full[sl], pol);
+            };
+            int64_t pre = 0;  // weight loads issued before the wait (slots 0 .. pre-1, first use)
+            if (!is_b)
+                for (int i = 0; i < n_items && pre < S; ++i) {
+                    const PItem it = ITEM(i);
+                    for (int ks = 0; ks < nks && pre < S; ks += 2, ++pre)
+                        load_w((int)pre, (int64_t)it.e * pairs + it.box, ks);
+                }
+            grid_dep_wait();
             for (int i = 0; i < n_items && ok; ++i) {
                 const PItem it = ITEM(i);
                 const int64_t box = (int64_t)it.e * pairs + it.box;
                 for (int ks = 0; ks < nks && ok; ks += is_b ? 1 : 2) {
                     for (int b = 0; b < (is_b ? NB : 1); ++b) {
-                        if (*abort_flag || !mbar_wait_bounded(&empty[s], ph ^ 1u, kPWaitNs)) {
-                            ok = false;
-                            break;
-                        }
-                        if (is_b) {
-                            mbar_arrive_expect_tx(&full[s], (uint32_t)kPBBytes);
-                            bulk_g2s_hint(sB + (size_t)s * kPBBytes,
-                                          p.act + ((it.pass * nks + ks) * NB + b) * (int64_t)kPBBytes, kPBBytes,
-                                          &full[s], pol);
-                        } else {
-                            const int64_t chunk = box * p.nchunk + (ks >> 2);  // 256-K chunk of the box
-                            mbar_arrive_expect_tx(&full[s], (uint32_t)(kPWBytes + kPSfBytes));
-                            tc::tma_load_2d(sW + (size_t)s * kPWBytes, &tmW, 64 * ((ks & 3) >> 1), (int)(chunk * 256),
-                                            &full[s], pol);
-                            bulk_g2s_hint(sSf + (size_t)s * kPSfBytes,
-                                          p.sf + chunk * 2048 + ((ks & 3) >> 1) * kPSfBytes, kPSfBytes, &full[s],
-                                          pol);
+                        if (issued >= pre) {
+                            if (*abort_flag || !mbar_wait_bounded(&empty[s], ph ^ 1u, kPWaitNs)) {
+                                ok = false;
+                                break;
+                            }
+                            if (is_b) {
+                                mbar_arrive_expect_tx(&full[s], (uint32_t)kPBBytes);
+                                bulk_g2s_hint(sB + (size_t)s * kPBBytes,
+                                              p.act + ((it.pass * nks + ks) * NB + b) * (int64_t)kPBBytes, kPBBytes,
+                                              &full[s], pol);
+                            } else {
+                                load_w(s, box, ks);
+                            }
                         }
                         ++issued;
                         if (++s == S) {
@@ -658,8 +686,8 @@ int launch_bf16_stage(const CUtensorMap &tmW, const PrefillParams &p, cudaStream
             return fail(MXMOE_ERR_CUDA, "ffn_bf16_kernel: cannot reserve %zu bytes of shared memory", kPSmem);
         configured_dev = dev;
     }
-    ffn_bf16_kernel<GATE_UP><<<num_sms(), kPThreads, kPSmem, st>>>(tmW, p);
-    return check_launch(GATE_UP ? "ffn_bf16_kernel<gate_up>" : "ffn_bf16_kernel<down>");
+    return launch_kernel(GATE_UP ? "ffn_bf16_kernel<gate_up>" : "ffn_bf16_kernel<down>", ffn_bf16_kernel<GATE_UP>,
+                         num_sms(), kPThreads, kPSmem, st, tmW, p);
 }
 
 }  // namespace
@@ -683,20 +711,19 @@ int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row,
                   int min_rows, int32_t *pass_start, int32_t *slot_row, uint8_t *x_tiled, int *status,
                   cudaStream_t st)
 {
-    prefill_passes_kernel<<<1, 1024, 0, st>>>(offsets, E, min_rows, pass_start, status);
-    if (int rc = check_launch("prefill_passes_kernel"))
+    if (int rc = launch_kernel("prefill_passes_kernel", prefill_passes_kernel, 1, 1024, 0, st, offsets, E, min_rows,
+                               pass_start, status))
         return rc;
     {
         const int blocks = (int)std::min<int64_t>(((int64_t)rows + 255) / 256, (int64_t)num_sms() * 4);
-        slot_rows_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(src_row, rows, slot_row);
-        if (int rc = check_launch("slot_rows_kernel"))
+        if (int rc = launch_kernel("slot_rows_kernel", slot_rows_kernel, blocks < 1 ? 1 : blocks, 256, 0, st, src_row,
+                                   rows, slot_row))
             return rc;
     }
     const int T = rows / k;
     const int blocks = (int)std::min<int64_t>(((int64_t)T + 7) / 8, (int64_t)num_sms() * 8);
-    x_tile_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(static_cast<const uint16_t *>(x), slot_row, offsets,
-                                                           pass_start, E, min_rows, k, T, H, x_tiled);
-    return check_launch("x_tile_kernel");
+    return launch_kernel("x_tile_kernel", x_tile_kernel, blocks < 1 ? 1 : blocks, 256, 0, st,
+                         static_cast<const uint16_t *>(x), slot_row, offsets, pass_start, E, min_rows, k, T, H, x_tiled);
 }
 
 // One FFN stage on bf16 tensor cores over the grouped rows.

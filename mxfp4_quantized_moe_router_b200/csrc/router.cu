@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
                                                           const float *__restrict__ bias, int T, int H, int E,
                                                           float *__restrict__ logits)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     __shared__ float red[kRgWarps][kRgExperts][kRgTokens + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -128,6 +130,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float *__res
                                                               const float *__restrict__ bias, int T, int E, int k,
                                                               int32_t *__restrict__ ids, float *__restrict__ w)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     __shared__ float s_bv[kRouteThreads / 32];
     __shared__ int s_bi[kRouteThreads / 32];
     __shared__ float s_sel_v[32];
@@ -243,6 +247,8 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict
                                                        int32_t *__restrict__ offsets, int32_t *__restrict__ src_row,
                                                        int32_t *__restrict__ dst_of)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     extern __shared__ int32_t sm[];
     int32_t *cursor = sm;            // [E]
     int32_t *wcnt = sm + E;          // [32][E]
@@ -320,6 +326,8 @@ __global__ void __launch_bounds__(256) route_warp_kernel(const float *__restrict
                                                          const float *__restrict__ bias, int T, int E, int k,
                                                          int32_t *__restrict__ ids, float *__restrict__ w)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (tok >= T)
@@ -407,6 +415,8 @@ constexpr int kPmMaxE = 1024;  // experts the grouping kernels take (shared memo
 __global__ void __launch_bounds__(kPmBlock) permute_count_kernel(const int32_t *__restrict__ ids, int n, int E,
                                                                  int32_t *__restrict__ counts)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     extern __shared__ int32_t cnt[];  // [E]
     const int tid = threadIdx.x, nb = gridDim.x;
     for (int e = tid; e < E; e += kPmBlock)
@@ -458,6 +468,8 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int32_t *s_warp, int 
 __global__ void __launch_bounds__(kPmBlock) permute_scan_kernel(int32_t *__restrict__ counts, int nb,
                                                                 int32_t *__restrict__ totals)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     __shared__ int32_t s_warp[33];
     int32_t *c = counts + (int64_t)blockIdx.x * nb;
     int carry = 0;
@@ -481,6 +493,8 @@ __global__ void __launch_bounds__(kPmBlock) permute_scatter_kernel(const int32_t
                                                                    int32_t *__restrict__ src_row,
                                                                    int32_t *__restrict__ dst_of)
 {
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
     extern __shared__ int32_t sm[];
     int32_t *base_e = sm;      // [E]: first position of this block's pairs of expert e
     int32_t *wcnt = sm + E;    // [32][E]: per warp, then exclusive over warps
@@ -548,10 +562,8 @@ extern "C" MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const 
     if (use_router_tc(T, H))
         return run_router_gemm_tc(x, wg, bias, T, H, E, logits, 1, nullptr, (cudaStream_t)stream);
     dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens, 1);
-    router_gemm_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(static_cast<const uint16_t *>(x),
-                                                              static_cast<const uint16_t *>(wg), bias, T, H, E,
-                                                              logits);
-    return check_launch("router_gemm_kernel");
+    return launch_kernel("router_gemm_kernel", router_gemm_kernel, grid, 256, 0, (cudaStream_t)stream,
+                         static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(wg), bias, T, H, E, logits);
 }
 
 namespace mxmoe {
@@ -563,20 +575,21 @@ int launch_route(const float *logits, int nsplit, const float *bias, int T, int 
 {
     if (E <= 1024) {  // a warp per token
         const int blocks = (T + 7) / 8;
+        int rc;
         if (E <= 128)
-            route_warp_kernel<4><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+            rc = launch_kernel("route_warp_kernel", route_warp_kernel<4>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
         else if (E <= 256)
-            route_warp_kernel<8><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+            rc = launch_kernel("route_warp_kernel", route_warp_kernel<8>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
         else if (E <= 384)
-            route_warp_kernel<12><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+            rc = launch_kernel("route_warp_kernel", route_warp_kernel<12>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
         else if (E <= 512)
-            route_warp_kernel<16><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
+            rc = launch_kernel("route_warp_kernel", route_warp_kernel<16>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
         else
-            route_warp_kernel<32><<<blocks, 256, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
-        return check_launch("route_warp_kernel");
+            rc = launch_kernel("route_warp_kernel", route_warp_kernel<32>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
+        return rc;
     }
-    route_kernel<32><<<T, kRouteThreads, 0, st>>>(logits, nsplit, bias, T, E, k, ids, w);
-    return check_launch("route_kernel");
+    return launch_kernel("route_kernel", route_kernel<32>, T, kRouteThreads, 0, st, logits, nsplit, bias, T, E, k, ids,
+                         w);
 }
 
 // K splits for the layer's router GEMM: enough CTAs to cover the GPU at
@@ -604,9 +617,9 @@ int run_router_and_route(const void *x, const void *wg, const float *bias, int T
         return launch_route(partials, nsplit, nsplit > 1 ? bias : nullptr, T, E, k, ids, w, st);
     }
     dim3 grid((E + kRgExperts - 1) / kRgExperts, (T + kRgTokens - 1) / kRgTokens, nsplit);
-    router_gemm_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(wg),
-                                             bias, T, H, E, partials);
-    if (int rc = check_launch("router_gemm_kernel"))
+    if (int rc = launch_kernel("router_gemm_kernel", router_gemm_kernel, grid, 256, 0, st,
+                               static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(wg), bias, T, H, E,
+                               partials))
         return rc;
     return launch_route(partials, nsplit, nsplit > 1 ? bias : nullptr, T, E, k, ids, w, st);
 }
@@ -653,14 +666,13 @@ int run_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32
             return fail(MXMOE_ERR_CUDA, "permute_scatter_kernel: cannot reserve shared memory");
         configured_dev = dev;
     }
-    permute_count_kernel<<<nb, kPmBlock, E * sizeof(int32_t), st>>>(ids, n, E, counts);
-    if (int rc = check_launch("permute_count_kernel"))
+    if (int rc = launch_kernel("permute_count_kernel", permute_count_kernel, nb, kPmBlock, E * sizeof(int32_t), st,
+                               ids, n, E, counts))
         return rc;
-    permute_scan_kernel<<<E, kPmBlock, 0, st>>>(counts, nb, totals);
-    if (int rc = check_launch("permute_scan_kernel"))
+    if (int rc = launch_kernel("permute_scan_kernel", permute_scan_kernel, E, kPmBlock, 0, st, counts, nb, totals))
         return rc;
-    permute_scatter_kernel<<<nb, kPmBlock, smem_scatter, st>>>(ids, n, E, counts, totals, offsets, src_row, dst_of);
-    return check_launch("permute_scatter_kernel");
+    return launch_kernel("permute_scatter_kernel", permute_scatter_kernel, nb, kPmBlock, smem_scatter, st, ids, n, E,
+                         counts, totals, offsets, src_row, dst_of);
 }
 
 }  // namespace mxmoe
@@ -685,8 +697,8 @@ extern "C" MXMOE_API int mxmoe_permute(const int32_t *ids, int T, int k, int E, 
             return fail(MXMOE_ERR_CUDA, "mxmoe_permute: cannot reserve shared memory");
         configured_dev = dev;
     }
-    permute_kernel<<<1, 1024, smem, (cudaStream_t)stream>>>(ids, T * k, E, offsets, src_row, dst_of);
-    return check_launch("permute_kernel");
+    return launch_kernel("permute_kernel", permute_kernel, 1, 1024, smem, (cudaStream_t)stream, ids, T * k, E, offsets,
+                         src_row, dst_of);
 }
 
 extern "C" MXMOE_API int64_t mxmoe_permute_scratch_size(int T, int k, int E)
@@ -709,6 +721,7 @@ extern "C" MXMOE_API int mxmoe_permute_ws(const int32_t *ids, int T, int k, int 
         return fail(MXMOE_ERR_NULL, "mxmoe_permute_ws: NULL pointer");
     if (int rc = check_device())
         return rc;
+    ChainScope chain;
     return run_permute(ids, T, k, E, offsets, src_row, dst_of, static_cast<int32_t *>(scratch),
                        (cudaStream_t)stream);
 }

@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(128, 1)
     uint32_t *tslot = reinterpret_cast<uint32_t *>(accfull + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
+    grid_dep_wait();  // the preceding kernel's results (chained launch); the next one starts as CTAs exit
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // item: expert tile fastest, so that the CTAs of one token tile run together and share x in L2
     const int et = blockIdx.x % p.etiles;
@@ -233,8 +234,7 @@ int run_router_gemm_tc(const void *x, const void *wg, const float *bias, int T, 
     p.out = out;
     p.status = status;
     const int grid = p.etiles * p.ttiles * nsplit;
-    router_tc_kernel<<<grid, 128, kRtSmem, st>>>(tmA, tmB, p);
-    return check_launch("router_tc_kernel");
+    return launch_kernel("router_tc_kernel", router_tc_kernel, grid, 128, kRtSmem, st, tmA, tmB, p);
 }
 
 }  // namespace mxmoe
