@@ -317,11 +317,33 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict
     }
 }
 
+// Routing key of (logit v, expert e): unsigned order is the selection order
+// (larger logit first, then the lower expert). The logit's bits are mapped to
+// an order-preserving unsigned value (negative: all bits flipped; otherwise
+// the sign bit set), with -0 taken as +0 so that the two tie; the low half is
+// the complement of e.
+__device__ __forceinline__ uint64_t route_key(float v, int e)
+{
+    uint32_t u = __float_as_uint(v);
+    if (u == 0x80000000u)
+        u = 0;
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((uint64_t)u << 32) | (uint32_t)~e;
+}
+
+__device__ __forceinline__ float route_key_value(uint64_t key)
+{
+    const uint32_t u = (uint32_t)(key >> 32);
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
 // One warp per token (E <= 32 * V): lane l holds the logits of experts
-// l, l + 32, ..., summed over the splits in split order plus the bias; k
-// rounds of a warp-wide arg-max (ties to the lower expert) pick the experts,
-// with no block-wide barrier, so that 8 tokens share a 256-thread block.
-template <int V>
+// l, l + 32, ..., summed over the splits in split order (G splits' loads in
+// flight at a time; G = 1 takes a single split) plus the bias, as routing
+// keys. k rounds of a warp-wide maximum of the keys not yet taken pick the
+// experts, with no block-wide barrier, so that 8 tokens share a 256-thread
+// block.
+template <int V, int G>
 __global__ void __launch_bounds__(256) route_warp_kernel(const float *__restrict__ logits, int nsplit,
                                                          const float *__restrict__ bias, int T, int E, int k,
                                                          int32_t *__restrict__ ids, float *__restrict__ w)
@@ -337,62 +359,71 @@ __global__ void __launch_bounds__(256) route_warp_kernel(const float *__restrict
 #pragma unroll
     for (int i = 0; i < V; ++i) {
         const int e = lane + 32 * i;
-        v[i] = e < E ? __ldg(l + e) : -FLT_MAX;
+        v[i] = e < E ? __ldg(l + e) : 0.f;
     }
-    for (int z = 1; z < nsplit; ++z) {  // the other splits, in split order
-        const float *lz = l + (int64_t)z * T * E;
+    if (G > 1) {
+        int z = 1;
+        for (; z + G - 1 < nsplit; z += G) {
+            float pz[G][V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int e = lane + 32 * i;
-            v[i] += e < E ? __ldg(lz + e) : 0.f;
-        }
-    }
-    if (bias) {
+            for (int g = 0; g < G; ++g) {
+                const float *lz = l + (int64_t)(z + g) * T * E;
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E)
-                v[i] += __ldg(bias + e);
-        }
-    }
-    uint32_t taken = 0;
-    float sel_v = 0.f;  // lane j < k: the j-th pick
-    int sel_i = 0;
-    for (int j = 0; j < k; ++j) {
-        float bv = -FLT_MAX;
-        int bi = 0x7FFFFFFF;
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && !((taken >> i) & 1u) && route_better(v[i], e, bv, bi)) {
-                bv = v[i];
-                bi = e;
+                for (int i = 0; i < V; ++i) {
+                    const int e = lane + 32 * i;
+                    pz[g][i] = e < E ? __ldg(lz + e) : 0.f;
+                }
             }
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    v[i] += pz[g][i];
+        }
+        for (; z < nsplit; ++z) {
+            const float *lz = l + (int64_t)z * T * E;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int e = lane + 32 * i;
+                v[i] += e < E ? __ldg(lz + e) : 0.f;
+            }
+        }
+    }
+    uint64_t key[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = e < E ? route_key(bias ? v[i] + __ldg(bias + e) : v[i], e) : 0ull;  // 0: never picked
+    }
+    uint64_t sel = 0;  // lane j < k: the key of the j-th pick
+    uint32_t taken = 0;  // bit i: key[i] already picked
+    for (int j = 0; j < k; ++j) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const uint64_t c = ((taken >> i) & 1u) ? 0ull : key[i];
+            best = c > best ? c : best;
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
-            if (route_better(ov, oi, bv, bi)) {
-                bv = ov;
-                bi = oi;
-            }
+            const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, best, off);
+            best = o > best ? o : best;
         }
-        if (bi != 0x7FFFFFFF && (bi & 31) == lane)
-            taken |= 1u << (bi >> 5);
-        if (lane == j) {
-            sel_v = bv;
-            sel_i = bi;
-        }
+        const uint32_t e = ~(uint32_t)best;
+        if (best != 0 && (e & 31u) == (uint32_t)lane)  // the owner drops the pick from its candidates
+            taken |= 1u << (e >> 5);
+        if (lane == j)
+            sel = best;
     }
     // weights: exp(l_j - l_max) / sum over the selected, summed in slot order
+    const float sel_v = route_key_value(sel);
     const float top = __shfl_sync(0xFFFFFFFFu, sel_v, 0);
     const float ex = lane < k ? expf(sel_v - top) : 0.f;
     float ssum = 0.f;
     for (int j = 0; j < k; ++j)
         ssum += __shfl_sync(0xFFFFFFFFu, ex, j);
     if (lane < k) {
-        ids[(int64_t)tok * k + lane] = sel_i;
+        ids[(int64_t)tok * k + lane] = (int32_t)~(uint32_t)sel;
         w[(int64_t)tok * k + lane] = ex / ssum;
     }
 }
@@ -568,6 +599,18 @@ extern "C" MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const 
 
 namespace mxmoe {
 
+template <int V>
+int launch_route_warp(const float *logits, int nsplit, const float *bias, int T, int E, int k, int32_t *ids, float *w,
+                      int blocks, cudaStream_t st)
+{
+    constexpr int G = V <= 16 ? 4 : 2;  // split loads in flight (registers)
+    if (nsplit == 1)
+        return launch_kernel("route_warp_kernel", route_warp_kernel<V, 1>, blocks, 256, 0, st, logits, nsplit, bias, T,
+                             E, k, ids, w);
+    return launch_kernel("route_warp_kernel", route_warp_kernel<V, G>, blocks, 256, 0, st, logits, nsplit, bias, T, E,
+                         k, ids, w);
+}
+
 // Top-k routing of T tokens: a warp per token up to 1024 experts, else the
 // block-per-token kernel.
 int launch_route(const float *logits, int nsplit, const float *bias, int T, int E, int k, int32_t *ids, float *w,
@@ -575,18 +618,15 @@ int launch_route(const float *logits, int nsplit, const float *bias, int T, int 
 {
     if (E <= 1024) {  // a warp per token
         const int blocks = (T + 7) / 8;
-        int rc;
         if (E <= 128)
-            rc = launch_kernel("route_warp_kernel", route_warp_kernel<4>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
-        else if (E <= 256)
-            rc = launch_kernel("route_warp_kernel", route_warp_kernel<8>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
-        else if (E <= 384)
-            rc = launch_kernel("route_warp_kernel", route_warp_kernel<12>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
-        else if (E <= 512)
-            rc = launch_kernel("route_warp_kernel", route_warp_kernel<16>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
-        else
-            rc = launch_kernel("route_warp_kernel", route_warp_kernel<32>, blocks, 256, 0, st, logits, nsplit, bias, T, E, k, ids, w);
-        return rc;
+            return launch_route_warp<4>(logits, nsplit, bias, T, E, k, ids, w, blocks, st);
+        if (E <= 256)
+            return launch_route_warp<8>(logits, nsplit, bias, T, E, k, ids, w, blocks, st);
+        if (E <= 384)
+            return launch_route_warp<12>(logits, nsplit, bias, T, E, k, ids, w, blocks, st);
+        if (E <= 512)
+            return launch_route_warp<16>(logits, nsplit, bias, T, E, k, ids, w, blocks, st);
+        return launch_route_warp<32>(logits, nsplit, bias, T, E, k, ids, w, blocks, st);
     }
     return launch_kernel("route_kernel", route_kernel<32>, T, kRouteThreads, 0, st, logits, nsplit, bias, T, E, k, ids,
                          w);

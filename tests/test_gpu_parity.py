@@ -98,16 +98,21 @@ def test_router_gemm(mx, T, H, E):
 
 
 # every expert-count bin of the warp-per-token kernel (128/256/384/512/1024),
-# the block kernel (E > 1024), and logits rounded to few levels (many ties,
-# which go to the lower expert index)
-@pytest.mark.parametrize("T,E,k,ties", [(64, 384, 8, False), (37, 16, 2, False), (5, 1000, 32, False),
-                                        (1, 8, 8, False), (200, 96, 1, False), (33, 256, 8, False),
-                                        (9, 512, 4, False), (17, 1024, 8, False), (3, 3000, 8, False),
-                                        (41, 384, 8, True), (7, 2500, 6, True)])
+# the block kernel (E > 1024), logits rounded to few levels (many ties, which
+# go to the lower expert index), and logits <= 0 whose maximum is a mix of
+# -0.0 and +0.0 (equal values: index order decides)
+@pytest.mark.parametrize("T,E,k,ties", [(64, 384, 8, ""), (37, 16, 2, ""), (5, 1000, 32, ""), (1, 8, 8, ""),
+                                        (200, 96, 1, ""), (33, 256, 8, ""), (9, 512, 4, ""), (17, 1024, 8, ""),
+                                        (3, 3000, 8, ""), (41, 384, 8, "rounded"), (7, 2500, 6, "rounded"),
+                                        (19, 384, 8, "zeros"), (5, 2000, 8, "zeros")])
 def test_route_bitexact(mx, T, E, k, ties):
     l = datagen.make_logits(T, E, seed=T + E)
     if ties:
         l = np.round(l * 2.0).astype(np.float32) / np.float32(2.0)
+    if ties == "zeros":
+        l = -np.abs(l)
+        l[:, 3::7] = np.float32(-0.0)
+        l[:, 5::7] = np.float32(0.0)
     ids_ref, w_ref = oracle.route(l, k)
     ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
     w = torch.empty((T, k), dtype=torch.float32, device=DEV)
