@@ -360,10 +360,11 @@ def run_native(args):
     lws = torch.empty(mx.mxmoe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
     lws_bytes = lws.numel()
 
-    def layer_step(b, x=None):
+    def layer_step(b, x=None, y_out=None):
         x = xs[b % nb] if x is None else x
-        rc = L.mxmoe_layer_forward(P(x), P(wg), P(bias), P(prepacked), T, H, I, E, k, P(y), P(ids), P(w), P(lws),
-                                   lws_bytes, sp)
+        y_out = y if y_out is None else y_out
+        rc = L.mxmoe_layer_forward(P(x), P(wg), P(bias), P(prepacked), T, H, I, E, k, P(y_out), P(ids), P(w),
+                                   P(lws), lws_bytes, sp)
         if rc:
             raise RuntimeError("mxmoe_layer_forward failed: " + mx.last_error())
 
@@ -433,24 +434,48 @@ def run_native(args):
     barrier()
     unit_ms = [a.elapsed_time(b) for a, b in ev_unit]
 
-    # --- end to end through the public API with host buffers
+    # --- end to end through the public API with host buffers: every step
+    # uploads its x from pinned host memory and downloads its y. The copies
+    # run on their own streams into double-buffered device x and y, ordered
+    # by events, so that step i+1's upload and step i-1's download overlap
+    # step i's layer, as in a serving loop.
     x_host = [xb.cpu().pin_memory() for xb in xs]
-    y_host = torch.empty((T, H), dtype=torch.float32).pin_memory()
-    x_dev = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    y_host = [torch.empty((T, H), dtype=torch.float32).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    y_dev = [torch.empty((T, H), dtype=torch.float32, device=dev) for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_ready, x_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
+    y_ready, y_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(b):
-        x_dev.copy_(x_host[b % nb], non_blocking=True)
-        layer_step(b, x_dev)
-        y_host.copy_(y, non_blocking=True)
+    def e2e_step(s):
+        j = s & 1
+        up.wait_event(x_free[j])  # the layer two steps back has read x_dev[j]
+        with torch.cuda.stream(up):
+            x_dev[j].copy_(x_host[s % nb], non_blocking=True)
+        x_ready[j].record(up)
+        stream.wait_event(x_ready[j])
+        stream.wait_event(y_free[j])  # y_dev[j] of two steps back is downloaded
+        layer_step(s, x_dev[j], y_dev[j])
+        x_free[j].record(stream)
+        y_ready[j].record(stream)
+        down.wait_event(y_ready[j])
+        with torch.cuda.stream(down):
+            y_host[j].copy_(y_dev[j], non_blocking=True)
+        y_free[j].record(down)
 
-    for i in range(args.warmup):
-        e2e_step(i)
+    def e2e_run(first, n):
+        for i in range(first, first + n):
+            e2e_step(i)
+        for j in range(2):  # the last downloads end the region
+            stream.wait_event(y_free[j])
+
+    e2e_run(0, args.warmup)
     barrier()
     torch.cuda.synchronize()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s2.record(stream)
-    for i in range(args.steps):
-        e2e_step(args.warmup + i)
+    up.wait_event(s2)
+    e2e_run(args.warmup, args.steps)
     e2.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -507,7 +532,8 @@ def run_native(args):
         "clocks": clk,
         "gpu_launches": kernels_per_step(T, k, E, H) * args.steps,
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
-                "d2h_bytes_per_step": T * H * 4, "api": "mxmoe_layer_forward with pinned host x/y copies"},
+                "d2h_bytes_per_step": T * H * 4, "api": "mxmoe_layer_forward with pinned host x/y copies on their own streams, "
+                       "double-buffered (step i+1's upload and step i-1's download overlap step i)"},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.seed, xs[0].cpu(), bias_np)
