@@ -23,6 +23,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -108,11 +109,16 @@ def load_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the term kernel's code (comments and blank lines left out), which
+    keys the committed traffic capture to the code it was taken on."""
     h = hashlib.sha256()
     for rel in ("mxfp4_quantized_moe_router_b200/csrc/ffn.cu", "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
                 "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("\n".join(line.rstrip() for line in src.splitlines() if line.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -15,10 +15,10 @@
 //    packed E2M1 activation codes, applies both operands' UE8M0 scales per 32
 //    elements of K in hardware and accumulates in fp32 in tensor memory. No
 //    instruction touches a weight element.
-//  * A block-scaled MMA costs about the same issue time at any N, so the
-//    weights are the N operand, 256 rows per MMA, and each MMA covers 8 KB of
-//    weight codes (256 rows x 64 values of K): enough that the weight stream,
-//    not the MMA issue, sets the pace.
+//  * The weights are the N operand, 256 rows per MMA, so that each MMA
+//    covers 8 KB of weight codes (256 rows x 64 values of K): the fewest MMAs
+//    per weight byte, and the weight stream, not the tensor pipe (about a
+//    third busy), sets the pace.
 //  * Activations become kT = 8 E2M1 terms per value: the balanced base-8
 //    digits (each in -4..4, all exact E2M1 values) of the value on the grid
 //    2^(E-22), E the exponent of its 32-value block's largest magnitude; term
@@ -804,10 +804,12 @@ constexpr int64_t kBf16Rows = 16384;
 bool use_bf16_path(int T, int k) { return (int64_t)T * k >= kBf16Rows; }
 
 // Below that, experts with at least kHotRows rows (a skewed router) still go
-// to the bf16 kernel, the rest to the E2M1-term kernel: an E2M1-term pass of 16
-// tokens costs about as much MMA issue as 1/5 of a 256-token bf16 pass, so the
-// bf16 kernel wins from about a hundred tokens per expert. Only token counts
-// that can produce such an expert (T >= kHotRows) launch its kernels.
+// to the bf16 kernel, the rest to the E2M1-term kernel: the E2M1-term kernel
+// multiplies 8 terms per activation value and re-streams the expert's weights
+// for every 16-token pass, so from about a hundred tokens per expert the bf16
+// kernel is cheaper (cuts of 64, 128, 256 and 512 rows measured within noise of
+// each other). Only token counts that can produce such an expert
+// (T >= kHotRows) launch its kernels.
 constexpr int kHotRows = 128;
 bool use_hybrid(int T, int k) { return !use_bf16_path(T, k) && T >= kHotRows; }
 int bf16_min_rows(int T, int k) { return use_bf16_path(T, k) ? 0 : kHotRows; }

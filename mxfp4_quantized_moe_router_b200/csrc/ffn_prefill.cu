@@ -19,15 +19,15 @@
 //  * A work item is (expert, pass of up to 256 tokens, one 256-row box of the
 //    prepacked blob) = two 128-row MMA tiles. A K step is 64 values.
 //  * Three rings in shared memory, each with its own producer or writer, so
-//    that no role waits on another's latency: activation steps (TMA, 3 x 32 KB;
-//    one step per K step for gate/up, two for down: hi then lo), packed weights
-//    with their scale images (TMA + bulk copy, 3 x 17 KB of two K steps each,
-//    issued by a second producer warp ahead), and dequantised bf16 weight tiles (2 x
-//    32 KB, written by sixteen warps, two threads per row, in the
-//    128-byte-swizzled K-major layout the MMA reads).
+//    that no role waits on another's latency: activation steps (bulk copies,
+//    2 x 32 KB; one step per K step for gate/up, two for down: hi then lo),
+//    packed weights with their scale images (TMA + bulk copy, 3 x 17 KB of two
+//    K steps each, issued by a second producer warp ahead), and dequantised
+//    bf16 weight tiles (3 x 32 KB, written by sixteen warps, two threads per
+//    row, in the 128-byte-swizzled K-major layout the MMA reads).
 //  * Two MMA warps each own one tile and one accumulator (128 lanes x 256
-//    columns, together all of tensor memory): an MMA costs about the same issue
-//    time whatever its shape, and two issuing threads double the rate.
+//    columns, together all of tensor memory), so that the tiles' MMAs are
+//    issued independently and each accumulator has its own epilogue warps.
 //  * Eight epilogue warps, four per accumulator, drain both at once: gate/up
 //    applies SwiGLU (tile row 32q + w is gate row 16q + w of the tile's 64,
 //    w < 16, or the matching up row) and writes h as bf16 hi/lo terms; down
@@ -52,9 +52,9 @@ constexpr uint64_t kPWaitNs = 2000000000ull;  // bounded waits: 2 s
 constexpr int kPThreads = 896;  // 28 warps: see the role list at the kernel
 constexpr int kPK = 64;         // K per step
 constexpr int kPTok = 256;      // tokens per pass
-constexpr int kPBStages = 3;    // activation ring
+constexpr int kPBStages = 2;    // activation ring
 constexpr int kPWStages = 3;    // packed weight ring (a slot holds two K steps)
-constexpr int kPAStages = 2;    // dequantised weight ring
+constexpr int kPAStages = 3;    // dequantised weight ring (a third slot measured faster than a third activation slot)
 constexpr int kPBBytes = kPTok * 128;  // activation step: 256 rows x 64 bf16
 constexpr int kPABytes = 128 * 128;    // one bf16 weight tile step: 128 rows x 64 bf16
 constexpr int kPWBytes = 256 * 64;     // packed codes of two K steps: 256 rows x 128 codes
