@@ -18,6 +18,13 @@ parameters in the model summary, 384 * 3 * 6144 * 2048 * 70 layers = 1.015T):
                   popularity follows Zipf(s=1.2)
 * ``prefill8192`` same layer, T 8192
 
+Block verification (``make_verify_inputs``): B sequences, each a block of K
+drafted tokens over a vocabulary of V. The full-size vocabulary 152064 is a
+stand-in: the pages name the drafter's mask token id 151669 (nxbn.cn article,
+DFlash configuration), so the vocabulary holds at least 151670 entries; 152064
+rounds that up to a multiple of 256. B = 1 and 32 match the verify8 and
+verify256 token counts (8 and 256 tokens = 1 and 32 blocks of 8).
+
 Distributions: activations x ~ N(0, 1), router weights ~ N(0, 0.02), expert
 weights ~ N(0, 0.02), each drawn in float32 by a seeded torch generator and
 rounded to bf16 (round to nearest even). Each tensor (and each expert's
@@ -57,7 +64,7 @@ CONFIGS = [
 ]
 BY_NAME = {c.name: c for c in CONFIGS}
 
-_TAGS = {"x": 1, "wg": 2, "w13": 3, "w2": 4, "bias": 5, "logits": 6, "ids": 7, "misc": 8}
+_TAGS = {"x": 1, "wg": 2, "w13": 3, "w2": 4, "bias": 5, "logits": 6, "ids": 7, "misc": 8, "verify": 9}
 
 
 def _seed(seed: int, tag: str, idx: int = 0) -> int:
@@ -159,3 +166,28 @@ def sample_tokens(T: int, n: int = 256, seed: int = 0) -> np.ndarray:
         return np.arange(T)
     rng = np.random.default_rng(int(seed) + 1)
     return np.sort(rng.choice(T, n, replace=False))
+
+
+VERIFY_VOCAB = 152064
+
+
+def make_verify_inputs(B: int, K: int, V: int, seed: int = 0, draft_noise: float = 0.4):
+    """Synthetic inputs of a block verification: float32 backbone logits
+    [B, K+1, V] (N(0, 1) plus, per row, one token raised by U(5, 12) so that
+    rows are peaked like a language model's), float32 drafter logits [B, K, V]
+    (the backbone's first K rows plus N(0, draft_noise^2)), int32 draft tokens
+    [B, K] (the argmax of each drafter row) and float32 uniforms [B, K+1] in
+    [0, 1). At V = 152064 these give mean accepted lengths of about 4
+    (sampling at temperature 1) and 6.4 (greedy), inside the 3.18-6.30 range
+    of the acceptance-length table on the model card (section 3). Only random
+    draws and an argmax; no verification arithmetic."""
+    rng = np.random.default_rng(_seed(seed, "verify"))
+    z = rng.standard_normal((B, K + 1, V), dtype=np.float32)
+    top = rng.integers(0, V, (B, K + 1))
+    boost = rng.uniform(5.0, 12.0, (B, K + 1)).astype(np.float32)
+    np.put_along_axis(z, top[..., None], np.take_along_axis(z, top[..., None], 2) + boost[..., None], 2)
+    w = z[:, :K] + rng.standard_normal((B, K, V), dtype=np.float32) * np.float32(draft_noise)
+    d = np.argmax(w, axis=2).astype(np.int32)
+    u = rng.random((B, K + 1), dtype=np.float32)
+    u = np.minimum(u, np.float32(1.0) - np.float32(2.0**-24))
+    return z, w.astype(np.float32), d, u

@@ -73,8 +73,11 @@ def _load():
         lib.mxo_combine.argtypes = [P, P, P, I64, I32, I64, P]
         lib.mxo_expert_ffn.argtypes = [P, P, P, I64, I64, I64, P, P]
         lib.mxo_expert_ffn_mxfp4.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
+        lib.mxo_verify_block.argtypes = [P, P, P, P, I64, I32, I64, ctypes.c_double, P, P, P, P]
+        lib.mxo_draw_interval.argtypes = [P, P, I64, ctypes.c_double, I64, P, P]
         for f in ("mxo_quantize", "mxo_dequantize", "mxo_router_logits", "mxo_route", "mxo_route_f32",
-                  "mxo_permute", "mxo_combine", "mxo_expert_ffn", "mxo_expert_ffn_mxfp4"):
+                  "mxo_permute", "mxo_combine", "mxo_expert_ffn", "mxo_expert_ffn_mxfp4", "mxo_verify_block",
+                  "mxo_draw_interval"):
             getattr(lib, f).restype = None
         _lib = lib
         return lib
@@ -244,3 +247,45 @@ def moe_layer(x, wg, bias, expert_fetch, k: int, threads: int = 1):
     y = combine(y_perm, dst_of, w, n, k)
     return dict(y=y, ids=ids, w=w, logits=logits, offsets=offsets, src_row=src_row, dst_of=dst_of,
                 touched=len(touched))
+
+
+# --- block verification of a speculative draft ----------------------------
+def verify_block(target: np.ndarray, draft, dtok: np.ndarray, u: np.ndarray, tau: float):
+    """Verify B drafted blocks of K tokens (see ``mxo_verify_block`` in the C
+    file for the reading of the pages' rejection-sampling verification).
+
+    target float32 [B, K+1, V]; draft float32 [B, K, V] (None when tau = 0);
+    dtok int32 [B, K]; u float32 [B, K+1] in [0, 1); tau >= 0 (0: greedy).
+    Returns (accepted int32 [B], tokens int32 [B, K+1], margin_acc float64
+    [B], margin_draw float64 [B])."""
+    target = np.ascontiguousarray(target, np.float32)
+    B, K1, V = target.shape
+    K = K1 - 1
+    dtok = np.ascontiguousarray(dtok, np.int32)
+    u = np.ascontiguousarray(u, np.float32)
+    assert dtok.shape == (B, K) and u.shape == (B, K + 1)
+    dp = None
+    if tau != 0.0:
+        draft = np.ascontiguousarray(draft, np.float32)
+        assert draft.shape == (B, K, V)
+        dp = _p(draft)
+    acc = np.empty(B, np.int32)
+    tokens = np.empty((B, K + 1), np.int32)
+    m_acc = np.empty(B, np.float64)
+    m_draw = np.empty(B, np.float64)
+    _load().mxo_verify_block(_p(target), dp, _p(dtok), _p(u), B, K, V, float(tau), _p(acc), _p(tokens), _p(m_acc),
+                             _p(m_draw))
+    return acc, tokens, m_acc, m_draw
+
+
+def draw_interval(z_row: np.ndarray, w_row, tau: float, v: int) -> tuple[float, float]:
+    """[lo, hi) that token v covers in the normalised running sum of a draw's
+    weights: the residual max(0, p - q) when a drafter row is given, else p."""
+    z_row = np.ascontiguousarray(z_row, np.float32)
+    wp = None
+    if w_row is not None:
+        w_row = np.ascontiguousarray(w_row, np.float32)
+        wp = _p(w_row)
+    lo, hi = ctypes.c_double(), ctypes.c_double()
+    _load().mxo_draw_interval(_p(z_row), wp, z_row.size, float(tau), int(v), ctypes.byref(lo), ctypes.byref(hi))
+    return lo.value, hi.value

@@ -351,3 +351,164 @@ void mxo_expert_ffn_mxfp4(const uint8_t *packed13, const uint8_t *sc13, const ui
     free(w13);
     free(w2);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Block verification of a speculative draft                                 */
+/* ------------------------------------------------------------------------ */
+
+/* softmax(z / tau) of one row of V float logits into p (double). */
+static void softmax_row(const float *z, int64_t V, double tau, double *p)
+{
+    double zmax = (double)z[0];
+    for (int64_t v = 1; v < V; ++v)
+        if ((double)z[v] > zmax)
+            zmax = (double)z[v];
+    double s = 0.0;
+    for (int64_t v = 0; v < V; ++v) {
+        p[v] = exp(((double)z[v] - zmax) / tau);
+        s += p[v];
+    }
+    for (int64_t v = 0; v < V; ++v)
+        p[v] /= s;
+}
+
+/* Index of the largest of V float logits, a tie going to the lower index. */
+static int64_t argmax_row(const float *z, int64_t V)
+{
+    int64_t best = 0;
+    for (int64_t v = 1; v < V; ++v)
+        if (z[v] > z[best])
+            best = v;
+    return best;
+}
+
+/* Verify B blocks of K drafted tokens against the backbone.
+ *
+ * "MiMo-V2.5-Pro-FP4-DFlash" (alphaneural mirror), section 3 "Block-Diffusion
+ * Speculative Decoding (DFlash)": the drafter fills a whole block of masked
+ * positions (at most 8) in one forward pass, the backbone verifies the block
+ * in one step, and the rejection-sampling verification keeps the output
+ * lossless. The pages give no formula; the reading here is the standard
+ * speculative-sampling test, taken position by position in block order:
+ *   p_i = softmax(z_i / tau) from the backbone's logits z_i at block position
+ *   i, q_i = softmax(w_i / tau) from the drafter's logits w_i;
+ *   draft token d_i is accepted when u_i * q_i(d_i) < p_i(d_i), u_i uniform
+ *   in [0, 1) and passed in;
+ *   at the first rejection j the output token is drawn from max(0, p_j - q_j)
+ *   normalised, and after K acceptances from p_K, both by inverse CDF in
+ *   token order with u_K: the smallest v whose running sum exceeds u_K times
+ *   the total (the last v with a non-zero weight if rounding leaves none).
+ * tau = 0 is greedy verification: d_i is accepted while it equals the argmax
+ * of z_i (a tie going to the lower token index); the output token is the
+ * argmax of z_n at the first mismatch n (n = K after K matches).
+ * A draft token outside [0, V) is never accepted.
+ *
+ * target float [B][K+1][V]; draft float [B][K][V] (not read when tau = 0);
+ * dtok int32 [B][K]; u float [B][K+1]; accepted int32 [B]; tokens int32
+ * [B][K+1]: the accepted drafts, then the output token, then -1.
+ * margin_acc, margin_draw (each may be NULL) double [B]: how far the
+ * decisions taken lie from their thresholds, for tests that compare with
+ * lower-precision arithmetic: the smallest |u q - p| / max(u q, p) over the
+ * acceptance tests taken, and the distance of u_K times the total from the
+ * nearer running-sum boundary of the drawn token, over the total; infinity for
+ * greedy verification, whose comparisons are exact. */
+void mxo_verify_block(const float *target, const float *draft, const int32_t *dtok, const float *u, int64_t B, int K,
+                      int64_t V, double tau, int32_t *accepted, int32_t *tokens, double *margin_acc,
+                      double *margin_draw)
+{
+    double *p = (double *)malloc(sizeof(double) * (size_t)V);
+    double *q = (double *)malloc(sizeof(double) * (size_t)V);
+    for (int64_t b = 0; b < B; ++b) {
+        const float *zb = target + b * (int64_t)(K + 1) * V;
+        const float *wb = draft ? draft + b * (int64_t)K * V : NULL;
+        const int32_t *db = dtok + b * K;
+        const float *ub = u + b * (K + 1);
+        double mg = INFINITY, mgd = INFINITY;
+        int n = 0;
+        int64_t out = 0;
+        if (tau == 0.0) {
+            while (n < K && db[n] >= 0 && db[n] < V && argmax_row(zb + (int64_t)n * V, V) == db[n])
+                ++n;
+            out = argmax_row(zb + (int64_t)n * V, V);
+        } else {
+            for (n = 0; n < K; ++n) {
+                const int32_t d = db[n];
+                if (d < 0 || d >= V)
+                    break;
+                softmax_row(zb + (int64_t)n * V, V, tau, p);
+                softmax_row(wb + (int64_t)n * V, V, tau, q);
+                const double lhs = (double)ub[n] * q[d], rhs = p[d];
+                const double den = lhs > rhs ? lhs : rhs;
+                if (den > 0.0 && fabs(lhs - rhs) / den < mg)
+                    mg = fabs(lhs - rhs) / den;
+                if (!(lhs < rhs))
+                    break;
+            }
+            /* the weights of the draw: residual at a rejection, else p_K */
+            softmax_row(zb + (int64_t)n * V, V, tau, p);
+            if (n < K) {
+                softmax_row(wb + (int64_t)n * V, V, tau, q);
+                for (int64_t v = 0; v < V; ++v)
+                    p[v] = p[v] > q[v] ? p[v] - q[v] : 0.0;
+            }
+            double total = 0.0;
+            for (int64_t v = 0; v < V; ++v)
+                total += p[v];
+            const double thr = (double)ub[K] * total;
+            double run = 0.0;
+            out = -1;
+            for (int64_t v = 0; v < V; ++v) {
+                const double before = run;
+                run += p[v];
+                if (run > thr) {
+                    out = v;
+                    const double gap = (thr - before) < (run - thr) ? (thr - before) : (run - thr);
+                    mgd = gap / total;
+                    break;
+                }
+            }
+            if (out < 0)
+                for (int64_t v = V - 1; v >= 0; --v)
+                    if (p[v] > 0.0) {
+                        out = v;
+                        break;
+                    }
+        }
+        accepted[b] = n;
+        for (int i = 0; i <= K; ++i)
+            tokens[b * (K + 1) + i] = i < n ? db[i] : (i == n ? (int32_t)out : -1);
+        if (margin_acc)
+            margin_acc[b] = mg;
+        if (margin_draw)
+            margin_draw[b] = mgd;
+    }
+    free(p);
+    free(q);
+}
+
+/* The interval [lo, hi) that token v covers in the normalised running sum of
+ * a draw's weights (the same weights as in mxo_verify_block): the residual
+ * max(0, p - q) when a drafter row w is given, else p; p = softmax(z / tau),
+ * q = softmax(w / tau). A draw with uniform u yields v exactly when
+ * lo <= u < hi. */
+void mxo_draw_interval(const float *z, const float *w, int64_t V, double tau, int64_t v, double *lo, double *hi)
+{
+    double *p = (double *)malloc(sizeof(double) * (size_t)V);
+    double *q = (double *)malloc(sizeof(double) * (size_t)V);
+    softmax_row(z, V, tau, p);
+    if (w) {
+        softmax_row(w, V, tau, q);
+        for (int64_t i = 0; i < V; ++i)
+            p[i] = p[i] > q[i] ? p[i] - q[i] : 0.0;
+    }
+    double total = 0.0, before = 0.0;
+    for (int64_t i = 0; i < V; ++i) {
+        if (i == v)
+            before = total;
+        total += p[i];
+    }
+    *lo = before / total;
+    *hi = (before + p[v]) / total;
+    free(p);
+    free(q);
+}
