@@ -77,6 +77,11 @@ def parse_args():
                     help="profiling only: shrink the layer to this many experts (0 = the workload's)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="profiling only: this many tokens per step (0 = the workload's)")
+    ap.add_argument("--workload", choices=["layer", "verify_block"], default="layer",
+                    help="layer: the MoE layer (the headline); verify_block: block verification of drafts")
+    ap.add_argument("--blocks", type=int, default=32, help="verify_block: drafted blocks per step")
+    ap.add_argument("--vocab", type=int, default=datagen.VERIFY_VOCAB, help="verify_block: vocabulary size")
+    ap.add_argument("--temperature", type=float, default=1.0, help="verify_block: 0 = greedy verification")
     return ap.parse_args()
 
 
@@ -548,9 +553,217 @@ def run_native(args):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------
+# block verification workload
+# ---------------------------------------------------------------------------
+VERIFY_K = 8  # drafted tokens per block (the model card's verify block)
+VERIFY_METRIC = "verified draft blocks/s (8 drafted tokens each); logit HBM GB/s as % of peak (1xB200)"
+VERIFY_UNIT = "blocks/s"
+
+
+def verify_config(args, world: int, nb: int):
+    mode = "greedy" if args.temperature == 0 else "rejection sampling, temperature %g" % args.temperature
+    return {
+        "workload": "verify_block: %d blocks of %d drafted tokens, vocabulary %d, %s"
+                    % (args.blocks, VERIFY_K, args.vocab, mode),
+        "blocks_per_step": args.blocks, "block_size": VERIFY_K, "vocab": args.vocab,
+        "temperature": args.temperature, "parallelism": "replicas x%d" % world,
+        "l2": "inputs larger than L2: %d rotating input batches of fp32 logits" % nb,
+    }
+
+
+def run_verify_reference(args):
+    """--impl reference --workload verify_block: the float64 oracle on host cores."""
+    import oracle
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    tau = args.temperature
+    z, w, d, u = datagen.make_verify_inputs(1, VERIFY_K, args.vocab, seed=args.seed)
+    times = []
+    for i in range(args.warmup + args.steps):  # one block per step: a bounded sample
+        t0 = time.perf_counter()
+        oracle.verify_block(z, w if tau > 0 else None, d, u, tau)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = len(times) / total
+    print(json.dumps({
+        "impl": "reference", "metric": VERIFY_METRIC, "value": value, "unit": VERIFY_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": verify_config(args, 1, 1),
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": VERIFY_UNIT,
+                         "sample": "each step: 1 block through the float64 C oracle, one thread"},
+        "e2e": {"value": value, "unit": VERIFY_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_verify(args):
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_quantized_moe_router_b200 as mx
+
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, K, V, tau = args.blocks, VERIFY_K, args.vocab, args.temperature
+    rows = 2 * K + 1 if tau > 0 else K + 1
+    step_bytes = B * rows * V * 4
+    nb = max(1, min(args.batches, 1 + (512 << 20) // max(step_bytes, 1)))  # rotate over more than L2
+    batches = []
+    for i in range(nb):
+        z, w, d, u = datagen.make_verify_inputs(B, K, V, seed=replica_input_seed(args.seed, rank, i))
+        batches.append((torch.from_numpy(z).to(dev), torch.from_numpy(w).to(dev) if tau > 0 else None,
+                        torch.from_numpy(d).to(dev), torch.from_numpy(u).to(dev)))
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    tok = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    ws = torch.empty(max(mx.mxmoe_verify_workspace_size(B, K, V), 1), dtype=torch.uint8, device=dev)
+    L = mx.load()
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    P = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+
+    def step(i, inputs=None, out=None):
+        zt, wt, dt, ut = inputs if inputs is not None else batches[i % nb]
+        a, t = out if out is not None else (acc, tok)
+        rc = L.mxmoe_verify_block(P(zt), P(wt), P(dt), P(ut), B, K, V, tau, P(a), P(t), P(ws), ws.numel(), sp)
+        if rc:
+            raise RuntimeError("mxmoe_verify_block failed: " + mx.last_error())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    accepted_mean = []
+    for i in range(nb):
+        step(i)
+        torch.cuda.synchronize()
+        accepted_mean.append(float(acc.float().mean()))
+    clocks = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.warmup):
+        step(i)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    clk = clocks.summary(t0, t1)
+    # end to end: each step uploads its logits, drafts and uniforms from pinned
+    # host memory and downloads the verdicts, copies on their own streams
+    # (double-buffered) so that they overlap the neighbouring steps' kernels
+    hosts = [tuple(None if x is None else x.cpu().pin_memory() for x in bt) for bt in batches[:2]]
+    devs = [tuple(None if x is None else torch.empty_like(x) for x in batches[0]) for _ in range(2)]
+    outs = [(torch.empty_like(acc), torch.empty_like(tok)) for _ in range(2)]
+    outs_h = [(torch.empty(B, dtype=torch.int32).pin_memory(), torch.empty((B, K + 1), dtype=torch.int32).pin_memory())
+              for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+    in_ready, in_free, out_ready, out_free = ev(), ev(), ev(), ev()
+
+    def e2e_step(s):
+        j = s & 1
+        up.wait_event(in_free[j])
+        with torch.cuda.stream(up):
+            for dst, src in zip(devs[j], hosts[s % len(hosts)]):
+                if dst is not None:
+                    dst.copy_(src, non_blocking=True)
+        in_ready[j].record(up)
+        stream.wait_event(in_ready[j])
+        stream.wait_event(out_free[j])
+        step(s, devs[j], outs[j])
+        in_free[j].record(stream)
+        out_ready[j].record(stream)
+        down.wait_event(out_ready[j])
+        with torch.cuda.stream(down):
+            outs_h[j][0].copy_(outs[j][0], non_blocking=True)
+            outs_h[j][1].copy_(outs[j][1], non_blocking=True)
+        out_free[j].record(down)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    up.wait_event(s2)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    for j in range(2):
+        stream.wait_event(out_free[j])
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(s2.elapsed_time(e2), world, dev)
+    clocks.stop()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    peak, _, peak_kind = load_peaks()
+    ms_step = ms / args.steps
+    achieved = step_bytes / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": VERIFY_METRIC, "value": B * args.steps * world / (ms / 1e3), "unit": VERIFY_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded datagen: peaked fp32 logits, drafts = the drafter's argmax, uniforms)",
+        "config": verify_config(args, world, nb),
+        "mean_accepted": float(np.mean(accepted_mean)),
+        "roofline": {"kernel": "mxmoe_verify_block (all %d kernels of the call)" % (4 if tau > 0 else 2),
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                     else "fallback 6.65 TB/s",
+                     "traffic": None, "unit_ms": ms_step, "algorithmic_bytes_per_launch": step_bytes},
+        "clocks": clk,
+        "gpu_launches": (4 if tau > 0 else 2) * args.steps,
+        "e2e": {"value": B * e2e_steps * world / (ms_e2e / 1e3), "unit": VERIFY_UNIT,
+                "h2d_bytes_per_step": step_bytes + B * K * 4 + B * (K + 1) * 4,
+                "d2h_bytes_per_step": B * 4 + B * (K + 1) * 4,
+                "api": "mxmoe_verify_block with pinned host logits/drafts/uniforms and verdict copies on their own "
+                       "streams (double-buffered)"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        z, w, d, u = datagen.make_verify_inputs(1, K, V, seed=args.seed)
+        t_cpu = time.perf_counter()
+        n_cpu = 0
+        while n_cpu < 3 or time.perf_counter() - t_cpu < 2.0:
+            oracle.verify_block(z, w if tau > 0 else None, d, u, tau)
+            n_cpu += 1
+        v_cpu = n_cpu / (time.perf_counter() - t_cpu)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": VERIFY_UNIT, "cores": 1, "kind": "oracle",
+                                "sample": "%d single blocks through the float64 C oracle, one thread" % n_cpu}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.workload == "verify_block":
+        if args.impl == "reference":
+            run_verify_reference(args)
+        else:
+            run_verify(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_native(args)

@@ -283,6 +283,51 @@ MXMOE_API int mxmoe_selftest_wait_timeout(int *status, int limit_us, void *strea
  *   workspace device (as passed to the call); *status host int. */
 MXMOE_API int mxmoe_read_status(const void *workspace, int *status, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Block verification of a speculative draft
+ *
+ * "MiMo-V2.5-Pro-FP4-DFlash" (alphaneural mirror), section 3
+ * "Block-Diffusion Speculative Decoding (DFlash)": the drafter proposes a
+ * block of tokens (at most 8) in one pass and the backbone verifies the whole
+ * block in one step; rejection-sampling verification keeps the output
+ * lossless. Reading (the pages give no formula): the standard
+ * speculative-sampling test in block order. With p_i = softmax(z_i / tau) of
+ * the backbone's logits at block position i and q_i = softmax(w_i / tau) of
+ * the drafter's, draft token d_i is accepted when u_i q_i(d_i) < p_i(d_i);
+ * at the first rejection j the emitted token is drawn from max(0, p_j - q_j),
+ * after K acceptances from p_K, both by inverse CDF in token order with u_K
+ * (the smallest v whose running sum exceeds u_K times the total). tau = 0 is
+ * greedy verification: d_i is accepted while it is the argmax of z_i (ties
+ * to the lower index) and the emitted token is the argmax at the first
+ * mismatch. A draft token outside [0, V) is never accepted. Arithmetic is
+ * fp32; a decision whose two sides are within float rounding of each other
+ * (a uniform on a threshold) may differ from an exact evaluation.
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes for mxmoe_verify_block with these sizes; -1 if invalid. */
+MXMOE_API int64_t mxmoe_verify_workspace_size(int B, int K, int64_t V);
+
+/* Verify B blocks of K drafted tokens.
+ *   target_logits device float [B, K+1, V]: the backbone's logits at the K
+ *       block positions and the position after the block.
+ *   draft_logits device float [B, K, V]: the drafter's logits (may be NULL
+ *       when temperature == 0).
+ *   draft_tokens device int32 [B, K]; uniforms device float [B, K+1] in
+ *       [0, 1): u_0 .. u_{K-1} for the acceptance tests, u_K for the draw.
+ *   temperature >= 0, finite (0: greedy).
+ *   accepted device int32 [B]: accepted drafts n (0 .. K).
+ *   tokens device int32 [B, K+1]: the n accepted drafts, then the emitted
+ *       token, then -1.
+ *   workspace device, >= mxmoe_verify_workspace_size(B, K, V) bytes,
+ *       256-byte aligned; contents not kept between calls.
+ * Errors: K < 1, K > 32, V < 1, V > 2^24, B < 0 -> INVALID_SHAPE;
+ * a negative or non-finite temperature -> INVALID_SHAPE; NULL pointers ->
+ * NULL; workspace too small -> WORKSPACE, misaligned -> ALIGNMENT. */
+MXMOE_API int mxmoe_verify_block(const float *target_logits, const float *draft_logits,
+                                 const int32_t *draft_tokens, const float *uniforms, int B, int K, int64_t V,
+                                 float temperature, int32_t *accepted, int32_t *tokens, void *workspace,
+                                 int64_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

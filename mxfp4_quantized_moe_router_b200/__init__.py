@@ -54,6 +54,8 @@ _SIGS = {
     "mxmoe_selftest_wait_timeout": (_I, [_P, _I, _P]),
     "mxmoe_permute_ws": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
     "mxmoe_permute_scratch_size": (_I64, [_I, _I, _I]),
+    "mxmoe_verify_workspace_size": (_I64, [_I, _I, _I64]),
+    "mxmoe_verify_block": (_I, [_P, _P, _P, _P, _I, _I, _I64, ctypes.c_float, _P, _P, _P, _I64, _P]),
 }
 
 _lib = None
@@ -383,3 +385,33 @@ class ExpertWeights:
     def prepack(self, stream=None):
         mxmoe_prepack_experts(self.packed13, self.sc13, self.packed2, self.sc2, self.E, self.H, self.I,
                               self.prepacked, stream)
+
+
+# ---------------------------------------------------------------------------
+# Block verification of a speculative draft
+# ---------------------------------------------------------------------------
+def mxmoe_verify_workspace_size(B, K, V) -> int:
+    return load().mxmoe_verify_workspace_size(B, K, V)
+
+
+def mxmoe_verify_block(target_logits, draft_logits, draft_tokens, uniforms, temperature, accepted, tokens, workspace,
+                       stream=None):
+    """Verify B drafted blocks (see include/mxmoe.h). target_logits float32
+    [B, K+1, V], draft_logits float32 [B, K, V] or None (greedy),
+    draft_tokens int32 [B, K], uniforms float32 [B, K+1], accepted int32 [B],
+    tokens int32 [B, K+1], workspace uint8 of mxmoe_verify_workspace_size."""
+    import torch
+
+    B, K1, V = target_logits.shape
+    K = K1 - 1
+    _need(target_logits, torch.float32, (B, K + 1, V), "target_logits")
+    if draft_logits is not None:
+        _need(draft_logits, torch.float32, (B, K, V), "draft_logits")
+    _need(draft_tokens, torch.int32, (B, K), "draft_tokens")
+    _need(uniforms, torch.float32, (B, K + 1), "uniforms")
+    _need(accepted, torch.int32, (B,), "accepted")
+    _need(tokens, torch.int32, (B, K + 1), "tokens")
+    _check("mxmoe_verify_block",
+           load().mxmoe_verify_block(_ptr(target_logits), _ptr(draft_logits), _ptr(draft_tokens), _ptr(uniforms), B,
+                                     K, V, float(temperature), _ptr(accepted), _ptr(tokens), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)))

@@ -138,3 +138,28 @@ def test_grouping_expert_limit(mx):
     assert lib.mxmoe_permute(None, 4, 2, 2000, None, None, None, None) == mx.ERR_INVALID_SHAPE
     assert lib.mxmoe_permute_scratch_size(4, 2, 1025) == -1
     assert lib.mxmoe_permute_scratch_size(4, 2, 1024) > 0
+
+
+def test_verify_block_queries_and_rejects_on_host(mx):
+    lib = mx.load()
+    V = 152064
+    ws = lib.mxmoe_verify_workspace_size(32, 8, V)
+    # partials of 17 rows x 19 chunks x 16 bytes per block, then per-block draw state and chunk sums
+    assert ws >= 32 * 17 * 19 * 16 and ws < 32 * 17 * 19 * 16 + 8192
+    assert lib.mxmoe_verify_workspace_size(1, 8, V) < ws
+    assert lib.mxmoe_verify_workspace_size(1, 0, V) == -1
+    assert lib.mxmoe_verify_workspace_size(1, 33, V) == -1
+    assert lib.mxmoe_verify_workspace_size(1, 8, 0) == -1
+    assert lib.mxmoe_verify_workspace_size(1, 8, (1 << 24) + 1) == -1
+    assert lib.mxmoe_verify_workspace_size(1, 8, 1 << 24) > 0
+    base = 1 << 20  # never dereferenced: rejected before anything is enqueued
+    big = 1 << 40
+    f = lib.mxmoe_verify_block
+    assert f(base, base, base, base, 1, 0, V, 1.0, base, base, base, big, None) == mx.ERR_INVALID_SHAPE
+    assert f(base, base, base, base, 1, 8, V, -1.0, base, base, base, big, None) == mx.ERR_INVALID_SHAPE
+    assert f(base, base, base, base, 1, 8, V, float("inf"), base, base, base, big, None) == mx.ERR_INVALID_SHAPE
+    assert f(base, base, base, base, 1, 8, V, float("nan"), base, base, base, big, None) == mx.ERR_INVALID_SHAPE
+    assert f(base, base, base, base, 1, 8, V, 1.0, base, base, base, 16, None) == mx.ERR_WORKSPACE
+    assert f(base, None, base, base, 1, 8, V, 1.0, base, base, base, big, None) == mx.ERR_NULL  # sampling needs q
+    assert f(base, base, base, base, 1, 8, V, 1.0, base, base, base + 16, big, None) == mx.ERR_ALIGNMENT
+    assert f(None, None, None, None, 0, 8, V, 0.0, None, None, None, 0, None) == mx.OK  # nothing to do
