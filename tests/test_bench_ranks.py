@@ -99,3 +99,24 @@ def test_launch_count_follows_the_dispatch():
     # verify8: one grouping kernel, E2M1-term FFN; verify256: hybrid; zipf1024: hybrid + multi-block grouping;
     # prefill8192: bf16 FFN + multi-block grouping
     assert [bench.kernels_per_step(T, 8, 384, 6144) for T in (8, 256, 1024, 8192)] == [7, 12, 14, 11]
+
+
+def test_verify_workload_reference_arm_prints_the_contract_line():
+    # the verification workload's reference arm: the float64 oracle on host
+    # cores, one block per step, printed as one JSON line with the base keys
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "verify_block", "--impl",
+                        "reference", "--steps", "2", "--warmup", "1", "--vocab", "3000"], capture_output=True,
+                       text=True, timeout=300, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["unit"] == "blocks/s" and line["value"] > 0
+    assert line["config"]["vocab"] == 3000 and line["config"]["block_size"] == 8
+    # off rank 0 the arm does nothing
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    q = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "verify_block", "--impl",
+                        "reference", "--steps", "2", "--warmup", "1", "--vocab", "3000"], capture_output=True,
+                       text=True, timeout=300, cwd=ROOT, env=env)
+    assert q.returncode == 0 and q.stdout.strip() == ""
