@@ -38,8 +38,10 @@
 //  * Stage 1 (gate/up): a 256-row tile is 128 gate rows and the matching 128
 //    up rows; SwiGLU and the term encoding of h (with its scale images) are
 //    fused into the epilogue. Stage 2 (down): a tile is 256 output rows.
-//  * Work items (expert, tile, token pass of up to NT tokens) are split
-//    contiguously over a persistent grid of one CTA per SM.
+//  * Work items (expert, tile, token pass of up to NT tokens) go round-robin
+//    over a persistent grid of one CTA per SM (CTA b takes items b, b + G,
+//    ...), so that the passes of one weight tile run side by side and share
+//    its boxes in L2.
 #include <float.h>
 #include <limits.h>
 
