@@ -22,8 +22,8 @@
 //  1. verify_rows_kernel: one CTA per (row, 8192-logit chunk) -- max, the sum
 //     of exp((z - max) / tau) and the argmax of the chunk, written as a
 //     partial; coalesced loads, one pass, no atomics.
-//  2. verify_decide_kernel: one CTA per block; its warps merge the rows'
-//     partials in chunk order (max, rescaled sums, argmax) in parallel, then
+//  2. verify_decide_kernel: one CTA per block, a warp per row, merging the
+//     rows' partials in chunk order (max, rescaled sums, argmax), then
 //     thread 0 takes the position-by-position decisions; greedy verification
 //     ends here.
 //  3. verify_draw_sums_kernel: one CTA per (block, chunk) of the drawn row,
@@ -34,6 +34,8 @@
 // Every reduction runs in a fixed order, so results are bit-reproducible.
 #include <float.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 
@@ -194,10 +196,10 @@ __device__ __forceinline__ void merge_row(const RowPart *__restrict__ part, int6
     arg = ai;
 }
 
-// One CTA per block: the eight warps merge the block's rows in parallel,
-// the drafts' logits are read in one round, and thread 0 takes the
-// position-by-position decisions from shared memory.
-__global__ void __launch_bounds__(256) verify_decide_kernel(const float *__restrict__ target,
+// One CTA per block, one warp per row (up to 32 warps): the warps merge the
+// block's rows in parallel, the drafts' logits are read in the same round,
+// and thread 0 takes the position-by-position decisions from shared memory.
+__global__ void __launch_bounds__(1024) verify_decide_kernel(const float *__restrict__ target,
                                                             const float *__restrict__ draft,
                                                             const int32_t *__restrict__ dtok,
                                                             const float *__restrict__ u, int K, int64_t V, int rows,
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(256) verify_decide_kernel(const float *__restr
         s_d[threadIdx.x] = db[threadIdx.x];
     if (threadIdx.x >= 64 && threadIdx.x <= 64 + K)
         s_u[threadIdx.x - 64] = u[(int64_t)b * (K + 1) + threadIdx.x - 64];
-    for (int r = warp; r < rows; r += 8) {
+    for (int r = warp; r < rows; r += (int)(blockDim.x >> 5)) {
         float m, s;
         int arg;
         merge_row(part, (int64_t)b * rows + r, nchunk, k, m, s, arg);
@@ -361,6 +363,7 @@ __global__ void __launch_bounds__(kVThreads) verify_draw_pick_kernel(const float
     __shared__ float s_w[kVChunk + kVChunk / 32];  // the chosen chunk's weights, one pad word per 32
     __shared__ int s_pick, s_last, s_cpick, s_clast;
     const int b = blockIdx.x, t = threadIdx.x;
+    const float uk = __ldg(u + (int64_t)b * (K + 1) + K);  // issued before the dependent loads
     const DrawInfo di = info[b];
     const float rp = 1.f / di.sp, rq = 1.f / di.sq;
     const float *zrow = target + ((int64_t)b * (K + 1) + di.n) * V;
@@ -388,7 +391,7 @@ __global__ void __launch_bounds__(kVThreads) verify_draw_pick_kernel(const float
     }
     __syncthreads();
     const float total = s_incl[nchunk - 1];
-    const float thr = u[(int64_t)b * (K + 1) + K] * total;
+    const float thr = uk * total;
     for (int c0 = t; c0 < nchunk; c0 += kVThreads)
         if (s_incl[c0] > thr)
             atomicMin(&s_cpick, c0);
@@ -519,7 +522,8 @@ extern "C" MXMOE_API int mxmoe_verify_block(const float *target_logits, const fl
     if (int rc = launch_kernel("verify_rows_kernel", verify_rows_kernel, dim3(nchunk, B * rows), kVThreads, 0, st,
                                target_logits, draft_logits, K, V, rows, k, nchunk, part))
         return rc;
-    if (int rc = launch_kernel("verify_decide_kernel", verify_decide_kernel, B, 256, 0, st, target_logits,
+    const int decide_threads = std::min(1024, std::max(128, 32 * rows));  // a warp per row
+    if (int rc = launch_kernel("verify_decide_kernel", verify_decide_kernel, B, decide_threads, 0, st, target_logits,
                                draft_logits, draft_tokens, uniforms, K, V, rows, k, nchunk, part, info, accepted,
                                tokens))
         return rc;

@@ -67,7 +67,7 @@ def check(mx, z, w, d, u, tau, max_skipped=0.1):
 
 @pytest.mark.parametrize("B,K,V,tau", [(5, 3, 50, 0.0), (5, 3, 50, 1.0), (37, 8, 1000, 1.0), (37, 8, 1000, 0.0),
                                        (9, 8, 20011, 1.0), (9, 8, 20011, 0.0), (3, 1, 8192, 0.7), (4, 2, 8193, 1.3),
-                                       (16, 8, 33000, 0.5)])
+                                       (16, 8, 33000, 0.5), (3, 32, 500, 1.0), (3, 32, 500, 0.0)])
 def test_verify_matches_oracle(mx, B, K, V, tau):
     z, w, d, u = datagen.make_verify_inputs(B, K, V, seed=B * 131 + V)
     check(mx, z, w, d, u, tau)
