@@ -243,7 +243,7 @@ MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *offsets, co
  * w[t, j] * y_perm[dst_of[t*k + j], c], float32.
  *   y_perm device float [T*k, H]; dst_of device int32 [T*k]; w device float
  *   [T, k]; y device float [T, H].
- * Errors: H % 4 != 0 -> INVALID_SHAPE; y_perm, y not 16-byte aligned ->
+ * Errors: H % 4 != 0 or T > 65535 -> INVALID_SHAPE; y_perm, y not 16-byte aligned ->
  * ALIGNMENT. */
 MXMOE_API int mxmoe_combine(const float *y_perm, const int32_t *dst_of, const float *w, int T, int k, int H,
                             float *y, void *stream);
@@ -262,7 +262,7 @@ MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, int k);
  *   [T, H]; ids_out device int32 [T, k] or NULL; w_out device float [T, k]
  *   or NULL; workspace device, >= mxmoe_workspace_size bytes, 256-byte
  *   aligned (its first 16 bytes hold the device status word).
- * Errors: the union of the steps' errors. */
+ * Errors: the union of the steps' errors (so T <= 65535, the combine's limit). */
 MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, const float *bias, const void *prepacked, int T,
                                   int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out,
                                   void *workspace, int64_t workspace_bytes, void *stream);
@@ -320,7 +320,7 @@ MXMOE_API int64_t mxmoe_verify_workspace_size(int B, int K, int64_t V);
  *       token, then -1.
  *   workspace device, >= mxmoe_verify_workspace_size(B, K, V) bytes,
  *       256-byte aligned; contents not kept between calls.
- * Errors: K < 1, K > 32, V < 1, V > 2^24, B < 0 -> INVALID_SHAPE;
+ * Errors: K < 1, K > 32, V < 1, V > 2^24, B < 0, B (2K + 1) > 65535 -> INVALID_SHAPE;
  * a negative or non-finite temperature -> INVALID_SHAPE; NULL pointers ->
  * NULL; workspace too small -> WORKSPACE, misaligned -> ALIGNMENT. */
 MXMOE_API int mxmoe_verify_block(const float *target_logits, const float *draft_logits,

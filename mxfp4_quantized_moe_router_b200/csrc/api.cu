@@ -167,9 +167,13 @@ extern "C" MXMOE_API const char *mxmoe_version(void) { return "mxmoe 0.1.0 (sm_1
 
 extern "C" MXMOE_API const char *mxmoe_last_error(void) { return g_err; }
 
+// Token limit of the layer and of the combine: one grid row per token.
+constexpr int kMaxLayerTokens = 65535;
+
 extern "C" MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, int k)
 {
-    if (T < 0 || k < 1 || k > 32 || k > E || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 64 || I % 32)
+    if (T < 0 || T > kMaxLayerTokens || k < 1 || k > 32 || k > E || E <= 0 || E > 1024 || H <= 0 || I <= 0 ||
+        H % 64 || I % 32)
         return -1;
     return layer_ws_layout(T, H, I, E, k, nullptr, nullptr);
 }
@@ -180,6 +184,9 @@ extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, cons
 {
     if (k > E)
         return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_layer_forward: k=%d > E=%d", k, E);
+    if (T > kMaxLayerTokens)
+        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_layer_forward: T=%d > %d (the combine's grid)", T,
+                    kMaxLayerTokens);
     if (int rc = validate_ffn_shapes(T, k, E, H, I))
         return rc;
     const int64_t need = layer_ws_layout(T, H, I, E, k, nullptr, nullptr);

@@ -1138,8 +1138,9 @@ extern "C" MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prep
 extern "C" MXMOE_API int mxmoe_combine(const float *y_perm, const int32_t *dst_of, const float *w, int T, int k,
                                        int H, float *y, void *stream)
 {
-    if (T < 0 || k < 1 || H <= 0 || H % 4)
-        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_combine: T=%d k=%d H=%d (H must be a multiple of 4)", T, k, H);
+    if (T < 0 || T > 65535 || k < 1 || H <= 0 || H % 4)
+        return fail(MXMOE_ERR_INVALID_SHAPE,
+                    "mxmoe_combine: T=%d k=%d H=%d (H must be a multiple of 4, T at most 65535)", T, k, H);
     if (T == 0)
         return MXMOE_OK;
     if (!y_perm || !dst_of || !w || !y)

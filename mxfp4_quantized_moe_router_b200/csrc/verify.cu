@@ -480,9 +480,12 @@ int64_t verify_ws_layout(int B, int K, int64_t V, bool sampling, RowPart **part,
 
 using namespace mxmoe;
 
+// Blocks per call: the row pass puts B (2K + 1) rows on the grid's y extent.
+static bool verify_blocks_ok(int B, int K) { return (int64_t)B * (2 * K + 1) <= 65535; }
+
 extern "C" MXMOE_API int64_t mxmoe_verify_workspace_size(int B, int K, int64_t V)
 {
-    if (B < 0 || K < 1 || K > 32 || V < 1 || V > (int64_t)kVMaxChunks * kVChunk)
+    if (B < 0 || K < 1 || K > 32 || V < 1 || V > (int64_t)kVMaxChunks * kVChunk || !verify_blocks_ok(B, K))
         return -1;
     return verify_ws_layout(B, K, V, true, nullptr, nullptr, nullptr, nullptr);
 }
@@ -492,9 +495,10 @@ extern "C" MXMOE_API int mxmoe_verify_block(const float *target_logits, const fl
                                             int64_t V, float temperature, int32_t *accepted, int32_t *tokens,
                                             void *workspace, int64_t workspace_bytes, void *stream)
 {
-    if (B < 0 || K < 1 || K > 32 || V < 1 || V > (int64_t)kVMaxChunks * kVChunk)
-        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_verify_block: B=%d K=%d V=%lld (need 1 <= K <= 32, V <= 2^24)", B,
-                    K, (long long)V);
+    if (B < 0 || K < 1 || K > 32 || V < 1 || V > (int64_t)kVMaxChunks * kVChunk || !verify_blocks_ok(B, K))
+        return fail(MXMOE_ERR_INVALID_SHAPE,
+                    "mxmoe_verify_block: B=%d K=%d V=%lld (need 1 <= K <= 32, V <= 2^24, B (2K+1) <= 65535)", B, K,
+                    (long long)V);
     if (!(temperature >= 0.f) || isinf(temperature))
         return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_verify_block: temperature must be finite and >= 0");
     const bool sampling = temperature > 0.f;

@@ -163,3 +163,18 @@ def test_verify_block_queries_and_rejects_on_host(mx):
     assert f(base, None, base, base, 1, 8, V, 1.0, base, base, base, big, None) == mx.ERR_NULL  # sampling needs q
     assert f(base, base, base, base, 1, 8, V, 1.0, base, base, base + 16, big, None) == mx.ERR_ALIGNMENT
     assert f(None, None, None, None, 0, 8, V, 0.0, None, None, None, 0, None) == mx.OK  # nothing to do
+
+
+def test_grid_limits_reject_on_host(mx):
+    # one grid row per token in the combine, per logit row in the verification's row pass
+    lib = mx.load()
+    base = 1 << 20  # never dereferenced: rejected before anything is enqueued
+    assert lib.mxmoe_combine(base, base, base, 65536, 8, 6144, base, None) == mx.ERR_INVALID_SHAPE
+    assert mx.mxmoe_workspace_size(65536, 6144, 2048, 384, 8) == -1
+    assert mx.mxmoe_workspace_size(65535, 6144, 2048, 384, 1) > 0
+    assert lib.mxmoe_layer_forward(base, base, None, base, 65536, 6144, 2048, 384, 8, base, None, None, base,
+                                   1 << 40, None) == mx.ERR_INVALID_SHAPE
+    assert lib.mxmoe_verify_workspace_size(3855, 8, 152064) > 0   # 3855 x 17 = 65535 rows
+    assert lib.mxmoe_verify_workspace_size(3856, 8, 152064) == -1
+    assert lib.mxmoe_verify_block(base, base, base, base, 3856, 8, 152064, 1.0, base, base, base, 1 << 40,
+                                  None) == mx.ERR_INVALID_SHAPE
