@@ -6,13 +6,18 @@ top-k routing, grouping by expert, gate/up + SwiGLU, down projection, weighted
 combine, through the library's C ABI. Metric: layer tokens/s, with the
 expert-weight HBM GB/s and its fraction of the measured HBM peak alongside.
 
-Default workload: one DFlash verify block (8 tokens, the block size of the
-"MiMo-V2.5-Pro-FP4-DFlash" model card, section 3) through a layer of 384 MXFP4
-experts, top-8, hidden 6144, expert intermediate 2048. Inputs are synthetic
-(datagen); the touched experts' weights (~1.2 GB per step) exceed the 126 MB L2,
-and the batches rotate so consecutive steps touch different experts.
+Default run: the five layer workloads in one process on one layer of 384 MXFP4
+experts (top-8, hidden 6144, expert intermediate 2048; the tiny one on its own
+small layer). The JSON line's headline is the largest single-GPU workload,
+prefill8192 (8192 tokens, tensor-bound); `per_config` holds the same fields
+for tiny, verify8 (one DFlash verify block of 8 tokens, the block size of the
+"MiMo-V2.5-Pro-FP4-DFlash" model card, section 3), verify256 (32 such blocks)
+and zipf1024 (1024 tokens, Zipf-skewed routing). Inputs are synthetic
+(datagen); every step streams the touched experts' weights (>1 GB) through
+HBM, far above the 126 MB L2.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                       [--config NAME] [--no-per-config]
 Under torchrun each rank runs an independent replica on its own GPU (no
 collective on the data path; weak scaling); rank 0 prints one JSON line.
 """
@@ -63,15 +68,24 @@ def kernels_per_step(T: int, k: int, E: int, H: int) -> int:
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
+HEADLINE = "prefill8192"  # the largest workload that fits one GPU
+
+
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--config", default="verify8", choices=[c.name for c in datagen.CONFIGS])
-    ap.add_argument("--batches", type=int, default=16, help="distinct rotating input batches")
+    ap.add_argument("--config", default=HEADLINE, choices=[c.name for c in datagen.CONFIGS],
+                    help="the workload of the line's headline value")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="measure the headline workload only (no per_config object)")
+    ap.add_argument("--min-timed-s", type=float, default=0.25,
+                    help="per_config entries: at least this many seconds of timed steps per workload")
+    ap.add_argument("--batches", type=int, default=16, help="distinct rotating input batches (small token counts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens of the oracle's timed CPU sample")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: shrink the layer to this many experts (0 = the workload's)")
@@ -86,6 +100,7 @@ def parse_args():
 
 
 def workload_config(cfg, world: int, batches: int):
+    big = cfg.T * cfg.k * cfg.H * 2 > (126 << 20)  # the step's x rows alone exceed L2
     return {
         "workload": "%s: MXFP4 MoE layer, T=%d tokens, H=%d, E=%d experts, top-%d, I=%d, block 32"
                     % (cfg.name, cfg.T, cfg.H, cfg.E, cfg.k, cfg.I),
@@ -97,8 +112,8 @@ def workload_config(cfg, world: int, batches: int):
         "intermediate": cfg.I,
         "router_bias_zipf": cfg.zipf_s,
         "parallelism": "replicas x%d" % world,
-        "l2": "inputs larger than L2: each step streams the touched experts' MXFP4 weights (>1 GB) and "
-              "%d input batches rotate" % batches,
+        "l2": "inputs larger than L2: each step streams the touched experts' MXFP4 weights (%s) and "
+              "%d input batches rotate" % (">7 GB" if big else ">0.4 MB" if cfg.E <= 16 else ">1 GB", batches),
     }
 
 
@@ -113,13 +128,24 @@ def load_peaks():
         return 6650.0, 1400.0, "fallback"
 
 
-def kernel_source_sha() -> str:
-    """Hash of the term kernel's code (comments, blank lines and the file's C
-    entry points left out), which keys the committed traffic capture to the
-    device code it was taken on."""
+# Device code whose DRAM traffic a committed ncu capture describes: the
+# E2M1-term gate/up kernel (decode-sized workloads) and the bf16 gate/up kernel
+# (from 16384 grouped rows).
+TRAFFIC_SOURCES = {
+    "ffn_gate_up": ("mxfp4_quantized_moe_router_b200/csrc/ffn.cu", "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
+                    "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"),
+    "ffn_bf16_gate_up": ("mxfp4_quantized_moe_router_b200/csrc/ffn_prefill.cu",
+                         "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
+                         "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"),
+}
+
+
+def kernel_source_sha(kind: str = "ffn_gate_up") -> str:
+    """Hash of a kernel's code (comments, blank lines and the file's C entry
+    points left out), which keys the committed traffic capture to the device
+    code it was taken on."""
     h = hashlib.sha256()
-    for rel in ("mxfp4_quantized_moe_router_b200/csrc/ffn.cu", "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
-                "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"):
+    for rel in TRAFFIC_SOURCES[kind]:
         with open(os.path.join(ROOT, rel)) as f:
             src = f.read()
         src = src.split('extern "C"', 1)[0]  # the kernels and their launchers, not the argument checks
@@ -129,16 +155,19 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, touched: float):
+def profiled_traffic(kind: str, workload: str, touched: float):
     """DRAM bytes (read + write) per launch of the gate/up stage, from the
     committed ncu capture of the same kernel source (null once the source has
-    changed). The capture's bytes per touched expert are scaled to this run's
-    mean number of touched experts per launch."""
+    changed). A capture keeps either its bytes per launch (taken on this very
+    workload) or its bytes per touched expert (taken on a shrunk layer), which
+    are scaled to this run's mean number of touched experts per launch."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
-        ent = d.get("ffn_gate_up", {}).get(workload)
-        if ent and ent.get("source_sha") == kernel_source_sha():
+        ent = d.get(kind, {}).get(workload)
+        if ent and ent.get("source_sha") == kernel_source_sha(kind):
+            if "dram_bytes_per_launch" in ent:
+                return float(ent["dram_bytes_per_launch"])
             return float(ent["dram_bytes_per_touched_expert"]) * touched
     except Exception:
         pass
@@ -180,25 +209,34 @@ def whole_job_rate(units_per_step_per_rank: int, steps: int, world: int, ms_max:
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples of this process's GPU,
+    every 50 ms from start() to stop(). start() returns once the first sample
+    has arrived (or after 3 s), so that every timed loop after it is covered;
+    summary() reads the samples that fall inside the given timed windows."""
+
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 50
 
     def __init__(self, uuid: str):
         self.uuid = uuid
         self.samples = []
         self.proc = None
         self.thread = None
+        self.first = threading.Event()
 
-    def start(self):
+    def start(self, wait_s: float = 3.0):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", str(self.PERIOD_MS)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        self.first.wait(wait_s)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -208,6 +246,7 @@ class ClockSampler:
             try:
                 self.samples.append(dict(t=time.time(), sm=float(parts[1]), max=float(parts[2]),
                                          hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                self.first.set()
             except ValueError:
                 pass
 
@@ -219,8 +258,18 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self, t0: float, t1: float):
-        win = [s for s in self.samples if t0 - 0.15 <= s["t"] <= t1 + 0.15] or self.samples[-3:]
+    def summary(self, windows):
+        """Median SM clock, max clock and active throttle reasons over the
+        samples taken inside the (t0, t1) windows (host time around each timed
+        loop, widened by one sampling period); if no sample fell inside a
+        window, the two samples nearest to it."""
+        pad = self.PERIOD_MS / 1e3
+        win = [s for s in self.samples if any(t0 - pad <= s["t"] <= t1 + pad for t0, t1 in windows)]
+        nearest = False
+        if not win and self.samples and windows:
+            mid = 0.5 * (windows[0][0] + windows[-1][1])
+            win = sorted(self.samples, key=lambda s: abs(s["t"] - mid))[:2]
+            nearest = True
         if not win:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         reasons = set()
@@ -229,13 +278,30 @@ class ClockSampler:
                               ("pcap", "sw_power_cap")):
                 if s[key].lower().startswith("active"):
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(s["sm"] for s in win), "sm_max_mhz": max(s["max"] for s in win),
-                "reasons": sorted(reasons), "samples": len(win)}
+        out = {"sm_mhz": statistics.median(s["sm"] for s in win), "sm_max_mhz": max(s["max"] for s in win),
+               "reasons": sorted(reasons), "samples": len(win), "period_ms": self.PERIOD_MS}
+        if nearest:
+            out["nearest_to_window"] = True
+        return out
 
 
 # ---------------------------------------------------------------------------
-# CPU oracle timing (baseline and reference arm)
+# host description and CPU oracle timing (baseline and reference arm)
 # ---------------------------------------------------------------------------
+def host_cpu():
+    """(logical cores the host offers, CPU model name)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 0, model
+
+
 def oracle_setup(cfg, seed, token_rows, x_bf16, bias):
     """Route the sample tokens with the oracle and quantise (untimed) the experts
     they touch. Returns the experts dict."""
@@ -265,15 +331,18 @@ def oracle_layer_time(cfg, wg, xs, bias, experts):
     return time.perf_counter() - t
 
 
-def cpu_baseline(cfg, seed, x_cpu, bias, n_tokens=2):
-    rows = list(range(min(n_tokens, cfg.T)))
+def cpu_baseline(cfg, seed, x_cpu, bias, n_tokens):
+    """The oracle as it stands on a seeded sample of the workload's tokens, one
+    thread on the host cores."""
+    rows = sorted(datagen.sample_tokens(cfg.T, min(n_tokens, cfg.T), seed).tolist())
     wg, xs, experts = oracle_setup(cfg, seed, rows, x_cpu, bias)
     dt = oracle_layer_time(cfg, wg, xs, bias, experts)
+    cores, model = host_cpu()
     return {"value": len(rows) / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "%d token(s) of the %s workload through the float64 C oracle (router, routing, %d experts "
+            "sample": "%d seeded token(s) of the %s workload through the float64 C oracle (router, routing, %d experts "
                       "decoded and run, combine; experts quantised beforehand, untimed), one thread"
                       % (len(rows), cfg.name, len(experts)),
-            "seconds": dt}
+            "seconds": dt, "host_cores": cores, "cpu_model": model}
 
 
 def run_reference(args):
@@ -286,7 +355,8 @@ def run_reference(args):
     x = datagen.make_x(cfg, args.seed)
     bias = datagen.make_router_bias(cfg, args.seed)
     # one token per step (all of its k experts); a step is a bounded sample
-    tokens = list(range(min(cfg.T, max(1, args.warmup + args.steps))))
+    n = min(cfg.T, max(1, args.warmup + args.steps))
+    tokens = sorted(datagen.sample_tokens(cfg.T, n, args.seed).tolist())
     steps_tokens = [[tokens[i % len(tokens)]] for i in range(args.warmup + args.steps)]
     need = sorted(set(t for s in steps_tokens for t in s))
     wg, _, experts = oracle_setup(cfg, args.seed, need, x, bias)
@@ -298,15 +368,16 @@ def run_reference(args):
             times.append(dt)
     total = sum(times)
     value = len(times) / total
+    cores, model = host_cpu()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(cfg, 1, 1),
         "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": UNIT,
-                         "sample": "each step: 1 token of the %s workload through the float64 C oracle "
+                         "sample": "each step: 1 seeded token of the %s workload through the float64 C oracle "
                                    "(router, routing, its %d experts decoded and run, combine), one thread"
-                                   % (cfg.name, cfg.k)},
+                                   % (cfg.name, cfg.k), "host_cores": cores, "cpu_model": model},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -315,45 +386,35 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # native arm
 # ---------------------------------------------------------------------------
-def run_native(args):
+def make_layer(mx, cfg, seed, dev):
+    """A layer's router weight and prepacked MXFP4 experts on the device
+    (generated by datagen, quantised and prepacked by the library)."""
+    import torch
+
+    wg = datagen.make_router_weight(cfg, seed, dev)
+    ew = mx.ExpertWeights(cfg.E, cfg.H, cfg.I, dev)
+    for e in range(cfg.E):
+        ew.quantize_expert(e, datagen.make_w13(cfg, e, seed, dev), datagen.make_w2(cfg, e, seed, dev))
+    ew.prepack()
+    torch.cuda.synchronize()
+    prepacked = ew.prepacked
+    del ew  # the kernels stream the prepacked blob only
+    torch.cuda.empty_cache()
+    return wg, prepacked
+
+
+def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev, clocks, want_e2e=True):
+    """Time one workload: the whole layer (device-resident inputs), its gate/up
+    unit (CUDA events on the launching stream), and the end-to-end leg with
+    host copies. Every rank takes the same collective steps."""
     import torch
     import torch.distributed as dist
 
-    import mxfp4_quantized_moe_router_b200 as mx
-
-    world, rank, local = dist_env()
-    if world > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", torch.cuda.current_device())
-    cfg = datagen.BY_NAME[args.config]
-    if args.experts:
-        import dataclasses
-
-        cfg = dataclasses.replace(cfg, name=cfg.name + "-E%d" % args.experts, E=args.experts)
-    if args.tokens:
-        import dataclasses
-
-        cfg = dataclasses.replace(cfg, name=cfg.name + "-T%d" % args.tokens, T=args.tokens)
     T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.k, cfg.I
-
-    # --- weights (same layer on every rank), quantised and prepacked on the device
-    wg = datagen.make_router_weight(cfg, args.seed, dev)
-    ew = mx.ExpertWeights(E, H, I, dev)
-    for e in range(E):
-        ew.quantize_expert(e, datagen.make_w13(cfg, e, args.seed, dev), datagen.make_w2(cfg, e, args.seed, dev))
-    ew.prepack()
-    torch.cuda.synchronize()
-    del ew.packed13, ew.sc13, ew.packed2, ew.sc2  # the kernels stream the prepacked blob only
-    torch.cuda.empty_cache()
-    prepacked = ew.prepacked
+    nb = max(1, args.batches if T * H * 2 <= (16 << 20) else 2)  # rotate batches of small token counts
+    xs = [datagen.make_x(cfg, replica_input_seed(args.seed, rank, b), dev) for b in range(nb)]
     bias_np = datagen.make_router_bias(cfg, args.seed)
     bias = torch.from_numpy(bias_np).to(dev) if bias_np is not None else None
-
-    # --- rotating input batches (per rank: its own tokens)
-    nb = max(1, args.batches)
-    xs = [datagen.make_x(cfg, replica_input_seed(args.seed, rank, b), dev) for b in range(nb)]
     logits = torch.empty((T, E), dtype=torch.float32, device=dev)
     ids = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
@@ -361,12 +422,11 @@ def run_native(args):
     src_row = torch.empty(T * k, dtype=torch.int32, device=dev)
     dst_of = torch.empty(T * k, dtype=torch.int32, device=dev)
     fws = torch.empty(mx.mxmoe_ffn_workspace_size(T, k, E, H, I), dtype=torch.uint8, device=dev)
+    pms = torch.empty(max(1, mx.mxmoe_permute_scratch_size(T, k, E)), dtype=torch.uint8, device=dev)
     y_perm = torch.empty((T * k, H), dtype=torch.float32, device=dev)
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
-
-    # raw C-ABI calls on one stream
     L = mx.load()
     P = lambda t: None if t is None else t.data_ptr()  # noqa: E731
     fws_bytes = fws.numel()
@@ -383,11 +443,11 @@ def run_native(args):
 
     def split_step(b, ev):
         """The same layer through the per-step entry points, with events around
-        the gate/up stage (the kernel that streams 2/3 of the weight bytes)."""
+        the gate/up stage (the unit that streams 2/3 of the weight bytes)."""
         x = xs[b % nb]
         rc = L.mxmoe_router_gemm(P(x), P(wg), P(bias), T, H, E, P(logits), sp)
         rc |= L.mxmoe_route(P(logits), T, E, k, P(ids), P(w), sp)
-        rc |= L.mxmoe_permute(P(ids), T, k, E, P(offsets), P(src_row), P(dst_of), sp)
+        rc |= L.mxmoe_permute_ws(P(ids), T, k, E, P(offsets), P(src_row), P(dst_of), P(pms), pms.numel(), sp)
         ev[0].record(stream)
         rc |= L.mxmoe_ffn_gate_up(P(x), P(offsets), P(src_row), P(prepacked), T, k, E, H, I, P(fws), fws_bytes, sp)
         ev[1].record(stream)
@@ -396,14 +456,6 @@ def run_native(args):
         if rc:
             raise RuntimeError("libmxmoe call failed: " + mx.last_error())
 
-    # touched experts per batch (untimed), for the weight-byte accounting
-    touched = []
-    for b in range(nb):
-        layer_step(b)
-        torch.cuda.synchronize()
-        touched.append(int(torch.unique(ids).numel()))
-    assert mx.mxmoe_read_status(lws) == mx.OK
-
     def barrier():
         if world > 1:
             dist.barrier()
@@ -411,39 +463,50 @@ def run_native(args):
     def rank_max(v: float) -> float:
         return max_over_ranks(v, world, dev)
 
-    uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    clocks = ClockSampler(uuid)
-    clocks.start()
-    time.sleep(0.3)
+    # touched experts per batch (untimed), for the weight-byte accounting; the
+    # same calls give a first step-time estimate
+    touched = []
+    est0 = time.perf_counter()
+    for b in range(nb):
+        layer_step(b)
+        torch.cuda.synchronize()
+        touched.append(int(torch.unique(ids).numel()))
+    est_s = (time.perf_counter() - est0) / nb
+    assert mx.mxmoe_read_status(lws) == mx.OK
+    if steps is None:  # per_config entries: at least min_timed_s of timed steps (same count on every rank)
+        steps = max(args.steps, int(np.ceil(rank_max(args.min_timed_s / max(est_s, 1e-6)))))
+        steps = min(steps, 20000)
+    windows = []
 
     # --- device-resident timed region: the whole layer per step
-    for i in range(args.warmup):
+    for i in range(warmup):
         layer_step(i)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     t0 = time.time()
     start.record(stream)
-    for i in range(args.steps):
-        layer_step(args.warmup + i)
+    for i in range(steps):
+        layer_step(warmup + i)
     end.record(stream)
     torch.cuda.synchronize()
-    t1 = time.time()
+    windows.append((t0, time.time()))
     barrier()
     ms = start.elapsed_time(end)
     ms_max = rank_max(ms)
-    clk = clocks.summary(t0, t1)
 
     # --- roofline region: same steps through the per-step entry points, with
     # CUDA events on the launching stream around the gate/up stage
-    for i in range(args.warmup):
+    for i in range(warmup):
         split_step(i, (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
-    ev_unit = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev_unit = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier()
     torch.cuda.synchronize()
-    for i in range(args.steps):
-        split_step(args.warmup + i, ev_unit[i])
+    t0 = time.time()
+    for i in range(steps):
+        split_step(warmup + i, ev_unit[i])
     torch.cuda.synchronize()
+    windows.append((t0, time.time()))
     barrier()
     unit_ms = [a.elapsed_time(b) for a, b in ev_unit]
 
@@ -452,61 +515,57 @@ def run_native(args):
     # run on their own streams into double-buffered device x and y, ordered
     # by events, so that step i+1's upload and step i-1's download overlap
     # step i's layer, as in a serving loop.
-    x_host = [xb.cpu().pin_memory() for xb in xs]
-    y_host = [torch.empty((T, H), dtype=torch.float32).pin_memory() for _ in range(2)]
-    x_dev = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    y_dev = [torch.empty((T, H), dtype=torch.float32, device=dev) for _ in range(2)]
-    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    x_ready, x_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
-    y_ready, y_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
+    ms_e2e = None
+    if want_e2e:
+        x_host = [xb.cpu().pin_memory() for xb in xs]
+        y_host = [torch.empty((T, H), dtype=torch.float32).pin_memory() for _ in range(2)]
+        x_dev = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        y_dev = [torch.empty((T, H), dtype=torch.float32, device=dev) for _ in range(2)]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        x_ready, x_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
+        y_ready, y_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(s):
-        j = s & 1
-        up.wait_event(x_free[j])  # the layer two steps back has read x_dev[j]
-        with torch.cuda.stream(up):
-            x_dev[j].copy_(x_host[s % nb], non_blocking=True)
-        x_ready[j].record(up)
-        stream.wait_event(x_ready[j])
-        stream.wait_event(y_free[j])  # y_dev[j] of two steps back is downloaded
-        layer_step(s, x_dev[j], y_dev[j])
-        x_free[j].record(stream)
-        y_ready[j].record(stream)
-        down.wait_event(y_ready[j])
-        with torch.cuda.stream(down):
-            y_host[j].copy_(y_dev[j], non_blocking=True)
-        y_free[j].record(down)
+        def e2e_step(s):
+            j = s & 1
+            up.wait_event(x_free[j])  # the layer two steps back has read x_dev[j]
+            with torch.cuda.stream(up):
+                x_dev[j].copy_(x_host[s % nb], non_blocking=True)
+            x_ready[j].record(up)
+            stream.wait_event(x_ready[j])
+            stream.wait_event(y_free[j])  # y_dev[j] of two steps back is downloaded
+            layer_step(s, x_dev[j], y_dev[j])
+            x_free[j].record(stream)
+            y_ready[j].record(stream)
+            down.wait_event(y_ready[j])
+            with torch.cuda.stream(down):
+                y_host[j].copy_(y_dev[j], non_blocking=True)
+            y_free[j].record(down)
 
-    def e2e_run(first, n):
-        for i in range(first, first + n):
-            e2e_step(i)
-        for j in range(2):  # the last downloads end the region
-            stream.wait_event(y_free[j])
+        def e2e_run(first, n):
+            for i in range(first, first + n):
+                e2e_step(i)
+            for j in range(2):  # the last downloads end the region
+                stream.wait_event(y_free[j])
 
-    e2e_run(0, args.warmup)
-    barrier()
-    torch.cuda.synchronize()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    up.wait_event(s2)
-    e2e_run(args.warmup, args.steps)
-    e2.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_e2e = rank_max(s2.elapsed_time(e2))
-    clocks.stop()
-
-    if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
-        return
+        e2e_run(0, warmup)
+        barrier()
+        torch.cuda.synchronize()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.time()
+        s2.record(stream)
+        up.wait_event(s2)
+        e2e_run(warmup, steps)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        windows.append((t0, time.time()))
+        barrier()
+        ms_e2e = rank_max(s2.elapsed_time(e2))
 
     peak, peak_tf, peak_kind = load_peaks()
-    steps_batches = [(args.warmup + i) % nb for i in range(args.steps)]
+    steps_batches = [(warmup + i) % nb for i in range(steps)]
     mean_touched = float(np.mean([touched[b] for b in steps_batches]))
-    tokens = T * args.steps * world
-    value = whole_job_rate(T, args.steps, world, ms_max)
-    weight_bytes_step = mean_touched * cfg.expert_bytes
-    weight_gbs = weight_bytes_step * args.steps / (ms / 1e3) / 1e9
+    value = whole_job_rate(T, steps, world, ms_max)
+    weight_gbs = mean_touched * cfg.expert_bytes * steps / (ms / 1e3) / 1e9
     unit_ms_mean = float(np.mean(unit_ms))
     if T * k >= BF16_PATH_ROWS:
         # dominant unit: mxmoe_ffn_gate_up on bf16 tensor cores (passes, slot rows, x_tile +
@@ -518,38 +577,117 @@ def run_native(args):
                     "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
                     "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops_sustained)" % peak_kind
                     if peak_kind == "measured" else "fallback 1.4 PFLOP/s sustained",
-                    "traffic": None, "unit_ms": unit_ms_mean, "algorithmic_flops_per_launch": unit_flops}
+                    "traffic": profiled_traffic("ffn_bf16_gate_up", cfg.name, mean_touched), "unit_ms": unit_ms_mean,
+                    "algorithmic_flops_per_launch": unit_flops}
+        dtype = "bf16 x dequantised e2m1 -> f32"
     else:
         # dominant unit: mxmoe_ffn_gate_up (x_terms + gate/up stage); algorithmic
         # bytes = gate/up MXFP4 bytes of the touched experts + x read + h written
         w13_bytes = 2 * I * H * 17 // 32
         unit_bytes = mean_touched * w13_bytes + T * H * 2 + T * k * I * 2
         achieved = unit_bytes / (unit_ms_mean / 1e3) / 1e9
-        roofline = {"kernel": "mxmoe_ffn_gate_up (act_terms_kernel + ffn_mxf4_kernel<gate_up>)",
+        hybrid = T >= 128
+        roofline = {"kernel": "mxmoe_ffn_gate_up (act_terms_kernel + ffn_mxf4_kernel<gate_up>%s)"
+                              % (" + the bf16 kernels for experts with >= 128 rows" if hybrid else ""),
                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
                     else "fallback 6.65 TB/s",
-                    "traffic": profiled_traffic(cfg.name, mean_touched), "unit_ms": unit_ms_mean,
+                    "traffic": profiled_traffic("ffn_gate_up", cfg.name, mean_touched), "unit_ms": unit_ms_mean,
                     "algorithmic_bytes_per_launch": unit_bytes}
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 x dequantised e2m1 -> f32" if T * k >= BF16_PATH_ROWS
-        else "e2m1 x e2m1 digit terms -> f32", "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert "
-                                          "W~N(0,0.02) quantised to MXFP4 by the library)",
-        "config": workload_config(cfg, world, nb),
-        "weight_gbs": weight_gbs,
-        "weight_frac_of_hbm_peak": weight_gbs / peak,
-        "touched_experts_per_step": mean_touched,
-        "roofline": roofline,
-        "clocks": clk,
-        "gpu_launches": kernels_per_step(T, k, E, H) * args.steps,
-        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
-                "d2h_bytes_per_step": T * H * 4, "api": "mxmoe_layer_forward with pinned host x/y copies on their own streams, "
-                       "double-buffered (step i+1's upload and step i-1's download overlap step i)"},
+        dtype = "e2m1 x e2m1 digit terms -> f32"
+    out = {
+        "value": value, "unit": UNIT, "steps": steps, "warmup": warmup, "ms_per_step": ms_max / steps,
+        "dtype": dtype, "config": workload_config(cfg, world, nb), "weight_gbs": weight_gbs,
+        "weight_frac_of_hbm_peak": weight_gbs / peak, "touched_experts_per_step": mean_touched,
+        "roofline": roofline, "clocks": clocks.summary(windows),
+        "gpu_launches": kernels_per_step(T, k, E, H) * steps,
     }
+    if ms_e2e is not None:
+        out["e2e"] = {"value": T * steps * world / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
+                      "d2h_bytes_per_step": T * H * 4,
+                      "api": "mxmoe_layer_forward with pinned host x/y copies on their own streams, double-buffered "
+                             "(step i+1's upload and step i-1's download overlap step i)"}
+    out["_x0"] = xs[0].cpu()
+    out["_bias"] = bias_np
+    return out
+
+
+def run_native(args):
+    import dataclasses
+
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_quantized_moe_router_b200 as mx
+
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def shaped(cfg):
+        if args.experts:
+            cfg = dataclasses.replace(cfg, name=cfg.name + "-E%d" % args.experts, E=args.experts)
+        if args.tokens:
+            cfg = dataclasses.replace(cfg, name=cfg.name + "-T%d" % args.tokens, T=args.tokens)
+        return cfg
+
+    head = shaped(datagen.BY_NAME[args.config])
+    names = [c.name for c in datagen.CONFIGS] if not args.no_per_config else [args.config]
+    cfgs = [shaped(datagen.BY_NAME[n]) for n in names]
+    # one set of weights per distinct layer (H, E, I); the tiny workload has its own
+    layers = {}
+    for c in cfgs:
+        key = (c.H, c.E, c.I)
+        if key not in layers:
+            layers[key] = make_layer(mx, c, args.seed, dev)
+
+    clocks = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    results = {}
+    for c in cfgs:  # the headline last, after the others have warmed the GPU
+        if c.name == head.name:
+            continue
+        wg, prepacked = layers[(c.H, c.E, c.I)]
+        results[c.name] = measure_layer(mx, c, wg, prepacked, args, None, args.warmup, world, rank, dev, clocks)
+        torch.cuda.empty_cache()
+    wg, prepacked = layers[(head.H, head.E, head.I)]
+    res = measure_layer(mx, head, wg, prepacked, args, args.steps, args.warmup, world, rank, dev, clocks)
+    clocks.stop()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    x0, bias_np = res.pop("_x0"), res.pop("_bias")
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": res["dtype"],
+        "data": "synthetic (seeded datagen: x~N(0,1), router W~N(0,0.02), expert W~N(0,0.02) quantised to MXFP4 by "
+                "the library)",
+        "config": res["config"],
+    }
+    for key in ("weight_gbs", "weight_frac_of_hbm_peak", "touched_experts_per_step", "roofline", "clocks",
+                "gpu_launches", "e2e"):
+        line[key] = res[key]
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, args.seed, xs[0].cpu(), bias_np)
+        line["cpu_baseline"] = cpu_baseline(head, args.seed, x0, bias_np, args.cpu_tokens)
+    if results:
+        line["per_config"] = {}
+        for c in cfgs:
+            if c.name == head.name:
+                r = dict(res)
+            else:
+                r = results[c.name]
+                r.pop("_x0")
+                r.pop("_bias")
+            line["per_config"][c.name] = {key: r[key] for key in (
+                "value", "unit", "ms_per_step", "steps", "dtype", "weight_gbs", "weight_frac_of_hbm_peak",
+                "touched_experts_per_step", "roofline", "e2e", "clocks", "gpu_launches") if key in r}
+            line["per_config"][c.name]["workload"] = r["config"]["workload"]
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -650,7 +788,6 @@ def run_verify(args):
         accepted_mean.append(float(acc.float().mean()))
     clocks = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
     clocks.start()
-    time.sleep(0.3)
     for i in range(args.warmup):
         step(i)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -665,7 +802,7 @@ def run_verify(args):
     t1 = time.time()
     barrier()
     ms = max_over_ranks(start.elapsed_time(end), world, dev)
-    clk = clocks.summary(t0, t1)
+    clk = clocks.summary([(t0, t1)])
     # end to end: each step uploads its logits, drafts and uniforms from pinned
     # host memory and downloads the verdicts, copies on their own streams
     # (double-buffered) so that they overlap the neighbouring steps' kernels

@@ -144,7 +144,12 @@ MXMOE_API int mxmoe_router_gemm(const void *x, const void *wg, const float *bias
  * Errors: k < 1, k > E, k > 32, E > 4096 or T < 0 -> INVALID_SHAPE. */
 MXMOE_API int mxmoe_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, void *stream);
 
-/* Group the T*k (token, slot) pairs by expert (stable).
+/* Group the T*k (token, slot) pairs by expert (stable), so that each
+ * expert's rows are contiguous for the grouped FFN. The pages route every
+ * token to 8 of 384 experts (nxbn.cn MiMo-V2.5-Pro-FP4-DFlash article,
+ * architecture section) and give no grouping rule; this is the plain
+ * counting-sort reading: experts ascending, pairs in (t, j) order within an
+ * expert.
  *   ids device int32 [T, k], every id in [0, E).
  *   offsets device int32 [E+1]: pairs routed to experts < e.
  *   src_row device int32 [T*k]: pair index t*k + j at each grouped position;
@@ -186,8 +191,15 @@ MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I);
  *   aligned. Its first 16 bytes hold the device status word of the call.
  * The products run on tcgen05 block-scaled tensor cores (E2M1 weights x E2M1
  * activation terms, UE8M0 scales per 32, fp32 accumulation): x and h each
- * enter as eight E2M1 terms per value, every term with its own scale per 32
- * values, together within 3^-8 of the 32-block's largest magnitude.
+ * enter as eight E2M1 terms per value (balanced base-8 digits on the grid
+ * 2^(E-22), E the exponent of the value's 32-block maximum), every term with
+ * its own scale per 32 values. That represents every bf16 x within 2^-15 of
+ * its block maximum exactly and any other value (smaller x, fp32 h) to within
+ * 2^-23 of the block maximum. From 16384 grouped rows (and, from 128 tokens,
+ * for experts with at least 128 rows) both stages run on bf16 tensor cores
+ * instead: the weights dequantised exactly (an E2M1 value times its
+ * power-of-two scale is a bf16 value), x as is, h as bf16 hi + lo (within
+ * 2^-15 of h).
  * Errors: H or I not a multiple of 128 or above 32768, k > 32, E > 1024,
  * T*k > 2^22, E*I*H >= 2^38 -> INVALID_SHAPE; workspace
  * too small -> WORKSPACE; x, y_perm not 16-byte or prepacked not 32-byte
@@ -228,8 +240,11 @@ MXMOE_API int mxmoe_ffn_down(const int32_t *offsets, const void *prepacked, int 
  * 6144/2048/top-8 layer fits up to 15 tokens).
  *   status  device int or NULL: when given, receives the call's device status
  *           word (MXMOE_OK or MXMOE_ERR_TIMEOUT) in stream order.
- * The first call on each device looks up the array's device address (once,
- * under a lock); make that first call before any stream capture. The call
+ * The first call in each CUDA context of a device looks up the array's
+ * device address (once per context, under a lock); make that first call
+ * before any stream capture. A device reset (cudaDeviceReset) or a new
+ * context reloads the library's device code, which invalidates an earlier
+ * lookup: the next call then looks the address up again. The call
  * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  * All calls share the one array and it keeps the last call's contents (the
  * call itself clears what must start at zero), so calls whose work overlaps
@@ -240,7 +255,10 @@ MXMOE_API int mxmoe_expert_ffn_noalloc(const void *x, const int32_t *offsets, co
                                        int *status, void *stream);
 
 /* Weighted combine: y[t, c] = sum over j = 0..k-1 (in order) of
- * w[t, j] * y_perm[dst_of[t*k + j], c], float32.
+ * w[t, j] * y_perm[dst_of[t*k + j], c], float32: each token's output is its
+ * selected experts' outputs weighted by its routing weights (the 8 activated
+ * experts of the nxbn.cn article's architecture section; the pages give no
+ * summation order, so slots are added in order).
  *   y_perm device float [T*k, H]; dst_of device int32 [T*k]; w device float
  *   [T, k]; y device float [T, H].
  * Errors: H % 4 != 0 or T > 65535 -> INVALID_SHAPE; y_perm, y not 16-byte aligned ->
@@ -252,7 +270,8 @@ MXMOE_API int mxmoe_combine(const float *y_perm, const int32_t *dst_of, const fl
 /* Whole layer                                                               */
 /* ------------------------------------------------------------------------ */
 
-/* Workspace bytes needed by mxmoe_layer_forward (-1 on bad sizes). */
+/* Workspace bytes needed by mxmoe_layer_forward; -1 for exactly the shapes
+ * that mxmoe_layer_forward rejects with INVALID_SHAPE. */
 MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, int k);
 
 /* The whole MoE expert layer for T tokens: router GEMM, route, permute,
@@ -321,7 +340,8 @@ MXMOE_API int64_t mxmoe_verify_workspace_size(int B, int K, int64_t V);
  *   workspace device, >= mxmoe_verify_workspace_size(B, K, V) bytes,
  *       256-byte aligned; contents not kept between calls.
  * Errors: K < 1, K > 32, V < 1, V > 2^24, B < 0, B (2K + 1) > 65535 -> INVALID_SHAPE;
- * a negative or non-finite temperature -> INVALID_SHAPE; NULL pointers ->
+ * a negative or non-finite temperature, or a positive one so small that
+ * log2(e) / temperature overflows float (below about 4e-39) -> INVALID_SHAPE; NULL pointers ->
  * NULL; workspace too small -> WORKSPACE, misaligned -> ALIGNMENT. */
 MXMOE_API int mxmoe_verify_block(const float *target_logits, const float *draft_logits,
                                  const int32_t *draft_tokens, const float *uniforms, int B, int K, int64_t V,

@@ -104,6 +104,7 @@ int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int 
                 cudaStream_t st);
 int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
+bool ffn_shapes_ok(int T, int k, int E, int H, int I);
 int router_splits(int T, int H, int E);
 int64_t permute_scratch_ints(int n, int E);
 int run_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row, int32_t *dst_of,
@@ -172,8 +173,8 @@ constexpr int kMaxLayerTokens = 65535;
 
 extern "C" MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, int k)
 {
-    if (T < 0 || T > kMaxLayerTokens || k < 1 || k > 32 || k > E || E <= 0 || E > 1024 || H <= 0 || I <= 0 ||
-        H % 64 || I % 32)
+    // exactly the shapes mxmoe_layer_forward accepts
+    if (T > kMaxLayerTokens || k > E || !ffn_shapes_ok(T, k, E, H, I))
         return -1;
     return layer_ws_layout(T, H, I, E, k, nullptr, nullptr);
 }

@@ -918,10 +918,16 @@ int launch_ffn(const void *codes, const uint8_t *act_terms, const FfnParams &p, 
 // 8 rows), else 16.
 int token_tile(int T) { return T <= 8 ? 8 : 16; }
 
+// The shapes every FFN entry point (and the layer) accepts.
+bool shapes_ok(int T, int k, int E, int H, int I)
+{
+    return !(T < 0 || k < 1 || k > 32 || E <= 0 || E > kMaxE || H <= 0 || I <= 0 || H % 128 || I % 128 ||
+             H > 32768 || I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31));
+}
+
 int validate_ffn(int T, int k, int E, int H, int I)
 {
-    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > kMaxE || H <= 0 || I <= 0 || H % 128 || I % 128 || H > 32768 ||
-        I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31))
+    if (!shapes_ok(T, k, E, H, I))
         return fail(MXMOE_ERR_INVALID_SHAPE,
                     "expert FFN: T=%d k=%d E=%d H=%d I=%d (need H, I multiples of 128 up to 32768, 1 <= k <= 32, "
                     "E <= 1024, T*k <= 2^22, E*I*H < 2^38)",
@@ -1054,6 +1060,7 @@ int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I)
 }
 
 int validate_ffn_shapes(int T, int k, int E, int H, int I) { return validate_ffn(T, k, E, H, I); }
+bool ffn_shapes_ok(int T, int k, int E, int H, int I) { return shapes_ok(T, k, E, H, I); }
 
 }  // namespace mxmoe
 
@@ -1061,8 +1068,7 @@ using namespace mxmoe;
 
 extern "C" MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I)
 {
-    if (T < 0 || k < 1 || k > 32 || E <= 0 || E > 1024 || H <= 0 || I <= 0 || H % 128 || I % 128 || H > 32768 ||
-        I > 32768 || (int64_t)T * k > (1 << 22) || (int64_t)E * I * H / 128 >= (1LL << 31))
+    if (!ffn_shapes_ok(T, k, E, H, I))
         return -1;
     return ffn_workspace_bytes(T, k, E, H, I);
 }

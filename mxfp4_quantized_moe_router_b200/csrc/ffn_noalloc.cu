@@ -9,6 +9,8 @@
 // allowed. Such a caller can pass its inputs and outputs and nothing else.
 #include <mutex>
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace mxmoe {
@@ -29,9 +31,35 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_ffn_scratch[kStaticScratchBytes];
 
 std::mutex g_setup_mutex;
-void *g_scratch_ptr[kMaxDevices] = {};
+// Looked-up addresses, one per device ordinal, each tagged with the CUDA
+// context it was looked up in. The array's address belongs to the module
+// loaded in that context: after cudaDeviceReset, or in another context on the
+// same device, the library's device code is loaded again and the array may sit
+// elsewhere, so a lookup made in an earlier context is never reused.
+struct ScratchEntry {
+    CUcontext ctx;
+    void *ptr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Resolve the scratch array's device address for the current device, once.
+PFN_cuCtxGetCurrent_v4000 ctx_getter()
+{
+    static std::once_flag once;
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    });
+    return fn;
+}
+
+// The scratch array's device address in the current device's current context.
+// The lookup (cudaGetSymbolAddress, which also makes the device's primary
+// context current if none is) runs on the first call in each context, under a
+// lock; later calls in the same context reuse it.
 int scratch_for_current_device(void **out)
 {
     int dev = -1;
@@ -40,16 +68,24 @@ int scratch_for_current_device(void **out)
         return mxmoe::fail(MXMOE_ERR_CUDA, "mxmoe_expert_ffn_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxDevices)
         return mxmoe::fail(MXMOE_ERR_DEVICE, "mxmoe_expert_ffn_noalloc: device ordinal %d out of range", dev);
+    auto get_ctx = ctx_getter();
+    if (!get_ctx)
+        return mxmoe::fail(MXMOE_ERR_CUDA, "mxmoe_expert_ffn_noalloc: cuCtxGetCurrent is not available");
+    CUcontext ctx = nullptr;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_ffn_scratch);
-        if (e != cudaSuccess || !p)
-            return mxmoe::fail(MXMOE_ERR_CUDA, "mxmoe_expert_ffn_noalloc: cudaGetSymbolAddress: %s",
-                               cudaGetErrorString(e));
-        g_scratch_ptr[dev] = p;
+    if (get_ctx(&ctx) == CUDA_SUCCESS && ctx && ctx == g_scratch[dev].ctx && g_scratch[dev].ptr) {
+        *out = g_scratch[dev].ptr;
+        return MXMOE_OK;
     }
-    *out = g_scratch_ptr[dev];
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_ffn_scratch);
+    if (e != cudaSuccess || !p)
+        return mxmoe::fail(MXMOE_ERR_CUDA, "mxmoe_expert_ffn_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+        return mxmoe::fail(MXMOE_ERR_CUDA, "mxmoe_expert_ffn_noalloc: no current CUDA context");
+    g_scratch[dev] = {ctx, p};
+    *out = p;
     return MXMOE_OK;
 }
 

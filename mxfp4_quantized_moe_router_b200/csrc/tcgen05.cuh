@@ -17,27 +17,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
 
-// Instruction descriptor of kind::mxf8f6f4.block_scale with A = E2M1, B = E4M3,
-// UE8M0 scales, both K-major, M = 128, N = n (multiple of 8), and the scale
-// byte `sf_id` (k32 block within a 4-block scale column) for A and B.
-__device__ __forceinline__ uint32_t idesc_e2m1_e4m3(int n, uint32_t sf_id)
-{
-    return (sf_id << 4) | (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | (8u << 24) |
-           (sf_id << 29);
-}
-
-__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
-}
-
-// 32 lanes x 128 bits from shared memory into tensor memory, replicated into
-// all four 32-lane sub-partitions (the scale-factor layout).
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, both
 // K-major, M = 128, N = n (a multiple of 16 up to 256).
 __device__ __forceinline__ uint32_t idesc_bf16(int n)
@@ -56,6 +35,8 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
+// 32 lanes x 128 bits from shared memory into tensor memory, replicated into
+// all four 32-lane sub-partitions (the scale-factor layout).
 __device__ __forceinline__ void cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc)
 {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
@@ -81,19 +62,6 @@ __device__ __forceinline__ void alloc(uint32_t *slot_smem, uint32_t ncols)
 __device__ __forceinline__ void dealloc(uint32_t taddr, uint32_t ncols)
 {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Eight consecutive 32-bit columns of this warp's 32 lanes.
-__device__ __forceinline__ void ld_32x32b_x8(uint32_t taddr, float (&v)[8])
-{
-    uint32_t r[8];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        v[i] = __uint_as_float(r[i]);
 }
 
 // 32 consecutive 32-bit columns of this warp's 32 lanes.
@@ -125,16 +93,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar,
-                                            uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
-        "{%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int y, int z, int w,
                                             uint64_t *bar, uint64_t policy)
 {
@@ -143,29 +101,6 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
         "{%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
-}
-
-// float -> E4M3 code (round to nearest even, saturating), and back (exact).
-__device__ __forceinline__ uint32_t f32_to_e4m3(float v)
-{
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.f), "f"(v));
-    return r & 0xFFu;
-}
-
-__device__ __forceinline__ float e4m3_to_f32(uint32_t code)
-{
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)code));
-    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-}
-
-// floor(log2 m) for m > 0 finite.
-__device__ __forceinline__ int floor_log2(float m)
-{
-    const uint32_t b = __float_as_uint(m);
-    const int be = (int)(b >> 23);
-    return be ? be - 127 : (31 - __clz((int)(b & 0x7FFFFF))) - 149;
 }
 
 }  // namespace tc

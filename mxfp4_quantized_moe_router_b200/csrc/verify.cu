@@ -502,6 +502,14 @@ extern "C" MXMOE_API int mxmoe_verify_block(const float *target_logits, const fl
     if (!(temperature >= 0.f) || isinf(temperature))
         return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_verify_block: temperature must be finite and >= 0");
     const bool sampling = temperature > 0.f;
+    // The kernels scale logits by log2(e) / temperature; a positive temperature
+    // so small that this factor overflows float would turn (z - max) * k into
+    // 0 * inf = NaN at the row maximum.
+    if (sampling && isinf(kLog2e / temperature))
+        return fail(MXMOE_ERR_INVALID_SHAPE,
+                    "mxmoe_verify_block: temperature %g is too small (log2(e) / temperature overflows float); "
+                    "use 0 for greedy verification",
+                    (double)temperature);
     if (workspace_bytes < mxmoe_verify_workspace_size(B, K, V))
         return fail(MXMOE_ERR_WORKSPACE, "mxmoe_verify_block: workspace of %lld bytes, need %lld",
                     (long long)workspace_bytes, (long long)mxmoe_verify_workspace_size(B, K, V));

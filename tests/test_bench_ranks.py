@@ -120,3 +120,53 @@ def test_verify_workload_reference_arm_prints_the_contract_line():
                         "reference", "--steps", "2", "--warmup", "1", "--vocab", "3000"], capture_output=True,
                        text=True, timeout=300, cwd=ROOT, env=env)
     assert q.returncode == 0 and q.stdout.strip() == ""
+
+
+def test_clock_summary_reads_the_timed_windows():
+    cs = bench.ClockSampler("GPU-x")
+    t = 1000.0
+
+    def sample(dt, sm, pcap="Not Active"):
+        return dict(t=t + dt, sm=sm, max=1965.0, hw="Not Active", hwt="Not Active", swt="Not Active", pcap=pcap)
+
+    cs.samples = [sample(0.0, 1965.0), sample(0.5, 1500.0, "Active"), sample(0.55, 1400.0, "Active"),
+                  sample(2.0, 1965.0)]
+    out = cs.summary([(t + 0.45, t + 0.6)])
+    assert out["samples"] == 2 and out["sm_mhz"] == 1450.0 and out["reasons"] == ["sw_power_cap"]
+    # two windows: the union of their samples
+    out = cs.summary([(t - 0.01, t + 0.01), (t + 1.99, t + 2.01)])
+    assert out["samples"] == 2 and out["sm_mhz"] == 1965.0 and out["reasons"] == []
+    # a window between samples falls back to the nearest ones, and says so
+    out = cs.summary([(t + 1.0, t + 1.01)])
+    assert out["samples"] == 2 and out.get("nearest_to_window")
+    assert bench.ClockSampler("GPU-y").summary([(t, t + 1)])["reasons"] == ["unsampled"]
+
+
+def test_host_cpu_names_cores_and_model():
+    cores, model = bench.host_cpu()
+    assert cores >= 1 and isinstance(model, str) and model
+
+
+def test_layer_reference_arm_prints_the_contract_line():
+    # the layer's reference arm on the tiny workload: the float64 oracle on
+    # host cores, one seeded token per step
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["host_cores"] >= 1 and line["cpu_baseline"]["cpu_model"]
+    assert line["config"]["workload"].startswith("tiny:")
+
+
+def test_headline_is_the_largest_single_gpu_workload():
+    assert bench.HEADLINE == max(datagen_configs(), key=lambda c: c.T).name
+
+
+def datagen_configs():
+    import datagen
+
+    return datagen.CONFIGS

@@ -73,6 +73,21 @@ def test_verify_matches_oracle(mx, B, K, V, tau):
     check(mx, z, w, d, u, tau)
 
 
+def test_verify_draw_beyond_one_round_of_chunks(mx):
+    # V just above 2^21 = 256 chunks of 8192: the draw's chunk scan carries its
+    # running sum across rounds of 256 chunks, and the first chunk of the second
+    # round is searched
+    V = (1 << 21) + 8193
+    z, w, d, u = datagen.make_verify_inputs(1, 2, V, seed=21)
+    check(mx, z, w, d, u, 1.0)
+    # a flat row (every weight equal) with u_K near 1 puts the draw in the last chunks
+    z2 = np.zeros_like(z)
+    w2 = np.zeros_like(w)
+    u2 = u.copy()
+    u2[:, -1] = np.float32(0.9999)
+    check(mx, z2, w2, d, u2, 1.0)
+
+
 @pytest.mark.parametrize("B,tau", [(32, 1.0), (32, 0.0), (1, 1.0), (1, 0.0)])
 def test_verify_full_size(mx, B, tau):
     # V = 152064, K = 8: one block (8 tokens) and 32 blocks (256 tokens)

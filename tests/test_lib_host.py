@@ -63,6 +63,12 @@ def test_workspace_queries(mx):
     assert mx.mxmoe_ffn_workspace_size((1 << 22) // 8 + 1, 8, 384, 6144, 2048) == -1
     # grows with T
     assert mx.mxmoe_workspace_size(256, 6144, 2048, 384, 8) > mx.mxmoe_workspace_size(8, 6144, 2048, 384, 8)
+    # the layer's size query refuses exactly what the layer refuses: H and I multiples of 128
+    assert mx.mxmoe_workspace_size(8, 192, 2048, 384, 8) == -1
+    assert mx.mxmoe_workspace_size(8, 6144, 2048 + 64, 384, 8) == -1
+    assert mx.mxmoe_workspace_size(8, 6144, 2048, 2000, 8) == -1  # E above the grouping's 1024
+    assert mx.mxmoe_workspace_size(65536, 256, 128, 16, 2) == -1  # T above the combine's 65535
+    assert mx.mxmoe_workspace_size(8, 256, 128, 4, 8) == -1  # k > E
 
 
 def _lib(mx):
@@ -159,6 +165,9 @@ def test_verify_block_queries_and_rejects_on_host(mx):
     assert f(base, base, base, base, 1, 8, V, -1.0, base, base, base, big, None) == mx.ERR_INVALID_SHAPE
     assert f(base, base, base, base, 1, 8, V, float("inf"), base, base, base, big, None) == mx.ERR_INVALID_SHAPE
     assert f(base, base, base, base, 1, 8, V, float("nan"), base, base, base, big, None) == mx.ERR_INVALID_SHAPE
+    # log2(e) / temperature overflows float below about 4e-39 (1e-40 is a float subnormal)
+    assert f(base, base, base, base, 1, 8, V, 1e-40, base, base, base, big, None) == mx.ERR_INVALID_SHAPE
+    assert "too small" in mx.last_error()
     assert f(base, base, base, base, 1, 8, V, 1.0, base, base, base, 16, None) == mx.ERR_WORKSPACE
     assert f(base, None, base, base, 1, 8, V, 1.0, base, base, base, big, None) == mx.ERR_NULL  # sampling needs q
     assert f(base, base, base, base, 1, 8, V, 1.0, base, base, base + 16, big, None) == mx.ERR_ALIGNMENT
