@@ -64,6 +64,13 @@ def _load():
         lib.mxo_e2m1_round.argtypes = [ctypes.c_double]
         lib.mxo_bf16_to_double.restype = ctypes.c_double
         lib.mxo_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.mxo_e4m3_value.restype = ctypes.c_double
+        lib.mxo_e4m3_value.argtypes = [I32]
+        lib.mxo_e4m3_round.restype = I32
+        lib.mxo_e4m3_round.argtypes = [ctypes.c_double]
+        lib.mxo_quantize_fp8.argtypes = [P, I64, I64, P, P]
+        lib.mxo_dequantize_fp8.argtypes = [P, P, I64, I64, P]
+        lib.mxo_expert_ffn_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
         lib.mxo_quantize.argtypes = [P, I64, I64, P, P]
         lib.mxo_dequantize.argtypes = [P, P, I64, I64, P]
         lib.mxo_router_logits.argtypes = [P, P, P, I64, I64, I64, P]
@@ -75,7 +82,7 @@ def _load():
         lib.mxo_expert_ffn_mxfp4.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
         lib.mxo_verify_block.argtypes = [P, P, P, P, I64, I32, I64, ctypes.c_double, P, P, P, P]
         lib.mxo_draw_interval.argtypes = [P, P, I64, ctypes.c_double, I64, P, P]
-        for f in ("mxo_quantize", "mxo_dequantize", "mxo_router_logits", "mxo_route", "mxo_route_f32",
+        for f in ("mxo_quantize_fp8", "mxo_dequantize_fp8", "mxo_expert_ffn_fp8", "mxo_quantize", "mxo_dequantize", "mxo_router_logits", "mxo_route", "mxo_route_f32",
                   "mxo_permute", "mxo_combine", "mxo_expert_ffn", "mxo_expert_ffn_mxfp4", "mxo_verify_block",
                   "mxo_draw_interval"):
             getattr(lib, f).restype = None
@@ -136,6 +143,48 @@ def dequantize(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
     out = np.empty((rows, K), np.float64)
     _load().mxo_dequantize(_p(packed), _p(scales), rows, K, _p(out))
     return out
+
+
+# --- FP8 expert weights (E4M3 elements, one E8M0 scale per 32) ---------------
+def e4m3_value(code: int) -> float:
+    return _load().mxo_e4m3_value(int(code))
+
+
+def e4m3_round(q: float) -> int:
+    return _load().mxo_e4m3_round(float(q))
+
+
+def quantize_fp8(w) -> tuple[np.ndarray, np.ndarray]:
+    """bf16 [rows, K] -> (E4M3 codes uint8 [rows, K], scales uint8 [rows, K/32])."""
+    wb = _bf16_bits(w)
+    rows, K = wb.shape
+    assert K % BLOCK == 0
+    codes = np.zeros((rows, K), np.uint8)
+    scales = np.zeros((rows, K // BLOCK), np.uint8)
+    _load().mxo_quantize_fp8(_p(wb), rows, K, _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequantize_fp8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, K = codes.shape
+    out = np.empty((rows, K), np.float64)
+    _load().mxo_dequantize_fp8(_p(codes), _p(scales), rows, K, _p(out))
+    return out
+
+
+def expert_ffn_fp8(c13, s13, c2, s2, x, want_h: bool = False):
+    """One FP8 expert (codes13 [2I, H], sc13 [2I, H/32], codes2 [H, I], sc2
+    [H, I/32]) decoded to float64, on rows x."""
+    c13, s13, c2, s2 = (np.ascontiguousarray(a, np.uint8) for a in (c13, s13, c2, s2))
+    xb = _bf16_bits(x)
+    n, H = xb.shape
+    I = c13.shape[0] // 2
+    y = np.empty((n, H), np.float64)
+    h = np.empty((n, I), np.float64) if want_h else None
+    _load().mxo_expert_ffn_fp8(_p(c13), _p(s13), _p(c2), _p(s2), _p(xb), n, H, I, _p(h) if want_h else None, _p(y))
+    return (y, h) if want_h else y
 
 
 # --- router -------------------------------------------------------------------
@@ -214,11 +263,13 @@ def expert_ffn_mxfp4(p13, s13, p2, s2, x, want_h: bool = False):
     return (y, h) if want_h else y
 
 
-def moe_layer(x, wg, bias, expert_fetch, k: int, threads: int = 1):
+def moe_layer(x, wg, bias, expert_fetch, k: int, threads: int = 1, fmt: str = "mxfp4"):
     """Whole MoE layer on the tokens in ``x`` (bf16 [n, H]).
 
     ``expert_fetch(e)`` returns the canonical MXFP4 arrays of expert e as
-    (packed13 [2I, H/2], sc13 [2I, H/32], packed2 [H, I/2], sc2 [H, I/32]).
+    (packed13 [2I, H/2], sc13 [2I, H/32], packed2 [H, I/2], sc2 [H, I/32]),
+    or with ``fmt="fp8"`` the FP8 arrays (codes13 [2I, H], sc13, codes2
+    [H, I], sc2).
     Steps: router logits (float64) -> route -> per expert, the rows routed
     to it -> combine in slot order. Returns dict with y, ids, w, logits,
     offsets, src_row, dst_of.
@@ -236,7 +287,8 @@ def moe_layer(x, wg, bias, expert_fetch, k: int, threads: int = 1):
         rows = src_row[offsets[e]:offsets[e + 1]]
         xe = np.ascontiguousarray(xb[rows // k])
         p13, s13, p2, s2 = expert_fetch(e)
-        y_perm[offsets[e]:offsets[e + 1]] = expert_ffn_mxfp4(p13, s13, p2, s2, xe)
+        ffn = expert_ffn_fp8 if fmt == "fp8" else expert_ffn_mxfp4
+        y_perm[offsets[e]:offsets[e + 1]] = ffn(p13, s13, p2, s2, xe)
 
     if threads > 1:
         with ThreadPoolExecutor(threads) as ex:

@@ -353,6 +353,127 @@ void mxo_expert_ffn_mxfp4(const uint8_t *packed13, const uint8_t *sc13, const ui
 }
 
 /* ------------------------------------------------------------------------ */
+/* FP8 expert weights (the pages' quality baseline)                          */
+/* ------------------------------------------------------------------------ */
+
+/* The model card's section 2 compares the MXFP4 experts with an FP8 baseline
+ * and its introduction says that lowering the bit width per parameter speeds
+ * up decoding; the pages give no FP8 layout. The reading here keeps the MX
+ * family of the FP4 experts: E4M3 elements with one E8M0 scale per 32
+ * elements along K (OCP MX FP8, "MXFP8"), the scale exponent chosen the same
+ * way as for E2M1 -- floor(log2 amax) minus the exponent of the element
+ * format's largest power of two (2 for E2M1, whose largest value is 1.5 * 2^2;
+ * 8 for E4M3, whose largest value is 1.75 * 2^8). */
+
+/* Value of one E4M3 code (OCP 8-bit floating point, E4M3).
+ * Bit 7 is the sign, bits 6..3 the exponent field e (bias 7), bits 2..0 the
+ * mantissa m. e == 0 is subnormal: (m / 8) * 2^-6. Otherwise
+ * 2^(e-7) * (1 + m/8). Codes 0x7F and 0xFF (e = 15, m = 7) are NaN; there is
+ * no infinity, so the largest finite magnitude is 2^8 * 1.75 = 448. */
+double mxo_e4m3_value(int code)
+{
+    int s = (code >> 7) & 1;
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    double mag = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Round a non-negative, exactly scaled magnitude q to an E4M3 magnitude code
+ * (0x00 .. 0x7E): the nearest finite E4M3 value; on a tie, the code whose
+ * mantissa's lowest bit is 0; anything above 448 saturates to 448 (0x7E).
+ * A plain search over the 127 finite magnitudes. */
+int mxo_e4m3_round(double q)
+{
+    if (q >= 448.0)
+        return 0x7E;
+    int best = 0;
+    double bestd = fabs(q - mxo_e4m3_value(0));
+    for (int c = 1; c <= 0x7E; ++c) {
+        double d = fabs(q - mxo_e4m3_value(c));
+        if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            bestd = d;
+        }
+    }
+    return best;
+}
+
+/* bf16 [rows, K] row-major -> E4M3 codes [rows, K] (one byte per element) +
+ * scales [rows, K/32].
+ * Per 32-element block along K:
+ *   amax = max |x|;
+ *   scale exponent e = floor(log2 amax) - 8, clamped to [-127, 127]; a block
+ *   whose amax is 0 gets e = -127 (scale byte 0);
+ *   scale byte S = e + 127 (E8M0);
+ *   each element: q = |x| / 2^e (exact), rounded to the nearest E4M3
+ *   magnitude (ties to the even mantissa, saturating at 448); the sign bit
+ *   of x is kept, also when the magnitude rounds to 0.
+ * K must be a multiple of 32. */
+void mxo_quantize_fp8(const uint16_t *w, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales)
+{
+    int64_t nblk = K / MXO_BLOCK;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            double v[MXO_BLOCK];
+            double amax = 0.0;
+            for (int i = 0; i < MXO_BLOCK; ++i) {
+                v[i] = bf16_to_double(w[r * K + b * MXO_BLOCK + i]);
+                if (fabs(v[i]) > amax)
+                    amax = fabs(v[i]);
+            }
+            int e;
+            if (amax == 0.0) {
+                e = -127;
+            } else {
+                int ex;
+                frexp(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1) */
+                e = (ex - 1) - 8; /* floor(log2 amax) - 8 */
+                if (e < -127)
+                    e = -127;
+                if (e > 127)
+                    e = 127;
+            }
+            scales[r * nblk + b] = (uint8_t)(e + 127);
+            for (int i = 0; i < MXO_BLOCK; ++i) {
+                double q = ldexp(fabs(v[i]), -e);
+                codes[r * K + b * MXO_BLOCK + i] = (uint8_t)(mxo_e4m3_round(q) | (signbit(v[i]) ? 0x80 : 0));
+            }
+        }
+    }
+}
+
+/* codes [rows, K] + scales [rows, K/32] -> double [rows, K]:
+ * element value = E4M3(code) * 2^(S - 127). */
+void mxo_dequantize_fp8(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K, double *out)
+{
+    int64_t nblk = K / MXO_BLOCK;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < nblk; ++b) {
+            double s = mxo_e8m0_value(scales[r * nblk + b]);
+            for (int64_t k = b * MXO_BLOCK; k < (b + 1) * MXO_BLOCK; ++k)
+                out[r * K + k] = mxo_e4m3_value(codes[r * K + k]) * s;
+        }
+}
+
+/* Decode one expert's FP8 weights to double and run it on n rows (the same
+ * SwiGLU expert as mxo_expert_ffn). codes13 [2I, H], sc13 [2I, H/32],
+ * codes2 [H, I], sc2 [H, I/32]. */
+void mxo_expert_ffn_fp8(const uint8_t *codes13, const uint8_t *sc13, const uint8_t *codes2, const uint8_t *sc2,
+                        const uint16_t *x, int64_t n, int64_t H, int64_t I, double *h_out, double *y)
+{
+    double *w13 = (double *)malloc(sizeof(double) * (size_t)(2 * I * H));
+    double *w2 = (double *)malloc(sizeof(double) * (size_t)(H * I));
+    mxo_dequantize_fp8(codes13, sc13, 2 * I, H, w13);
+    mxo_dequantize_fp8(codes2, sc2, H, I, w2);
+    mxo_expert_ffn(w13, w2, x, n, H, I, h_out, y);
+    free(w13);
+    free(w2);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Block verification of a speculative draft                                 */
 /* ------------------------------------------------------------------------ */
 
