@@ -386,13 +386,14 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # native arm
 # ---------------------------------------------------------------------------
-def make_layer(mx, cfg, seed, dev):
-    """A layer's router weight and prepacked MXFP4 experts on the device
-    (generated by datagen, quantised and prepacked by the library)."""
+def make_layer(mx, cfg, seed, dev, fmt="mxfp4"):
+    """A layer's router weight and prepacked experts on the device (generated
+    by datagen, quantised and prepacked by the library): MXFP4, or with
+    fmt="fp8" FP8 (E4M3, one E8M0 scale per 32)."""
     import torch
 
     wg = datagen.make_router_weight(cfg, seed, dev)
-    ew = mx.ExpertWeights(cfg.E, cfg.H, cfg.I, dev)
+    ew = (mx.ExpertWeightsFp8 if fmt == "fp8" else mx.ExpertWeights)(cfg.E, cfg.H, cfg.I, dev)
     for e in range(cfg.E):
         ew.quantize_expert(e, datagen.make_w13(cfg, e, seed, dev), datagen.make_w2(cfg, e, seed, dev))
     ew.prepack()
@@ -403,10 +404,18 @@ def make_layer(mx, cfg, seed, dev):
     return wg, prepacked
 
 
-def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev, clocks, want_e2e=True):
-    """Time one workload: the whole layer (device-resident inputs), its gate/up
-    unit (CUDA events on the launching stream), and the end-to-end leg with
-    host copies. Every rank takes the same collective steps."""
+def fp8_expert_bytes(cfg) -> int:
+    """FP8 bytes of one expert: 3*H*I one-byte codes plus one scale byte per 32."""
+    n = 3 * cfg.H * cfg.I
+    return n + n // 32
+
+
+def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev, clocks, want_e2e=True, fmt="mxfp4"):
+    """Time one workload: the whole layer (device-resident inputs), its
+    dominant unit (CUDA events on the launching stream: the gate/up stage, or
+    for FP8 experts the whole expert FFN), and the end-to-end leg with host
+    copies. Every rank takes the same collective steps."""
+    fp8 = fmt == "fp8"
     import torch
     import torch.distributed as dist
 
@@ -421,7 +430,8 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     src_row = torch.empty(T * k, dtype=torch.int32, device=dev)
     dst_of = torch.empty(T * k, dtype=torch.int32, device=dev)
-    fws = torch.empty(mx.mxmoe_ffn_workspace_size(T, k, E, H, I), dtype=torch.uint8, device=dev)
+    fws = torch.empty((mx.mxmoe_ffn_workspace_size_fp8 if fp8 else mx.mxmoe_ffn_workspace_size)(T, k, E, H, I),
+                      dtype=torch.uint8, device=dev)
     pms = torch.empty(max(1, mx.mxmoe_permute_scratch_size(T, k, E)), dtype=torch.uint8, device=dev)
     y_perm = torch.empty((T * k, H), dtype=torch.float32, device=dev)
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
@@ -430,14 +440,15 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
     L = mx.load()
     P = lambda t: None if t is None else t.data_ptr()  # noqa: E731
     fws_bytes = fws.numel()
-    lws = torch.empty(mx.mxmoe_workspace_size(T, H, I, E, k), dtype=torch.uint8, device=dev)
+    lws = torch.empty((mx.mxmoe_workspace_size_fp8 if fp8 else mx.mxmoe_workspace_size)(T, H, I, E, k),
+                      dtype=torch.uint8, device=dev)
+    forward = L.mxmoe_layer_forward_fp8 if fp8 else L.mxmoe_layer_forward
     lws_bytes = lws.numel()
 
     def layer_step(b, x=None, y_out=None):
         x = xs[b % nb] if x is None else x
         y_out = y if y_out is None else y_out
-        rc = L.mxmoe_layer_forward(P(x), P(wg), P(bias), P(prepacked), T, H, I, E, k, P(y_out), P(ids), P(w),
-                                   P(lws), lws_bytes, sp)
+        rc = forward(P(x), P(wg), P(bias), P(prepacked), T, H, I, E, k, P(y_out), P(ids), P(w), P(lws), lws_bytes, sp)
         if rc:
             raise RuntimeError("mxmoe_layer_forward failed: " + mx.last_error())
 
@@ -448,10 +459,17 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
         rc = L.mxmoe_router_gemm(P(x), P(wg), P(bias), T, H, E, P(logits), sp)
         rc |= L.mxmoe_route(P(logits), T, E, k, P(ids), P(w), sp)
         rc |= L.mxmoe_permute_ws(P(ids), T, k, E, P(offsets), P(src_row), P(dst_of), P(pms), pms.numel(), sp)
-        ev[0].record(stream)
-        rc |= L.mxmoe_ffn_gate_up(P(x), P(offsets), P(src_row), P(prepacked), T, k, E, H, I, P(fws), fws_bytes, sp)
-        ev[1].record(stream)
-        rc |= L.mxmoe_ffn_down(P(offsets), P(prepacked), T, k, E, H, I, P(y_perm), P(fws), fws_bytes, sp)
+        if fp8:  # the FP8 FFN has no separate stage entry points: the unit is the whole expert FFN
+            ev[0].record(stream)
+            rc |= L.mxmoe_expert_ffn_fp8(P(x), P(offsets), P(src_row), P(prepacked), T, k, E, H, I, P(y_perm),
+                                         P(fws), fws_bytes, sp)
+            ev[1].record(stream)
+        else:
+            ev[0].record(stream)
+            rc |= L.mxmoe_ffn_gate_up(P(x), P(offsets), P(src_row), P(prepacked), T, k, E, H, I, P(fws), fws_bytes,
+                                      sp)
+            ev[1].record(stream)
+            rc |= L.mxmoe_ffn_down(P(offsets), P(prepacked), T, k, E, H, I, P(y_perm), P(fws), fws_bytes, sp)
         rc |= L.mxmoe_combine(P(y_perm), P(dst_of), P(w), T, k, H, P(y), sp)
         if rc:
             raise RuntimeError("libmxmoe call failed: " + mx.last_error())
@@ -565,9 +583,21 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
     steps_batches = [(warmup + i) % nb for i in range(steps)]
     mean_touched = float(np.mean([touched[b] for b in steps_batches]))
     value = whole_job_rate(T, steps, world, ms_max)
-    weight_gbs = mean_touched * cfg.expert_bytes * steps / (ms / 1e3) / 1e9
+    expert_bytes = fp8_expert_bytes(cfg) if fp8 else cfg.expert_bytes
+    weight_gbs = mean_touched * expert_bytes * steps / (ms / 1e3) / 1e9
     unit_ms_mean = float(np.mean(unit_ms))
-    if T * k >= BF16_PATH_ROWS:
+    if fp8:
+        # dominant unit: mxmoe_expert_ffn_fp8 (act_terms + both FP8 stages); algorithmic bytes = the touched
+        # experts' FP8 bytes + x read + h written and read back + y_perm written
+        unit_bytes = mean_touched * expert_bytes + T * H * 2 + 2 * T * k * I * 2 + T * k * H * 4
+        achieved = unit_bytes / (unit_ms_mean / 1e3) / 1e9
+        roofline = {"kernel": "mxmoe_expert_ffn_fp8 (act_terms_kernel + ffn_mxf4_kernel<gate_up|down, fp8 weights>)",
+                    "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                    else "fallback 6.65 TB/s", "traffic": None, "unit_ms": unit_ms_mean,
+                    "algorithmic_bytes_per_launch": unit_bytes}
+        dtype = "e2m1 digit terms x e4m3 -> f32"
+    elif T * k >= BF16_PATH_ROWS:
         # dominant unit: mxmoe_ffn_gate_up on bf16 tensor cores (passes, slot rows, x_tile +
         # ffn_bf16_kernel<gate_up>); algorithmic work = the dense gate/up
         # contraction of every grouped row: 2 * rows * 2I * H flops
@@ -600,8 +630,11 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
         "dtype": dtype, "config": workload_config(cfg, world, nb), "weight_gbs": weight_gbs,
         "weight_frac_of_hbm_peak": weight_gbs / peak, "touched_experts_per_step": mean_touched,
         "roofline": roofline, "clocks": clocks.summary(windows),
-        "gpu_launches": kernels_per_step(T, k, E, H) * steps,
+        "gpu_launches": (kernels_per_step(T, k, E, H) if not fp8 else (3 if T * k > 4096 and E <= 1024 else 1) + 6)
+        * steps,
     }
+    if fp8:
+        out["weight_format"] = "fp8 (E4M3, one E8M0 scale per 32)"
     if ms_e2e is not None:
         out["e2e"] = {"value": T * steps * world / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
                       "d2h_bytes_per_step": T * H * 4,
@@ -653,6 +686,16 @@ def run_native(args):
         wg, prepacked = layers[(c.H, c.E, c.I)]
         results[c.name] = measure_layer(mx, c, wg, prepacked, args, None, args.warmup, world, rank, dev, clocks)
         torch.cuda.empty_cache()
+    fp8_name = None
+    if not args.no_per_config and not args.experts and not args.tokens:
+        # the verify8 workload with FP8 experts (the pages' 8-bit baseline), to set its weight stream against MXFP4's
+        c = datagen.BY_NAME["verify8"]
+        wg8, pre8 = make_layer(mx, c, args.seed, dev, fmt="fp8")
+        fp8_name = "verify8_fp8"
+        results[fp8_name] = measure_layer(mx, c, wg8, pre8, args, None, args.warmup, world, rank, dev, clocks,
+                                          fmt="fp8")
+        del wg8, pre8
+        torch.cuda.empty_cache()
     wg, prepacked = layers[(head.H, head.E, head.I)]
     res = measure_layer(mx, head, wg, prepacked, args, args.steps, args.warmup, world, rank, dev, clocks)
     clocks.stop()
@@ -677,17 +720,17 @@ def run_native(args):
         line["cpu_baseline"] = cpu_baseline(head, args.seed, x0, bias_np, args.cpu_tokens)
     if results:
         line["per_config"] = {}
-        for c in cfgs:
-            if c.name == head.name:
+        for name in [c.name for c in cfgs] + ([fp8_name] if fp8_name else []):
+            if name == head.name:
                 r = dict(res)
             else:
-                r = results[c.name]
+                r = results[name]
                 r.pop("_x0")
                 r.pop("_bias")
-            line["per_config"][c.name] = {key: r[key] for key in (
+            line["per_config"][name] = {key: r[key] for key in (
                 "value", "unit", "ms_per_step", "steps", "dtype", "weight_gbs", "weight_frac_of_hbm_peak",
-                "touched_experts_per_step", "roofline", "e2e", "clocks", "gpu_launches") if key in r}
-            line["per_config"][c.name]["workload"] = r["config"]["workload"]
+                "touched_experts_per_step", "roofline", "e2e", "clocks", "gpu_launches", "weight_format") if key in r}
+            line["per_config"][name]["workload"] = r["config"]["workload"]
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -286,6 +286,81 @@ MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, const float *bi
                                   int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out,
                                   void *workspace, int64_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------ */
+/* FP8 expert weights                                                        */
+/* ------------------------------------------------------------------------ */
+/* The model card's section 2 ("FP4 Quantization") sets the MXFP4 experts
+ * against an FP8 baseline, and its introduction says that even 8-bit weights
+ * carry heavy memory-bandwidth costs at this scale, so lowering the bit width
+ * speeds up decoding. These entry points run the same layer with FP8 expert
+ * weights, to measure that. The pages give no FP8 layout; the reading is the
+ * MX scheme of the FP4 experts with E4M3 elements ("MXFP8"): one E8M0 scale
+ * per 32 elements along K, scale exponent e = floor(log2 amax) - 8 clamped to
+ * [-127, 127] (-127 for an all-zero block; 8 is the exponent of E4M3's
+ * largest power of two), each element |x| / 2^e rounded to nearest E4M3 with
+ * ties to the even mantissa, saturating at 448, sign bit copied. E4M3 codes:
+ * bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa; exponent 0 is
+ * subnormal; 0x7F / 0xFF (NaN) are never produced. */
+
+/* bf16 [rows, K] -> E4M3 codes uint8 [rows, K] (one byte per element) and
+ * scales uint8 [rows, K/32], all device memory.
+ * Errors: K % 32 != 0 or rows/K <= 0 -> INVALID_SHAPE; NULL -> NULL; w not
+ * 16-byte or codes not 8-byte aligned -> ALIGNMENT. */
+MXMOE_API int mxmoe_quantize_fp8(const void *w, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales,
+                                 void *stream);
+
+/* out[r, k] = E4M3(codes[r, k]) * 2^(scales[r, k/32] - 127) as float (device
+ * memory). Errors as for mxmoe_quantize_fp8. */
+MXMOE_API int mxmoe_dequantize_fp8(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K, float *out,
+                                   void *stream);
+
+/* Bytes of the prepacked FP8 blob: E * (2*I*H + Hp*I) * 33/32, Hp = H rounded
+ * up to a multiple of 256. -1 unless H and I are positive multiples of 128. */
+MXMOE_API int64_t mxmoe_prepacked_size_fp8(int E, int H, int I);
+
+/* Re-tile FP8 expert weights for the FP8 FFN (a byte permutation plus
+ * zero padding of the down rows to a multiple of 256).
+ *   codes13 device uint8 [E, 2I, H], sc13 [E, 2I, H/32] (gate rows 0..I-1,
+ *   up rows I..2I-1); codes2 [E, H, I], sc2 [E, H, I/32] (down);
+ *   prepacked device, mxmoe_prepacked_size_fp8 bytes, 32-byte aligned.
+ * Layout: [gate/up code boxes][down code boxes][gate/up scale images][down
+ * scale images]. A code box is a 256-row tile by 128 values of K (256 rows of
+ * 128 bytes, 32 KB, contiguous), boxes ordered by (expert, tile, K chunk);
+ * gate/up tile t holds gate rows 128t .. 128t+127, then the matching up rows.
+ * A box's scale images are two 512-byte images, one per row half g: byte
+ * (r % 32) * 16 + (r / 32) * 4 + kb is the scale of tile row 128g + r, k32
+ * block kb of the box.
+ * Errors: shapes -> INVALID_SHAPE; NULL -> NULL; prepacked not 32-byte or
+ * codes13/codes2 not 16-byte aligned -> ALIGNMENT. */
+MXMOE_API int mxmoe_prepack_experts_fp8(const uint8_t *codes13, const uint8_t *sc13, const uint8_t *codes2,
+                                        const uint8_t *sc2, int E, int H, int I, void *prepacked, void *stream);
+
+/* Workspace bytes for mxmoe_expert_ffn_fp8 (-1 on bad sizes). */
+MXMOE_API int64_t mxmoe_ffn_workspace_size_fp8(int T, int k, int E, int H, int I);
+
+/* mxmoe_expert_ffn with FP8 expert weights (blob from
+ * mxmoe_prepack_experts_fp8): the same grouped SwiGLU FFN, arguments, layout
+ * and errors, workspace from mxmoe_ffn_workspace_size_fp8. Both stages run on
+ * tcgen05.mma.kind::mxf8f6f4.block_scale at every token count: E4M3 weights
+ * as stored times the E2M1 digit terms of x and h (the same terms, and the
+ * same error bound, as the MXFP4 kernel), UE8M0 scales per 32 applied in
+ * hardware, fp32 accumulation. */
+MXMOE_API int mxmoe_expert_ffn_fp8(const void *x, const int32_t *offsets, const int32_t *src_row,
+                                   const void *prepacked, int T, int k, int E, int H, int I, float *y_perm,
+                                   void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Workspace bytes for mxmoe_layer_forward_fp8 (-1 for exactly the shapes it
+ * rejects with INVALID_SHAPE). */
+MXMOE_API int64_t mxmoe_workspace_size_fp8(int T, int H, int I, int E, int k);
+
+/* mxmoe_layer_forward with FP8 expert weights: router GEMM, route, permute,
+ * mxmoe_expert_ffn_fp8's FFN, combine. Arguments and errors as for
+ * mxmoe_layer_forward, prepacked from mxmoe_prepack_experts_fp8, workspace
+ * from mxmoe_workspace_size_fp8. */
+MXMOE_API int mxmoe_layer_forward_fp8(const void *x, const void *wg, const float *bias, const void *prepacked, int T,
+                                      int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out,
+                                      void *workspace, int64_t workspace_bytes, void *stream);
+
 /* Test of the device-side timeout path (failure detection): one thread waits
  * on a shared-memory mbarrier that nothing ever arrives on, through the same
  * bounded wait that every wait of the FFN and router kernels uses, with a

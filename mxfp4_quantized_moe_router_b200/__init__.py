@@ -54,6 +54,14 @@ _SIGS = {
     "mxmoe_selftest_wait_timeout": (_I, [_P, _I, _P]),
     "mxmoe_permute_ws": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
     "mxmoe_permute_scratch_size": (_I64, [_I, _I, _I]),
+    "mxmoe_quantize_fp8": (_I, [_P, _I64, _I64, _P, _P, _P]),
+    "mxmoe_dequantize_fp8": (_I, [_P, _P, _I64, _I64, _P, _P]),
+    "mxmoe_prepacked_size_fp8": (_I64, [_I, _I, _I]),
+    "mxmoe_prepack_experts_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "mxmoe_ffn_workspace_size_fp8": (_I64, [_I, _I, _I, _I, _I]),
+    "mxmoe_expert_ffn_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I64, _P]),
+    "mxmoe_workspace_size_fp8": (_I64, [_I, _I, _I, _I, _I]),
+    "mxmoe_layer_forward_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
     "mxmoe_verify_workspace_size": (_I64, [_I, _I, _I64]),
     "mxmoe_verify_block": (_I, [_P, _P, _P, _P, _I, _I, _I64, ctypes.c_float, _P, _P, _P, _I64, _P]),
 }
@@ -385,6 +393,132 @@ class ExpertWeights:
     def prepack(self, stream=None):
         mxmoe_prepack_experts(self.packed13, self.sc13, self.packed2, self.sc2, self.E, self.H, self.I,
                               self.prepacked, stream)
+
+
+# ---------------------------------------------------------------------------
+# FP8 expert weights (E4M3, one E8M0 scale per 32)
+# ---------------------------------------------------------------------------
+def mxmoe_quantize_fp8(w, codes, scales, stream=None):
+    import torch
+
+    rows, K = w.shape
+    _need(w, torch.bfloat16, (rows, K), "w")
+    _need(codes, torch.uint8, (rows, K), "codes")
+    _need(scales, torch.uint8, (rows, K // 32), "scales")
+    _check("mxmoe_quantize_fp8",
+           load().mxmoe_quantize_fp8(_ptr(w), rows, K, _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def quantize_fp8(w, stream=None):
+    """bf16 [rows, K] -> (E4M3 codes uint8 [rows, K], scales uint8 [rows, K/32])."""
+    import torch
+
+    rows, K = w.shape
+    codes = torch.empty((rows, K), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((rows, K // 32), dtype=torch.uint8, device=w.device)
+    mxmoe_quantize_fp8(w.contiguous(), codes, scales, stream)
+    return codes, scales
+
+
+def mxmoe_dequantize_fp8(codes, scales, out, stream=None):
+    import torch
+
+    rows, K = out.shape
+    _need(codes, torch.uint8, (rows, K), "codes")
+    _need(scales, torch.uint8, (rows, K // 32), "scales")
+    _need(out, torch.float32, (rows, K), "out")
+    _check("mxmoe_dequantize_fp8",
+           load().mxmoe_dequantize_fp8(_ptr(codes), _ptr(scales), rows, K, _ptr(out), _stream(stream)))
+
+
+def dequantize_fp8(codes, scales, stream=None):
+    import torch
+
+    out = torch.empty(tuple(codes.shape), dtype=torch.float32, device=codes.device)
+    mxmoe_dequantize_fp8(codes, scales, out, stream)
+    return out
+
+
+def mxmoe_prepacked_size_fp8(E: int, H: int, I: int) -> int:
+    return load().mxmoe_prepacked_size_fp8(E, H, I)
+
+
+def mxmoe_prepack_experts_fp8(codes13, sc13, codes2, sc2, E, H, I, prepacked, stream=None):
+    import torch
+
+    _need(codes13, torch.uint8, (E, 2 * I, H), "codes13")
+    _need(sc13, torch.uint8, (E, 2 * I, H // 32), "sc13")
+    _need(codes2, torch.uint8, (E, H, I), "codes2")
+    _need(sc2, torch.uint8, (E, H, I // 32), "sc2")
+    _need(prepacked, torch.uint8, (mxmoe_prepacked_size_fp8(E, H, I),), "prepacked")
+    _check("mxmoe_prepack_experts_fp8",
+           load().mxmoe_prepack_experts_fp8(_ptr(codes13), _ptr(sc13), _ptr(codes2), _ptr(sc2), E, H, I,
+                                            _ptr(prepacked), _stream(stream)))
+
+
+def mxmoe_ffn_workspace_size_fp8(T, k, E, H, I) -> int:
+    return load().mxmoe_ffn_workspace_size_fp8(T, k, E, H, I)
+
+
+def mxmoe_expert_ffn_fp8(x, offsets, src_row, prepacked, k, E, I, y_perm, workspace, stream=None):
+    import torch
+
+    T, H = x.shape
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(src_row, torch.int32, (T * k,), "src_row")
+    _need(y_perm, torch.float32, (T * k, H), "y_perm")
+    _check("mxmoe_expert_ffn_fp8",
+           load().mxmoe_expert_ffn_fp8(_ptr(x), _ptr(offsets), _ptr(src_row), _ptr(prepacked), T, k, E, H, I,
+                                       _ptr(y_perm), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))
+
+
+def mxmoe_workspace_size_fp8(T, H, I, E, k) -> int:
+    return load().mxmoe_workspace_size_fp8(T, H, I, E, k)
+
+
+def mxmoe_layer_forward_fp8(x, wg, bias, prepacked, I, k, y, workspace, ids_out=None, w_out=None, stream=None):
+    import torch
+
+    T, H = x.shape
+    E = wg.shape[0]
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(wg, torch.bfloat16, (E, H), "wg")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    _need(y, torch.float32, (T, H), "y")
+    if ids_out is not None:
+        _need(ids_out, torch.int32, (T, k), "ids_out")
+    if w_out is not None:
+        _need(w_out, torch.float32, (T, k), "w_out")
+    _check("mxmoe_layer_forward_fp8",
+           load().mxmoe_layer_forward_fp8(_ptr(x), _ptr(wg), _ptr(bias), _ptr(prepacked), T, H, I, E, k, _ptr(y),
+                                          _ptr(ids_out), _ptr(w_out), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+class ExpertWeightsFp8:
+    """FP8 expert weights of one layer on the device: E4M3 codes and scales
+    (canonical) plus the prepacked blob the FP8 FFN streams."""
+
+    def __init__(self, E: int, H: int, I: int, device="cuda"):
+        import torch
+
+        self.E, self.H, self.I = E, H, I
+        self.codes13 = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
+        self.sc13 = torch.empty((E, 2 * I, H // 32), dtype=torch.uint8, device=device)
+        self.codes2 = torch.empty((E, H, I), dtype=torch.uint8, device=device)
+        self.sc2 = torch.empty((E, H, I // 32), dtype=torch.uint8, device=device)
+        self.prepacked = torch.empty((mxmoe_prepacked_size_fp8(E, H, I),), dtype=torch.uint8, device=device)
+
+    def quantize_expert(self, e: int, w13, w2, stream=None):
+        mxmoe_quantize_fp8(w13, self.codes13[e], self.sc13[e], stream)
+        mxmoe_quantize_fp8(w2, self.codes2[e], self.sc2[e], stream)
+
+    def prepack(self, stream=None):
+        mxmoe_prepack_experts_fp8(self.codes13, self.sc13, self.codes2, self.sc2, self.E, self.H, self.I,
+                                  self.prepacked, stream)
 
 
 # ---------------------------------------------------------------------------

@@ -103,6 +103,9 @@ int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row
 int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int T, int k, int H, float *y,
                 cudaStream_t st);
 int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
+int run_expert_ffn_fp8(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
+                       int k, int E, int H, int I, float *y_perm, void *workspace, bool clear_status, cudaStream_t st);
+int64_t ffn_workspace_bytes_fp8(int T, int k, int E, int H, int I);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
 bool ffn_shapes_ok(int T, int k, int E, int H, int I);
 int router_splits(int T, int H, int E);
@@ -126,7 +129,7 @@ struct LayerWs {
     float *y_perm;
 };
 
-int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *base)
+int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *base, bool fp8 = false)
 {
     int64_t off = 0;
     auto take = [&](int64_t bytes) {
@@ -135,7 +138,7 @@ int64_t layer_ws_layout(int T, int H, int I, int E, int k, LayerWs *ws, void *ba
         return o;
     };
     const int64_t n = (int64_t)T * k;
-    const int64_t o_ffn = take(ffn_workspace_bytes(T, k, E, H, I));
+    const int64_t o_ffn = take(fp8 ? ffn_workspace_bytes_fp8(T, k, E, H, I) : ffn_workspace_bytes(T, k, E, H, I));
     const int64_t o_logits = take((int64_t)router_splits(T, H, E) * T * E * 4);
     const int64_t o_ids = take(n * 4);
     const int64_t o_w = take(n * 4);
@@ -179,33 +182,34 @@ extern "C" MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, in
     return layer_ws_layout(T, H, I, E, k, nullptr, nullptr);
 }
 
-extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, const float *bias, const void *prepacked,
-                                             int T, int H, int I, int E, int k, float *y, int32_t *ids_out,
-                                             float *w_out, void *workspace, int64_t workspace_bytes, void *stream)
+namespace {
+// The whole layer; fp8 selects the FP8-weight expert FFN (prepacked by
+// mxmoe_prepack_experts_fp8) instead of the MXFP4 one.
+int layer_forward(const char *fn, bool fp8, const void *x, const void *wg, const float *bias, const void *prepacked,
+                  int T, int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out, void *workspace,
+                  int64_t workspace_bytes, void *stream)
 {
     if (k > E)
-        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_layer_forward: k=%d > E=%d", k, E);
+        return fail(MXMOE_ERR_INVALID_SHAPE, "%s: k=%d > E=%d", fn, k, E);
     if (T > kMaxLayerTokens)
-        return fail(MXMOE_ERR_INVALID_SHAPE, "mxmoe_layer_forward: T=%d > %d (the combine's grid)", T,
-                    kMaxLayerTokens);
+        return fail(MXMOE_ERR_INVALID_SHAPE, "%s: T=%d > %d (the combine's grid)", fn, T, kMaxLayerTokens);
     if (int rc = validate_ffn_shapes(T, k, E, H, I))
         return rc;
-    const int64_t need = layer_ws_layout(T, H, I, E, k, nullptr, nullptr);
+    const int64_t need = layer_ws_layout(T, H, I, E, k, nullptr, nullptr, fp8);
     if (!workspace || workspace_bytes < need)
-        return fail(MXMOE_ERR_WORKSPACE, "mxmoe_layer_forward: workspace of %lld bytes, need %lld",
-                    (long long)workspace_bytes, (long long)need);
+        return fail(MXMOE_ERR_WORKSPACE, "%s: workspace of %lld bytes, need %lld", fn, (long long)workspace_bytes,
+                    (long long)need);
     if (T == 0)
         return MXMOE_OK;
     if (!x || !wg || !prepacked || !y)
-        return fail(MXMOE_ERR_NULL, "mxmoe_layer_forward: NULL pointer");
+        return fail(MXMOE_ERR_NULL, "%s: NULL pointer", fn);
     if (!aligned16(x) || !aligned16(wg) || !aligned16(prepacked) || !aligned16(y) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255))
-        return fail(MXMOE_ERR_ALIGNMENT,
-                    "mxmoe_layer_forward: x, wg, prepacked, y need 16-byte and workspace 256-byte alignment");
+        return fail(MXMOE_ERR_ALIGNMENT, "%s: x, wg, prepacked, y need 16-byte and workspace 256-byte alignment", fn);
     if (int rc = check_device())
         return rc;
     LayerWs ws;
-    layer_ws_layout(T, H, I, E, k, &ws, workspace);
+    layer_ws_layout(T, H, I, E, k, &ws, workspace, fp8);
     int32_t *ids = ids_out ? ids_out : ws.ids;
     float *w = w_out ? w_out : ws.w;
     cudaStream_t st = (cudaStream_t)stream;
@@ -213,16 +217,44 @@ extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, cons
     // of the router kernel survives to mxmoe_read_status
     int *status = static_cast<int *>(ws.ffn);
     if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess)
-        return fail(MXMOE_ERR_CUDA, "mxmoe_layer_forward: cannot clear the status word");
+        return fail(MXMOE_ERR_CUDA, "%s: cannot clear the status word", fn);
     ChainScope chain;  // the router GEMM starts after the clear; every later kernel is chained
     if (int rc = run_router_and_route(x, wg, bias, T, H, E, k, ws.logits, router_splits(T, H, E), ids, w, status,
                                       st))
         return rc;
     if (int rc = run_permute(ids, T, k, E, ws.offsets, ws.src_row, ws.dst_of, ws.permute_scratch, st))
         return rc;
-    if (int rc = run_expert_ffn(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn, false, st))
+    if (int rc = fp8 ? run_expert_ffn_fp8(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn,
+                                          false, st)
+                     : run_expert_ffn(x, ws.offsets, ws.src_row, prepacked, T, k, E, H, I, ws.y_perm, ws.ffn, false,
+                                      st))
         return rc;
     return run_combine(ws.y_perm, ws.dst_of, w, T, k, H, y, st);
+}
+}  // namespace
+
+extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, const float *bias, const void *prepacked,
+                                             int T, int H, int I, int E, int k, float *y, int32_t *ids_out,
+                                             float *w_out, void *workspace, int64_t workspace_bytes, void *stream)
+{
+    return layer_forward("mxmoe_layer_forward", false, x, wg, bias, prepacked, T, H, I, E, k, y, ids_out, w_out,
+                         workspace, workspace_bytes, stream);
+}
+
+extern "C" MXMOE_API int64_t mxmoe_workspace_size_fp8(int T, int H, int I, int E, int k)
+{
+    if (T > kMaxLayerTokens || k > E || !ffn_shapes_ok(T, k, E, H, I))
+        return -1;
+    return layer_ws_layout(T, H, I, E, k, nullptr, nullptr, true);
+}
+
+extern "C" MXMOE_API int mxmoe_layer_forward_fp8(const void *x, const void *wg, const float *bias,
+                                                 const void *prepacked, int T, int H, int I, int E, int k, float *y,
+                                                 int32_t *ids_out, float *w_out, void *workspace,
+                                                 int64_t workspace_bytes, void *stream)
+{
+    return layer_forward("mxmoe_layer_forward_fp8", true, x, wg, bias, prepacked, T, H, I, E, k, y, ids_out, w_out,
+                         workspace, workspace_bytes, stream);
 }
 
 namespace mxmoe {

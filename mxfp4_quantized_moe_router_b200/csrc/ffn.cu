@@ -42,6 +42,12 @@
 //    over a persistent grid of one CTA per SM (CTA b takes items b, b + G,
 //    ...), so that the passes of one weight tile run side by side and share
 //    its boxes in L2.
+//  * FP8 expert weights (E4M3 codes, one E8M0 scale per 32; the pages' FP8
+//    baseline, model card section 2) run through the same kernel with
+//    tcgen05.mma.kind::mxf8f6f4.block_scale: the E4M3 weights are the N
+//    operand as they are stored (256 rows x 128 values of K per 32 KB box),
+//    the activations the same E2M1 digit terms, unpacked to one byte per
+//    value by the TMA (16U4_ALIGN16B), with the same UE8M0 scale images.
 #include <float.h>
 #include <limits.h>
 
@@ -162,6 +168,28 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
+// Instruction descriptor of kind::mxf8f6f4.block_scale with A = E2M1 (the
+// activation terms, one per byte), B = E4M3 (FP8 weights), UE8M0 scales, both
+// K-major, M = 128, N = n, scale byte sf_id (0..3: the k32 block of a 4-block
+// scale column) for both operands.
+__device__ __forceinline__ uint32_t idesc_e2m1_x_e4m3(int n, uint32_t sf_id)
+{
+    return (sf_id << 4) | (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | (8u << 24) |
+           (sf_id << 29);
+}
+
+// D (+)= A * B^T over 32 values of K, one UE8M0 scale per 32 values for each
+// operand (the scale bytes picked by the descriptor's sf_id).
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // Work items of one FFN stage: (expert, 256-row tile, token pass), expert-major,
 // then tile, then pass. CTA b takes items b, b + G, b + 2G, ... (G CTAs), so
 // the passes of one weight tile run on neighbouring CTAs at about the same
@@ -240,7 +268,10 @@ __device__ __forceinline__ void act_digits(float v, int E, uint32_t (&code)[kT])
 // One FFN stage over all experts.
 // GATE_UP = true: stage 1 (x terms in; h terms and their scale images out).
 // GATE_UP = false: stage 2 (h terms in; float rows out).
-template <int NT, bool GATE_UP>
+// FP8 = true: E4M3 weights (128 values of K per box, kind::mxf8f6f4, the
+// activation terms unpacked to a byte each by the TMA); else MXFP4 weights
+// (256 values of K per box, kind::mxf4).
+template <int NT, bool GATE_UP, bool FP8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_mxf4_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
                     const FfnParams p)
@@ -315,8 +346,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t G = gridDim.x, total = s_items[E];
     const int n_items = (int)(total > blockIdx.x ? (total - blockIdx.x + G - 1) / G : 0);
 #define ITEM(i) decode_item<NT>(blockIdx.x + (int64_t)(i) * G, s_items, p.offsets, E, tiles)
-    const int nchunk = (p.K + kKC - 1) / kKC;  // the last chunk may hold one 128-column half
+    // MXFP4: 256-value chunks (the last may hold one 128-column half);
+    // FP8: 128-value chunks, each one half
+    const int nchunk = FP8 ? p.K / 128 : (p.K + kKC - 1) / kKC;
     const int khalves = p.K / 128;
+    constexpr int kWSfBox = FP8 ? 1024 : kWSf;  // a box's weight scale images
     // Chained launch: the producer fills the weight ring before waiting for
     // the preceding kernel (weights and offsets are older than it; the
     // activation terms, their scale images and the pass table are its
@@ -336,9 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int64_t issued_w = 0, issued_a = 0;
             bool ok = true;
             auto load_w = [&](int sl, int64_t box) {  // weight box and its scale images into slot sl
-                mbar_arrive_expect_tx(&fullW[sl], (uint32_t)(kWBox + kWSf));
+                mbar_arrive_expect_tx(&fullW[sl], (uint32_t)(kWBox + kWSfBox));
                 tc::tma_load_2d(sW + (size_t)sl * kWBox, &tmW, 0, (int)(box * 256), &fullW[sl], pol_w);
-                bulk_g2s_hint(sSfw + sl * kWSf, p.wsf + box * kWSf, kWSf, &fullW[sl], pol_w);
+                bulk_g2s_hint(sSfw + sl * kWSf, p.wsf + box * kWSfBox, kWSfBox, &fullW[sl], pol_w);
             };
             int64_t pre_w = 0;  // weight boxes issued before the wait (slots 0 .. pre_w-1, first use)
             for (int i = 0; i < n_items && pre_w < C::kStagesW; ++i) {
@@ -366,11 +400,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    const int nh = min(2, khalves - 2 * c);  // K halves in this chunk
-                    mbar_arrive_expect_tx(&fullA[sa], (uint32_t)(C::kATx + nh * kSFImg));
-                    tc::tma_load_4d(sA + (size_t)sa * kAStage, &tmA, 0, 0, r0, c, &fullA[sa], pol_a);
-                    bulk_g2s_hint(sSfa + sa * 2 * kSFImg, p.asf + (pass_id * khalves + 2 * c) * kSFImg,
-                                  (uint32_t)(nh * kSFImg), &fullA[sa], pol_a);
+                    if (FP8) {
+                        // K half c of the packed terms, unpacked to a byte per value (the transaction
+                        // counts the packed bytes: 64 per row), and its one scale image
+                        mbar_arrive_expect_tx(&fullA[sa], (uint32_t)(C::kM * 64 + kSFImg));
+                        tc::tma_load_4d(sA + (size_t)sa * kAStage, &tmA, 128 * (c & 1), 0, r0, c >> 1, &fullA[sa],
+                                        pol_a);
+                        bulk_g2s_hint(sSfa + sa * 2 * kSFImg, p.asf + (pass_id * khalves + c) * kSFImg, kSFImg,
+                                      &fullA[sa], pol_a);
+                    } else {
+                        const int nh = min(2, khalves - 2 * c);  // K halves in this chunk
+                        mbar_arrive_expect_tx(&fullA[sa], (uint32_t)(C::kATx + nh * kSFImg));
+                        tc::tma_load_4d(sA + (size_t)sa * kAStage, &tmA, 0, 0, r0, c, &fullA[sa], pol_a);
+                        bulk_g2s_hint(sSfa + sa * 2 * kSFImg, p.asf + (pass_id * khalves + 2 * c) * kSFImg,
+                                      (uint32_t)(nh * kSFImg), &fullA[sa], pol_a);
+                    }
                     ++issued_a;
                     if (++sw == C::kStagesW) {
                         sw = 0;
@@ -422,13 +466,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sfa_t = tmem + C::kSfaCol0 + 8 * sa;   // + 4 per K half
                     const uint32_t a_base = smem_u32(sA + (size_t)sa * kAStage);
                     const uint32_t w_base = smem_u32(sW + (size_t)sw * kWBox);
-                    const int nk = 2 * min(2, khalves - 2 * c);  // a half chunk takes two MMAs
-                    for (int k = 0; k < nk; ++k) {  // 64 values of K per MMA
-                        const uint32_t h = (uint32_t)(k >> 1), id = 2u * (uint32_t)(k & 1);
-                        mma_mxf4(tmem, tc::smem_desc(a_base + k * 32, 16, 1024, 2),
-                                 tc::smem_desc(w_base + k * 32, 16, 1024, 2), idesc_mxf4(256, id),
-                                 (c > 0 || k > 0) ? 1u : 0u, (sfa_t + 4 * h) | (id << 30),
-                                 (sfw_t + 8 * h) | (id << 30));
+                    if (FP8) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {  // 32 values of K (32 bytes of both operands) per MMA
+                            const uint32_t id = (uint32_t)k;
+                            mma_mxf8f6f4(tmem, tc::smem_desc(a_base + k * 32, 16, 1024, 2),
+                                         tc::smem_desc(w_base + k * 32, 16, 1024, 2), idesc_e2m1_x_e4m3(256, id),
+                                         (c > 0 || k > 0) ? 1u : 0u, sfa_t | (id << 30), sfw_t | (id << 30));
+                        }
+                    } else {
+                        const int nk = 2 * min(2, khalves - 2 * c);  // a half chunk takes two MMAs
+                        for (int k = 0; k < nk; ++k) {  // 64 values of K per MMA
+                            const uint32_t h = (uint32_t)(k >> 1), id = 2u * (uint32_t)(k & 1);
+                            mma_mxf4(tmem, tc::smem_desc(a_base + k * 32, 16, 1024, 2),
+                                     tc::smem_desc(w_base + k * 32, 16, 1024, 2), idesc_mxf4(256, id),
+                                     (c > 0 || k > 0) ? 1u : 0u, (sfa_t + 4 * h) | (id << 30),
+                                     (sfw_t + 8 * h) | (id << 30));
+                        }
                     }
                     tc::commit(&emptyW[sw]);  // frees both stages once these MMAs are done
                     tc::commit(&emptyA[sa]);
@@ -480,9 +534,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t sfw_s = smem_u32(sSfw + sw * kWSf);
                 const uint32_t sfa_s = smem_u32(sSfa + sa * 2 * kSFImg);
 #pragma unroll
-                for (int img = 0; img < 4; ++img)
+                for (int img = 0; img < (FP8 ? 2 : 4); ++img)
                     tc::cp_32x128b_warpx4(sfw_t + 4 * img, tc::smem_desc(sfw_s + img * kSFImg, 16, 128, 0));
-                for (int h = 0; h < min(2, khalves - 2 * c); ++h)
+                for (int h = 0; h < (FP8 ? 1 : min(2, khalves - 2 * c)); ++h)
                     tc::cp_32x128b_warpx4(sfa_t + 4 * h, tc::smem_desc(sfa_s + h * kSFImg, 16, 128, 0));
                 tc::commit(&sfready[sa]);
                 any = true;
@@ -816,7 +870,8 @@ constexpr int kHotRows = 128;
 bool use_hybrid(int T, int k) { return !use_bf16_path(T, k) && T >= kHotRows; }
 int bf16_min_rows(int T, int k) { return use_bf16_path(T, k) ? 0 : kHotRows; }
 
-int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
+// fp8: the FP8-weight FFN, which runs every expert on the E2M1-term kernel.
+int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base, bool fp8 = false)
 {
     int64_t off = 0;
     auto take = [&](int64_t bytes) {
@@ -828,8 +883,8 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
     const int64_t passes = max_passes(rows);
     const int64_t o_status = take(16);
     const int64_t o_ps = take((kMaxE + 1) * 4);
-    const bool terms = !use_bf16_path(T, k);                 // the E2M1-term kernel runs
-    const bool bf16 = !terms || use_hybrid(T, k);           // the bf16 kernel runs
+    const bool terms = fp8 || !use_bf16_path(T, k);        // the E2M1-term kernel runs
+    const bool bf16 = !fp8 && (!terms || use_hybrid(T, k));  // the bf16 kernel runs
     const int64_t o_xt = take(terms ? rows * kT * pad256(H) / 2 : 0);
     const int64_t o_xs = take(terms ? passes * (H / 128) * kSFImg : 0);
     const int64_t o_ht = take(terms ? rows * kT * pad256(I) / 2 : 0);
@@ -857,15 +912,15 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base)
 
 
 int encode(CUtensorMap *m, int rank, const void *base, const cuuint64_t *dims, const cuuint64_t *strides,
-           const cuuint32_t *box, CUtensorMapL2promotion promo, const char *what)
+           const cuuint32_t *box, CUtensorMapL2promotion promo, const char *what,
+           CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_UINT8)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
-                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(m, type, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (%s) failed: %d", what, (int)r);
     return MXMOE_OK;
@@ -892,26 +947,41 @@ int encode_terms(CUtensorMap *m, const void *base, int64_t rows, int K, int nt)
     return encode(m, 4, base, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, "activation terms");
 }
 
-template <int NT, bool GATE_UP>
+// The same terms for the FP8 kernel: the 4-bit codes unpacked by the TMA into
+// one byte per value (16U4_ALIGN16B; dims and box counted in values), a
+// request bringing one 128-value K half of all terms of nt rows.
+int encode_terms_unpacked(CUtensorMap *m, const void *base, int64_t rows, int K, int nt)
+{
+    const cuuint64_t dims[4] = {256, (cuuint64_t)kT, (cuuint64_t)rows, (cuuint64_t)((K + kKC - 1) / kKC)};
+    const cuuint64_t strides[3] = {128, (cuuint64_t)(kT * 128), (cuuint64_t)(rows * kT * 128)};
+    const cuuint32_t box[4] = {128, (cuuint32_t)kT, (cuuint32_t)nt, 1};
+    return encode(m, 4, base, dims, strides, box, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, "unpacked activation terms",
+                  CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B);
+}
+
+template <int NT, bool GATE_UP, bool FP8 = false>
 int launch_ffn(const void *codes, const uint8_t *act_terms, const FfnParams &p, cudaStream_t st)
 {
     using C = Cfg<NT>;
+    auto kernel = ffn_mxf4_kernel<NT, GATE_UP, FP8>;
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        if (cudaFuncSetAttribute(ffn_mxf4_kernel<NT, GATE_UP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::kSmem) != cudaSuccess)
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem) != cudaSuccess)
             return fail(MXMOE_ERR_CUDA, "ffn_mxf4_kernel: cannot reserve %zu bytes of shared memory", C::kSmem);
         configured_dev = dev;
     }
     CUtensorMap tmW, tmA;
-    if (int rc = encode_weights(&tmW, codes, (int64_t)p.E * p.tiles * ((p.K + kKC - 1) / kKC)))
+    const int64_t chunks = FP8 ? p.K / 128 : (p.K + kKC - 1) / kKC;
+    if (int rc = encode_weights(&tmW, codes, (int64_t)p.E * p.tiles * chunks))
         return rc;
-    if (int rc = encode_terms(&tmA, act_terms, p.rows, p.K, NT))
+    if (int rc = FP8 ? encode_terms_unpacked(&tmA, act_terms, p.rows, p.K, NT)
+                     : encode_terms(&tmA, act_terms, p.rows, p.K, NT))
         return rc;
-    return launch_kernel(GATE_UP ? "ffn_mxf4_kernel<gate_up>" : "ffn_mxf4_kernel<down>", ffn_mxf4_kernel<NT, GATE_UP>,
-                         num_sms(), kThreads, C::kSmem, st, tmW, tmA, p);
+    const char *name = FP8 ? (GATE_UP ? "ffn_mxf4_kernel<gate_up, fp8 weights>" : "ffn_mxf4_kernel<down, fp8 weights>")
+                           : (GATE_UP ? "ffn_mxf4_kernel<gate_up>" : "ffn_mxf4_kernel<down>");
+    return launch_kernel(name, kernel, num_sms(), kThreads, C::kSmem, st, tmW, tmA, p);
 }
 
 // Token rows per pass: 8 up to 8 tokens (an expert then never sees more than
@@ -1039,6 +1109,72 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
                           ws.status, st);
 }
 
+// The FP8-weight FFN: both stages on the E2M1-term kernel with kind::mxf8f6f4
+// for every expert and token count.
+struct Fp8Blob {
+    const uint8_t *w13, *w2, *sf13, *sf2;
+};
+
+Fp8Blob fp8_blob_parts(const void *prepacked, int E, int H, int I)
+{
+    const uint8_t *b = static_cast<const uint8_t *>(prepacked);
+    const int64_t Hp = pad256(H);
+    Fp8Blob o;
+    o.w13 = b;
+    o.w2 = o.w13 + (int64_t)E * 2 * I * H;
+    o.sf13 = o.w2 + (int64_t)E * Hp * I;
+    o.sf2 = o.sf13 + (int64_t)E * 2 * I * (H / 32);
+    return o;
+}
+
+int run_expert_ffn_fp8(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
+                       int k, int E, int H, int I, float *y_perm, void *workspace, bool clear_status, cudaStream_t st)
+{
+    FfnWs ws;
+    ffn_ws_layout(T, k, E, H, I, &ws, workspace, true);
+    const int rows = T * k;
+    const int nt = token_tile(T);
+    const Fp8Blob bl = fp8_blob_parts(prepacked, E, H, I);
+    const int64_t warps = (int64_t)rows * ((H + kKC - 1) / kKC);
+    const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 8);
+    if (int rc = launch_kernel("act_terms_kernel", act_terms_kernel, blocks < 1 ? 1 : blocks, 256, 0, st,
+                               static_cast<const uint16_t *>(x), src_row, offsets, E, k, rows, H, nt, INT_MAX,
+                               ws.x_terms, ws.x_sf, ws.pass_start, clear_status ? ws.status : nullptr))
+        return rc;
+    FfnParams p{};
+    p.tiles = I / 128;
+    p.K = H;
+    p.rows = rows;
+    p.wsf = bl.sf13;
+    p.asf = ws.x_sf;
+    p.offsets = offsets;
+    p.pass_start = ws.pass_start;
+    p.E = E;
+    p.h_terms = ws.h_terms;
+    p.h_sf = ws.h_sf;
+    p.I = I;
+    p.H = H;
+    p.hot_rows = INT_MAX;
+    p.status = ws.status;
+    if (int rc = nt == 8 ? launch_ffn<8, true, true>(bl.w13, ws.x_terms, p, st)
+                         : launch_ffn<16, true, true>(bl.w13, ws.x_terms, p, st))
+        return rc;
+    p.tiles = (int)(pad256(H) / 256);
+    p.K = I;
+    p.wsf = bl.sf2;
+    p.asf = ws.h_sf;
+    p.h_terms = nullptr;
+    p.h_sf = nullptr;
+    p.y_out = y_perm;
+    return nt == 8 ? launch_ffn<8, false, true>(bl.w2, ws.h_terms, p, st)
+                   : launch_ffn<16, false, true>(bl.w2, ws.h_terms, p, st);
+}
+
+int64_t ffn_workspace_bytes_fp8(int T, int k, int E, int H, int I)
+{
+    return ffn_ws_layout(T, k, E, H, I, nullptr, nullptr, true);
+}
+
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
                    int k, int E, int H, int I, float *y_perm, void *workspace, bool clear_status, cudaStream_t st)
 {
@@ -1073,13 +1209,15 @@ extern "C" MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H
     return ffn_workspace_bytes(T, k, E, H, I);
 }
 
-static int check_ffn_args(const char *fn, int T, int k, int E, int H, int I, void *workspace, int64_t workspace_bytes)
+static int check_ffn_args(const char *fn, int T, int k, int E, int H, int I, void *workspace, int64_t workspace_bytes,
+                          bool fp8 = false)
 {
     if (int rc = validate_ffn_shapes(T, k, E, H, I))
         return rc;
-    if (!workspace || workspace_bytes < ffn_workspace_bytes(T, k, E, H, I))
+    const int64_t need = fp8 ? ffn_workspace_bytes_fp8(T, k, E, H, I) : ffn_workspace_bytes(T, k, E, H, I);
+    if (!workspace || workspace_bytes < need)
         return fail(MXMOE_ERR_WORKSPACE, "%s: workspace of %lld bytes, need %lld", fn, (long long)workspace_bytes,
-                    (long long)ffn_workspace_bytes(T, k, E, H, I));
+                    (long long)need);
     if (reinterpret_cast<uintptr_t>(workspace) & 255)
         return fail(MXMOE_ERR_ALIGNMENT, "%s: workspace needs 256-byte alignment", fn);
     return MXMOE_OK;
@@ -1156,4 +1294,31 @@ extern "C" MXMOE_API int mxmoe_combine(const float *y_perm, const int32_t *dst_o
     if (int rc = check_device())
         return rc;
     return run_combine(y_perm, dst_of, w, T, k, H, y, (cudaStream_t)stream);
+}
+
+extern "C" MXMOE_API int64_t mxmoe_ffn_workspace_size_fp8(int T, int k, int E, int H, int I)
+{
+    if (!ffn_shapes_ok(T, k, E, H, I))
+        return -1;
+    return ffn_workspace_bytes_fp8(T, k, E, H, I);
+}
+
+extern "C" MXMOE_API int mxmoe_expert_ffn_fp8(const void *x, const int32_t *offsets, const int32_t *src_row,
+                                              const void *prepacked, int T, int k, int E, int H, int I, float *y_perm,
+                                              void *workspace, int64_t workspace_bytes, void *stream)
+{
+    if (int rc = check_ffn_args("mxmoe_expert_ffn_fp8", T, k, E, H, I, workspace, workspace_bytes, true))
+        return rc;
+    if (T == 0)
+        return MXMOE_OK;
+    if (!x || !offsets || !src_row || !prepacked || !y_perm)
+        return fail(MXMOE_ERR_NULL, "mxmoe_expert_ffn_fp8: NULL pointer");
+    if (!aligned16(x) || !aligned32(prepacked) || !aligned16(y_perm))
+        return fail(MXMOE_ERR_ALIGNMENT,
+                    "mxmoe_expert_ffn_fp8: x and y_perm need 16-byte, prepacked 32-byte alignment");
+    if (int rc = check_device())
+        return rc;
+    ChainScope chain;
+    return run_expert_ffn_fp8(x, offsets, src_row, prepacked, T, k, E, H, I, y_perm, workspace, true,
+                              (cudaStream_t)stream);
 }
