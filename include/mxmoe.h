@@ -361,6 +361,58 @@ MXMOE_API int mxmoe_layer_forward_fp8(const void *x, const void *wg, const float
                                       int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out,
                                       void *workspace, int64_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------ */
+/* Expert parallelism                                                        */
+/* ------------------------------------------------------------------------ */
+/* The pages serve the model with expert parallelism (--ep-size 16 in the
+ * SGLang launch of the "MiMo-V2.5-Pro-FP4-DFlash" model card's deployment
+ * section and of the nxbn.cn article's SGLang deployment section). With G
+ * ranks, rank g holds experts [g E/G, (g+1) E/G) (E a multiple of G) as its
+ * own prepacked blob, and each rank routes its own tokens. One layer step on
+ * rank g:
+ *   1. mxmoe_router_gemm + mxmoe_route on its tokens (all E experts);
+ *   2. mxmoe_permute: pairs grouped by expert -- also by owner rank;
+ *   3. mxmoe_ep_dispatch: the rows to send, their local expert ids and the
+ *      row count per destination rank;
+ *   4. all-to-all of the counts, then of the rows and ids (the caller's
+ *      collective library, e.g. NCCL through torch.distributed);
+ *   5. mxmoe_ep_expert_ffn on the received rows with the rank's experts;
+ *   6. all-to-all back (the reverse splits): the output rows land in the
+ *      grouped order of step 2;
+ *   7. mxmoe_combine with step 2's dst_of and step 1's weights.
+ * The result equals mxmoe_layer_forward of the whole layer on the rank's
+ * tokens up to float summation order. */
+
+/* Sender side of the dispatch, after mxmoe_permute.
+ *   x device bf16 [T, H]; offsets, src_row from mxmoe_permute over E experts.
+ *   send_x device bf16 [T*k, H]: send_x[r] = x[src_row[r] / k] (grouped
+ *   order, so rank g's rows are offsets[g E/G] .. offsets[(g+1) E/G]).
+ *   send_local device int32 [T*k]: the expert of row r minus the first
+ *   expert of its owner rank.
+ *   send_counts device int32 [G]: rows destined to each rank.
+ * Errors: E > 1024 or not a multiple of G, k > 32, H % 8 != 0, T*k > 2^24 ->
+ * INVALID_SHAPE; NULL -> NULL; x, send_x not 16-byte aligned -> ALIGNMENT. */
+MXMOE_API int mxmoe_ep_dispatch(const void *x, const int32_t *offsets, const int32_t *src_row, int T, int k, int E,
+                                int G, int H, void *send_x, int32_t *send_local, int32_t *send_counts, void *stream);
+
+/* Workspace bytes for mxmoe_ep_expert_ffn (-1 on bad sizes). */
+MXMOE_API int64_t mxmoe_ep_workspace_size(int n_recv, int E_local, int H, int I);
+
+/* Receiver side: the rank's experts applied to the rows it received.
+ *   x_recv device bf16 [n_recv, H]; recv_local device int32 [n_recv], each
+ *   in [0, E_local); prepacked_local: mxmoe_prepack_experts of the rank's
+ *   E_local experts; y_recv device float [n_recv, H]: y_recv[i] = the FFN of
+ *   expert recv_local[i] on x_recv[i] (receive order); workspace device,
+ *   >= mxmoe_ep_workspace_size bytes, 256-byte aligned (its first 16 bytes
+ *   hold the device status word, read with mxmoe_read_status).
+ * The rows are grouped by local expert (mxmoe_permute with k = 1), run
+ * through mxmoe_expert_ffn and gathered back into receive order.
+ * Errors: the expert FFN's shapes with T = n_recv, k = 1 -> INVALID_SHAPE;
+ * workspace -> WORKSPACE / ALIGNMENT; NULL -> NULL. */
+MXMOE_API int mxmoe_ep_expert_ffn(const void *x_recv, const int32_t *recv_local, int n_recv, int E_local, int H,
+                                  int I, const void *prepacked_local, float *y_recv, void *workspace,
+                                  int64_t workspace_bytes, void *stream);
+
 /* Test of the device-side timeout path (failure detection): one thread waits
  * on a shared-memory mbarrier that nothing ever arrives on, through the same
  * bounded wait that every wait of the FFN and router kernels uses, with a

@@ -62,6 +62,9 @@ _SIGS = {
     "mxmoe_expert_ffn_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I64, _P]),
     "mxmoe_workspace_size_fp8": (_I64, [_I, _I, _I, _I, _I]),
     "mxmoe_layer_forward_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
+    "mxmoe_ep_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "mxmoe_ep_workspace_size": (_I64, [_I, _I, _I, _I]),
+    "mxmoe_ep_expert_ffn": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _I64, _P]),
     "mxmoe_verify_workspace_size": (_I64, [_I, _I, _I64]),
     "mxmoe_verify_block": (_I, [_P, _P, _P, _P, _I, _I, _I64, ctypes.c_float, _P, _P, _P, _I64, _P]),
 }
@@ -519,6 +522,41 @@ class ExpertWeightsFp8:
     def prepack(self, stream=None):
         mxmoe_prepack_experts_fp8(self.codes13, self.sc13, self.codes2, self.sc2, self.E, self.H, self.I,
                                   self.prepacked, stream)
+
+
+# ---------------------------------------------------------------------------
+# Expert parallelism (compute steps; the exchanges are in .ep)
+# ---------------------------------------------------------------------------
+def mxmoe_ep_dispatch(x, offsets, src_row, k, E, G, send_x, send_local, send_counts, stream=None):
+    import torch
+
+    T, H = x.shape
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(src_row, torch.int32, (T * k,), "src_row")
+    _need(send_x, torch.bfloat16, (T * k, H), "send_x")
+    _need(send_local, torch.int32, (T * k,), "send_local")
+    _need(send_counts, torch.int32, (G,), "send_counts")
+    _check("mxmoe_ep_dispatch",
+           load().mxmoe_ep_dispatch(_ptr(x), _ptr(offsets), _ptr(src_row), T, k, E, G, H, _ptr(send_x),
+                                    _ptr(send_local), _ptr(send_counts), _stream(stream)))
+
+
+def mxmoe_ep_workspace_size(n_recv, E_local, H, I) -> int:
+    return load().mxmoe_ep_workspace_size(n_recv, E_local, H, I)
+
+
+def mxmoe_ep_expert_ffn(x_recv, recv_local, E_local, I, prepacked_local, y_recv, workspace, stream=None):
+    import torch
+
+    n, H = x_recv.shape
+    _need(x_recv, torch.bfloat16, (n, H), "x_recv")
+    _need(recv_local, torch.int32, (n,), "recv_local")
+    _need(y_recv, torch.float32, (n, H), "y_recv")
+    _check("mxmoe_ep_expert_ffn",
+           load().mxmoe_ep_expert_ffn(_ptr(x_recv), _ptr(recv_local), n, E_local, H, I, _ptr(prepacked_local),
+                                      _ptr(y_recv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(stream)))
 
 
 # ---------------------------------------------------------------------------
