@@ -45,6 +45,7 @@ import datagen  # noqa: E402
 METRIC = "MXFP4 MoE-layer tokens/s; expert-weight HBM GB/s as % of peak (1×B200)"
 UNIT = "tokens/s"
 BF16_PATH_ROWS = 16384  # grouped rows (tokens x top-k) from which both FFN stages run on bf16 tensor cores
+PERSISTENT_MAX_TOKENS = 16  # mxmoe_layer_forward runs one persistent kernel up to this many tokens
 
 
 def kernels_per_step(T: int, k: int, E: int, H: int) -> int:
@@ -410,7 +411,8 @@ def fp8_expert_bytes(cfg) -> int:
     return n + n // 32
 
 
-def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev, clocks, want_e2e=True, fmt="mxfp4"):
+def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev, clocks, want_e2e=True, fmt="mxfp4",
+                  path="auto"):
     """Time one workload: the whole layer (device-resident inputs), its
     dominant unit (CUDA events on the launching stream: the gate/up stage, or
     for FP8 experts the whole expert FFN), and the end-to-end leg with host
@@ -442,7 +444,9 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
     fws_bytes = fws.numel()
     lws = torch.empty((mx.mxmoe_workspace_size_fp8 if fp8 else mx.mxmoe_workspace_size)(T, H, I, E, k),
                       dtype=torch.uint8, device=dev)
-    forward = L.mxmoe_layer_forward_fp8 if fp8 else L.mxmoe_layer_forward
+    forward = (L.mxmoe_layer_forward_fp8 if fp8 else
+               {"auto": L.mxmoe_layer_forward, "chained": L.mxmoe_layer_forward_chained,
+                "persistent": L.mxmoe_layer_forward_persistent}[path])
     lws_bytes = lws.numel()
 
     def layer_step(b, x=None, y_out=None):
@@ -635,6 +639,10 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
     }
     if fp8:
         out["weight_format"] = "fp8 (E4M3, one E8M0 scale per 32)"
+    persistent = path == "persistent" or (path == "auto" and not fp8 and T <= PERSISTENT_MAX_TOKENS and E <= 384)
+    out["layer_path"] = "persistent kernel" if persistent else "chained launches"
+    if persistent:  # one cooperative launch per step (plus the status clear)
+        out["gpu_launches"] = steps
     if ms_e2e is not None:
         out["e2e"] = {"value": T * steps * world / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": T * H * 2,
                       "d2h_bytes_per_step": T * H * 4,
@@ -687,7 +695,17 @@ def run_native(args):
         results[c.name] = measure_layer(mx, c, wg, prepacked, args, None, args.warmup, world, rank, dev, clocks)
         torch.cuda.empty_cache()
     fp8_name = None
+    extra = []
     if not args.no_per_config and not args.experts and not args.tokens:
+        # the persistent layer kernel against the chained launches, on the decode-sized workloads
+        for name, path in (("verify8", "chained"), ("verify256", "persistent")):
+            c = datagen.BY_NAME[name]
+            wg_c, pre_c = layers[(c.H, c.E, c.I)]
+            key = "%s_%s" % (name, path)
+            results[key] = measure_layer(mx, c, wg_c, pre_c, args, None, args.warmup, world, rank, dev, clocks,
+                                         want_e2e=False, path=path)
+            extra.append(key)
+            torch.cuda.empty_cache()
         # the verify8 workload with FP8 experts (the pages' 8-bit baseline), to set its weight stream against MXFP4's
         c = datagen.BY_NAME["verify8"]
         wg8, pre8 = make_layer(mx, c, args.seed, dev, fmt="fp8")
@@ -720,7 +738,7 @@ def run_native(args):
         line["cpu_baseline"] = cpu_baseline(head, args.seed, x0, bias_np, args.cpu_tokens)
     if results:
         line["per_config"] = {}
-        for name in [c.name for c in cfgs] + ([fp8_name] if fp8_name else []):
+        for name in [c.name for c in cfgs] + extra + ([fp8_name] if fp8_name else []):
             if name == head.name:
                 r = dict(res)
             else:
@@ -729,7 +747,8 @@ def run_native(args):
                 r.pop("_bias")
             line["per_config"][name] = {key: r[key] for key in (
                 "value", "unit", "ms_per_step", "steps", "dtype", "weight_gbs", "weight_frac_of_hbm_peak",
-                "touched_experts_per_step", "roofline", "e2e", "clocks", "gpu_launches", "weight_format") if key in r}
+                "touched_experts_per_step", "roofline", "e2e", "clocks", "gpu_launches", "weight_format",
+                "layer_path") if key in r}
             line["per_config"][name]["workload"] = r["config"]["workload"]
     print(json.dumps(line), flush=True)
     if world > 1:

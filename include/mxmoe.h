@@ -413,6 +413,38 @@ MXMOE_API int mxmoe_ep_expert_ffn(const void *x_recv, const int32_t *recv_local,
                                   int I, const void *prepacked_local, float *y_recv, void *workspace,
                                   int64_t workspace_bytes, void *stream);
 
+/* The layer of mxmoe_layer_forward as one persistent kernel: one CTA per SM,
+ * all resident (a cooperative launch), running the router GEMM, routing,
+ * grouping, the activation terms, both FFN stages (tcgen05 block-scaled MMA,
+ * the same items as mxmoe_expert_ffn's E2M1-term kernel) and the combine as
+ * phases separated by grid-wide barriers, so that no launch boundary sits
+ * between the layer's steps and the weight stream of the gate/up stage starts
+ * while the activation terms are still being encoded. This is the execution
+ * model of the pages' serving engine, applied to this layer: a persistent
+ * engine kernel that stays resident, removes the gaps at operator boundaries
+ * and keeps prefetching while the tensor cores compute ("Xiaomi
+ * MiMo-V2.5-Pro-UltraSpeed 發佈說明", agentlenshq.com, section "TileRT 執行模型").
+ * mxmoe_layer_forward takes this path by itself up to 16 tokens (the
+ * decode-sized steps, e.g. one verify block of 8); this entry point takes it
+ * for any supported size, mxmoe_layer_forward_chained never.
+ * Arguments, layout, results and workspace as for mxmoe_layer_forward (ids and
+ * weights identical; y equal up to float summation order, which is the same
+ * as the chained path's). Every grid-wide wait is bounded (2 s): a CTA that
+ * gives up records MXMOE_ERR_TIMEOUT in the status word (mxmoe_read_status)
+ * and the others stop at their next barrier.
+ * Errors: those of mxmoe_layer_forward; and T > 256, T*k > 4096 or E > 384 ->
+ * INVALID_SHAPE. */
+MXMOE_API int mxmoe_layer_forward_persistent(const void *x, const void *wg, const float *bias, const void *prepacked,
+                                             int T, int H, int I, int E, int k, float *y, int32_t *ids_out,
+                                             float *w_out, void *workspace, int64_t workspace_bytes, void *stream);
+
+/* mxmoe_layer_forward as the chain of separate launches at every size (never
+ * the persistent kernel). Arguments, results and errors as for
+ * mxmoe_layer_forward. */
+MXMOE_API int mxmoe_layer_forward_chained(const void *x, const void *wg, const float *bias, const void *prepacked,
+                                          int T, int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out,
+                                          void *workspace, int64_t workspace_bytes, void *stream);
+
 /* Test of the device-side timeout path (failure detection): one thread waits
  * on a shared-memory mbarrier that nothing ever arrives on, through the same
  * bounded wait that every wait of the FFN and router kernels uses, with a

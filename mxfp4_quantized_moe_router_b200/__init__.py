@@ -50,6 +50,8 @@ _SIGS = {
     "mxmoe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "mxmoe_workspace_size": (_I64, [_I, _I, _I, _I, _I]),
     "mxmoe_layer_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
+    "mxmoe_layer_forward_persistent": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
+    "mxmoe_layer_forward_chained": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
     "mxmoe_read_status": (_I, [_P, _P, _P]),
     "mxmoe_selftest_wait_timeout": (_I, [_P, _I, _P]),
     "mxmoe_permute_ws": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I64, _P]),
@@ -334,6 +336,35 @@ def mxmoe_layer_forward(x, wg, bias, prepacked, I, k, y, workspace, ids_out=None
            load().mxmoe_layer_forward(_ptr(x), _ptr(wg), _ptr(bias), _ptr(prepacked), T, H, I, E, k, _ptr(y),
                                    _ptr(ids_out), _ptr(w_out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def _layer_call(name, x, wg, bias, prepacked, I, k, y, workspace, ids_out, w_out, stream):
+    import torch
+
+    T, H = x.shape
+    E = wg.shape[0]
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(wg, torch.bfloat16, (E, H), "wg")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    _need(y, torch.float32, (T, H), "y")
+    if ids_out is not None:
+        _need(ids_out, torch.int32, (T, k), "ids_out")
+    if w_out is not None:
+        _need(w_out, torch.float32, (T, k), "w_out")
+    _check(name, getattr(load(), name)(_ptr(x), _ptr(wg), _ptr(bias), _ptr(prepacked), T, H, I, E, k, _ptr(y),
+                                       _ptr(ids_out), _ptr(w_out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def mxmoe_layer_forward_persistent(x, wg, bias, prepacked, I, k, y, workspace, ids_out=None, w_out=None, stream=None):
+    """mxmoe_layer_forward as one persistent kernel (T <= 256, T*k <= 4096, E <= 384)."""
+    _layer_call("mxmoe_layer_forward_persistent", x, wg, bias, prepacked, I, k, y, workspace, ids_out, w_out, stream)
+
+
+def mxmoe_layer_forward_chained(x, wg, bias, prepacked, I, k, y, workspace, ids_out=None, w_out=None, stream=None):
+    """mxmoe_layer_forward as chained launches at every size."""
+    _layer_call("mxmoe_layer_forward_chained", x, wg, bias, prepacked, I, k, y, workspace, ids_out, w_out, stream)
 
 
 def mxmoe_read_status(workspace, stream=None) -> int:

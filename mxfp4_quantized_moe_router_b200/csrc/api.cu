@@ -106,6 +106,10 @@ int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I);
 int run_expert_ffn_fp8(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,
                        int k, int E, int H, int I, float *y_perm, void *workspace, bool clear_status, cudaStream_t st);
 int64_t ffn_workspace_bytes_fp8(int T, int k, int E, int H, int I);
+bool fused_layer_ok(int T, int k, int E, int H, int I);
+int run_fused_layer(const void *x, const void *wg, const float *bias, const void *prepacked, int T, int H, int I,
+                    int E, int k, int nsplit, float *partials, int32_t *ids, float *w, int32_t *offsets,
+                    int32_t *src_row, int32_t *dst_of, float *y_perm, float *y, void *ffn_ws, cudaStream_t st);
 int validate_ffn_shapes(int T, int k, int E, int H, int I);
 bool ffn_shapes_ok(int T, int k, int E, int H, int I);
 int router_splits(int T, int H, int E);
@@ -183,9 +187,17 @@ extern "C" MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, in
 }
 
 namespace {
+// Token counts up to which mxmoe_layer_forward runs the whole layer as one
+// persistent kernel (decode-sized steps, where the chained launches' gaps and
+// the small kernels' latency weigh most).
+constexpr int kPersistentMaxTokens = 16;
+
+enum class LayerPath { kAuto, kChained, kPersistent };
+
 // The whole layer; fp8 selects the FP8-weight expert FFN (prepacked by
-// mxmoe_prepack_experts_fp8) instead of the MXFP4 one.
-int layer_forward(const char *fn, bool fp8, const void *x, const void *wg, const float *bias, const void *prepacked,
+// mxmoe_prepack_experts_fp8) instead of the MXFP4 one; path picks the chained
+// launches or the persistent kernel (kAuto: by size).
+int layer_forward(const char *fn, bool fp8, LayerPath path, const void *x, const void *wg, const float *bias, const void *prepacked,
                   int T, int H, int I, int E, int k, float *y, int32_t *ids_out, float *w_out, void *workspace,
                   int64_t workspace_bytes, void *stream)
 {
@@ -206,6 +218,10 @@ int layer_forward(const char *fn, bool fp8, const void *x, const void *wg, const
     if (!aligned16(x) || !aligned16(wg) || !aligned16(prepacked) || !aligned16(y) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255))
         return fail(MXMOE_ERR_ALIGNMENT, "%s: x, wg, prepacked, y need 16-byte and workspace 256-byte alignment", fn);
+    if (path == LayerPath::kPersistent && (fp8 || !fused_layer_ok(T, k, E, H, I)))
+        return fail(MXMOE_ERR_INVALID_SHAPE,
+                    "%s: T=%d k=%d E=%d (the persistent layer takes 1 <= T <= 256, T*k <= 4096, k <= E <= 384)", fn,
+                    T, k, E);
     if (int rc = check_device())
         return rc;
     LayerWs ws;
@@ -213,6 +229,11 @@ int layer_forward(const char *fn, bool fp8, const void *x, const void *wg, const
     int32_t *ids = ids_out ? ids_out : ws.ids;
     float *w = w_out ? w_out : ws.w;
     cudaStream_t st = (cudaStream_t)stream;
+    const bool persistent = path == LayerPath::kPersistent ||
+                            (path == LayerPath::kAuto && !fp8 && T <= kPersistentMaxTokens && fused_layer_ok(T, k, E, H, I));
+    if (persistent)
+        return run_fused_layer(x, wg, bias, prepacked, T, H, I, E, k, router_splits(T, H, E), ws.logits, ids, w,
+                               ws.offsets, ws.src_row, ws.dst_of, ws.y_perm, y, ws.ffn, st);
     // one status record for the whole layer (the FFN workspace's first word): cleared here, so that a timeout
     // of the router kernel survives to mxmoe_read_status
     int *status = static_cast<int *>(ws.ffn);
@@ -237,8 +258,26 @@ extern "C" MXMOE_API int mxmoe_layer_forward(const void *x, const void *wg, cons
                                              int T, int H, int I, int E, int k, float *y, int32_t *ids_out,
                                              float *w_out, void *workspace, int64_t workspace_bytes, void *stream)
 {
-    return layer_forward("mxmoe_layer_forward", false, x, wg, bias, prepacked, T, H, I, E, k, y, ids_out, w_out,
-                         workspace, workspace_bytes, stream);
+    return layer_forward("mxmoe_layer_forward", false, LayerPath::kAuto, x, wg, bias, prepacked, T, H, I, E, k, y,
+                         ids_out, w_out, workspace, workspace_bytes, stream);
+}
+
+extern "C" MXMOE_API int mxmoe_layer_forward_chained(const void *x, const void *wg, const float *bias,
+                                                     const void *prepacked, int T, int H, int I, int E, int k, float *y,
+                                                     int32_t *ids_out, float *w_out, void *workspace,
+                                                     int64_t workspace_bytes, void *stream)
+{
+    return layer_forward("mxmoe_layer_forward_chained", false, LayerPath::kChained, x, wg, bias, prepacked, T, H, I,
+                         E, k, y, ids_out, w_out, workspace, workspace_bytes, stream);
+}
+
+extern "C" MXMOE_API int mxmoe_layer_forward_persistent(const void *x, const void *wg, const float *bias,
+                                                        const void *prepacked, int T, int H, int I, int E, int k,
+                                                        float *y, int32_t *ids_out, float *w_out, void *workspace,
+                                                        int64_t workspace_bytes, void *stream)
+{
+    return layer_forward("mxmoe_layer_forward_persistent", false, LayerPath::kPersistent, x, wg, bias, prepacked, T,
+                         H, I, E, k, y, ids_out, w_out, workspace, workspace_bytes, stream);
 }
 
 extern "C" MXMOE_API int64_t mxmoe_workspace_size_fp8(int T, int H, int I, int E, int k)
@@ -253,8 +292,8 @@ extern "C" MXMOE_API int mxmoe_layer_forward_fp8(const void *x, const void *wg, 
                                                  int32_t *ids_out, float *w_out, void *workspace,
                                                  int64_t workspace_bytes, void *stream)
 {
-    return layer_forward("mxmoe_layer_forward_fp8", true, x, wg, bias, prepacked, T, H, I, E, k, y, ids_out, w_out,
-                         workspace, workspace_bytes, stream);
+    return layer_forward("mxmoe_layer_forward_fp8", true, LayerPath::kChained, x, wg, bias, prepacked, T, H, I, E, k,
+                         y, ids_out, w_out, workspace, workspace_bytes, stream);
 }
 
 namespace mxmoe {

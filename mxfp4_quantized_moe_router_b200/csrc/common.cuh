@@ -207,6 +207,12 @@ __device__ __forceinline__ uint64_t policy_evict_last()
     return p;
 }
 
+// Named barrier over `nthreads` threads (multiple of 32) of the block.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Tensor-core and conversion primitives
 // ---------------------------------------------------------------------------

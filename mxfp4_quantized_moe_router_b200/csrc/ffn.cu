@@ -57,6 +57,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "router_dev.cuh"
 #include "tcgen05.cuh"
 
 namespace mxmoe {
@@ -134,7 +135,8 @@ struct Cfg {
     static constexpr size_t kOffSfa = kOffSfw + (size_t)kStagesW * kWSf;
     static constexpr size_t kOffBar = kOffSfa + (size_t)kStagesA * 2 * kSFImg;
     static constexpr int kBars = 2 * kStagesW + 2 * kStagesA + 3 + kStagesA + 1;
-    static constexpr size_t kOffMisc = (kOffBar + kBars * 8 + 15) & ~size_t(15);
+    // two barrier sets: the persistent layer kernel gives each FFN stage its own
+    static constexpr size_t kOffMisc = (kOffBar + 2 * kBars * 8 + 15) & ~size_t(15);
     static constexpr size_t kOffItems = kOffMisc + 64;  // items before each expert [kMaxE + 1]
     static constexpr size_t kSmem = 1024 + kOffItems + (kMaxE + 1) * 4;
     // Tensor memory: the accumulator (128 lanes x 256 columns), then per weight
@@ -265,38 +267,48 @@ __device__ __forceinline__ void act_digits(float v, int E, uint32_t (&code)[kT])
     code[0] = e2m1_digit_code(u >> 21);
 }
 
-// One FFN stage over all experts.
-// GATE_UP = true: stage 1 (x terms in; h terms and their scale images out).
-// GATE_UP = false: stage 2 (h terms in; float rows out).
-// FP8 = true: E4M3 weights (128 values of K per box, kind::mxf8f6f4, the
-// activation terms unpacked to a byte each by the TMA); else MXFP4 weights
-// (256 values of K per box, kind::mxf4).
-template <int NT, bool GATE_UP, bool FP8 = false>
-__global__ void __launch_bounds__(kThreads, 1)
-    ffn_mxf4_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
-                    const FfnParams p)
+// Shared-memory view of one FFN stage: rings, scale images, barrier set
+// `set` (0 or 1) and the per-expert item table.
+template <int NT>
+struct StageSmem {
+    uint8_t *sW, *sA, *sSfw, *sSfa;
+    uint64_t *fullW, *emptyW, *fullA, *emptyA, *accfull, *accempty, *mma_done, *sfready, *cp_done;
+    uint32_t *tslot;
+    volatile int *abort_flag;
+    int32_t *s_items;
+    __device__ __forceinline__ StageSmem(uint8_t *smem, int set)
+    {
+        using C = Cfg<NT>;
+        sW = smem;
+        sA = smem + C::kOffA;
+        sSfw = smem + C::kOffSfw;
+        sSfa = smem + C::kOffSfa;
+        fullW = reinterpret_cast<uint64_t *>(smem + C::kOffBar) + set * C::kBars;
+        emptyW = fullW + C::kStagesW;
+        fullA = emptyW + C::kStagesW;
+        emptyA = fullA + C::kStagesA;
+        accfull = emptyA + C::kStagesA;
+        accempty = accfull + 1;
+        mma_done = accempty + 1;
+        sfready = mma_done + 1;  // [kStagesA]: a chunk's scale images are in tensor memory
+        cp_done = sfready + C::kStagesA;
+        tslot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
+        abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+        s_items = reinterpret_cast<int32_t *>(smem + C::kOffItems);
+    }
+};
+
+// Items of every expert and their prefix (s_items), the stage's barriers,
+// a cleared abort flag. Called by every thread of the block; ends with a
+// block-wide barrier.
+template <int NT>
+__device__ __forceinline__ void stage_prepare(const FfnParams &p, const StageSmem<NT> &S)
 {
     using C = Cfg<NT>;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sW = smem, *sA = smem + C::kOffA, *sSfw = smem + C::kOffSfw, *sSfa = smem + C::kOffSfa;
-    uint64_t *fullW = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
-    uint64_t *emptyW = fullW + C::kStagesW;
-    uint64_t *fullA = emptyW + C::kStagesW;
-    uint64_t *emptyA = fullA + C::kStagesA;
-    uint64_t *accfull = emptyA + C::kStagesA;
-    uint64_t *accempty = accfull + 1;
-    uint64_t *mma_done = accempty + 1;
-    uint64_t *sfready = mma_done + 1;        // [kStagesA]: a chunk's scale images are in tensor memory
-    uint64_t *cp_done = sfready + C::kStagesA;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = p.E, tiles = p.tiles;
-
-    int32_t *s_items = reinterpret_cast<int32_t *>(smem + C::kOffItems);
-    for (int e = tid; e < E; e += kThreads) {  // items of expert e: tiles * ceil(n_e / NT), none if it is hot
+    int32_t *s_items = S.s_items;
+    for (int e = tid; e < E; e += blockDim.x) {  // items of expert e: tiles * ceil(n_e / NT), none if it is hot
         const int n_e = p.offsets[e + 1] - p.offsets[e];
         s_items[e] = n_e >= p.hot_rows ? 0 : tiles * ((n_e + NT - 1) / NT);
     }
@@ -321,28 +333,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 32) {
         for (int s = 0; s < C::kStagesW; ++s) {
-            mbar_init(&fullW[s], 1);
-            mbar_init(&emptyW[s], 1);
+            mbar_init(&S.fullW[s], 1);
+            mbar_init(&S.emptyW[s], 1);
         }
         for (int s = 0; s < C::kStagesA; ++s) {
-            mbar_init(&fullA[s], 1);
-            mbar_init(&emptyA[s], 1);
+            mbar_init(&S.fullA[s], 1);
+            mbar_init(&S.emptyA[s], 1);
         }
-        mbar_init(accfull, 1);
-        mbar_init(accempty, 4);
-        mbar_init(mma_done, 1);
+        mbar_init(S.accfull, 1);
+        mbar_init(S.accempty, 4);
+        mbar_init(S.mma_done, 1);
         for (int s = 0; s < C::kStagesA; ++s)
-            mbar_init(&sfready[s], 1);
-        mbar_init(cp_done, 1);
-        *abort_flag = 0;
+            mbar_init(&S.sfready[s], 1);
+        mbar_init(S.cp_done, 1);
+        *S.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1)
-        tc::alloc(tslot, C::kTmemCols);
-    tc::fence_before();
     __syncthreads();
-    tc::fence_after();
-    const uint32_t tmem = *tslot;
+}
+
+// The chained launch's producer wait: the preceding kernel's results.
+struct WaitChained {
+    __device__ __forceinline__ bool operator()() const
+    {
+        grid_dep_wait();
+        return true;
+    }
+};
+
+// The roles of one FFN stage, warps 0..6 of the block (warp 0 producer, 1 MMA,
+// 2..5 epilogue, 6 scale copies; any further warps return at once). The
+// producer fills its weight ring first, then calls producer_wait() (false:
+// give up) before it loads any activation; every other role must have waited
+// for its inputs before it is called. No block-wide barrier inside; the
+// caller ends the stage with tc::fence_before() and __syncthreads().
+// GATE_UP = true: stage 1 (x terms in; h terms and their scale images out).
+// GATE_UP = false: stage 2 (h terms in; float rows out).
+// FP8 = true: E4M3 weights (128 values of K per box, kind::mxf8f6f4, the
+// activation terms unpacked to a byte each by the TMA); else MXFP4 weights
+// (256 values of K per box, kind::mxf4).
+template <int NT, bool GATE_UP, bool FP8, class ProducerWait>
+__device__ __forceinline__ void stage_roles(const CUtensorMap &tmW, const CUtensorMap &tmA, const FfnParams &p,
+                                            const StageSmem<NT> &S, uint32_t tmem, ProducerWait producer_wait)
+{
+    using C = Cfg<NT>;
+    uint8_t *sW = S.sW, *sA = S.sA, *sSfw = S.sSfw, *sSfa = S.sSfa;
+    uint64_t *fullW = S.fullW, *emptyW = S.emptyW, *fullA = S.fullA, *emptyA = S.emptyA;
+    uint64_t *accfull = S.accfull, *accempty = S.accempty, *mma_done = S.mma_done, *sfready = S.sfready;
+    uint64_t *cp_done = S.cp_done;
+    volatile int *abort_flag = S.abort_flag;
+    const int32_t *s_items = S.s_items;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = p.E, tiles = p.tiles;
     const int64_t G = gridDim.x, total = s_items[E];
     const int n_items = (int)(total > blockIdx.x ? (total - blockIdx.x + G - 1) / G : 0);
 #define ITEM(i) decode_item<NT>(blockIdx.x + (int64_t)(i) * G, s_items, p.offsets, E, tiles)
@@ -351,14 +393,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nchunk = FP8 ? p.K / 128 : (p.K + kKC - 1) / kKC;
     const int khalves = p.K / 128;
     constexpr int kWSfBox = FP8 ? 1024 : kWSf;  // a box's weight scale images
-    // Chained launch: the producer fills the weight ring before waiting for
-    // the preceding kernel (weights and offsets are older than it; the
-    // activation terms, their scale images and the pass table are its
-    // results); every other thread waits here. The next kernel is let start
-    // only as this one's CTAs exit: triggered earlier, its CTAs sat resident
-    // and waiting beside these, which measured slower.
-    if (!(warp == 0 && lane == 0))
-        grid_dep_wait();
 
     if (warp == 0) {
         // ----------------------------------------------------------- producer
@@ -381,7 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < nchunk && pre_w < C::kStagesW; ++c, ++pre_w)
                     load_w((int)pre_w, box0 + c);
             }
-            grid_dep_wait();
+            if (!producer_wait())
+                ok = false;
             for (int i = 0; i < n_items && ok; ++i) {
                 const Item it = ITEM(i);
                 const int64_t box0 = ((int64_t)it.e * tiles + it.tile) * nchunk;
@@ -430,7 +465,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 set_status(p.status, MXMOE_ERR_TIMEOUT);
                 *abort_flag = 1;
             }
-            // Drain: no copy of ours may still be landing when the CTA ends.
+            // Drain: no copy of ours may still be landing when the CTA ends (the
+            // weight loads issued before the wait included).
+            issued_w = issued_w > pre_w ? issued_w : pre_w;
             for (int64_t f = issued_w > C::kStagesW ? issued_w - C::kStagesW : 0; f < issued_w; ++f)
                 if (!mbar_wait_bounded(&fullW[f % C::kStagesW], (uint32_t)((f / C::kStagesW) & 1), kWaitLimitNs)) {
                     set_status(p.status, MXMOE_ERR_TIMEOUT);
@@ -560,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     set_status(p.status, MXMOE_ERR_TIMEOUT);
             }
         }
-    } else {
+    } else if (warp <= 5) {
         // ----------------------------------------------------------- epilogue
         // Warp quarter q reads accumulator lanes 32q .. 32q+31: tokens 4q .. 4q+3
         // of the pass, term tl = lane % 8 in each. A warp that gives up on a wait
@@ -677,13 +714,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
+#undef ITEM
+}
+
+// One FFN stage over all experts as its own (chained) launch.
+template <int NT, bool GATE_UP, bool FP8 = false>
+__global__ void __launch_bounds__(kThreads, 1)
+    ffn_mxf4_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
+                    const FfnParams p)
+{
+    using C = Cfg<NT>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const StageSmem<NT> S(smem, 0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    stage_prepare<NT>(p, S);
+    if (warp == 1)
+        tc::alloc(S.tslot, C::kTmemCols);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *S.tslot;
+    // Chained launch: the producer fills the weight ring before waiting for
+    // the preceding kernel (weights and offsets are older than it; the
+    // activation terms, their scale images and the pass table are its
+    // results); every other thread waits here. The next kernel is let start
+    // only as this one's CTAs exit: triggered earlier, its CTAs sat resident
+    // and waiting beside these, which measured slower.
+    if (!(warp == 0 && lane == 0))
+        grid_dep_wait();
+    stage_roles<NT, GATE_UP, FP8>(tmW, tmA, p, S, tmem, WaitChained{});
     tc::fence_before();
     __syncthreads();
     if (warp == 1) {
         tc::fence_after();
         tc::dealloc(tmem, C::kTmemCols);
     }
-#undef ITEM
 }
 
 // Token passes of each expert: pass_start[e] = sum over e' < e of
@@ -709,15 +775,89 @@ __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
     }
 }
 
-// Activation rows -> kT E2M1 terms per value in grouped row order, in the
-// term_offset layout, with their scale images (one per token pass and 128
-// columns), from x rows (bf16), row r holding token src_row[r] / k. One warp
-// per (row, 256-value chunk): lane l holds values 8l .. 8l+7 of the chunk (one
-// 16-byte load), a 32-value block is four lanes, and each of the kT terms of
-// the chunk leaves as one 128-byte row of 32-bit stores. Rows of experts with
-// at least hot_rows rows are skipped (the bf16 kernel takes those experts).
-// Block 0 also writes pass_start for the FFN stages and clears the status word
-// (when given).
+// One unit (grouped row r, 256-value chunk c; u = r * chunks + c) of the
+// activation terms: row r holds token src_row[r] / k; one warp, lane l holding
+// values 8l .. 8l+7 of the chunk (one 16-byte load), a 32-value block being
+// four lanes; each of the kT terms of the chunk leaves as one 128-byte row of
+// 32-bit stores, in the term_offset layout, with their scale images (one per
+// token pass and 128 columns). Rows of experts with at least hot_rows rows are
+// skipped (the bf16 kernel takes those experts). s_off / s_pass: the offsets
+// and the token-pass prefix in shared memory. COHERENT: src_row was written
+// earlier in the same launch (read through L2, not the read-only path).
+template <bool COHERENT>
+__device__ __forceinline__ void act_terms_unit(int64_t u, const uint16_t *__restrict__ act,
+                                               const int32_t *__restrict__ src_row, const int32_t *s_off,
+                                               const int32_t *s_pass, int E, int k, int rows, int H, int nt,
+                                               int hot_rows, uint8_t *__restrict__ terms, uint8_t *__restrict__ sf)
+{
+    const int lane = threadIdx.x & 31;
+    const int nch = (H + kKC - 1) / kKC;
+    const int kb = lane >> 2, q = lane & 3;  // the lane's 32-block within the chunk; its place in the block
+    const int r = (int)(u / nch), c = (int)(u % nch);
+    int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_off[mid] <= r)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    if (s_off[lo + 1] - s_off[lo] >= hot_rows)  // the bf16 kernel takes this expert
+        return;
+    const int local = r - s_off[lo];
+    const int64_t img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
+    const int n = local % nt;
+    const int tok = (COHERENT ? __ldcg(src_row + r) : __ldg(src_row + r)) / k;
+    const int col = c * kKC + 8 * lane;
+    const bool live = col < H;  // H % 128 == 0: in a half chunk lanes 0..15 are live
+    float v[8];
+    if (live) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(act + (int64_t)tok * H + col));
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[2 * j] = __uint_as_float(w4[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            v[j] = 0.f;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        m = fmaxf(m, fabsf(v[j]));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    const int E_blk = act_block_exp(m);
+    uint32_t word[kT];
+#pragma unroll
+    for (int t = 0; t < kT; ++t)
+        word[t] = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {  // value j of the lane: nibble j (element 2i in the low nibble of byte i)
+        uint32_t code[kT];
+        act_digits(v[j], E_blk, code);
+#pragma unroll
+        for (int t = 0; t < kT; ++t)
+            word[t] |= code[t] << (4 * j);
+    }
+    if (live) {
+        uint32_t *tp = reinterpret_cast<uint32_t *>(terms + term_offset(rows, 0, r, col));
+#pragma unroll
+        for (int t = 0; t < kT; ++t)  // term t sits 128 bytes after term t-1
+            tp[32 * t] = word[t];
+        // scales of the block: lane q of it writes terms q and q + 4
+        uint8_t *sp = sf + (img_row + 2 * c + (kb >> 2)) * kSFImg;
+        sp[image_byte(n, q, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * q + 127);
+        sp[image_byte(n, q + 4, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * (q + 4) + 127);
+    }
+}
+
+// Activation rows -> kT E2M1 terms per value in grouped row order (act_terms_unit
+// over every (row, 256-value chunk)). Block 0 also writes pass_start for the FFN
+// stages and clears the status word (when given).
 __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restrict__ act, const int32_t *__restrict__ src_row,
                                                       const int32_t *__restrict__ offsets, int E, int k, int rows,
                                                       int H, int nt, int hot_rows, uint8_t *__restrict__ terms,
@@ -727,7 +867,7 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
     grid_dep_wait();  // the preceding kernel's results (chained launch)
     grid_dep_launch();
     __shared__ int32_t s_off[kMaxE + 1], s_pass[kMaxE + 1];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5;
     for (int e = threadIdx.x; e <= E; e += blockDim.x)
         s_off[e] = offsets[e];
     __syncthreads();
@@ -746,69 +886,8 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
     const int nch = (H + kKC - 1) / kKC;
     const int64_t total = (int64_t)rows * nch;
     const int64_t nwarps = (int64_t)gridDim.x * 8, gw = (int64_t)blockIdx.x * 8 + warp;
-    const int kb = lane >> 2, q = lane & 3;  // the lane's 32-block within the chunk; its place in the block
-    for (int64_t u = gw; u < total; u += nwarps) {
-        const int r = (int)(u / nch), c = (int)(u % nch);
-        int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (s_off[mid] <= r)
-                lo = mid;
-            else
-                hi = mid;
-        }
-        if (s_off[lo + 1] - s_off[lo] >= hot_rows)  // the bf16 kernel takes this expert
-            continue;
-        const int local = r - s_off[lo];
-        const int64_t img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
-        const int n = local % nt;
-        const int tok = __ldg(src_row + r) / k;
-        const int col = c * kKC + 8 * lane;
-        const bool live = col < H;  // H % 128 == 0: in a half chunk lanes 0..15 are live
-        float v[8];
-        if (live) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(act + (int64_t)tok * H + col));
-            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[2 * j] = __uint_as_float(w4[j] << 16);
-                v[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                v[j] = 0.f;
-        }
-        float m = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            m = fmaxf(m, fabsf(v[j]));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        const int E_blk = act_block_exp(m);
-        uint32_t word[kT];
-#pragma unroll
-        for (int t = 0; t < kT; ++t)
-            word[t] = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {  // value j of the lane: nibble j (element 2i in the low nibble of byte i)
-            uint32_t code[kT];
-            act_digits(v[j], E_blk, code);
-#pragma unroll
-            for (int t = 0; t < kT; ++t)
-                word[t] |= code[t] << (4 * j);
-        }
-        if (live) {
-            uint32_t *tp = reinterpret_cast<uint32_t *>(terms + term_offset(rows, 0, r, col));
-#pragma unroll
-            for (int t = 0; t < kT; ++t)  // term t sits 128 bytes after term t-1
-                tp[32 * t] = word[t];
-            // scales of the block: lane q of it writes terms q and q + 4
-            uint8_t *sp = sf + (img_row + 2 * c + (kb >> 2)) * kSFImg;
-            sp[image_byte(n, q, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * q + 127);
-            sp[image_byte(n, q + 4, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * (q + 4) + 127);
-        }
-    }
+    for (int64_t u = gw; u < total; u += nwarps)
+        act_terms_unit<false>(u, act, src_row, s_off, s_pass, E, k, rows, H, nt, hot_rows, terms, sf);
 }
 
 // y[t, c] = sum_j w[t, j] * y_perm[dst_of[t*k + j], c], j in order.
@@ -833,6 +912,294 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
         acc.w = fmaf(wj, v.w, acc.w);
     }
     reinterpret_cast<float4 *>(y + (int64_t)t * H)[c4] = acc;
+}
+
+// ---------------------------------------------------------------------------
+// The whole layer as one persistent kernel (decode-sized token counts): the
+// execution model of the pages' serving engine -- a resident engine kernel
+// that removes the gaps at operator boundaries and keeps prefetching while
+// the tensor cores compute ("Xiaomi MiMo-V2.5-Pro-UltraSpeed 發佈說明",
+// agentlenshq.com, section "TileRT 執行模型").
+// ---------------------------------------------------------------------------
+// One CTA per SM, all co-resident (cooperative launch), 8 warps. The layer's
+// steps run as phases separated by grid-wide barriers, so no launch boundary
+// sits between them:
+//   1. router GEMM tiles (all warps; the same tiles and split sums as the
+//      chained router_gemm_kernel);                                  barrier 1
+//   2. routing, a warp per token;                                    barrier 2
+//   3. grouping by expert (CTA 0; offsets, src_row, dst_of, passes); barrier 3
+//   4. gate/up: warps 1..7 encode the activation terms while the producer warp
+//      already streams its first weight boxes; then the FFN roles; barrier 4
+//      is the terms' completion, which only the producer's activation loads
+//      and the other roles wait for;
+//   5. down: the FFN roles again (second barrier set);              barrier 5
+//   6. the weighted combine (all warps).                            barrier 6
+// Every barrier wait is bounded (2 s); a CTA that gives up records
+// MXMOE_ERR_TIMEOUT in the status word, which every waiter polls, so the
+// others stop at their next barrier. Memory written by one phase and read by
+// the next crosses CTAs through L2 (a release fence and atomic arrival, an
+// acquire load, then ld.global.cg or the TMA), and generic-proxy writes read by
+// the TMA are ordered with proxy fences on both sides.
+constexpr int kFusedThreads = 256;
+constexpr int kFusedMaxE = 384;      // routing keeps 12 logits per lane
+constexpr int kFusedMaxPairs = 4096;  // grouping in one CTA's shared memory
+
+struct FusedParams {
+    const uint16_t *x, *wg;
+    const float *bias;
+    int T, H, I, E, k, nsplit;
+    float *partials;  // router partial sums [nsplit, T, E]
+    int32_t *ids;
+    float *w;
+    int32_t *offsets, *src_row, *dst_of;  // the grouping (offsets also in gu / dn)
+    int32_t *pass_start;                  // token passes before each expert (also in gu / dn)
+    uint8_t *x_terms, *x_sf;              // the activation terms of x and their scale images
+    float *y_perm, *y;
+    unsigned *barrier;  // grid barrier arrivals, zero at launch
+    int *status;
+    FfnParams gu, dn;
+};
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Arrival of the CTA at the next grid barrier, by one thread, after a
+// block-wide barrier that followed every thread's writes of the phase (and
+// each thread's proxy fence, so that the TMA of other CTAs sees them).
+__device__ __forceinline__ void grid_arrive(unsigned *ctr)
+{
+    __threadfence();
+    atomicAdd(ctr, 1u);
+}
+
+// Waits until `target` arrivals; false on a timeout (recorded) or when another
+// CTA has recorded a failure.
+__device__ __forceinline__ bool grid_wait(const unsigned *ctr, unsigned target, int *status)
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_u32(ctr) < target) {
+        if (*reinterpret_cast<volatile int *>(status) != 0)
+            return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            set_status(status, MXMOE_ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(64);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+}
+
+__device__ __forceinline__ void proxy_fence_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Block-wide: arrive at barrier n and wait for it (every thread gets the verdict).
+__device__ __forceinline__ bool grid_sync(const FusedParams &fp, unsigned n, int *s_flag)
+{
+    proxy_fence_global();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        grid_arrive(fp.barrier);
+        *s_flag = grid_wait(fp.barrier, n * gridDim.x, fp.status);
+    }
+    __syncthreads();
+    return *s_flag != 0;
+}
+
+// The producer's wait before its first activation load: barrier n.
+struct WaitGrid {
+    const unsigned *ctr;
+    unsigned target;
+    int *status;
+    __device__ __forceinline__ bool operator()() const { return grid_wait(ctr, target, status); }
+};
+
+// Grouping of the T*k pairs by expert in one CTA (phase 3): counts, prefix,
+// then each expert's pairs in index order (stable), token passes of NT rows.
+template <int NT>
+__device__ void fused_group(const FusedParams &fp, int32_t *s_ids, int32_t *s_cnt, int32_t *s_off)
+{
+    const int n = fp.T * fp.k, E = fp.E;
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int q = tid; q < n; q += blockDim.x)
+        s_ids[q] = __ldcg(fp.ids + q);
+    for (int e = tid; e < E; e += blockDim.x)
+        s_cnt[e] = 0;
+    __syncthreads();
+    for (int q = tid; q < n; q += blockDim.x)
+        atomicAdd(&s_cnt[s_ids[q]], 1);
+    __syncthreads();
+    if (tid < 32) {  // exclusive prefixes of the counts (offsets) and of ceil(count / NT) (passes)
+        int carry = 0, carry_p = 0;
+        for (int b = 0; b <= E; b += 32) {
+            const int e = b + lane;
+            const int c = e < E ? s_cnt[e] : 0, cp = (c + NT - 1) / NT;
+            int incl = c, incl_p = cp;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                const int op = __shfl_up_sync(0xFFFFFFFFu, incl_p, off);
+                if (lane >= off) {
+                    incl += o;
+                    incl_p += op;
+                }
+            }
+            if (e <= E) {
+                s_off[e] = carry + incl - c;
+                fp.offsets[e] = carry + incl - c;
+                fp.pass_start[e] = carry_p + incl_p - cp;
+            }
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            carry_p += __shfl_sync(0xFFFFFFFFu, incl_p, 31);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) {
+        int pos = s_off[e];
+        for (int q = 0; q < n && pos < s_off[e + 1]; ++q)
+            if (s_ids[q] == e) {
+                fp.src_row[pos] = q;
+                fp.dst_of[q] = pos;
+                ++pos;
+            }
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    fused_layer_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmH,
+                       const FusedParams fp)
+{
+    using C = Cfg<NT>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const StageSmem<NT> S1(smem, 0), S2(smem, 1);
+    // two flags in the spare words after the stages' tensor-memory slot and abort flag
+    int &s_flag = *reinterpret_cast<int *>(smem + C::kOffMisc + 8);
+    int &s_flag2 = *reinterpret_cast<int *>(smem + C::kOffMisc + 12);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int T = fp.T, E = fp.E, k = fp.k, H = fp.H;
+    const int G = gridDim.x;
+    if (warp == 1)
+        tc::alloc(S1.tslot, C::kTmemCols);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *S1.tslot;
+    int32_t *s_scratch = reinterpret_cast<int32_t *>(S1.sA);  // the activation ring is free until stage 1 loads
+
+    // 1. router GEMM tiles
+    {
+        RouterRed &red = *reinterpret_cast<RouterRed *>(S1.sA);
+        const int ex = (E + kRgExperts - 1) / kRgExperts, ty = (T + kRgTokens - 1) / kRgTokens;
+        const int ntiles = ex * ty * fp.nsplit;
+        for (int vt = blockIdx.x; vt < ntiles; vt += G)
+            router_tile(fp.x, fp.wg, fp.bias, T, H, E, fp.partials, vt % ex, (vt / ex) % ty, vt / (ex * ty), fp.nsplit,
+                        red);
+    }
+    bool alive = grid_sync(fp, 1, &s_flag);
+    // 2. routing, a warp per token (the partial sums were written in this launch by other CTAs and were never
+    // read before on this SM, so the read-only path holds no stale copy of them)
+    if (alive)
+        for (int tok = blockIdx.x * 8 + warp; tok < T; tok += G * 8)
+            route_token<kFusedMaxE / 32, 4>(fp.partials, fp.nsplit, fp.nsplit > 1 ? fp.bias : nullptr, T, E, k,
+                                            fp.ids, fp.w, tok);
+    alive = alive && grid_sync(fp, 2, &s_flag);
+    // 3. grouping (CTA 0)
+    if (alive && blockIdx.x == 0)
+        fused_group<NT>(fp, s_scratch, s_scratch + kFusedMaxPairs, s_scratch + kFusedMaxPairs + kFusedMaxE);
+    alive = alive && grid_sync(fp, 3, &s_flag);
+
+    // 4. gate/up: warps 1..7 encode the activation terms while the producer (warp 0) streams its first weight
+    // boxes and then waits for barrier 4 before loading activations
+    if (alive) {
+        int32_t *s_off = s_scratch, *s_pass = s_scratch + kFusedMaxE + 1;
+        for (int e = tid; e <= E; e += blockDim.x) {
+            s_off[e] = __ldcg(fp.offsets + e);
+            s_pass[e] = __ldcg(fp.pass_start + e);
+        }
+        stage_prepare<NT>(fp.gu, S1);  // ends with a block-wide barrier
+        const WaitGrid w4{fp.barrier, 4u * G, fp.status};
+        if (warp == 0) {
+            stage_roles<NT, true, false>(tmW13, tmX, fp.gu, S1, tmem, w4);
+        } else {
+            const int nch = (H + kKC - 1) / kKC;
+            const int64_t total = (int64_t)T * k * nch;
+            const int64_t nworkers = (int64_t)G * 7, gw = (int64_t)blockIdx.x * 7 + (warp - 1);
+            for (int64_t u = gw; u < total; u += nworkers)
+                act_terms_unit<true>(u, fp.x, fp.src_row, s_off, s_pass, E, k, T * k, H, NT, INT_MAX, fp.x_terms,
+                                     fp.x_sf);
+            proxy_fence_global();
+            named_bar_sync(1, 7 * 32);  // warps 1..7: this CTA's terms are written
+            if (tid == 32) {
+                grid_arrive(fp.barrier);
+                s_flag2 = w4();
+            }
+            named_bar_sync(1, 7 * 32);
+            if (s_flag2)
+                stage_roles<NT, true, false>(tmW13, tmX, fp.gu, S1, tmem, w4);
+            else if (tid == 32)
+                *S1.abort_flag = 1;
+        }
+        tc::fence_before();
+        __syncthreads();
+        if (tid == 0)  // one verdict for the whole CTA
+            s_flag = s_flag2 != 0 && *reinterpret_cast<volatile int *>(fp.status) == 0;
+        __syncthreads();
+        alive = s_flag != 0;
+    }
+    // 5. down
+    if (alive) {
+        proxy_fence_global();  // this thread's h writes, for the other CTAs' TMA
+        __syncthreads();
+        if (tid == 0)
+            grid_arrive(fp.barrier);
+        stage_prepare<NT>(fp.dn, S2);
+        const WaitGrid w5{fp.barrier, 5u * G, fp.status};
+        if (warp == 0) {
+            stage_roles<NT, false, false>(tmW2, tmH, fp.dn, S2, tmem, w5);
+        } else {
+            if (tid == 32)
+                s_flag2 = w5();
+            named_bar_sync(1, 7 * 32);
+            if (s_flag2)
+                stage_roles<NT, false, false>(tmW2, tmH, fp.dn, S2, tmem, w5);
+            else if (tid == 32)
+                *S2.abort_flag = 1;
+        }
+        tc::fence_before();
+        __syncthreads();
+        alive = s_flag2 != 0;
+    }
+    // 6. combine: y[t, c] = sum over j, in order, of w[t, j] * y_perm[dst_of[t*k + j], c]
+    alive = alive && grid_sync(fp, 6, &s_flag);
+    if (alive) {
+        const int H4 = H / 4;
+        for (int64_t u = (int64_t)blockIdx.x * blockDim.x + tid; u < (int64_t)T * H4; u += (int64_t)G * blockDim.x) {
+            const int t = (int)(u / H4), c4 = (int)(u % H4);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < k; ++j) {
+                const float wj = __ldcg(fp.w + (int64_t)t * k + j);
+                const int r = __ldcg(fp.dst_of + (int64_t)t * k + j);
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(fp.y_perm + (int64_t)r * H) + c4);
+                acc.x = fmaf(wj, v.x, acc.x);
+                acc.y = fmaf(wj, v.y, acc.y);
+                acc.z = fmaf(wj, v.z, acc.z);
+                acc.w = fmaf(wj, v.w, acc.w);
+            }
+            reinterpret_cast<float4 *>(fp.y + (int64_t)t * H)[c4] = acc;
+        }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after();
+        tc::dealloc(tmem, C::kTmemCols);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1173,6 +1540,126 @@ int run_expert_ffn_fp8(const void *x, const int32_t *offsets, const int32_t *src
 int64_t ffn_workspace_bytes_fp8(int T, int k, int E, int H, int I)
 {
     return ffn_ws_layout(T, k, E, H, I, nullptr, nullptr, true);
+}
+
+// Whether the persistent layer kernel takes these sizes: every expert on the
+// E2M1-term kernel, the grouping in one CTA, routing with 12 logits a lane.
+bool fused_layer_ok(int T, int k, int E, int H, int I)
+{
+    return T >= 1 && T <= 256 && (int64_t)T * k <= kFusedMaxPairs && E <= kFusedMaxE && E >= k && k <= 32 &&
+           shapes_ok(T, k, E, H, I);
+}
+
+template <int NT>
+int launch_fused(const FusedParams &fp, const uint8_t *w13, const uint8_t *w2, const uint8_t *h_terms,
+                 cudaStream_t st)
+{
+    using C = Cfg<NT>;
+    auto kernel = fused_layer_kernel<NT>;
+    static thread_local int configured_dev = -1;
+    static thread_local int grid = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem) != cudaSuccess)
+            return fail(MXMOE_ERR_CUDA, "fused_layer_kernel: cannot reserve %zu bytes of shared memory", C::kSmem);
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kFusedThreads, C::kSmem) != cudaSuccess ||
+            per_sm < 1)
+            return fail(MXMOE_ERR_CUDA, "fused_layer_kernel: no CTA fits on an SM");
+        grid = num_sms();  // one CTA per SM, all resident at once
+        configured_dev = dev;
+    }
+    CUtensorMap tmW13, tmX, tmW2, tmH;
+    const int rows = fp.T * fp.k;
+    if (int rc = encode_weights(&tmW13, w13, (int64_t)fp.E * fp.gu.tiles * ((fp.H + kKC - 1) / kKC)))
+        return rc;
+    if (int rc = encode_terms(&tmX, fp.x_terms, rows, fp.H, NT))
+        return rc;
+    if (int rc = encode_weights(&tmW2, w2, (int64_t)fp.E * fp.dn.tiles * ((fp.I + kKC - 1) / kKC)))
+        return rc;
+    if (int rc = encode_terms(&tmH, h_terms, rows, fp.I, NT))
+        return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // the grid-wide barriers need every CTA resident
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tmW13, tmX, tmW2, tmH, fp);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MXMOE_ERR_CUDA, "fused_layer_kernel: %s", cudaGetErrorString(e));
+    }
+    return check_launch("fused_layer_kernel");
+}
+
+// The whole layer in one persistent launch (fused_layer_ok sizes). ffn_ws: the
+// FFN workspace of (T, k, E, H, I); its first 16 bytes (status word, barrier
+// counter) are cleared here, before the launch. partials: [nsplit, T, E].
+int run_fused_layer(const void *x, const void *wg, const float *bias, const void *prepacked, int T, int H, int I,
+                    int E, int k, int nsplit, float *partials, int32_t *ids, float *w, int32_t *offsets,
+                    int32_t *src_row, int32_t *dst_of, float *y_perm, float *y, void *ffn_ws, cudaStream_t st)
+{
+    FfnWs ws;
+    ffn_ws_layout(T, k, E, H, I, &ws, ffn_ws);
+    if (cudaMemsetAsync(ws.status, 0, 16, st) != cudaSuccess)
+        return fail(MXMOE_ERR_CUDA, "persistent layer: cannot clear the status word");
+    const Blob bl = blob_parts(prepacked, E, H, I);
+    const int nt = token_tile(T);
+    FusedParams fp{};
+    fp.x = static_cast<const uint16_t *>(x);
+    fp.wg = static_cast<const uint16_t *>(wg);
+    fp.bias = bias;
+    fp.T = T;
+    fp.H = H;
+    fp.I = I;
+    fp.E = E;
+    fp.k = k;
+    fp.nsplit = nsplit;
+    fp.partials = partials;
+    fp.ids = ids;
+    fp.w = w;
+    fp.offsets = offsets;
+    fp.src_row = src_row;
+    fp.dst_of = dst_of;
+    fp.pass_start = ws.pass_start;
+    fp.x_terms = ws.x_terms;
+    fp.x_sf = ws.x_sf;
+    fp.y_perm = y_perm;
+    fp.y = y;
+    fp.barrier = reinterpret_cast<unsigned *>(reinterpret_cast<uint8_t *>(ws.status) + 8);
+    fp.status = ws.status;
+    FfnParams &gu = fp.gu;
+    gu.tiles = I / 128;
+    gu.K = H;
+    gu.rows = T * k;
+    gu.wsf = bl.sf13;
+    gu.asf = ws.x_sf;
+    gu.offsets = offsets;
+    gu.pass_start = ws.pass_start;
+    gu.E = E;
+    gu.h_terms = ws.h_terms;
+    gu.h_sf = ws.h_sf;
+    gu.I = I;
+    gu.H = H;
+    gu.hot_rows = INT_MAX;
+    gu.status = ws.status;
+    FfnParams &dn = fp.dn;
+    dn = gu;
+    dn.tiles = (int)(pad256(H) / 256);
+    dn.K = I;
+    dn.wsf = bl.sf2;
+    dn.asf = ws.h_sf;
+    dn.h_terms = nullptr;
+    dn.h_sf = nullptr;
+    dn.y_out = y_perm;
+    return nt == 8 ? launch_fused<8>(fp, bl.w13, bl.w2, ws.h_terms, st)
+                   : launch_fused<16>(fp, bl.w13, bl.w2, ws.h_terms, st);
 }
 
 int run_expert_ffn(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked, int T,

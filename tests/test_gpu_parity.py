@@ -239,21 +239,21 @@ def test_combine(mx):
 # ---------------------------------------------------------------------------
 # Whole layer
 # ---------------------------------------------------------------------------
-def run_layer(mx, layer, x, bias):
+def run_layer(mx, layer, x, bias, forward=None):
     cfg = layer.cfg
     T = x.shape[0]
     ws = torch.empty(mx.mxmoe_workspace_size(T, cfg.H, cfg.I, cfg.E, cfg.k), dtype=torch.uint8, device=DEV)
     y = torch.empty((T, cfg.H), dtype=torch.float32, device=DEV)
     ids = torch.empty((T, cfg.k), dtype=torch.int32, device=DEV)
     w = torch.empty((T, cfg.k), dtype=torch.float32, device=DEV)
-    mx.mxmoe_layer_forward(x, layer.wg, bias, layer.ew.prepacked, cfg.I, cfg.k, y, ws, ids, w)
+    (forward or mx.mxmoe_layer_forward)(x, layer.wg, bias, layer.ew.prepacked, cfg.I, cfg.k, y, ws, ids, w)
     assert mx.mxmoe_read_status(ws) == mx.OK
     return y.cpu().numpy(), ids.cpu().numpy(), w.cpu().numpy()
 
 
-def check_layer(mx, layer, ox, x, bias, sample, check_bytes=False):
+def check_layer(mx, layer, ox, x, bias, sample, check_bytes=False, forward=None):
     cfg = layer.cfg
-    y, ids, w = run_layer(mx, layer, x.to(DEV), None if bias is None else torch.from_numpy(bias).to(DEV))
+    y, ids, w = run_layer(mx, layer, x.to(DEV), None if bias is None else torch.from_numpy(bias).to(DEV), forward)
     xs = x[torch.from_numpy(sample)]
     fetch = ox
     if check_bytes:
