@@ -943,6 +943,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 constexpr int kFusedThreads = 256;
 constexpr int kFusedMaxE = 384;      // routing keeps 12 logits per lane
 constexpr int kFusedMaxPairs = 4096;  // grouping in one CTA's shared memory
+constexpr int kFusedLocalRoute = 64;  // up to this many tokens CTA 0 routes them (no grid-wide barrier)
 
 struct FusedParams {
     const uint16_t *x, *wg;
@@ -1018,7 +1019,9 @@ struct WaitGrid {
 };
 
 // Grouping of the T*k pairs by expert in one CTA (phase 3): counts, prefix,
-// then each expert's pairs in index order (stable), token passes of NT rows.
+// token passes of NT rows, then the pairs placed in index order by warp 0, 32
+// at a time: lanes holding the same expert (match_any) take consecutive
+// places in lane order after that expert's earlier pairs (stable).
 template <int NT>
 __device__ void fused_group(const FusedParams &fp, int32_t *s_ids, int32_t *s_cnt, int32_t *s_off)
 {
@@ -1057,14 +1060,25 @@ __device__ void fused_group(const FusedParams &fp, int32_t *s_ids, int32_t *s_cn
         }
     }
     __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-        int pos = s_off[e];
-        for (int q = 0; q < n && pos < s_off[e + 1]; ++q)
-            if (s_ids[q] == e) {
+    if (tid < 32) {  // s_cnt becomes each expert's next free place
+        for (int e = lane; e < E; e += 32)
+            s_cnt[e] = s_off[e];
+        __syncwarp();
+        for (int base = 0; base < n; base += 32) {
+            const int q = base + lane;
+            const int e = q < n ? s_ids[q] : -1;
+            const uint32_t same = __match_any_sync(0xFFFFFFFFu, e);
+            const int rank = __popc(same & ((1u << lane) - 1u));
+            const int pos = e >= 0 ? s_cnt[e] + rank : 0;
+            __syncwarp();
+            if (e >= 0 && rank == 0)
+                s_cnt[e] += __popc(same);
+            __syncwarp();
+            if (q < n) {
                 fp.src_row[pos] = q;
                 fp.dst_of[q] = pos;
-                ++pos;
             }
+        }
     }
 }
 
@@ -1101,18 +1115,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             router_tile(fp.x, fp.wg, fp.bias, T, H, E, fp.partials, vt % ex, (vt / ex) % ty, vt / (ex * ty), fp.nsplit,
                         red);
     }
-    bool alive = grid_sync(fp, 1, &s_flag);
+    unsigned nbar = 1;
+    bool alive = grid_sync(fp, nbar, &s_flag);
     // 2. routing, a warp per token (the partial sums were written in this launch by other CTAs and were never
-    // read before on this SM, so the read-only path holds no stale copy of them)
-    if (alive)
-        for (int tok = blockIdx.x * 8 + warp; tok < T; tok += G * 8)
+    // read before on this SM, so the read-only path holds no stale copy of them). Up to kFusedLocalRoute
+    // tokens CTA 0 routes them all itself and goes on to the grouping without a grid-wide barrier.
+    const bool local_route = T <= kFusedLocalRoute;
+    if (alive && (!local_route || blockIdx.x == 0))
+        for (int tok = (local_route ? 0 : blockIdx.x * 8) + warp; tok < T; tok += local_route ? 8 : G * 8)
             route_token<kFusedMaxE / 32, 4>(fp.partials, fp.nsplit, fp.nsplit > 1 ? fp.bias : nullptr, T, E, k,
                                             fp.ids, fp.w, tok);
-    alive = alive && grid_sync(fp, 2, &s_flag);
+    if (!local_route)
+        alive = alive && grid_sync(fp, ++nbar, &s_flag);
+    else
+        __syncthreads();  // CTA 0's ids and weights, for its own grouping
     // 3. grouping (CTA 0)
     if (alive && blockIdx.x == 0)
         fused_group<NT>(fp, s_scratch, s_scratch + kFusedMaxPairs, s_scratch + kFusedMaxPairs + kFusedMaxE);
-    alive = alive && grid_sync(fp, 3, &s_flag);
+    alive = alive && grid_sync(fp, ++nbar, &s_flag);
 
     // 4. gate/up: warps 1..7 encode the activation terms while the producer (warp 0) streams its first weight
     // boxes and then waits for barrier 4 before loading activations
@@ -1123,7 +1143,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             s_pass[e] = __ldcg(fp.pass_start + e);
         }
         stage_prepare<NT>(fp.gu, S1);  // ends with a block-wide barrier
-        const WaitGrid w4{fp.barrier, 4u * G, fp.status};
+        const WaitGrid w4{fp.barrier, (++nbar) * G, fp.status};
         if (warp == 0) {
             stage_roles<NT, true, false>(tmW13, tmX, fp.gu, S1, tmem, w4);
         } else {
@@ -1159,7 +1179,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (tid == 0)
             grid_arrive(fp.barrier);
         stage_prepare<NT>(fp.dn, S2);
-        const WaitGrid w5{fp.barrier, 5u * G, fp.status};
+        const WaitGrid w5{fp.barrier, (++nbar) * G, fp.status};
         if (warp == 0) {
             stage_roles<NT, false, false>(tmW2, tmH, fp.dn, S2, tmem, w5);
         } else {
@@ -1176,7 +1196,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         alive = s_flag2 != 0;
     }
     // 6. combine: y[t, c] = sum over j, in order, of w[t, j] * y_perm[dst_of[t*k + j], c]
-    alive = alive && grid_sync(fp, 6, &s_flag);
+    alive = alive && grid_sync(fp, ++nbar, &s_flag);
     if (alive) {
         const int H4 = H / 4;
         for (int64_t u = (int64_t)blockIdx.x * blockDim.x + tid; u < (int64_t)T * H4; u += (int64_t)G * blockDim.x) {

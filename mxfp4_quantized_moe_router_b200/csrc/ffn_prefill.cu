@@ -16,23 +16,22 @@
 // accumulation): x as it is (exact), h as two bf16 terms hi + lo (within 2^-15
 // of h), which the down stage stacks along K so that one accumulator column
 // sums both.
-//  * A work item is (expert, pass of up to 256 tokens, one 128-row MMA tile
-//    -- half of a 256-row box of the prepacked blob). A K step is 64 values.
+//  * A work item is (expert, pass of up to 256 tokens, one 256-row box of the
+//    prepacked blob) = two 128-row MMA tiles. A K step is 64 values.
 //  * Three rings in shared memory, each with its own producer or writer, so
 //    that no role waits on another's latency: activation steps (bulk copies,
-//    3 x 32 KB; one step per K step for gate/up, two for down: hi then lo),
-//    packed weights with their scale images (two TMA boxes of 64 rows + a bulk
-//    copy, 4 x 9 KB of two K steps each, issued by a second producer warp
-//    ahead), and dequantised bf16 weight tiles (5 x 16 KB, written by sixteen
-//    warps, four threads per row, in the 128-byte-swizzled K-major layout the
-//    MMA reads).
-//  * One MMA warp, two accumulators (128 lanes x 256 columns each, together all
-//    of tensor memory) used by alternate items, so that the epilogue of item i
-//    overlaps the MMAs of item i + 1.
-//  * Eight epilogue warps, four per accumulator, each group draining the items
-//    of its accumulator: gate/up applies SwiGLU (tile row 32q + w is gate row
-//    16q + w of the tile's 64, w < 16, or the matching up row) and writes h as
-//    bf16 hi/lo terms; down writes y in fp32.
+//    2 x 32 KB; one step per K step for gate/up, two for down: hi then lo),
+//    packed weights with their scale images (TMA + bulk copy, 3 x 17 KB of two
+//    K steps each, issued by a second producer warp ahead), and dequantised
+//    bf16 weight tiles (3 x 32 KB, written by sixteen warps, two threads per
+//    row, in the 128-byte-swizzled K-major layout the MMA reads).
+//  * Two MMA warps each own one tile and one accumulator (128 lanes x 256
+//    columns, together all of tensor memory), so that the tiles' MMAs are
+//    issued independently and each accumulator has its own epilogue warps.
+//  * Eight epilogue warps, four per accumulator, drain both at once: gate/up
+//    applies SwiGLU (tile row 32q + w is gate row 16q + w of the tile's 64,
+//    w < 16, or the matching up row) and writes h as bf16 hi/lo terms; down
+//    writes y in fp32.
 //  * Items go round-robin over a persistent grid of one CTA per SM, so the
 //    few expert passes in flight keep their activations in L2 while every
 //    weight box is read once per pass.
@@ -50,16 +49,16 @@ namespace mxmoe {
 namespace {
 
 constexpr uint64_t kPWaitNs = 2000000000ull;  // bounded waits: 2 s
-constexpr int kPThreads = 864;  // 27 warps: see the role list at the kernel
+constexpr int kPThreads = 896;  // 28 warps: see the role list at the kernel
 constexpr int kPK = 64;         // K per step
 constexpr int kPTok = 256;      // tokens per pass
-constexpr int kPBStages = 3;    // activation ring
-constexpr int kPWStages = 4;    // packed weight ring (a slot holds two K steps of one tile)
-constexpr int kPAStages = 5;    // dequantised weight ring (one tile a slot)
+constexpr int kPBStages = 2;    // activation ring
+constexpr int kPWStages = 3;    // packed weight ring (a slot holds two K steps)
+constexpr int kPAStages = 3;    // dequantised weight ring (a third slot measured faster than a third activation slot)
 constexpr int kPBBytes = kPTok * 128;  // activation step: 256 rows x 64 bf16
 constexpr int kPABytes = 128 * 128;    // one bf16 weight tile step: 128 rows x 64 bf16
-constexpr int kPWBytes = 128 * 64;     // packed codes of two K steps of a tile: 128 rows x 128 codes
-constexpr int kPSfBytes = 1024;        // the box's scale images of that K half (both row halves)
+constexpr int kPWBytes = 256 * 64;     // packed codes of two K steps: 256 rows x 128 codes
+constexpr int kPSfBytes = 1024;        // their two scale images (one K half of a chunk, both row halves)
 struct PrefillParams {
     int pairs;                // 256-row blob boxes per expert: I/128 (gate/up) or Hp/256 (down)
     int K;                    // H (gate/up) or I (down)
@@ -74,13 +73,14 @@ struct PrefillParams {
     int *status;
 };
 
-// shared memory: activation ring | dequantised ring | packed ring | scale images | barriers | misc
+// shared memory: activation ring | dequantised ring (2 tiles a step) | packed ring | scale images | barriers |
+// misc
 constexpr size_t kPOffA = (size_t)kPBStages * kPBBytes;
-constexpr size_t kPOffW = kPOffA + (size_t)kPAStages * kPABytes;
+constexpr size_t kPOffW = kPOffA + (size_t)kPAStages * 2 * kPABytes;
 constexpr size_t kPOffSf = kPOffW + (size_t)kPWStages * kPWBytes;
 constexpr size_t kPOffBar = kPOffSf + (size_t)kPWStages * kPSfBytes;
-// full_b, empty_b, full_w, empty_w, aready, aempty, accfull[2], accempty[2], mma_done
-constexpr int kPBars = 2 * kPBStages + 2 * kPWStages + 2 * kPAStages + 5;
+// full_b, empty_b, full_w, empty_w, aready, aempty, accfull[2], accempty[2], mma_done[2]
+constexpr int kPBars = 2 * kPBStages + 2 * kPWStages + 2 * kPAStages + 6;
 constexpr size_t kPOffMisc = (kPOffBar + kPBars * 8 + 15) & ~size_t(15);
 constexpr size_t kPSmem = 1024 + kPOffMisc + 64;
 static_assert(kPSmem <= 232448, "shared memory");
@@ -199,14 +199,13 @@ __global__ void __launch_bounds__(256) x_tile_kernel(const uint16_t *__restrict_
     }
 }
 
-// Work items: (pass of up to 256 tokens, 128-row tile), passes in expert
-// order: item i is tile i % (2 pairs) of pass i / (2 pairs), i.e. half j =
-// tile % 2 of blob box tile / 2. CTA b takes items b, b + G, b + 2G, ... (G
-// CTAs), so that at any time the grid works on a few consecutive passes and
-// their activation steps stay in L2 while every weight box is read once per
-// pass. Every role decodes the same items.
+// Work items: (pass of up to 256 tokens, 256-row blob box), passes in expert
+// order: item i is box i % pairs of pass i / pairs. CTA b takes items b,
+// b + G, b + 2G, ... (G CTAs), so that at any time the grid works on a few
+// consecutive passes and their activation steps stay in L2 while every weight
+// box is read once per pass. Every role decodes the same items.
 struct PItem {
-    int e, box, j, r0, nt;
+    int e, box, r0, nt;
     int64_t pass;  // global pass index: the block row of the tiled activations
 };
 
@@ -214,10 +213,8 @@ __device__ __forceinline__ PItem decode_item(int64_t idx, const int32_t *__restr
                                              const int32_t *__restrict__ off, int E, int pairs)
 {
     PItem it;
-    it.pass = idx / (2 * pairs);
-    const int tile = (int)(idx % (2 * pairs));
-    it.box = tile >> 1;
-    it.j = tile & 1;
+    it.pass = idx / pairs;
+    it.box = (int)(idx % pairs);
     int lo = 0, hi = E;  // expert of the pass: largest e with pass_start[e] <= pass
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -306,12 +303,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __shfl_sync(0xFFFFFFFFu, okv, 0) != 0;
 }
 
-// Warp roles (27 warps).
+// Warp roles (28 warps).
 constexpr int kPWarpB = 0;      // activation producer
-constexpr int kPWarpMma = 1;    // MMA warp (both accumulators, alternate items)
-constexpr int kPWarpW = 2;      // packed weight producer
-constexpr int kPDeqWarp0 = 3;   // dequantising warps 3 .. 18
-constexpr int kPEpiWarp0 = 19;  // epilogue warps 19 .. 26 (accumulator (w - 19) / 4, lane quarter w % 4)
+constexpr int kPWarpMma = 1;    // MMA warps 1, 2 (tile / accumulator 0, 1)
+constexpr int kPWarpW = 3;      // packed weight producer
+constexpr int kPDeqWarp0 = 4;   // dequantising warps 4 .. 19
+constexpr int kPEpiWarp0 = 20;  // epilogue warps 20 .. 27 (accumulator (w - 20) / 4, lane quarter w % 4)
 constexpr int kPDeqWarps = kPEpiWarp0 - kPDeqWarp0;
 static_assert(kPThreads == 32 * (kPEpiWarp0 + 8), "warp roles");
 
@@ -334,30 +331,6 @@ struct Ring {
     }
 };
 
-// The packed-ring row of tile row m (and, through box_row, the blob box row
-// that holds its scales). Gate/up tile j of a box is its gate rows
-// 64j .. 64j+63 and the matching up rows 128+64j .. 128+64j+63, loaded as the
-// slot's rows 0..63 and 64..127; tile row 32q + w is gate row 16q + w of the
-// 64 for w < 16, else the up row of the same h column. Down tile j is box rows
-// 128j .. 128j+127, in order.
-template <bool GATE_UP>
-__device__ __forceinline__ int tile_slot_row(int m)
-{
-    if (!GATE_UP)
-        return m;
-    const int q = m >> 5, w = m & 31;
-    return (w < 16 ? 0 : 64) + 16 * q + (w & 15);
-}
-
-template <bool GATE_UP>
-__device__ __forceinline__ int tile_box_row(int m, int j)
-{
-    if (!GATE_UP)
-        return 128 * j + m;
-    const int q = m >> 5, w = m & 31;
-    return (w < 16 ? 0 : 128) + 64 * j + 16 * q + (w & 15);
-}
-
 template <bool GATE_UP>
 __global__ void __launch_bounds__(kPThreads, 1)
     ffn_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const PrefillParams p)
@@ -377,9 +350,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     uint64_t *empty_w = full_w + kPWStages;
     uint64_t *aready = empty_w + kPWStages;
     uint64_t *aempty = aready + kPAStages;
-    uint64_t *accfull = aempty + kPAStages;  // [2]: per accumulator
+    uint64_t *accfull = aempty + kPAStages;  // [2]: one accumulator per MMA warp
     uint64_t *accempty = accfull + 2;        // [2]
-    uint64_t *mma_done = accempty + 2;
+    uint64_t *mma_done = accempty + 2;       // [2]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + kPOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -388,7 +361,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (tid == 32) {
         for (int s = 0; s < kPBStages; ++s) {
             mbar_init(&full_b[s], 1);
-            mbar_init(&empty_b[s], 1);
+            mbar_init(&empty_b[s], 2);
         }
         for (int s = 0; s < kPWStages; ++s) {
             mbar_init(&full_w[s], 1);
@@ -396,13 +369,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         for (int s = 0; s < kPAStages; ++s) {
             mbar_init(&aready[s], kPDeqWarps);
-            mbar_init(&aempty[s], 1);
+            mbar_init(&aempty[s], 2);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&accfull[b], 1);
-            mbar_init(&accempty[b], 4);
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&accfull[j], 1);
+            mbar_init(&accempty[j], 4);
+            mbar_init(&mma_done[j], 1);
         }
-        mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -412,7 +385,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = *tslot;
-    const int64_t total = (int64_t)__ldg(p.pass_start + E) * 2 * pairs;
+    const int64_t total = (int64_t)__ldg(p.pass_start + E) * pairs;
     const int64_t G = gridDim.x;
     const int n_items = (int)(total > blockIdx.x ? (total - blockIdx.x + G - 1) / G : 0);
 #define ITEM(i) decode_item(blockIdx.x + (int64_t)(i) * G, p.pass_start, p.offsets, E, pairs)
@@ -428,9 +401,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // ---------------------------------------------------------- producers
         // Warp 0: the activation steps (x rows of the pass; for down h's hi
         // rows then lo rows), one bulk copy of a tiled 32 KB block each, kept
-        // in L2 for the other tiles of the pass.
-        // Warp 2: packed weights of two K steps of the item's tile (two TMA
-        // boxes of 64 rows x 64 bytes) with the box's scale images of that K half.
+        // in L2 for the other boxes of the pass.
+        // Warp 3: packed weights of two K steps (64 bytes of each of the box's
+        // 256 rows) with their scale images.
         if (lane == 0) {
             const bool is_b = warp == kPWarpB;
             const int S = is_b ? kPBStages : kPWStages;
@@ -441,15 +414,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
             uint32_t ph = 0;
             int64_t issued = 0;
             bool ok = true;
-            // packed weights and scale images of K steps ks, ks + 1 of tile j of a box into slot sl
-            auto load_w = [&](int sl, int64_t box, int j, int ks) {
+            // packed weights and scale images of K steps ks, ks + 1 of a box into slot sl
+            auto load_w = [&](int sl, int64_t box, int ks) {
                 const int64_t chunk = box * p.nchunk + (ks >> 2);  // 256-K chunk of the box
-                const int x = 64 * ((ks & 3) >> 1);
-                const int y0 = (int)(chunk * 256) + (GATE_UP ? 64 * j : 128 * j);
-                const int y1 = GATE_UP ? y0 + 128 : y0 + 64;
                 mbar_arrive_expect_tx(&full[sl], (uint32_t)(kPWBytes + kPSfBytes));
-                tc::tma_load_2d(sW + (size_t)sl * kPWBytes, &tmW, x, y0, &full[sl], pol);
-                tc::tma_load_2d(sW + (size_t)sl * kPWBytes + 64 * 64, &tmW, x, y1, &full[sl], pol);
+                tc::tma_load_2d(sW + (size_t)sl * kPWBytes, &tmW, 64 * ((ks & 3) >> 1), (int)(chunk * 256), &full[sl],
+                                pol);
                 bulk_g2s_hint(sSf + (size_t)sl * kPSfBytes, p.sf + chunk * 2048 + ((ks & 3) >> 1) * kPSfBytes,
                               kPSfBytes, &full[sl], pol);
             };
@@ -458,7 +428,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 for (int i = 0; i < n_items && pre < S; ++i) {
                     const PItem it = ITEM(i);
                     for (int ks = 0; ks < nks && pre < S; ks += 2, ++pre)
-                        load_w((int)pre, (int64_t)it.e * pairs + it.box, it.j, ks);
+                        load_w((int)pre, (int64_t)it.e * pairs + it.box, ks);
                 }
             grid_dep_wait();
             for (int i = 0; i < n_items && ok; ++i) {
@@ -477,7 +447,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                                               p.act + ((it.pass * nks + ks) * NB + b) * (int64_t)kPBBytes, kPBBytes,
                                               &full[s], pol);
                             } else {
-                                load_w(s, box, it.j, ks);
+                                load_w(s, box, ks);
                             }
                         }
                         ++issued;
@@ -499,31 +469,31 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     break;
                 }
         }
-    } else if (warp == kPWarpMma) {
+    } else if (warp == kPWarpMma || warp == kPWarpMma + 1) {
         // ---------------------------------------------------------------- MMA
-        // Item i goes to accumulator i % 2 (tensor memory columns 256 (i % 2)
-        // ..): D[row][n] += A[row][k] * B[n][k], A the item's dequantised tile,
+        // Warp 1 + j multiplies weight tile j of every K step into accumulator
+        // j (tensor memory columns 256j ..): D[row][n] += A_j[row][k] * B[n][k],
         // B the step's activation rows (down: hi, then lo, into the same D).
         if (lane == 0) {
+            const int j = warp - kPWarpMma;
+            const uint32_t d_tmem = tmem + (uint32_t)j * 256;
             Ring<kPBStages> rb;
             Ring<kPAStages> ra;
             bool ok = true, any = false;
             for (int i = 0; i < n_items && ok; ++i) {
                 const PItem it = ITEM(i);
-                const int buf = i & 1;
-                if (*abort_flag || !mbar_wait_bounded(&accempty[buf], (uint32_t)((i >> 1) & 1) ^ 1u, kPWaitNs)) {
+                if (*abort_flag || !mbar_wait_bounded(&accempty[j], (uint32_t)(i & 1) ^ 1u, kPWaitNs)) {
                     ok = false;
                     break;
                 }
                 tc::fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)buf * 256;
                 const uint32_t idesc = tc::idesc_bf16((it.nt + 15) & ~15);  // N: the pass's tokens, rounded up to 16
                 for (int ks = 0; ks < nks && ok; ++ks) {
                     if (*abort_flag || !mbar_wait_bounded(&aready[ra.slot], ra.phase, kPWaitNs)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t a_base = smem_u32(sA + (size_t)ra.slot * kPABytes);
+                    const uint32_t a_base = smem_u32(sA + (size_t)(2 * ra.slot + j) * kPABytes);
                     for (int b = 0; b < NB; ++b) {
                         if (*abort_flag || !mbar_wait_bounded(&full_b[rb.slot], rb.phase, kPWaitNs)) {
                             ok = false;
@@ -534,8 +504,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4)  // 16 values of K per MMA
                             tc::mma_bf16(d_tmem, tc::smem_desc(a_base + 32 * k4, 16, 1024, 2),
-                                         tc::smem_desc(b_base + 32 * k4, 16, 1024, 2), idesc,
-                                         (ks > 0 || b > 0 || k4 > 0) ? 1u : 0u);
+                                     tc::smem_desc(b_base + 32 * k4, 16, 1024, 2), idesc,
+                                     (ks > 0 || b > 0 || k4 > 0) ? 1u : 0u);
                         tc::commit(&empty_b[rb.slot]);
                         any = true;
                         rb.next();
@@ -545,48 +515,51 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     ra.next();
                 }
                 if (ok)
-                    tc::commit(&accfull[buf]);
+                    tc::commit(&accfull[j]);
             }
             if (!ok) {
                 set_status(p.status, MXMOE_ERR_TIMEOUT);
                 *abort_flag = 1;
             }
             if (any) {
-                tc::commit(mma_done);
-                if (!mbar_wait_bounded(mma_done, 0, kPWaitNs))
+                tc::commit(&mma_done[j]);
+                if (!mbar_wait_bounded(&mma_done[j], 0, kPWaitNs))
                     set_status(p.status, MXMOE_ERR_TIMEOUT);
             }
         }
     } else if (warp >= kPDeqWarp0 && warp < kPEpiWarp0) {
         // ------------------------------------------------------ dequantising
-        // Thread (kq, m) writes quarter kq (16 values) of row m of the item's
-        // tile: bf16 values (exact: an E2M1 value times a power of two) from
-        // the packed step and the E8M0 scale of its 32-value block, by table
-        // lookups (no conversion instructions per value), in the 128-byte
-        // swizzle (16-byte chunk c of row m at chunk c ^ (m % 8); quarter kq is
-        // chunks 2kq, 2kq + 1).
+        // Thread (k, j, m) writes half k of row m of weight tile j: 32 bf16
+        // values (exact: an E2M1 value times a power of two) from the packed
+        // step and the E8M0 scale of its 32-value block, by table lookups (no
+        // conversion instructions per value), in the 128-byte swizzle (16-byte
+        // chunk c of row m at chunk c ^ (m % 8); half k is chunks 4k .. 4k+3).
+        //  gate/up: tile j holds gate rows 64j .. 64j+63 of the box (its rows
+        //           0..127) and the matching up rows (box rows 128..255); row
+        //           32q + w is gate row 16q + w of the 64 for w < 16, else the
+        //           up row of the same h column;
+        //  down:    tile j is box rows 128j .. 128j+127.
         const int d = tid - 32 * kPDeqWarp0;
-        const int kq = d >> 7, m = d & 127;
-        const int srow = tile_slot_row<GATE_UP>(m);
+        const int k = d >> 8, j = (d >> 7) & 1, m = d & 127;
+        const int q = m >> 5, w = m & 31;
+        const int R = GATE_UP ? (w < 16 ? 0 : 128) + 64 * j + 16 * q + (w & 15) : 128 * j + m;  // box row
+        const int img = R >> 7, rr = R & 127;
+        const int sf_byte = img * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
         Ring<kPWStages> rw;
         Ring<kPAStages> ra;
         bool aborted = false;
         for (int i = 0; i < n_items; ++i) {
-            const PItem it = ITEM(i);
-            const int R = tile_box_row<GATE_UP>(m, it.j);  // the row's place in the box: its scale image byte
-            const int img = R >> 7, rr = R & 127;
-            const int sf_byte = img * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
             for (int ks = 0; ks < nks; ++ks) {
                 if (!aborted && !(ks & 1))  // a packed slot holds steps ks, ks + 1
                     aborted = !warp_wait(&full_w[rw.slot], rw.phase, abort_flag, p.status);
-                uint2 c = make_uint2(0, 0);
+                uint4 c = make_uint4(0, 0, 0, 0);
                 uint32_t e = 0;
                 if (!aborted) {
-                    c = *reinterpret_cast<const uint2 *>(sW + (size_t)rw.slot * kPWBytes + srow * 64 + 32 * (ks & 1) +
-                                                         8 * kq);
-                    // k32 block 2(ks%4) + kq/2 of the chunk: byte 2(ks%2) + kq/2 of the row's scale word in the
+                    c = *reinterpret_cast<const uint4 *>(sW + (size_t)rw.slot * kPWBytes + R * 64 + 32 * (ks & 1) +
+                                                         16 * k);
+                    // k32 block 2(ks%4) + k of the chunk: byte 2(ks%2) + k of the row's scale word in the
                     // image of this K half
-                    e = sSf[(size_t)rw.slot * kPSfBytes + sf_byte + 2 * (ks & 1) + (kq >> 1)];
+                    e = sSf[(size_t)rw.slot * kPSfBytes + sf_byte + 2 * (ks & 1) + k];
                 }
                 if (ks & 1) {
                     __syncwarp();
@@ -598,9 +571,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     aborted = !warp_wait(&aempty[ra.slot], ra.phase ^ 1u, abort_flag, p.status);
                 if (!aborted) {
                     const Bf16Tab t = e2m1_table(e);
-                    uint8_t *arow = sA + (size_t)ra.slot * kPABytes + m * 128;
-                    *reinterpret_cast<uint4 *>(arow + (((2 * kq) ^ (m & 7)) << 4)) = e2m1x8_to_bf16x8(c.x, t);
-                    *reinterpret_cast<uint4 *>(arow + (((2 * kq + 1) ^ (m & 7)) << 4)) = e2m1x8_to_bf16x8(c.y, t);
+                    uint8_t *arow = sA + (size_t)(2 * ra.slot + j) * kPABytes + m * 128;
+                    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {  // 8 values per 16-byte chunk
+                        const int ch = 4 * k + q4;
+                        *reinterpret_cast<uint4 *>(arow + ((ch ^ (m & 7)) << 4)) = e2m1x8_to_bf16x8(words[q4], t);
+                    }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 }
                 __syncwarp();
@@ -611,18 +588,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
     } else if (warp >= kPEpiWarp0) {
         // ----------------------------------------------------------- epilogue
-        // Warps 19..22 drain accumulator 0 (items 0, 2, 4, ...), warps 23..26
-        // accumulator 1 (items 1, 3, ...); warp quarter q = warp % 4 reads
-        // lanes 32q .. 32q+31, 32 columns (tokens) at a time.
-        const int g = (warp - kPEpiWarp0) >> 2, q = warp & 3;
-        const uint32_t acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(256 * g);
+        // Warps 12..15 drain accumulator 0, warps 16..19 accumulator 1; warp
+        // quarter q reads lanes 32q .. 32q+31, 32 columns (tokens) at a time.
+        const int j = (warp - kPEpiWarp0) >> 2, q = warp & 3;
+        const uint32_t acc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(256 * j);
         bool aborted = false;
-        for (int i = g; i < n_items; i += 2) {
+        for (int i = 0; i < n_items; ++i) {
             const PItem it = ITEM(i);
-            const int nt = it.nt, j = it.j;
+            const int nt = it.nt;
             const int64_t r0 = it.r0;
             if (!aborted)
-                aborted = !warp_wait(&accfull[g], (uint32_t)((i >> 1) & 1), abort_flag, p.status);
+                aborted = !warp_wait(&accfull[j], (uint32_t)(i & 1), abort_flag, p.status);
             tc::fence_after();
             if (GATE_UP) {
                 // lane w < 16 holds the gate rows of h column 128 box + 64j + 16q + w, lane w + 16 the up rows.
@@ -641,9 +617,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     for (int t = 0; t < 16; ++t) {
                         const float send = upper ? v[t] : v[t + 16];
                         const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
-                        const float gv = upper ? recv : v[t];
+                        const float g = upper ? recv : v[t];
                         const float u = upper ? v[t + 16] : recv;
-                        const float h = silu_fast(gv) * u;
+                        const float h = silu_fast(g) * u;
                         const uint32_t hi = (__float_as_uint(h) + 0x8000u) & 0xFFFF0000u;
                         const uint32_t lo = __float_as_uint(h - __uint_as_float(hi));
                         const int m = n0 + t + (upper ? 16 : 0);  // row of the pass
@@ -671,7 +647,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             tc::fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&accempty[g]);
+                mbar_arrive(&accempty[j]);
         }
     }
     tc::fence_before();
@@ -768,7 +744,7 @@ int run_bf16_stage(bool gate_up, const uint8_t *act_tiled, const int32_t *offset
     const int pairs = gate_up ? I / 128 : (H + 255) / 256;
     const int64_t blob_rows = (int64_t)E * pairs * nchunk * 256;
     CUtensorMap tmW;
-    if (int rc = encode2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, 128, (uint64_t)blob_rows, 128, 64, 64,
+    if (int rc = encode2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, 128, (uint64_t)blob_rows, 128, 64, 256,
                           CU_TENSOR_MAP_SWIZZLE_NONE, "bf16 stage weights"))
         return rc;
     PrefillParams p{};

@@ -457,14 +457,16 @@ int launch_route(const float *logits, int nsplit, const float *bias, int T, int 
                          w);
 }
 
-// K splits for the layer's router GEMM: enough CTAs to cover the GPU at
-// decode sizes, each split at least 8 k32 blocks (one per warp).
+// K splits for the layer's router GEMM: as many as keep all tiles in one
+// wave of one tile per SM (the persistent layer kernel runs a tile per CTA;
+// the chained kernel's CTAs all fit at once either way), at most 8, each
+// split at least 8 k32 blocks (one per warp).
 int router_splits(int T, int H, int E)
 {
     if (use_router_tc(T, H))
         return router_tc_splits(T, H, E);
     const int64_t base = (int64_t)((E + kRgExperts - 1) / kRgExperts) * ((T + kRgTokens - 1) / kRgTokens);
-    int z = (int)((2 * 148 + base / 2) / std::max<int64_t>(base, 1));
+    int z = (int)(num_sms() / std::max<int64_t>(base, 1));
     z = std::max(1, std::min(z, 8));
     z = std::min(z, std::max(1, (H / 32) / 8));
     return z;
