@@ -782,47 +782,62 @@ __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
 // 32-bit stores, in the term_offset layout, with their scale images (one per
 // token pass and 128 columns). Rows of experts with at least hot_rows rows are
 // skipped (the bf16 kernel takes those experts). s_off / s_pass: the offsets
-// and the token-pass prefix in shared memory. COHERENT: src_row was written
-// earlier in the same launch (read through L2, not the read-only path).
+// and the token-pass prefix in shared memory. The three steps (locate, load,
+// encode) are separate so that a warp can keep several units' loads in
+// flight. COHERENT: src_row was written earlier in the same launch (read
+// through L2, not the read-only path).
+struct ActUnit {
+    int r, c, n, tok;
+    int64_t img_row;
+    bool skip;
+};
+
 template <bool COHERENT>
-__device__ __forceinline__ void act_terms_unit(int64_t u, const uint16_t *__restrict__ act,
-                                               const int32_t *__restrict__ src_row, const int32_t *s_off,
-                                               const int32_t *s_pass, int E, int k, int rows, int H, int nt,
-                                               int hot_rows, uint8_t *__restrict__ terms, uint8_t *__restrict__ sf)
+__device__ __forceinline__ ActUnit act_unit_locate(int64_t u, const int32_t *__restrict__ src_row,
+                                                   const int32_t *s_off, const int32_t *s_pass, int E, int k, int H,
+                                                   int nt, int hot_rows)
 {
-    const int lane = threadIdx.x & 31;
     const int nch = (H + kKC - 1) / kKC;
-    const int kb = lane >> 2, q = lane & 3;  // the lane's 32-block within the chunk; its place in the block
-    const int r = (int)(u / nch), c = (int)(u % nch);
+    ActUnit a;
+    a.r = (int)(u / nch);
+    a.c = (int)(u % nch);
     int lo = 0, hi = E;  // expert of row r: largest e with s_off[e] <= r
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (s_off[mid] <= r)
+        if (s_off[mid] <= a.r)
             lo = mid;
         else
             hi = mid;
     }
-    if (s_off[lo + 1] - s_off[lo] >= hot_rows)  // the bf16 kernel takes this expert
-        return;
-    const int local = r - s_off[lo];
-    const int64_t img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
-    const int n = local % nt;
-    const int tok = (COHERENT ? __ldcg(src_row + r) : __ldg(src_row + r)) / k;
-    const int col = c * kKC + 8 * lane;
-    const bool live = col < H;  // H % 128 == 0: in a half chunk lanes 0..15 are live
+    a.skip = s_off[lo + 1] - s_off[lo] >= hot_rows;  // the bf16 kernel takes this expert
+    const int local = a.r - s_off[lo];
+    a.img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
+    a.n = local % nt;
+    a.tok = a.skip ? 0 : (COHERENT ? __ldcg(src_row + a.r) : __ldg(src_row + a.r)) / k;
+    return a;
+}
+
+__device__ __forceinline__ uint4 act_unit_load(const ActUnit &a, const uint16_t *__restrict__ act, int H)
+{
+    const int col = a.c * kKC + 8 * (threadIdx.x & 31);
+    if (a.skip || col >= H)  // H % 128 == 0: in a half chunk lanes 0..15 are live
+        return make_uint4(0, 0, 0, 0);
+    return __ldg(reinterpret_cast<const uint4 *>(act + (int64_t)a.tok * H + col));
+}
+
+__device__ __forceinline__ void act_unit_encode(const ActUnit &a, uint4 raw, int rows, int H,
+                                                uint8_t *__restrict__ terms, uint8_t *__restrict__ sf)
+{
+    const int lane = threadIdx.x & 31;
+    const int kb = lane >> 2, q = lane & 3;  // the lane's 32-block within the chunk; its place in the block
+    const int col = a.c * kKC + 8 * lane;
+    const bool live = col < H;
     float v[8];
-    if (live) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(act + (int64_t)tok * H + col));
-        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[2 * j] = __uint_as_float(w4[j] << 16);
-            v[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            v[j] = 0.f;
+    for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(w4[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
     }
     float m = 0.f;
 #pragma unroll
@@ -844,14 +859,14 @@ __device__ __forceinline__ void act_terms_unit(int64_t u, const uint16_t *__rest
             word[t] |= code[t] << (4 * j);
     }
     if (live) {
-        uint32_t *tp = reinterpret_cast<uint32_t *>(terms + term_offset(rows, 0, r, col));
+        uint32_t *tp = reinterpret_cast<uint32_t *>(terms + term_offset(rows, 0, a.r, col));
 #pragma unroll
         for (int t = 0; t < kT; ++t)  // term t sits 128 bytes after term t-1
             tp[32 * t] = word[t];
         // scales of the block: lane q of it writes terms q and q + 4
-        uint8_t *sp = sf + (img_row + 2 * c + (kb >> 2)) * kSFImg;
-        sp[image_byte(n, q, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * q + 127);
-        sp[image_byte(n, q + 4, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * (q + 4) + 127);
+        uint8_t *sp = sf + (a.img_row + 2 * a.c + (kb >> 2)) * kSFImg;
+        sp[image_byte(a.n, q, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * q + 127);
+        sp[image_byte(a.n, q + 4, kb & 3)] = (uint8_t)(E_blk - 1 - 3 * (q + 4) + 127);
     }
 }
 
@@ -886,8 +901,11 @@ __global__ void __launch_bounds__(256) act_terms_kernel(const uint16_t *__restri
     const int nch = (H + kKC - 1) / kKC;
     const int64_t total = (int64_t)rows * nch;
     const int64_t nwarps = (int64_t)gridDim.x * 8, gw = (int64_t)blockIdx.x * 8 + warp;
-    for (int64_t u = gw; u < total; u += nwarps)
-        act_terms_unit<false>(u, act, src_row, s_off, s_pass, E, k, rows, H, nt, hot_rows, terms, sf);
+    for (int64_t u = gw; u < total; u += nwarps) {
+        const ActUnit a = act_unit_locate<false>(u, src_row, s_off, s_pass, E, k, H, nt, hot_rows);
+        if (!a.skip)
+            act_unit_encode(a, act_unit_load(a, act, H), rows, H, terms, sf);
+    }
 }
 
 // y[t, c] = sum_j w[t, j] * y_perm[dst_of[t*k + j], c], j in order.
@@ -1150,9 +1168,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int nch = (H + kKC - 1) / kKC;
             const int64_t total = (int64_t)T * k * nch;
             const int64_t nworkers = (int64_t)G * 7, gw = (int64_t)blockIdx.x * 7 + (warp - 1);
-            for (int64_t u = gw; u < total; u += nworkers)
-                act_terms_unit<true>(u, fp.x, fp.src_row, s_off, s_pass, E, k, T * k, H, NT, INT_MAX, fp.x_terms,
-                                     fp.x_sf);
+            // four units per warp at a time: their row lookups, then their x loads, in flight together
+            for (int64_t u0 = gw; u0 < total; u0 += 4 * nworkers) {
+                ActUnit a[4];
+                uint4 raw[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t u = u0 + j * nworkers;
+                    a[j] = act_unit_locate<true>(u < total ? u : u0, fp.src_row, s_off, s_pass, E, k, H, NT, INT_MAX);
+                    a[j].skip = u >= total;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    raw[j] = act_unit_load(a[j], fp.x, H);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (!a[j].skip)
+                        act_unit_encode(a[j], raw[j], T * k, H, fp.x_terms, fp.x_sf);
+            }
             proxy_fence_global();
             named_bar_sync(1, 7 * 32);  // warps 1..7: this CTA's terms are written
             if (tid == 32) {
