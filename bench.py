@@ -45,7 +45,7 @@ import datagen  # noqa: E402
 METRIC = "MXFP4 MoE-layer tokens/s; expert-weight HBM GB/s as % of peak (1×B200)"
 UNIT = "tokens/s"
 BF16_PATH_ROWS = 16384  # grouped rows (tokens x top-k) from which both FFN stages run on bf16 tensor cores
-PERSISTENT_MAX_TOKENS = 16  # mxmoe_layer_forward runs one persistent kernel up to this many tokens
+PERSISTENT_MAX_TOKENS = 0  # mxmoe_layer_forward runs one persistent kernel up to this many tokens
 
 
 def kernels_per_step(T: int, k: int, E: int, H: int) -> int:
@@ -698,7 +698,7 @@ def run_native(args):
     extra = []
     if not args.no_per_config and not args.experts and not args.tokens:
         # the persistent layer kernel against the chained launches, on the decode-sized workloads
-        for name, path in (("verify8", "chained"), ("verify256", "persistent")):
+        for name, path in (("verify8", "persistent"), ("verify256", "persistent")):
             c = datagen.BY_NAME[name]
             wg_c, pre_c = layers[(c.H, c.E, c.I)]
             key = "%s_%s" % (name, path)

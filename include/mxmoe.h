@@ -424,9 +424,10 @@ MXMOE_API int mxmoe_ep_expert_ffn(const void *x_recv, const int32_t *recv_local,
  * engine kernel that stays resident, removes the gaps at operator boundaries
  * and keeps prefetching while the tensor cores compute ("Xiaomi
  * MiMo-V2.5-Pro-UltraSpeed 發佈說明", agentlenshq.com, section "TileRT 執行模型").
- * mxmoe_layer_forward takes this path by itself up to 16 tokens (the
- * decode-sized steps, e.g. one verify block of 8); this entry point takes it
- * for any supported size, mxmoe_layer_forward_chained never.
+ * This entry point takes the path for any supported size,
+ * mxmoe_layer_forward_chained never; mxmoe_layer_forward keeps the chained
+ * launches (measured as fast or faster: on one verify block the grid-wide
+ * barriers cost about what the chained launches' gaps do).
  * Arguments, layout, results and workspace as for mxmoe_layer_forward (ids and
  * weights identical; y equal up to float summation order, which is the same
  * as the chained path's). Every grid-wide wait is bounded (2 s): a CTA that

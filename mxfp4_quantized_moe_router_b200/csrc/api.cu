@@ -188,9 +188,11 @@ extern "C" MXMOE_API int64_t mxmoe_workspace_size(int T, int H, int I, int E, in
 
 namespace {
 // Token counts up to which mxmoe_layer_forward runs the whole layer as one
-// persistent kernel (decode-sized steps, where the chained launches' gaps and
-// the small kernels' latency weigh most).
-constexpr int kPersistentMaxTokens = 16;
+// persistent kernel. None: measured on one verify block (8 tokens), the
+// persistent kernel's grid-wide barriers cost about as much as the chained
+// launches' gaps, which programmatic dependent launch already hides (0.2494
+// vs 0.2459 ms per layer step), so the chained launches stay the default.
+constexpr int kPersistentMaxTokens = 0;
 
 enum class LayerPath { kAuto, kChained, kPersistent };
 
