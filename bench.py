@@ -130,14 +130,14 @@ def load_peaks():
 
 
 # Device code whose DRAM traffic a committed ncu capture describes: the
-# E2M1-term gate/up kernel (decode-sized workloads) and the bf16 gate/up kernel
-# (from 16384 grouped rows).
+# E2M1-term gate/up kernel (decode-sized workloads) and the large-token gate/up
+# kernel (from 16384 grouped rows).
 TRAFFIC_SOURCES = {
     "ffn_gate_up": ("mxfp4_quantized_moe_router_b200/csrc/ffn.cu", "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
                     "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"),
-    "ffn_bf16_gate_up": ("mxfp4_quantized_moe_router_b200/csrc/ffn_prefill.cu",
-                         "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
-                         "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"),
+    "ffn_f8_gate_up": ("mxfp4_quantized_moe_router_b200/csrc/ffn_prefill8.cu",
+                       "mxfp4_quantized_moe_router_b200/csrc/common.cuh",
+                       "mxfp4_quantized_moe_router_b200/csrc/tcgen05.cuh"),
 }
 
 
@@ -602,18 +602,22 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
                     "algorithmic_bytes_per_launch": unit_bytes}
         dtype = "e2m1 digit terms x e4m3 -> f32"
     elif T * k >= BF16_PATH_ROWS:
-        # dominant unit: mxmoe_ffn_gate_up on bf16 tensor cores (passes, slot rows, x_tile +
-        # ffn_bf16_kernel<gate_up>); algorithmic work = the dense gate/up
-        # contraction of every grouped row: 2 * rows * 2I * H flops
+        # dominant unit: mxmoe_ffn_gate_up on block-scaled tensor cores (passes, slot rows, x8_terms +
+        # ffn_f8_kernel<gate_up>); algorithmic work = the dense gate/up contraction of every grouped row,
+        # 2 * rows * 2I * H flops, against the bf16 peak: x enters as two E4M3 terms on the fp8 kind,
+        # whose rate is twice bf16's, so the two terms take the time of one bf16 contraction (the same
+        # fraction as the issued term work against the fp8 peak)
         unit_flops = 2.0 * T * k * 2 * I * H
         achieved = unit_flops / (unit_ms_mean / 1e3) / 1e12
-        roofline = {"kernel": "mxmoe_ffn_gate_up (x_tile_kernel + ffn_bf16_kernel<gate_up>)", "bound": "tensor",
+        roofline = {"kernel": "mxmoe_ffn_gate_up (x8_terms_kernel + ffn_f8_kernel<gate_up>)", "bound": "tensor",
                     "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops_sustained)" % peak_kind
+                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops_sustained; the fp8 kind's issued two-term "
+                                   "work is twice the flops at twice the rate)" % peak_kind
                     if peak_kind == "measured" else "fallback 1.4 PFLOP/s sustained",
-                    "traffic": profiled_traffic("ffn_bf16_gate_up", cfg.name, mean_touched), "unit_ms": unit_ms_mean,
-                    "algorithmic_flops_per_launch": unit_flops}
-        dtype = "bf16 x dequantised e2m1 -> f32"
+                    "traffic": profiled_traffic("ffn_f8_gate_up", cfg.name, mean_touched), "unit_ms": unit_ms_mean,
+                    "algorithmic_flops_per_launch": unit_flops,
+                    "issued_fp8_frac": 2 * achieved / (2 * peak_tf)}
+        dtype = "e2m1 x e4m3 terms -> f32"
     else:
         # dominant unit: mxmoe_ffn_gate_up (x_terms + gate/up stage); algorithmic
         # bytes = gate/up MXFP4 bytes of the touched experts + x read + h written

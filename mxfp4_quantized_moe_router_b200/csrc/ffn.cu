@@ -68,6 +68,15 @@ int run_bf16_stage(bool gate_up, const uint8_t *act_tiled, const int32_t *offset
                    const uint8_t *w, const uint8_t *sf, int rows, int E, int H, int I, uint8_t *h_tiled, float *y,
                    int *status, cudaStream_t st);
 int64_t bf16_max_passes(int64_t rows, int E, int min_rows);
+int64_t f8_max_passes(int64_t rows, int E, int min_rows);
+int64_t f8_terms_bytes(int64_t passes, int K, int nterms);
+int64_t f8_sf_bytes(int64_t passes, int K, int nterms);
+int run_f8_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
+                int min_rows, int32_t *pass_start, int32_t *slot_row, uint8_t *x_terms, uint8_t *x_sf, int *status,
+                cudaStream_t st);
+int run_f8_stage(bool gate_up, const uint8_t *terms, const uint8_t *terms_sf, const int32_t *offsets,
+                 const int32_t *pass_start, const uint8_t *w, const uint8_t *sf, int E, int H, int I, uint8_t *h_terms,
+                 uint8_t *h_sf, float *y, int *status, cudaStream_t st);
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
@@ -1265,10 +1274,12 @@ struct FfnWs {
     uint8_t *x_sf;        // scale images [pass][H/128][512]
     uint8_t *h_terms;     // term_offset layout, K = I
     uint8_t *h_sf;        // scale images [pass][I/128][512]
-    int32_t *bf_pass_start;  // bf16 kernel: its 256-token passes before each expert [kMaxE + 1]
-    int32_t *slot_row;    // bf16 kernel: grouped row of each (token, slot) [rows]
-    uint8_t *x_tiled;     // bf16 kernel: x per (pass, K step) as the shared-memory image
-    uint8_t *h_tiled;     // bf16 kernel: h hi, lo per (pass, K step, term) likewise
+    int32_t *bf_pass_start;  // large-token kernel: its token passes before each expert [kMaxE + 1]
+    int32_t *slot_row;    // large-token kernel: grouped row of each (token, slot) [rows]
+    uint8_t *x_tiled;     // large-token kernel: x's two E4M3 terms per (pass, stage, term) as the shared-memory image
+    uint8_t *x8_sf;       // their scale images
+    uint8_t *h_tiled;     // large-token kernel: h's three E4M3 terms likewise
+    uint8_t *h8_sf;       // their scale images
 };
 
 // Token counts at which both FFN stages run on bf16 tensor cores for every
@@ -1311,9 +1322,11 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base, 
     const int64_t o_hs = take(terms ? passes * (I / 128) * kSFImg : 0);
     const int64_t o_bps = take(bf16 ? (kMaxE + 1) * 4 : 0);
     const int64_t o_sr = take(bf16 ? rows * 4 : 0);
-    const int64_t bp = bf16 ? bf16_max_passes(rows, E, bf16_min_rows(T, k)) : 0;  // 256-token passes, at most
-    const int64_t o_xp = take(bp * 256 * H * 2);
-    const int64_t o_h2 = take(bp * 256 * I * 4);
+    const int64_t bp = bf16 ? f8_max_passes(rows, E, bf16_min_rows(T, k)) : 0;  // 224-token passes, at most
+    const int64_t o_xp = take(f8_terms_bytes(bp, H, 2));
+    const int64_t o_x8s = take(f8_sf_bytes(bp, H, 2));
+    const int64_t o_h2 = take(f8_terms_bytes(bp, I, 3));
+    const int64_t o_h8s = take(f8_sf_bytes(bp, I, 3));
     if (ws && base) {
         uint8_t *b = static_cast<uint8_t *>(base);
         ws->status = reinterpret_cast<int *>(b + o_status);
@@ -1325,7 +1338,9 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base, 
         ws->bf_pass_start = bf16 ? reinterpret_cast<int32_t *>(b + o_bps) : nullptr;
         ws->slot_row = bf16 ? reinterpret_cast<int32_t *>(b + o_sr) : nullptr;
         ws->x_tiled = bf16 ? b + o_xp : nullptr;
+        ws->x8_sf = bf16 ? b + o_x8s : nullptr;
         ws->h_tiled = bf16 ? b + o_h2 : nullptr;
+        ws->h8_sf = bf16 ? b + o_h8s : nullptr;
     }
     return off;
 }
@@ -1486,12 +1501,13 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
         if (!use_hybrid(T, k))
             return MXMOE_OK;
     }
-    // bf16 kernel: every expert, or (hybrid) those with at least kHotRows rows; h leaves as bf16 hi, lo terms
-    if (int rc = run_bf16_prep(x, offsets, src_row, k, rows, E, H, bf16_min_rows(T, k), ws.bf_pass_start,
-                               ws.slot_row, ws.x_tiled, clear, st))
+    // large-token kernel: every expert, or (hybrid) those with at least kHotRows rows; x as two E4M3 terms,
+    // h leaves as three
+    if (int rc = run_f8_prep(x, offsets, src_row, k, rows, E, H, bf16_min_rows(T, k), ws.bf_pass_start, ws.slot_row,
+                             ws.x_tiled, ws.x8_sf, clear, st))
         return rc;
-    return run_bf16_stage(true, ws.x_tiled, offsets, ws.bf_pass_start, bl.w13, bl.sf13, rows, E, H, I, ws.h_tiled,
-                          nullptr, ws.status, st);
+    return run_f8_stage(true, ws.x_tiled, ws.x8_sf, offsets, ws.bf_pass_start, bl.w13, bl.sf13, E, H, I, ws.h_tiled,
+                        ws.h8_sf, nullptr, ws.status, st);
 }
 
 int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, int E, int H, int I, float *y_perm,
@@ -1525,8 +1541,8 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
         if (!use_hybrid(T, k))
             return MXMOE_OK;
     }
-    return run_bf16_stage(false, ws.h_tiled, offsets, ws.bf_pass_start, bl.w2, bl.sf2, rows, E, H, I, nullptr, y_perm,
-                          ws.status, st);
+    return run_f8_stage(false, ws.h_tiled, ws.h8_sf, offsets, ws.bf_pass_start, bl.w2, bl.sf2, E, H, I, nullptr,
+                        nullptr, y_perm, ws.status, st);
 }
 
 // The FP8-weight FFN: both stages on the E2M1-term kernel with kind::mxf8f6f4

@@ -85,12 +85,12 @@ constexpr size_t kPOffMisc = (kPOffBar + kPBars * 8 + 15) & ~size_t(15);
 constexpr size_t kPSmem = 1024 + kPOffMisc + 64;
 static_assert(kPSmem <= 232448, "shared memory");
 
-// Token passes of up to 256 rows before each expert: pass_start[e] = sum over
-// e' < e of ceil(n_e' / 256), e = 0 .. E (E <= 1024), counting only experts
-// with at least min_rows rows (the others run on the E2M1-term kernel). One
-// block of 1024 threads; also clears the status word (when given).
+// Token passes of up to `tok` rows before each expert: pass_start[e] = sum
+// over e' < e of ceil(n_e' / tok), e = 0 .. E (E <= 1024), counting only
+// experts with at least min_rows rows (the others run on the E2M1-term
+// kernel). One block of 1024 threads; also clears the status word (when given).
 __global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__restrict__ offsets, int E,
-                                                              int min_rows, int32_t *__restrict__ pass_start,
+                                                              int min_rows, int tok, int32_t *__restrict__ pass_start,
                                                               int *status)
 {
     grid_dep_wait();  // the preceding kernel's results (chained launch)
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__r
     __shared__ int32_t s_warp[32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     const int n_e = e < E ? __ldg(offsets + e + 1) - __ldg(offsets + e) : 0;
-    const int c = n_e >= min_rows ? (n_e + kPTok - 1) / kPTok : 0;
+    const int c = n_e >= min_rows ? (n_e + tok - 1) / tok : 0;
     int incl = c;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -693,6 +693,15 @@ int launch_bf16_stage(const CUtensorMap &tmW, const PrefillParams &p, cudaStream
 
 }  // namespace
 
+// A 2-D tensor map (rows of row_bytes bytes, `inner` elements of `type` each),
+// for the other prefill kernel file.
+int encode2d_any(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle,
+                 const char *what)
+{
+    return encode2d(m, type, base, inner, outer, row_bytes, box_inner, box_outer, swizzle, what);
+}
+
 // Upper bound on the 256-token passes of `rows` grouped rows over E experts
 // when only experts with at least min_rows rows count: sum of ceil(n_e / 256)
 // <= rows / 256 + (number of such experts). Sizes the tiled activations.
@@ -708,19 +717,31 @@ int64_t bf16_max_passes(int64_t rows, int E, int min_rows)
 // 2 bytes), through slot_row (rows ints: the grouped row of each (token,
 // slot)); clears the status word when status is given. E <= 1024 and
 // k <= 32 (every accepted shape).
+// Passes of up to `tok` rows before each expert with at least min_rows rows
+// (pass_start, E + 1 ints; E <= 1024); clears the status word when given.
+int run_pass_prefix(const int32_t *offsets, int E, int min_rows, int tok, int32_t *pass_start, int *status,
+                    cudaStream_t st)
+{
+    return launch_kernel("prefill_passes_kernel", prefill_passes_kernel, 1, 1024, 0, st, offsets, E, min_rows, tok,
+                         pass_start, status);
+}
+
+// slot_row[src_row[r]] = r for the rows grouped pairs.
+int run_slot_rows(const int32_t *src_row, int rows, int32_t *slot_row, cudaStream_t st)
+{
+    const int blocks = (int)std::min<int64_t>(((int64_t)rows + 255) / 256, (int64_t)num_sms() * 4);
+    return launch_kernel("slot_rows_kernel", slot_rows_kernel, blocks < 1 ? 1 : blocks, 256, 0, st, src_row, rows,
+                         slot_row);
+}
+
 int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
                   int min_rows, int32_t *pass_start, int32_t *slot_row, uint8_t *x_tiled, int *status,
                   cudaStream_t st)
 {
-    if (int rc = launch_kernel("prefill_passes_kernel", prefill_passes_kernel, 1, 1024, 0, st, offsets, E, min_rows,
-                               pass_start, status))
+    if (int rc = run_pass_prefix(offsets, E, min_rows, kPTok, pass_start, status, st))
         return rc;
-    {
-        const int blocks = (int)std::min<int64_t>(((int64_t)rows + 255) / 256, (int64_t)num_sms() * 4);
-        if (int rc = launch_kernel("slot_rows_kernel", slot_rows_kernel, blocks < 1 ? 1 : blocks, 256, 0, st, src_row,
-                                   rows, slot_row))
-            return rc;
-    }
+    if (int rc = run_slot_rows(src_row, rows, slot_row, st))
+        return rc;
     const int T = rows / k;
     const int blocks = (int)std::min<int64_t>(((int64_t)T + 7) / 8, (int64_t)num_sms() * 8);
     return launch_kernel("x_tile_kernel", x_tile_kernel, blocks < 1 ? 1 : blocks, 256, 0, st,
