@@ -31,10 +31,11 @@
 //    tiles: M = 128, N = the pass's tokens rounded up to 16, K = 32.
 //  * Accumulators: tile 0 at tensor-memory column 0, tile 1 at 256 (224
 //    columns each); the scale slots sit in the columns between and after.
-//  * Four epilogue warps: gate/up computes h = silu(g) u for each token (lane
-//    = h column, so a warp holds one 32-block of h per token: its maximum is
-//    one redux.sync), encodes h into its three E4M3 terms in the layout the
-//    down stage reads; down writes y in fp32.
+//  * Eight epilogue warps, two per accumulator lane quarter taking alternate
+//    32-token chunks: gate/up computes h = silu(g) u for each token (lane = h
+//    column, so a warp holds one 32-block of h per token: its maximum is one
+//    redux.sync), encodes h into its three E4M3 terms in the layout the down
+//    stage reads; down writes y in fp32.
 //  * Items go round-robin over a persistent grid of one CTA per SM.
 // All waits are bounded; on a timeout the kernel records MXMOE_ERR_TIMEOUT in
 // the workspace status word and returns.
@@ -52,7 +53,7 @@ int encode2d_any(CUtensorMap *m, CUtensorMapDataType type, const void *base, uin
 namespace {
 
 constexpr uint64_t kQWaitNs = 2000000000ull;  // bounded waits: 2 s
-constexpr int kQThreads = 256;                // 8 warps: see the role list at the kernel
+constexpr int kQThreads = 384;                // 12 warps: see the role list at the kernel
 constexpr int kQTok = 224;                    // tokens per pass (N <= 224)
 constexpr int kQK = 128;                      // K per stage
 constexpr int kQAStages = 3;                  // weight ring
@@ -129,6 +130,30 @@ __device__ __forceinline__ float q8_e4m3_value(uint32_t code)
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)code));
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// E4M3 codes of two values in one conversion: lo's code in bits 0..7, hi's in 8..15.
+__device__ __forceinline__ uint32_t q8_e4m3x2(float lo, float hi)
+{
+    uint16_t pair;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(hi), "f"(lo));
+    return pair;
+}
+
+// The values of two E4M3 codes (bits 0..7 and 8..15). Every E4M3 value is a
+// normal f16 or zero, so one conversion to f16x2 and a widening of the bits
+// (f16 exponent bias 15 -> f32 bias 127) give them exactly.
+__device__ __forceinline__ float q8_f16_bits_to_f32(uint32_t h)
+{
+    const uint32_t mag = h & 0x7FFFu;
+    return __uint_as_float(((h & 0x8000u) << 16) | (mag ? (mag << 13) + (112u << 23) : 0u));
+}
+
+__device__ __forceinline__ float2 q8_e4m3x2_values(uint32_t codes)
+{
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)codes));
+    return make_float2(q8_f16_bits_to_f32(h2 & 0xFFFFu), q8_f16_bits_to_f32(h2 >> 16));
 }
 
 // Instruction descriptor of kind::mxf8f6f4.block_scale: A = E2M1 (the
@@ -280,11 +305,13 @@ __global__ void __launch_bounds__(256) x8_terms_kernel(const uint16_t *__restric
     }
 }
 
-// Warp roles (8 warps).
+// Warp roles (12 warps).
 constexpr int kQWarpB = 0;      // activation-term producer
 constexpr int kQWarpMma = 1;    // MMA thread (and the scale-image copies)
 constexpr int kQWarpA = 2;      // weight producer
-constexpr int kQEpiWarp0 = 4;   // epilogue warps 4..7 (lane quarter w % 4)
+constexpr int kQEpiWarp0 = 4;   // epilogue warps 4..11 (lane quarter w % 4, token chunks of parity (w - 4) / 4)
+constexpr int kQEpiWarps = 8;
+static_assert(kQThreads == 32 * (kQEpiWarp0 + kQEpiWarps), "warp roles");
 
 __device__ __forceinline__ float q8_silu(float g) { return __fdividef(g, 1.f + __expf(-g)); }
 
@@ -323,7 +350,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
             mbar_init(&empty_b[s], 1);
         }
         mbar_init(accfull, 1);
-        mbar_init(accempty, 4);
+        mbar_init(accempty, kQEpiWarps);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -387,9 +414,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
                                 break;
                             }
                             if (is_b) {
+                                // the pass's rows only (the MMA reads N = nt rounded up to 16 of them)
                                 const int64_t tile = (it.pass * nkb + kb) * NTERMS + t;
-                                mbar_arrive_expect_tx(&full[s], (uint32_t)(kQBBytes + kQSfBytes));
-                                bulk_g2s_hint(sB + (size_t)s * kQBBytes, p.act + tile * kQBBytes, kQBBytes, &full[s],
+                                const uint32_t bytes = (uint32_t)((it.nt + 15) & ~15) * kQK;
+                                mbar_arrive_expect_tx(&full[s], bytes + (uint32_t)kQSfBytes);
+                                bulk_g2s_hint(sB + (size_t)s * kQBBytes, p.act + tile * kQBBytes, bytes, &full[s],
                                               pol);
                                 bulk_g2s_hint(sBsf + (size_t)s * kQSfBytes, p.act_sf + tile * kQSfBytes, kQSfBytes,
                                               &full[s], pol);
@@ -420,84 +449,94 @@ __global__ void __launch_bounds__(kQThreads, 1)
         // ---------------------------------------------------------------- MMA
         // For every stage: the weight scale images into slot sa's columns, then
         // per term its scale images into slot sb's columns and, for each of the
-        // stage's four 32-blocks, one MMA per tile: D_j += A_j * B_t^T.
-        if (lane == 0) {
-            int sa = 0, sb = 0;
-            uint32_t pha = 0, phb = 0;
-            bool ok = true, any = false;
-            for (int i = 0; i < n_items && ok; ++i) {
-                const QItem it = ITEM(i);
-                if (*abort_flag || !mbar_wait_bounded(accempty, ((uint32_t)i & 1u) ^ 1u, kQWaitNs)) {
-                    ok = false;
+        // stage's four 32-blocks, one MMA per tile: D_j += A_j * B_t^T. The
+        // whole warp runs the loop (lane 0 waits, the verdict is shared); one
+        // elected lane issues. Descriptors are stepped from per-ring bases.
+        const bool leader = tc::elect_one();
+        const uint64_t a_desc0 = tc::smem_desc(smem_u32(sA), 16, 1024, 2);
+        const uint64_t b_desc0 = tc::smem_desc(smem_u32(sB), 16, 1024, 2);
+        const uint32_t sfa_s0 = smem_u32(sAsf), sfb_s0 = smem_u32(sBsf);
+        int sa = 0, sb = 0;
+        uint32_t pha = 0, phb = 0;
+        bool ok = true, any = false;
+        for (int i = 0; i < n_items && ok; ++i) {
+            const QItem it = ITEM(i);
+            ok = q8_warp_wait(accempty, ((uint32_t)i & 1u) ^ 1u, abort_flag, p.status);
+            if (!ok)
+                break;
+            tc::fence_after();
+            const int n = (it.nt + 15) & ~15;
+            uint32_t idesc[4];
+#pragma unroll
+            for (int k32 = 0; k32 < 4; ++k32)
+                idesc[k32] = q8_idesc(n, (uint32_t)k32);
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+                ok = q8_warp_wait(&full_a[sa], pha, abort_flag, p.status);
+                if (!ok)
                     break;
-                }
                 tc::fence_after();
-                const int n = (it.nt + 15) & ~15;
-                for (int kb = 0; kb < nkb && ok; ++kb) {
-                    if (*abort_flag || !mbar_wait_bounded(&full_a[sa], pha, kQWaitNs)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after();
-                    const uint32_t sfa_t = tmem + kQSfaCol0 + 8 * sa;
-                    const uint32_t sfa_s = smem_u32(sAsf + (size_t)sa * kQSfBytes);
+                const uint32_t sfa_t = tmem + kQSfaCol0 + 8 * sa;
+                const uint64_t a_desc = a_desc0 + (uint64_t)((sa * kQABytes) >> 4);
+                if (leader) {
+                    const uint32_t sfa_s = sfa_s0 + sa * kQSfBytes;
                     tc::cp_32x128b_warpx4(sfa_t, tc::smem_desc(sfa_s, 16, 128, 0));
                     tc::cp_32x128b_warpx4(sfa_t + 4, tc::smem_desc(sfa_s + 512, 16, 128, 0));
-                    const uint32_t a_base = smem_u32(sA + (size_t)sa * kQABytes);
-                    for (int t = 0; t < NTERMS; ++t) {
-                        if (*abort_flag || !mbar_wait_bounded(&full_b[sb], phb, kQWaitNs)) {
-                            ok = false;
-                            break;
-                        }
-                        tc::fence_after();
+                }
+                for (int t = 0; t < NTERMS; ++t) {
+                    ok = q8_warp_wait(&full_b[sb], phb, abort_flag, p.status);
+                    if (!ok)
+                        break;
+                    tc::fence_after();
+                    if (leader) {
                         const uint32_t sfb_t = tmem + kQSfbCol0 + 8 * sb;
-                        const uint32_t sfb_s = smem_u32(sBsf + (size_t)sb * kQSfBytes);
+                        const uint32_t sfb_s = sfb_s0 + sb * kQSfBytes;
                         tc::cp_32x128b_warpx4(sfb_t, tc::smem_desc(sfb_s, 16, 128, 0));
                         tc::cp_32x128b_warpx4(sfb_t + 4, tc::smem_desc(sfb_s + 512, 16, 128, 0));
-                        const uint32_t b_base = smem_u32(sB + (size_t)sb * kQBBytes);
+                        const uint64_t b_desc = b_desc0 + (uint64_t)((sb * kQBBytes) >> 4);
+                        const uint32_t first = (kb > 0 || t > 0) ? 1u : 0u;
 #pragma unroll
-                        for (int k32 = 0; k32 < 4; ++k32) {
-                            const uint32_t idesc = q8_idesc(n, (uint32_t)k32);
+                        for (int k32 = 0; k32 < 4; ++k32)
 #pragma unroll
-                            for (int j = 0; j < 2; ++j)
-                                q8_mma(tmem + (uint32_t)j * kQAccCols,
-                                       tc::smem_desc(a_base + (uint32_t)j * (128 * kQK) + 32 * k32, 16, 1024, 2),
-                                       tc::smem_desc(b_base + 32 * k32, 16, 1024, 2), idesc,
-                                       (kb > 0 || t > 0 || k32 > 0) ? 1u : 0u, (sfa_t + 4 * j) | ((uint32_t)k32 << 30),
-                                       sfb_t | ((uint32_t)k32 << 30));
-                        }
+                            for (int j = 0; j < 2; ++j)  // + 32 bytes of K per 32-block, + 16 KB per tile
+                                q8_mma(tmem + (uint32_t)j * kQAccCols, a_desc + (uint64_t)(2 * k32 + 1024 * j),
+                                       b_desc + (uint64_t)(2 * k32), idesc[k32], k32 > 0 ? 1u : first,
+                                       (sfa_t + 4 * j) | ((uint32_t)k32 << 30), sfb_t | ((uint32_t)k32 << 30));
                         tc::commit(&empty_b[sb]);
-                        any = true;
-                        if (++sb == kQBStages) {
-                            sb = 0;
-                            phb ^= 1u;
-                        }
                     }
-                    if (ok)
-                        tc::commit(&empty_a[sa]);
-                    if (++sa == kQAStages) {
-                        sa = 0;
-                        pha ^= 1u;
+                    __syncwarp();
+                    any = true;
+                    if (++sb == kQBStages) {
+                        sb = 0;
+                        phb ^= 1u;
                     }
                 }
-                if (ok)
-                    tc::commit(accfull);
+                if (ok && leader)
+                    tc::commit(&empty_a[sa]);
+                __syncwarp();
+                if (++sa == kQAStages) {
+                    sa = 0;
+                    pha ^= 1u;
+                }
             }
-            if (!ok) {
-                set_status(p.status, MXMOE_ERR_TIMEOUT);
-                *abort_flag = 1;
-            }
-            if (any) {  // every MMA and copy of ours completes before tensor memory is released
-                tc::commit(mma_done);
-                if (!mbar_wait_bounded(mma_done, 0, kQWaitNs))
-                    set_status(p.status, MXMOE_ERR_TIMEOUT);
-            }
+            if (ok && leader)
+                tc::commit(accfull);
+            __syncwarp();
         }
+        if (!ok && lane == 0) {
+            set_status(p.status, MXMOE_ERR_TIMEOUT);
+            *abort_flag = 1;
+        }
+        if (any && leader) {  // every MMA and copy of ours completes before tensor memory is released
+            tc::commit(mma_done);
+            if (!mbar_wait_bounded(mma_done, 0, kQWaitNs))
+                set_status(p.status, MXMOE_ERR_TIMEOUT);
+        }
+        __syncwarp();
     } else if (warp >= kQEpiWarp0) {
         // ----------------------------------------------------------- epilogue
         // Warp quarter q reads accumulator lanes 32q .. 32q+31 of both tiles,
-        // 32 columns (tokens) at a time.
-        const int q = warp & 3;
+        // 32 columns (tokens) at a time: chunks 2c + half for half = (warp - 4) / 4.
+        const int q = warp & 3, half = (warp - kQEpiWarp0) >> 2;
         const uint32_t acc0 = tmem + ((uint32_t)(32 * q) << 16), acc1 = acc0 + kQAccCols;
         bool aborted = false;
         for (int i = 0; i < n_items; ++i) {
@@ -513,29 +552,49 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 uint8_t *hb = p.h_terms + ((it.pass * nkb_d + it.box) * 3) * (int64_t)kQBBytes;
                 uint8_t *hs = p.h_sf + ((it.pass * nkb_d + it.box) * 3) * (int64_t)kQSfBytes;
                 const int bcol = 32 * q + lane;
-                for (int n0 = 0; n0 < nt && !aborted; n0 += 32) {
+                for (int n0 = 32 * half; n0 < nt && !aborted; n0 += 64) {
                     float g[32], u[32];
                     tc::ld_32x32b_x32(acc0 + (uint32_t)n0, g);
                     tc::ld_32x32b_x32(acc1 + (uint32_t)n0, u);
-                    for (int t = 0; t < 32 && n0 + t < nt; ++t) {
-                        const int m = n0 + t;  // row of the pass
-                        const float h = q8_silu(g[t]) * u[t];
-                        const uint32_t mbits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(h) & 0x7FFFFFFFu);
-                        const int Eb = max((int)(mbits >> 23) - 127, -112);
-                        const uint32_t c0 = q8_e4m3(h * q8_pow2(7 - Eb));
-                        const float r1 = h - q8_e4m3_value(c0) * q8_pow2(Eb - 7);
-                        const uint32_t c1 = q8_e4m3(r1 * q8_pow2(11 - Eb));
-                        const float r2 = r1 - q8_e4m3_value(c1) * q8_pow2(Eb - 11);
-                        const uint32_t c2 = q8_e4m3(r2 * q8_pow2(15 - Eb));
-                        const int off = q8_swz(m, bcol);
-                        hb[off] = (uint8_t)c0;
-                        hb[kQBBytes + off] = (uint8_t)c1;
-                        hb[2 * kQBBytes + off] = (uint8_t)c2;
+                    // two tokens (rows m, m + 1 of the pass) per step, their codes converted together
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const int m = n0 + t;
+                        if (m >= nt)
+                            break;
+                        const float ha = q8_silu(g[t]) * u[t], hb2 = q8_silu(g[t + 1]) * u[t + 1];
+                        const uint32_t ma = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(ha) & 0x7FFFFFFFu);
+                        const uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hb2) & 0x7FFFFFFFu);
+                        const int Ea = max((int)(ma >> 23) - 127, -112), Eb = max((int)(mb >> 23) - 127, -112);
+                        const uint32_t c0 = q8_e4m3x2(ha * q8_pow2(7 - Ea), hb2 * q8_pow2(7 - Eb));
+                        const float2 v0 = q8_e4m3x2_values(c0);
+                        const float ra = fmaf(-v0.x, q8_pow2(Ea - 7), ha), rb = fmaf(-v0.y, q8_pow2(Eb - 7), hb2);
+                        const uint32_t c1 = q8_e4m3x2(ra * q8_pow2(11 - Ea), rb * q8_pow2(11 - Eb));
+                        const float2 v1 = q8_e4m3x2_values(c1);
+                        const float sa = fmaf(-v1.x, q8_pow2(Ea - 11), ra), sb = fmaf(-v1.y, q8_pow2(Eb - 11), rb);
+                        const uint32_t c2 = q8_e4m3x2(sa * q8_pow2(15 - Ea), sb * q8_pow2(15 - Eb));
+                        const int offa = q8_swz(m, bcol);
+                        hb[offa] = (uint8_t)c0;
+                        hb[kQBBytes + offa] = (uint8_t)c1;
+                        hb[2 * kQBBytes + offa] = (uint8_t)c2;
+                        const bool second = m + 1 < nt;
+                        if (second) {
+                            const int offb = q8_swz(m + 1, bcol);
+                            hb[offb] = (uint8_t)(c0 >> 8);
+                            hb[kQBBytes + offb] = (uint8_t)(c1 >> 8);
+                            hb[2 * kQBBytes + offb] = (uint8_t)(c2 >> 8);
+                        }
                         if (lane == 0) {
-                            const int sb = q8_sf_byte(m, q);
-                            hs[sb] = (uint8_t)(Eb - 7 + 127);
-                            hs[kQSfBytes + sb] = (uint8_t)(Eb - 11 + 127);
-                            hs[2 * kQSfBytes + sb] = (uint8_t)(Eb - 15 + 127);
+                            const int fa = q8_sf_byte(m, q);
+                            hs[fa] = (uint8_t)(Ea - 7 + 127);
+                            hs[kQSfBytes + fa] = (uint8_t)(Ea - 11 + 127);
+                            hs[2 * kQSfBytes + fa] = (uint8_t)(Ea - 15 + 127);
+                            if (second) {
+                                const int fb = q8_sf_byte(m + 1, q);
+                                hs[fb] = (uint8_t)(Eb - 7 + 127);
+                                hs[kQSfBytes + fb] = (uint8_t)(Eb - 11 + 127);
+                                hs[2 * kQSfBytes + fb] = (uint8_t)(Eb - 15 + 127);
+                            }
                         }
                     }
                 }
@@ -543,7 +602,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 // lane: y columns 256 box + 32q + lane (tile 0) and 256 box + 128 + 32q + lane (tile 1)
                 const int c0 = 256 * it.box + 32 * q + lane, c1 = c0 + 128;
                 float *dst = p.y + (int64_t)it.r0 * p.H;
-                for (int n0 = 0; n0 < nt && !aborted; n0 += 32) {
+                for (int n0 = 32 * half; n0 < nt && !aborted; n0 += 64) {
                     float v0[32], v1[32];
                     tc::ld_32x32b_x32(acc0 + (uint32_t)n0, v0);
                     tc::ld_32x32b_x32(acc1 + (uint32_t)n0, v1);
