@@ -626,7 +626,7 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
         achieved = unit_bytes / (unit_ms_mean / 1e3) / 1e9
         hybrid = T >= 128
         roofline = {"kernel": "mxmoe_ffn_gate_up (act_terms_kernel + ffn_mxf4_kernel<gate_up>%s)"
-                              % (" + the bf16 kernels for experts with >= 128 rows" if hybrid else ""),
+                              % (" + the large-token kernels for experts with >= 128 rows" if hybrid else ""),
                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
                     else "fallback 6.65 TB/s",

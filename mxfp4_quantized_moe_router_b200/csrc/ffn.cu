@@ -61,13 +61,6 @@
 #include "tcgen05.cuh"
 
 namespace mxmoe {
-int run_bf16_prep(const void *x, const int32_t *offsets, const int32_t *src_row, int k, int rows, int E, int H,
-                  int min_rows, int32_t *pass_start, int32_t *slot_row, uint8_t *x_tiled, int *status,
-                  cudaStream_t st);
-int run_bf16_stage(bool gate_up, const uint8_t *act_tiled, const int32_t *offsets, const int32_t *pass_start,
-                   const uint8_t *w, const uint8_t *sf, int rows, int E, int H, int I, uint8_t *h_tiled, float *y,
-                   int *status, cudaStream_t st);
-int64_t bf16_max_passes(int64_t rows, int E, int min_rows);
 int64_t f8_max_passes(int64_t rows, int E, int min_rows);
 int64_t f8_terms_bytes(int64_t passes, int K, int nterms);
 int64_t f8_sf_bytes(int64_t passes, int K, int nterms);
@@ -103,7 +96,7 @@ struct FfnParams {
     int I;
     float *y_out;               // down output: [rows, H]
     int H;
-    int hot_rows;               // experts with at least this many rows are left to the bf16 kernel
+    int hot_rows;               // experts with at least this many rows are left to the large-token kernel
     int *status;
 };
 
@@ -790,7 +783,7 @@ __device__ void pass_prefix(const int32_t *offsets, int E, int nt, int32_t *out)
 // four lanes; each of the kT terms of the chunk leaves as one 128-byte row of
 // 32-bit stores, in the term_offset layout, with their scale images (one per
 // token pass and 128 columns). Rows of experts with at least hot_rows rows are
-// skipped (the bf16 kernel takes those experts). s_off / s_pass: the offsets
+// skipped (the large-token kernel takes those experts). s_off / s_pass: the offsets
 // and the token-pass prefix in shared memory. The three steps (locate, load,
 // encode) are separate so that a warp can keep several units' loads in
 // flight. COHERENT: src_row was written earlier in the same launch (read
@@ -818,7 +811,7 @@ __device__ __forceinline__ ActUnit act_unit_locate(int64_t u, const int32_t *__r
         else
             hi = mid;
     }
-    a.skip = s_off[lo + 1] - s_off[lo] >= hot_rows;  // the bf16 kernel takes this expert
+    a.skip = s_off[lo + 1] - s_off[lo] >= hot_rows;  // the large-token kernel takes this expert
     const int local = a.r - s_off[lo];
     a.img_row = ((int64_t)s_pass[lo] + local / nt) * (H / 128);
     a.n = local % nt;
@@ -1274,7 +1267,7 @@ struct FfnWs {
     uint8_t *x_sf;        // scale images [pass][H/128][512]
     uint8_t *h_terms;     // term_offset layout, K = I
     uint8_t *h_sf;        // scale images [pass][I/128][512]
-    int32_t *bf_pass_start;  // large-token kernel: its token passes before each expert [kMaxE + 1]
+    int32_t *f8_pass_start;  // large-token kernel: its token passes before each expert [kMaxE + 1]
     int32_t *slot_row;    // large-token kernel: grouped row of each (token, slot) [rows]
     uint8_t *x_tiled;     // large-token kernel: x's two E4M3 terms per (pass, stage, term) as the shared-memory image
     uint8_t *x8_sf;       // their scale images
@@ -1282,24 +1275,24 @@ struct FfnWs {
     uint8_t *h8_sf;       // their scale images
 };
 
-// Token counts at which both FFN stages run on bf16 tensor cores for every
-// expert (weights dequantised in shared memory; x as is, h as two bf16 terms)
-// instead of the E2M1-term MMAs: from 16384 grouped rows (2048 tokens at
-// top-8), where experts see hundreds of tokens and the stages are bound by the
-// tensor cores.
-constexpr int64_t kBf16Rows = 16384;
-bool use_bf16_path(int T, int k) { return (int64_t)T * k >= kBf16Rows; }
+// Token counts at which both FFN stages run on the large-token kernel
+// (ffn_prefill8.cu: block-scaled fp8-kind tensor cores, the E2M1 weights as
+// stored, x as two E4M3 terms and h as three) for every expert, instead of
+// the E2M1-term MMAs: from 16384 grouped rows (2048 tokens at top-8), where
+// experts see hundreds of tokens and the stages are bound by the tensor cores.
+constexpr int64_t kLargeRows = 16384;
+bool use_large_path(int T, int k) { return (int64_t)T * k >= kLargeRows; }
 
 // Below that, experts with at least kHotRows rows (a skewed router) still go
-// to the bf16 kernel, the rest to the E2M1-term kernel: the E2M1-term kernel
-// multiplies 8 terms per activation value and re-streams the expert's weights
-// for every 16-token pass, so from about a hundred tokens per expert the bf16
-// kernel is cheaper (cuts of 64, 128, 256 and 512 rows measured within noise of
-// each other). Only token counts that can produce such an expert
-// (T >= kHotRows) launch its kernels.
+// to the large-token kernel, the rest to the E2M1-term kernel: the E2M1-term
+// kernel multiplies 8 terms per activation value and re-streams the expert's
+// weights for every 16-token pass, so from about a hundred tokens per expert
+// the large-token kernel is cheaper (cuts of 64, 128, 256 and 512 rows
+// measured within noise of each other). Only token counts that can produce
+// such an expert (T >= kHotRows) launch its kernels.
 constexpr int kHotRows = 128;
-bool use_hybrid(int T, int k) { return !use_bf16_path(T, k) && T >= kHotRows; }
-int bf16_min_rows(int T, int k) { return use_bf16_path(T, k) ? 0 : kHotRows; }
+bool use_hybrid(int T, int k) { return !use_large_path(T, k) && T >= kHotRows; }
+int large_min_rows(int T, int k) { return use_large_path(T, k) ? 0 : kHotRows; }
 
 // fp8: the FP8-weight FFN, which runs every expert on the E2M1-term kernel.
 int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base, bool fp8 = false)
@@ -1314,15 +1307,15 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base, 
     const int64_t passes = max_passes(rows);
     const int64_t o_status = take(16);
     const int64_t o_ps = take((kMaxE + 1) * 4);
-    const bool terms = fp8 || !use_bf16_path(T, k);        // the E2M1-term kernel runs
-    const bool bf16 = !fp8 && (!terms || use_hybrid(T, k));  // the bf16 kernel runs
+    const bool terms = fp8 || !use_large_path(T, k);        // the E2M1-term kernel runs
+    const bool large = !fp8 && (!terms || use_hybrid(T, k));  // the large-token kernel runs
     const int64_t o_xt = take(terms ? rows * kT * pad256(H) / 2 : 0);
     const int64_t o_xs = take(terms ? passes * (H / 128) * kSFImg : 0);
     const int64_t o_ht = take(terms ? rows * kT * pad256(I) / 2 : 0);
     const int64_t o_hs = take(terms ? passes * (I / 128) * kSFImg : 0);
-    const int64_t o_bps = take(bf16 ? (kMaxE + 1) * 4 : 0);
-    const int64_t o_sr = take(bf16 ? rows * 4 : 0);
-    const int64_t bp = bf16 ? f8_max_passes(rows, E, bf16_min_rows(T, k)) : 0;  // 224-token passes, at most
+    const int64_t o_bps = take(large ? (kMaxE + 1) * 4 : 0);
+    const int64_t o_sr = take(large ? rows * 4 : 0);
+    const int64_t bp = large ? f8_max_passes(rows, E, large_min_rows(T, k)) : 0;  // 224-token passes, at most
     const int64_t o_xp = take(f8_terms_bytes(bp, H, 2));
     const int64_t o_x8s = take(f8_sf_bytes(bp, H, 2));
     const int64_t o_h2 = take(f8_terms_bytes(bp, I, 3));
@@ -1335,12 +1328,12 @@ int64_t ffn_ws_layout(int T, int k, int E, int H, int I, FfnWs *ws, void *base, 
         ws->x_sf = b + o_xs;
         ws->h_terms = b + o_ht;
         ws->h_sf = b + o_hs;
-        ws->bf_pass_start = bf16 ? reinterpret_cast<int32_t *>(b + o_bps) : nullptr;
-        ws->slot_row = bf16 ? reinterpret_cast<int32_t *>(b + o_sr) : nullptr;
-        ws->x_tiled = bf16 ? b + o_xp : nullptr;
-        ws->x8_sf = bf16 ? b + o_x8s : nullptr;
-        ws->h_tiled = bf16 ? b + o_h2 : nullptr;
-        ws->h8_sf = bf16 ? b + o_h8s : nullptr;
+        ws->f8_pass_start = large ? reinterpret_cast<int32_t *>(b + o_bps) : nullptr;
+        ws->slot_row = large ? reinterpret_cast<int32_t *>(b + o_sr) : nullptr;
+        ws->x_tiled = large ? b + o_xp : nullptr;
+        ws->x8_sf = large ? b + o_x8s : nullptr;
+        ws->h_tiled = large ? b + o_h2 : nullptr;
+        ws->h8_sf = large ? b + o_h8s : nullptr;
     }
     return off;
 }
@@ -1470,7 +1463,7 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     const int rows = T * k;
     const int nt = token_tile(T);
     const Blob bl = blob_parts(prepacked, E, H, I);
-    if (!use_bf16_path(T, k)) {  // E2M1-term kernel: every expert, or (hybrid) those below kHotRows rows
+    if (!use_large_path(T, k)) {  // E2M1-term kernel: every expert, or (hybrid) those below kHotRows rows
         const int hot_rows = use_hybrid(T, k) ? kHotRows : INT_MAX;
         const int64_t warps = (int64_t)rows * ((H + kKC - 1) / kKC);
         const int blocks = (int)std::min<int64_t>((warps + 7) / 8, (int64_t)num_sms() * 8);
@@ -1503,10 +1496,10 @@ int run_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_ro
     }
     // large-token kernel: every expert, or (hybrid) those with at least kHotRows rows; x as two E4M3 terms,
     // h leaves as three
-    if (int rc = run_f8_prep(x, offsets, src_row, k, rows, E, H, bf16_min_rows(T, k), ws.bf_pass_start, ws.slot_row,
+    if (int rc = run_f8_prep(x, offsets, src_row, k, rows, E, H, large_min_rows(T, k), ws.f8_pass_start, ws.slot_row,
                              ws.x_tiled, ws.x8_sf, clear, st))
         return rc;
-    return run_f8_stage(true, ws.x_tiled, ws.x8_sf, offsets, ws.bf_pass_start, bl.w13, bl.sf13, E, H, I, ws.h_tiled,
+    return run_f8_stage(true, ws.x_tiled, ws.x8_sf, offsets, ws.f8_pass_start, bl.w13, bl.sf13, E, H, I, ws.h_tiled,
                         ws.h8_sf, nullptr, ws.status, st);
 }
 
@@ -1518,7 +1511,7 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
     const int rows = T * k;
     const int nt = token_tile(T);
     const Blob bl = blob_parts(prepacked, E, H, I);
-    if (!use_bf16_path(T, k)) {
+    if (!use_large_path(T, k)) {
         FfnParams p{};
         p.tiles = (int)(pad256(H) / 256);
         p.K = I;
@@ -1541,7 +1534,7 @@ int run_ffn_down(const int32_t *offsets, const void *prepacked, int T, int k, in
         if (!use_hybrid(T, k))
             return MXMOE_OK;
     }
-    return run_f8_stage(false, ws.h_tiled, ws.h8_sf, offsets, ws.bf_pass_start, bl.w2, bl.sf2, E, H, I, nullptr,
+    return run_f8_stage(false, ws.h_tiled, ws.h8_sf, offsets, ws.f8_pass_start, bl.w2, bl.sf2, E, H, I, nullptr,
                         nullptr, y_perm, ws.status, st);
 }
 

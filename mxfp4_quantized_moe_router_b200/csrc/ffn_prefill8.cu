@@ -47,9 +47,6 @@
 #include "tcgen05.cuh"
 
 namespace mxmoe {
-int encode2d_any(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t inner, uint64_t outer,
-                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle,
-                 const char *what);
 namespace {
 
 constexpr uint64_t kQWaitNs = 2000000000ull;  // bounded waits: 2 s
@@ -98,6 +95,58 @@ struct Q8Params {
     float *y;                   // down out: [rows, H]
     int *status;
 };
+
+// Token passes of up to `tok` rows before each expert: pass_start[e] = sum
+// over e' < e of ceil(n_e' / tok), e = 0 .. E (E <= 1024), counting only
+// experts with at least min_rows rows (the others run on the E2M1-term
+// kernel). One block of 1024 threads; also clears the status word (when given).
+__global__ void __launch_bounds__(1024) prefill_passes_kernel(const int32_t *__restrict__ offsets, int E,
+                                                              int min_rows, int tok, int32_t *__restrict__ pass_start,
+                                                              int *status)
+{
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
+    __shared__ int32_t s_warp[32];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    const int n_e = e < E ? __ldg(offsets + e + 1) - __ldg(offsets + e) : 0;
+    const int c = n_e >= min_rows ? (n_e + tok - 1) / tok : 0;
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off)
+            incl += o;
+    }
+    if (lane == 31)
+        s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = s_warp[lane], wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xFFFFFFFFu, wi, off);
+            if (lane >= off)
+                wi += o;
+        }
+        s_warp[lane] = wi - w;  // passes before this warp's experts
+    }
+    __syncthreads();
+    const int excl = s_warp[warp] + incl - c;
+    if (e <= E)
+        pass_start[e] = excl;  // e == E: the total
+    if (e == 0 && status)
+        *status = 0;
+}
+
+// slot_row[src_row[r]] = r: the grouped row of each (token, slot) pair.
+__global__ void __launch_bounds__(256) slot_rows_kernel(const int32_t *__restrict__ src_row, int rows,
+                                                        int32_t *__restrict__ slot_row)
+{
+    grid_dep_wait();  // the preceding kernel's results (chained launch)
+    grid_dep_launch();
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x)
+        slot_row[__ldg(src_row + r)] = r;
+}
 
 // Byte of the scale of activation row m (of the pass), 32-block kb of a
 // stage, in the term's two 512-byte images (rows 0..127, 128..255): lane
@@ -649,9 +698,40 @@ int launch_f8_stage(const CUtensorMap &tmW, const Q8Params &p, cudaStream_t st)
 
 }  // namespace
 
+// A 2-D tensor map: `outer` rows of row_bytes bytes, `inner` elements of
+// `type` each, boxes of box_inner x box_outer.
+int encode2d_any(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t inner, uint64_t outer,
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle, const char *what)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc)
+        return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer}, es[2] = {1, 1};
+    CUresult r = enc(m, type, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (%s) failed: %d", what, (int)r);
+    return MXMOE_OK;
+}
+
+// Token passes of up to `tok` rows before each expert with at least min_rows
+// rows (pass_start, E + 1 ints; E <= 1024); clears the status word when given.
 int run_pass_prefix(const int32_t *offsets, int E, int min_rows, int tok, int32_t *pass_start, int *status,
-                    cudaStream_t st);
-int run_slot_rows(const int32_t *src_row, int rows, int32_t *slot_row, cudaStream_t st);
+                    cudaStream_t st)
+{
+    return launch_kernel("prefill_passes_kernel", prefill_passes_kernel, 1, 1024, 0, st, offsets, E, min_rows, tok,
+                         pass_start, status);
+}
+
+// slot_row[src_row[r]] = r for the rows grouped pairs.
+int run_slot_rows(const int32_t *src_row, int rows, int32_t *slot_row, cudaStream_t st)
+{
+    const int blocks = (int)std::min<int64_t>(((int64_t)rows + 255) / 256, (int64_t)num_sms() * 4);
+    return launch_kernel("slot_rows_kernel", slot_rows_kernel, blocks < 1 ? 1 : blocks, 256, 0, st, src_row, rows,
+                         slot_row);
+}
 
 // Upper bound on the 224-token passes of `rows` grouped rows over E experts
 // when only experts with at least min_rows rows count.

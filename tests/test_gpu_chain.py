@@ -7,7 +7,7 @@ what older kernels wrote (offsets, pass tables, weights). A read of a buffer
 from the wrong call or before it is written would change bits here. Before
 each call a torch kernel rewrites x, so the first kernel of a call must not
 overlap the caller's own work either. Each FFN path: E2M1-term kernels,
-hybrid, and bf16 kernels (with the tcgen05 router and the multi-block
+hybrid, and large-token kernels (with the tcgen05 router and the multi-block
 grouping)."""
 import pytest
 import torch

@@ -1,6 +1,6 @@
 """Parity of the expert FFN with the oracle at the format's numeric edges, on
-both tensor-core paths (the E2M1-term kernel at small token counts, the bf16
-kernel from 16384 grouped rows), through the C ABI.
+both tensor-core paths (the E2M1-term kernel at small token counts, the
+large-token fp8-kind kernel from 16384 grouped rows), through the C ABI.
 
 The MXFP4 format (model card, section 2 "FP4 Quantization": E2M1 elements,
 one E8M0 scale per 32 values along K) reaches its edges where a block's scale
@@ -84,8 +84,8 @@ def _x_row(kind, H, rng, j):
 @pytest.mark.parametrize("H,I,E,T,path", [
     (256, 256, 4, 64, "terms"),       # 16 tokens per expert: one 16-token pass each, E2M1-term kernel
     (384, 128, 4, 40, "terms"),       # ragged: a trailing half K chunk, a down tile of 128 real rows
-    (256, 256, 4, 16384, "bf16"),     # 16384 grouped rows: both stages on the bf16 kernel
-    (384, 128, 4, 16384, "bf16"),     # bf16 kernel with half K chunks and a half-real down box
+    (256, 256, 4, 16384, "large"),    # 16384 grouped rows: both stages on the large-token (fp8-kind) kernel
+    (384, 128, 4, 16384, "large"),    # large-token kernel with half K chunks and a half-real down box
 ])
 def test_expert_ffn_format_edges(mx, H, I, E, T, path):
     rng = np.random.default_rng(H * 7 + T)
@@ -117,7 +117,7 @@ def test_expert_ffn_format_edges(mx, H, I, E, T, path):
     xbits = bf16_bits(xb)
     for e in range(E):
         rows = src[off[e]:off[e + 1]]
-        if T > 256:  # the bf16 cases: a seeded sample of each expert's rows keeps the oracle quick
+        if T > 256:  # the large-token cases: a seeded sample of each expert's rows keeps the oracle quick
             pick = np.sort(np.random.default_rng(e).choice(len(rows), 256, replace=False))
             rows = rows[pick]
             grouped = off[e] + pick

@@ -1,6 +1,6 @@
 """The whole layer call is capturable in a CUDA graph (no synchronisation or
 allocation inside), and a replay gives the same bits as the eager call, on
-each FFN path: E2M1-term kernels, hybrid, and bf16 kernels (with the tcgen05
+each FFN path: E2M1-term kernels, hybrid, and large-token kernels (with the tcgen05
 router and the multi-block grouping)."""
 import pytest
 import torch

@@ -180,7 +180,7 @@ def test_permute_skewed(mx):
 # ---------------------------------------------------------------------------
 FFN_CASES = [
     # H, I, E, k, T : several 256-row tiles along I and H, several K chunks,
-    # more work items than SMs, the bf16 tensor-core path from 16384 rows,
+    # more work items than SMs, the large-token (fp8-kind tensor-core) path from 16384 rows,
     # ragged token passes (8-token passes for T <= 8, 16-token passes
     # otherwise); H or I = 128 mod 256 gives a trailing half K chunk and, for
     # H, a down tile of 128 real rows
@@ -192,10 +192,10 @@ FFN_CASES = [
     (1024, 128, 2, 2, 1),     # one token: 7 of the 8 pass rows unused
     (1024, 1024, 64, 4, 64),  # more items than SMs in both stages
     (1024, 512, 64, 8, 8),    # ~180 items of one pass each
-    (256, 128, 12, 2, 800),   # ~133 rows per expert: hybrid, experts above 128 rows on the bf16 kernel
+    (256, 128, 12, 2, 800),   # ~133 rows per expert: hybrid, experts above 128 rows on the large-token kernel
     (640, 384, 10, 2, 640),   # hybrid with ragged H and I: ~128 rows per expert, either side of the cut
-    (256, 128, 7, 2, 8192),   # 16384 grouped rows: both stages on bf16 tensor cores, ragged passes
-    (640, 384, 5, 2, 8192),   # bf16 path with 3 gate/up boxes, a half-real down box and half K chunks
+    (256, 128, 7, 2, 8192),   # 16384 grouped rows: both stages on the large-token kernel, ragged passes
+    (640, 384, 5, 2, 8192),   # large-token path with 3 gate/up boxes, a half-real down box and half K chunks
 ]
 
 
