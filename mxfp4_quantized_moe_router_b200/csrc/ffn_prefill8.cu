@@ -272,28 +272,36 @@ __device__ __forceinline__ bool q8_warp_wait(uint64_t *bar, uint32_t parity, vol
 // whose largest magnitude has exponent E (at least -116, so that every scale
 // stays a normal UE8M0 value): term 0 = x / 2^(E-7) rounded to E4M3, term 1 =
 // the exact remainder / 2^(E-11) rounded to E4M3. Rows of experts with fewer
-// than min_rows rows are skipped (the E2M1-term kernel takes them). One warp
-// per token: lane j < k finds where slot j goes, then the warp reads x[t] once
-// (lane l: values 4l .. 4l+3 of each 128-value stage, a 32-block being eight
-// lanes) and writes every such place.
+// than min_rows rows are skipped (the E2M1-term kernel takes them).
+// A warp takes (token t, a range of the 128-value stages; `groups` ranges
+// per token so that small token counts still fill the GPU): lane j < k finds
+// where slot j goes, every lane keeps each slot's tile row offset for its own
+// 4 bytes, then per stage the warp reads x[t] once (lane l: values 4l .. 4l+3,
+// a 32-block being eight lanes), encodes, and writes every slot's two terms;
+// lane j writes slot j's four block scales of both terms as one word each.
 constexpr int kQMaxK = 32;
 
+template <int KMAX>
 __global__ void __launch_bounds__(256) x8_terms_kernel(const uint16_t *__restrict__ x,
                                                        const int32_t *__restrict__ slot_row,
                                                        const int32_t *__restrict__ offsets,
                                                        const int32_t *__restrict__ pass_start, int E, int min_rows,
-                                                       int k, int T, int H, uint8_t *__restrict__ terms,
+                                                       int k, int T, int H, int groups, uint8_t *__restrict__ terms,
                                                        uint8_t *__restrict__ sf)
 {
     grid_dep_wait();  // the preceding kernel's results (chained launch)
     grid_dep_launch();
-    __shared__ int64_t s_pass[8][kQMaxK];  // per warp: pass of slot j, or -1
-    __shared__ int s_row[8][kQMaxK];       // its row within the pass
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int nkb = H / kQK;
+    const int per = (nkb + groups - 1) / groups;
     if (__ldg(pass_start + E) == 0)  // no expert for this kernel
         return;
-    for (int t = blockIdx.x * 8 + wl; t < T; t += gridDim.x * 8) {
+    const int64_t units = (int64_t)T * groups;
+    for (int64_t u = (int64_t)blockIdx.x * 8 + wl; u < units; u += (int64_t)gridDim.x * 8) {
+        const int t = (int)(u / groups), g = (int)(u % groups);
+        const int kb0 = g * per, kb1 = min(nkb, kb0 + per);
+        int64_t my_pass = -1;  // lane j < k: slot j's pass (or -1: the E2M1-term kernel's expert) and row
+        int my_row = 0;
         if (lane < k) {
             const int r = __ldg(slot_row + (int64_t)t * k + lane);
             int lo = 0, hi = E;  // expert of row r: largest e with offsets[e] <= r
@@ -305,15 +313,22 @@ __global__ void __launch_bounds__(256) x8_terms_kernel(const uint16_t *__restric
                     hi = mid;
             }
             const int local = r - __ldg(offsets + lo);
-            int64_t pass = -1;
             if (__ldg(offsets + lo + 1) - __ldg(offsets + lo) >= min_rows)
-                pass = __ldg(pass_start + lo) + local / kQTok;
-            s_pass[wl][lane] = pass;
-            s_row[wl][lane] = local % kQTok;
+                my_pass = __ldg(pass_start + lo) + local / kQTok;
+            my_row = local % kQTok;
         }
-        __syncwarp();
+        if (!__any_sync(0xFFFFFFFFu, my_pass >= 0) || kb0 >= kb1)
+            continue;
+        int64_t tb[KMAX];  // slot j: byte offset of this lane's 4 bytes in the slot's row of stage 0, term 0
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            const long long pj = __shfl_sync(0xFFFFFFFFu, (long long)my_pass, j);
+            const int rj = __shfl_sync(0xFFFFFFFFu, my_row, j);
+            tb[j] = (j < k && pj >= 0) ? pj * nkb * 2 * (int64_t)kQBBytes + q8_swz(rj, 4 * lane) : -1;
+        }
+        const int64_t sbase = my_pass >= 0 ? my_pass * nkb * 2 * (int64_t)kQSfBytes + q8_sf_byte(my_row, 0) : -1;
         const uint2 *src = reinterpret_cast<const uint2 *>(x + (int64_t)t * H);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
             const uint2 raw = __ldg(src + kb * 32 + lane);
             float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
                           __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
@@ -335,22 +350,24 @@ __global__ void __launch_bounds__(256) x8_terms_kernel(const uint16_t *__restric
                 w0 |= c0 << (8 * j);
                 w1 |= c1 << (8 * j);
             }
-            for (int j = 0; j < k; ++j) {
-                const int64_t pass = s_pass[wl][j];
-                if (pass < 0)
-                    continue;
-                const int row = s_row[wl][j];
-                const int64_t tile0 = ((pass * nkb + kb) * 2) * (int64_t)kQBBytes;
-                *reinterpret_cast<uint32_t *>(terms + tile0 + q8_swz(row, 4 * lane)) = w0;
-                *reinterpret_cast<uint32_t *>(terms + tile0 + kQBBytes + q8_swz(row, 4 * lane)) = w1;
-                if ((lane & 7) == 0) {
-                    uint8_t *s0 = sf + ((pass * nkb + kb) * 2) * (int64_t)kQSfBytes;
-                    s0[q8_sf_byte(row, lane >> 3)] = (uint8_t)(Eb - 7 + 127);
-                    s0[kQSfBytes + q8_sf_byte(row, lane >> 3)] = (uint8_t)(Eb - 11 + 127);
+            // the stage's four block scale bytes of term 0 (E - 7 + 127); term 1's are 4 less (E - 11 + 127)
+            const uint32_t s0 = (uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 0) + 120) |
+                                ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 8) + 120) << 8) |
+                                ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 16) + 120) << 16) |
+                                ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 24) + 120) << 24);
+            const int64_t koff = (int64_t)kb * 2 * kQBBytes;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (tb[j] >= 0) {
+                    *reinterpret_cast<uint32_t *>(terms + tb[j] + koff) = w0;
+                    *reinterpret_cast<uint32_t *>(terms + tb[j] + koff + kQBBytes) = w1;
                 }
+            if (sbase >= 0) {
+                uint8_t *s = sf + sbase + (int64_t)kb * 2 * kQSfBytes;
+                *reinterpret_cast<uint32_t *>(s) = s0;
+                *reinterpret_cast<uint32_t *>(s + kQSfBytes) = s0 - 0x04040404u;
             }
         }
-        __syncwarp();
     }
 }
 
@@ -760,10 +777,18 @@ int run_f8_prep(const void *x, const int32_t *offsets, const int32_t *src_row, i
     if (int rc = run_slot_rows(src_row, rows, slot_row, st))
         return rc;
     const int T = rows / k;
-    const int blocks = (int)std::min<int64_t>(((int64_t)T + 7) / 8, (int64_t)num_sms() * 8);
-    return launch_kernel("x8_terms_kernel", x8_terms_kernel, blocks < 1 ? 1 : blocks, 256, 0, st,
-                         static_cast<const uint16_t *>(x), slot_row, offsets, pass_start, E, min_rows, k, T, H, x_terms,
-                         x_sf);
+    // stage ranges per token: about 48 warps per SM in all
+    const int nkb = H / kQK;
+    const int groups = (int)std::max<int64_t>(1, std::min<int64_t>(nkb, ((int64_t)num_sms() * 48 + T - 1) / T));
+    const int64_t units = (int64_t)T * groups;
+    const int blocks = (int)std::min<int64_t>((units + 7) / 8, (int64_t)num_sms() * 8);
+    if (k <= 8)
+        return launch_kernel("x8_terms_kernel", x8_terms_kernel<8>, blocks < 1 ? 1 : blocks, 256, 0, st,
+                             static_cast<const uint16_t *>(x), slot_row, offsets, pass_start, E, min_rows, k, T, H,
+                             groups, x_terms, x_sf);
+    return launch_kernel("x8_terms_kernel", x8_terms_kernel<kQMaxK>, blocks < 1 ? 1 : blocks, 256, 0, st,
+                         static_cast<const uint16_t *>(x), slot_row, offsets, pass_start, E, min_rows, k, T, H, groups,
+                         x_terms, x_sf);
 }
 
 // One FFN stage on the block-scaled fp8-kind tensor cores.
