@@ -116,6 +116,10 @@ int router_splits(int T, int H, int E);
 int64_t permute_scratch_ints(int n, int E);
 int run_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *src_row, int32_t *dst_of,
                 int32_t *scratch, cudaStream_t st);
+bool front_ok(int T, int k, int E, int H, int I);
+int run_layer_front(const void *x, const void *wg, const float *bias, const void *prepacked, int T, int H, int I,
+                    int E, int k, int nsplit, float *partials, int32_t *ids, float *w, int32_t *offsets,
+                    int32_t *src_row, int32_t *dst_of, float *y_perm, float *y, void *ffn_ws, cudaStream_t st);
 int run_router_and_route(const void *x, const void *wg, const float *bias, int T, int H, int E, int k,
                          float *partials, int nsplit, int32_t *ids, float *w, int *status, cudaStream_t st);
 
@@ -235,6 +239,11 @@ int layer_forward(const char *fn, bool fp8, LayerPath path, const void *x, const
                             (path == LayerPath::kAuto && !fp8 && T <= kPersistentMaxTokens && fused_layer_ok(T, k, E, H, I));
     if (persistent)
         return run_fused_layer(x, wg, bias, prepacked, T, H, I, E, k, router_splits(T, H, E), ws.logits, ids, w,
+                               ws.offsets, ws.src_row, ws.dst_of, ws.y_perm, y, ws.ffn, st);
+    // decode-sized steps: router, routing, grouping and the activation terms in one cooperative launch, then the
+    // FFN stages and the combine chained (mxmoe_layer_forward_chained keeps one launch per step)
+    if (path == LayerPath::kAuto && !fp8 && front_ok(T, k, E, H, I))
+        return run_layer_front(x, wg, bias, prepacked, T, H, I, E, k, router_splits(T, H, E), ws.logits, ids, w,
                                ws.offsets, ws.src_row, ws.dst_of, ws.y_perm, y, ws.ffn, st);
     // one status record for the whole layer (the FFN workspace's first word): cleared here, so that a timeout
     // of the router kernel survives to mxmoe_read_status

@@ -98,6 +98,7 @@ struct FfnParams {
     int H;
     int hot_rows;               // experts with at least this many rows are left to the large-token kernel
     int *status;
+    int wait_first;             // chained after a kernel that wrote the offsets: every thread waits first
 };
 
 __host__ __device__ __forceinline__ int64_t pad256(int64_t v) { return (v + 255) & ~int64_t(255); }
@@ -730,6 +731,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const StageSmem<NT> S(smem, 0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (p.wait_first)  // the offsets and the pass table are the preceding kernel's results
+        grid_dep_wait();
     stage_prepare<NT>(p, S);
     if (warp == 1)
         tc::alloc(S.tslot, C::kTmemCols);
@@ -1275,6 +1278,69 @@ struct FfnWs {
     uint8_t *h8_sf;       // their scale images
 };
 
+// The front of a decode-sized layer step as one cooperative launch: router
+// GEMM tiles, routing, grouping and the activation terms -- the persistent
+// layer kernel's first phases (the same device code, so the results are
+// bit-identical to the chained kernels'), with only two grid-wide barriers up
+// to kFusedLocalRoute tokens (CTA 0 routes and groups them alone) and no
+// launch boundary between the steps. The FFN stages follow as chained launches.
+constexpr size_t kFrontSmem = sizeof(RouterRed) > (size_t)(kFusedMaxPairs + 2 * kFusedMaxE + 1) * 4
+                                  ? sizeof(RouterRed)
+                                  : (size_t)(kFusedMaxPairs + 2 * kFusedMaxE + 1) * 4;
+
+template <int NT>
+__global__ void __launch_bounds__(kFusedThreads, 1) front_kernel(const FusedParams fp)
+{
+    extern __shared__ __align__(16) uint8_t front_smem[];
+    __shared__ int s_flag;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int T = fp.T, E = fp.E, k = fp.k, H = fp.H;
+    const int G = gridDim.x;
+    int32_t *s_scratch = reinterpret_cast<int32_t *>(front_smem);
+    // 1. router GEMM tiles
+    {
+        RouterRed &red = *reinterpret_cast<RouterRed *>(front_smem);
+        const int ex = (E + kRgExperts - 1) / kRgExperts, ty = (T + kRgTokens - 1) / kRgTokens;
+        const int ntiles = ex * ty * fp.nsplit;
+        for (int vt = blockIdx.x; vt < ntiles; vt += G)
+            router_tile(fp.x, fp.wg, fp.bias, T, H, E, fp.partials, vt % ex, (vt / ex) % ty, vt / (ex * ty), fp.nsplit,
+                        red);
+    }
+    unsigned nbar = 1;
+    bool alive = grid_sync(fp, nbar, &s_flag);
+    // 2. routing, a warp per token (partial sums written in this launch by other CTAs, never read before on this
+    // SM); up to kFusedLocalRoute tokens CTA 0 routes them all and groups them without another grid barrier
+    const bool local_route = T <= kFusedLocalRoute;
+    if (alive && (!local_route || blockIdx.x == 0))
+        for (int tok = (local_route ? 0 : blockIdx.x * 8) + warp; tok < T; tok += local_route ? 8 : G * 8)
+            route_token<kFusedMaxE / 32, 4>(fp.partials, fp.nsplit, fp.nsplit > 1 ? fp.bias : nullptr, T, E, k,
+                                            fp.ids, fp.w, tok);
+    if (!local_route)
+        alive = alive && grid_sync(fp, ++nbar, &s_flag);
+    else
+        __syncthreads();
+    // 3. grouping (CTA 0): offsets, src_row, dst_of and the token passes
+    if (alive && blockIdx.x == 0)
+        fused_group<NT>(fp, s_scratch, s_scratch + kFusedMaxPairs, s_scratch + kFusedMaxPairs + kFusedMaxE);
+    alive = alive && grid_sync(fp, ++nbar, &s_flag);
+    // 4. the activation terms of every grouped row (all warps, round-robin over (row, 256-value chunk))
+    if (alive) {
+        int32_t *s_off = s_scratch, *s_pass = s_scratch + kFusedMaxE + 1;
+        for (int e = tid; e <= E; e += blockDim.x) {
+            s_off[e] = __ldcg(fp.offsets + e);
+            s_pass[e] = __ldcg(fp.pass_start + e);
+        }
+        __syncthreads();
+        const int nch = (H + kKC - 1) / kKC;
+        const int64_t total = (int64_t)T * k * nch;
+        const int64_t nworkers = (int64_t)G * (kFusedThreads / 32), gw = (int64_t)blockIdx.x * (kFusedThreads / 32) + warp;
+        for (int64_t u = gw; u < total; u += nworkers) {
+            const ActUnit a = act_unit_locate<true>(u, fp.src_row, s_off, s_pass, E, k, H, NT, INT_MAX);
+            act_unit_encode(a, act_unit_load(a, fp.x, H), T * k, H, fp.x_terms, fp.x_sf);
+        }
+    }
+}
+
 // Token counts at which both FFN stages run on the large-token kernel
 // (ffn_prefill8.cu: block-scaled fp8-kind tensor cores, the E2M1 weights as
 // stored, x as two E4M3 terms and h as three) for every expert, instead of
@@ -1737,6 +1803,112 @@ int run_combine(const float *y_perm, const int32_t *dst_of, const float *w, int 
 {
     dim3 grid((H / 4 + 255) / 256, T);
     return launch_kernel("combine_kernel", combine_kernel, grid, 256, 0, st, y_perm, dst_of, w, T, k, H, y);
+}
+
+// Shapes the front kernel takes: the E2M1-term path without hot experts
+// (T < kHotRows), at most kFusedMaxPairs pairs and kFusedMaxE experts, and
+// the mma.sync router (T < 512).
+bool front_ok(int T, int k, int E, int H, int I)
+{
+    return T >= 1 && T < kHotRows && !use_large_path(T, k) && (int64_t)T * k <= kFusedMaxPairs && k <= E &&
+           E <= kFusedMaxE && shapes_ok(T, k, E, H, I);
+}
+
+template <int NT>
+int launch_front(const FusedParams &fp, cudaStream_t st)
+{
+    auto kernel = front_kernel<NT>;
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFrontSmem) != cudaSuccess)
+            return fail(MXMOE_ERR_CUDA, "front_kernel: cannot reserve %zu bytes of shared memory", kFrontSmem);
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kFusedThreads, kFrontSmem) != cudaSuccess ||
+            per_sm < 1)
+            return fail(MXMOE_ERR_CUDA, "front_kernel: no CTA fits on an SM");
+        configured_dev = dev;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms());  // one CTA per SM, all resident at once
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = kFrontSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // the grid-wide barriers need every CTA resident
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    chain_next();  // a plain launch, first of the layer's chain
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, fp);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MXMOE_ERR_CUDA, "front_kernel: %s", cudaGetErrorString(e));
+    }
+    return check_launch("front_kernel");
+}
+
+// The layer for front_ok shapes: the front kernel (router, routing, grouping,
+// activation terms), then the gate/up and down stages on the E2M1-term kernel
+// and the combine, chained. The gate/up stage reads the grouping that its
+// predecessor wrote, so all its threads wait for it first (FfnParams::wait_first).
+int run_layer_front(const void *x, const void *wg, const float *bias, const void *prepacked, int T, int H, int I,
+                    int E, int k, int nsplit, float *partials, int32_t *ids, float *w, int32_t *offsets,
+                    int32_t *src_row, int32_t *dst_of, float *y_perm, float *y, void *ffn_ws, cudaStream_t st)
+{
+    FfnWs ws;
+    ffn_ws_layout(T, k, E, H, I, &ws, ffn_ws);
+    if (cudaMemsetAsync(ws.status, 0, 16, st) != cudaSuccess)  // the status word and the grid barrier's count
+        return fail(MXMOE_ERR_CUDA, "layer: cannot clear the status word");
+    const Blob bl = blob_parts(prepacked, E, H, I);
+    const int nt = token_tile(T);
+    FusedParams fp{};
+    fp.x = static_cast<const uint16_t *>(x);
+    fp.wg = static_cast<const uint16_t *>(wg);
+    fp.bias = bias;
+    fp.T = T;
+    fp.H = H;
+    fp.I = I;
+    fp.E = E;
+    fp.k = k;
+    fp.nsplit = nsplit;
+    fp.partials = partials;
+    fp.ids = ids;
+    fp.w = w;
+    fp.offsets = offsets;
+    fp.src_row = src_row;
+    fp.dst_of = dst_of;
+    fp.pass_start = ws.pass_start;
+    fp.x_terms = ws.x_terms;
+    fp.x_sf = ws.x_sf;
+    fp.barrier = reinterpret_cast<unsigned *>(reinterpret_cast<uint8_t *>(ws.status) + 8);
+    fp.status = ws.status;
+    ChainScope chain;
+    if (int rc = nt == 8 ? launch_front<8>(fp, st) : launch_front<16>(fp, st))
+        return rc;
+    FfnParams p{};
+    p.tiles = I / 128;
+    p.K = H;
+    p.rows = T * k;
+    p.wsf = bl.sf13;
+    p.asf = ws.x_sf;
+    p.offsets = offsets;
+    p.pass_start = ws.pass_start;
+    p.E = E;
+    p.h_terms = ws.h_terms;
+    p.h_sf = ws.h_sf;
+    p.I = I;
+    p.y_out = nullptr;
+    p.H = H;
+    p.hot_rows = INT_MAX;
+    p.status = ws.status;
+    p.wait_first = 1;
+    if (int rc = nt == 8 ? launch_ffn<8, true>(bl.w13, ws.x_terms, p, st) : launch_ffn<16, true>(bl.w13, ws.x_terms, p, st))
+        return rc;
+    if (int rc = run_ffn_down(offsets, prepacked, T, k, E, H, I, y_perm, ffn_ws, st))
+        return rc;
+    return run_combine(y_perm, dst_of, w, T, k, H, y, st);
 }
 
 int64_t ffn_workspace_bytes(int T, int k, int E, int H, int I)
