@@ -622,6 +622,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                     float g[32], u[32];
                     tc::ld_32x32b_x32(acc0 + (uint32_t)n0, g);
                     tc::ld_32x32b_x32(acc1 + (uint32_t)n0, u);
+                    int Eown = 0;  // the block exponent of token n0 + lane, for the scale bytes written below
                     // two tokens (rows m, m + 1 of the pass) per step, their codes converted together
 #pragma unroll
                     for (int t = 0; t < 32; t += 2) {
@@ -650,18 +651,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
                             hb[kQBBytes + offb] = (uint8_t)(c1 >> 8);
                             hb[2 * kQBBytes + offb] = (uint8_t)(c2 >> 8);
                         }
-                        if (lane == 0) {
-                            const int fa = q8_sf_byte(m, q);
-                            hs[fa] = (uint8_t)(Ea - 7 + 127);
-                            hs[kQSfBytes + fa] = (uint8_t)(Ea - 11 + 127);
-                            hs[2 * kQSfBytes + fa] = (uint8_t)(Ea - 15 + 127);
-                            if (second) {
-                                const int fb = q8_sf_byte(m + 1, q);
-                                hs[fb] = (uint8_t)(Eb - 7 + 127);
-                                hs[kQSfBytes + fb] = (uint8_t)(Eb - 11 + 127);
-                                hs[2 * kQSfBytes + fb] = (uint8_t)(Eb - 15 + 127);
-                            }
-                        }
+                        Eown = lane == t ? Ea : (lane == t + 1 ? Eb : Eown);
+                    }
+                    // scale bytes of the three terms: lane j those of token n0 + j, 32-block q of the stage
+                    if (n0 + lane < nt) {
+                        const int f = q8_sf_byte(n0 + lane, q);
+                        hs[f] = (uint8_t)(Eown - 7 + 127);
+                        hs[kQSfBytes + f] = (uint8_t)(Eown - 11 + 127);
+                        hs[2 * kQSfBytes + f] = (uint8_t)(Eown - 15 + 127);
                     }
                 }
             } else {
