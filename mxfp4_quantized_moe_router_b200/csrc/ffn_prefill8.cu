@@ -633,13 +633,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
                         const uint32_t ma = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(ha) & 0x7FFFFFFFu);
                         const uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hb2) & 0x7FFFFFFFu);
                         const int Ea = max((int)(ma >> 23) - 127, -112), Eb = max((int)(mb >> 23) - 127, -112);
-                        const uint32_t c0 = q8_e4m3x2(ha * q8_pow2(7 - Ea), hb2 * q8_pow2(7 - Eb));
+                        // on the scale of term 0 (h / 2^(E-7), below 256 in magnitude); each remainder is exact
+                        // and times 16 is the next term's scale (2^(E-11), then 2^(E-15))
+                        const float aa = ha * q8_pow2(7 - Ea), ab = hb2 * q8_pow2(7 - Eb);
+                        const uint32_t c0 = q8_e4m3x2(aa, ab);
                         const float2 v0 = q8_e4m3x2_values(c0);
-                        const float ra = fmaf(-v0.x, q8_pow2(Ea - 7), ha), rb = fmaf(-v0.y, q8_pow2(Eb - 7), hb2);
-                        const uint32_t c1 = q8_e4m3x2(ra * q8_pow2(11 - Ea), rb * q8_pow2(11 - Eb));
+                        const float ba = (aa - v0.x) * 16.f, bb = (ab - v0.y) * 16.f;
+                        const uint32_t c1 = q8_e4m3x2(ba, bb);
                         const float2 v1 = q8_e4m3x2_values(c1);
-                        const float sa = fmaf(-v1.x, q8_pow2(Ea - 11), ra), sb = fmaf(-v1.y, q8_pow2(Eb - 11), rb);
-                        const uint32_t c2 = q8_e4m3x2(sa * q8_pow2(15 - Ea), sb * q8_pow2(15 - Eb));
+                        const uint32_t c2 = q8_e4m3x2((ba - v1.x) * 16.f, (bb - v1.y) * 16.f);
                         const int offa = q8_swz(m, bcol);
                         hb[offa] = (uint8_t)c0;
                         hb[kQBBytes + offa] = (uint8_t)c1;
