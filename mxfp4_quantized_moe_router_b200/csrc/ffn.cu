@@ -242,32 +242,72 @@ __device__ __forceinline__ int act_block_exp(float m)
     return max((int)(b >> 23) - 127, -104);
 }
 
-// The kT balanced base-8 digits of an activation value v in a block of
-// exponent E, as E2M1 codes: v ~= sum_t d_t * 2^(E - 1 - 3t), d_t in
-// {-4..4} (all exact E2M1 values), t = 0 most significant. The digits are
-// exact for any v that is a multiple of 2^(E - 22) -- every bf16 value within
-// 2^-15 of its block maximum -- and otherwise represent v rounded to that
-// grid (within 2^-23 of the block maximum).
-__device__ __forceinline__ uint32_t e2m1_digit_code(int d)  // d in [-4, 4]
+__device__ __forceinline__ uint32_t byte_perm(uint32_t a, uint32_t b, uint32_t sel)
 {
-    const int mag = d < 0 ? -d : d;
-    // E2M1 codes of 0, 1, 2, 3, 4 are 0x0, 0x2, 0x4, 0x5, 0x6; bit 3 is the sign
-    return ((0x65420u >> (4 * mag)) & 0xFu) | (d < 0 ? 8u : 0u);
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
 }
 
-__device__ __forceinline__ void act_digits(float v, int E, uint32_t (&code)[kT])
+// The kT balanced base-8 digits of 8 activation values v[0..7] of a block of
+// exponent E, as E2M1 codes: v ~= sum_t d_t * 2^(E - 1 - 3t), d_t in {-4..4}
+// (all exact E2M1 values), t = 0 most significant; word[t] holds value j's
+// code of d_t in nibble j. The digits are exact for any v that is a multiple
+// of 2^(E - 22) -- every bf16 value within 2^-15 of its block maximum -- and
+// otherwise represent v rounded to that grid (within 2^-23 of the block
+// maximum).
+// iv = v * 2^(22 - E) rounded, |iv| <= 2^23. Adding 4 at each of the 7 low
+// base-8 positions (u = iv + 4 * (8^0 + ... + 8^6)) turns the low digits, in
+// [-4, 3], into plain base-8 digits d + 4 (no carries), and what is left
+// above them (an arithmetic shift by 21) is the top digit, in [-4, 4]. Each
+// value's seven low digits + 4 are spread to nibbles 0..6 of a word and its
+// top digit + 4 (0..8) put in nibble 7; an 8 x 8 nibble transpose (two
+// byte-permute stages, one of nibble masks) gathers digit t of the 8 values
+// into one word, in the nibble order 0 2 4 6 1 3 5 7; a byte-permute lookup
+// turns four digits into their codes at a time, bytes of even and odd values
+// then interleaved to nibbles. A selector nibble of 8 (a top digit of 4)
+// reads 0 (the sign of table byte 0) and takes code 6 from a second lookup.
+__device__ __forceinline__ void act_words(const float (&v)[8], int E, uint32_t (&word)[kT])
 {
-    const int iv = (int)rintf(v * pow2f(22 - E));  // |iv| <= 2^23
-    // Balanced base-8 digits: the 7 low ones in [-4, 3], the top one in
-    // [-4, 4]. Adding 4 at each of the 7 low positions turns the low digits
-    // into plain base-8 digits d + 4 (no carries), and what is left above
-    // them (an arithmetic shift) is the top digit. Codes of d = -4 .. 3 by
-    // d + 4: 0xE, 0xD, 0xC, 0xA, 0x0, 0x2, 0x4, 0x5 (bit 3 the sign).
-    const int u = iv + 0x124924;  // 4 * (8^0 + 8^1 + ... + 8^6)
+    static_assert(kT == 8, "one word per digit of 8 values");
+    const float s = pow2f(22 - E);
+    uint32_t x[8];
 #pragma unroll
-    for (int t = kT - 1; t > 0; --t)  // term kT-1 holds the lowest digit
-        code[t] = (0x5420ACDEu >> (4 * ((u >> (3 * (kT - 1 - t))) & 7))) & 0xFu;
-    code[0] = e2m1_digit_code(u >> 21);
+    for (int p = 0; p < 8; ++p) {
+        const int u = (int)rintf(v[p < 4 ? 2 * p : 2 * p - 7] * s) + 0x124924;
+        uint32_t f = (uint32_t)u;
+        f = (f & 0xFFFu) | ((f << 4) & 0x01FF0000u);        // digits 4..6 to bits 16..24
+        f = (f & 0x003F003Fu) | ((f << 2) & 0x3F003F00u);   // digits 2, 3 and 6 to the odd bytes
+        f = (f & 0x07070707u) | ((f << 1) & 0x70707070u);   // odd digits to the high nibbles
+        x[p] = f | (((uint32_t)(u + 0x800000) << 7) & 0xF0000000u);
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {  // 4 x 4 blocks of nibbles
+        const uint32_t a = x[p], b = x[p + 4];
+        x[p] = byte_perm(a, b, 0x5410u);
+        x[p + 4] = byte_perm(a, b, 0x7632u);
+    }
+#pragma unroll
+    for (int p = 0; p < 8; p += (p & 1) ? 3 : 1) {  // 2 x 2 blocks: pairs (0,2) (1,3) (4,6) (5,7)
+        const uint32_t a = x[p], b = x[p + 2];
+        x[p] = byte_perm(a, b, 0x6240u);
+        x[p + 2] = byte_perm(a, b, 0x7351u);
+    }
+#pragma unroll
+    for (int p = 0; p < 8; p += 2) {  // single nibbles
+        const uint32_t a = x[p], b = x[p + 1];
+        x[p] = (a & 0x0F0F0F0Fu) | ((b << 4) & 0xF0F0F0F0u);
+        x[p + 1] = ((a >> 4) & 0x0F0F0F0Fu) | (b & 0xF0F0F0F0u);
+    }
+    // codes of digit + 4 = 0..7 (d = -4..3): 0xE 0xD 0xC 0xA 0x0 0x2 0x4 0x5 (bit 3 the sign)
+    constexpr uint32_t kLo = 0x0A0C0D0Eu, kHi = 0x05040200u;
+#pragma unroll
+    for (int m = 0; m < 7; ++m)  // x[m]: the digits of weight 8^m, term kT - 1 - m
+        word[kT - 1 - m] = byte_perm(kLo, kHi, x[m]) | (byte_perm(kLo, kHi, x[m] >> 16) << 4);
+    const uint32_t y = x[7];
+    const uint32_t lo = byte_perm(kLo, kHi, y) | (byte_perm(0x80u, 0u, y) & 0x06060606u);
+    const uint32_t hi = byte_perm(kLo, kHi, y >> 16) | (byte_perm(0x80u, 0u, y >> 16) & 0x06060606u);
+    word[0] = lo | (hi << 4);
 }
 
 // Shared-memory view of one FFN stage: rings, scale images, barrier set
@@ -681,17 +721,7 @@ __device__ __forceinline__ void stage_roles(const CUtensorMap &tmW, const CUtens
                     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                     const int E_blk = act_block_exp(m);
                     uint32_t word[kT];
-#pragma unroll
-                    for (int t = 0; t < kT; ++t)
-                        word[t] = 0;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint32_t code[kT];
-                        act_digits(hv[b][j], E_blk, code);
-#pragma unroll
-                        for (int t = 0; t < kT; ++t)
-                            word[t] |= code[t] << (4 * j);
-                    }
+                    act_words(hv[b], E_blk, word);
                     if (valid) {
                         const int col = 128 * it.tile + 64 * b + 8 * tl;
 #pragma unroll
@@ -851,18 +881,8 @@ __device__ __forceinline__ void act_unit_encode(const ActUnit &a, uint4 raw, int
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     const int E_blk = act_block_exp(m);
-    uint32_t word[kT];
-#pragma unroll
-    for (int t = 0; t < kT; ++t)
-        word[t] = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {  // value j of the lane: nibble j (element 2i in the low nibble of byte i)
-        uint32_t code[kT];
-        act_digits(v[j], E_blk, code);
-#pragma unroll
-        for (int t = 0; t < kT; ++t)
-            word[t] |= code[t] << (4 * j);
-    }
+    uint32_t word[kT];  // value j of the lane: nibble j (element 2i in the low nibble of byte i)
+    act_words(v, E_blk, word);
     if (live) {
         uint32_t *tp = reinterpret_cast<uint32_t *>(terms + term_offset(rows, 0, a.r, col));
 #pragma unroll

@@ -189,20 +189,13 @@ __device__ __forceinline__ uint32_t q8_e4m3x2(float lo, float hi)
     return pair;
 }
 
-// The values of two E4M3 codes (bits 0..7 and 8..15). Every E4M3 value is a
-// normal f16 or zero, so one conversion to f16x2 and a widening of the bits
-// (f16 exponent bias 15 -> f32 bias 127) give them exactly.
-__device__ __forceinline__ float q8_f16_bits_to_f32(uint32_t h)
-{
-    const uint32_t mag = h & 0x7FFFu;
-    return __uint_as_float(((h & 0x8000u) << 16) | (mag ? (mag << 13) + (112u << 23) : 0u));
-}
-
+// The values of two E4M3 codes (bits 0..7 and 8..15): every E4M3 value is an
+// f16 value, so a conversion to f16x2 and two widenings give them exactly.
 __device__ __forceinline__ float2 q8_e4m3x2_values(uint32_t codes)
 {
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)codes));
-    return make_float2(q8_f16_bits_to_f32(h2 & 0xFFFFu), q8_f16_bits_to_f32(h2 >> 16));
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h2));
 }
 
 // Instruction descriptor of kind::mxf8f6f4.block_scale: A = E2M1 (the
@@ -618,7 +611,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 uint8_t *hb = p.h_terms + ((it.pass * nkb_d + it.box) * 3) * (int64_t)kQBBytes;
                 uint8_t *hs = p.h_sf + ((it.pass * nkb_d + it.box) * 3) * (int64_t)kQSfBytes;
                 const int bcol = 32 * q + lane;
+                // the lane's byte in a row of swizzle phase c (16-byte chunk bcol / 16 at chunk (bcol / 16) ^ c)
+                int sw[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    sw[c] = (((bcol >> 4) ^ c) << 4) + (bcol & 15);
                 for (int n0 = 32 * half; n0 < nt && !aborted; n0 += 64) {
+                    uint8_t *hrow = hb + (int64_t)n0 * 128;  // row n0 of the tiles; n0 % 8 == 0, so row n0 + t has phase t % 8
                     float g[32], u[32];
                     tc::ld_32x32b_x32(acc0 + (uint32_t)n0, g);
                     tc::ld_32x32b_x32(acc1 + (uint32_t)n0, u);
@@ -642,16 +641,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
                         const uint32_t c1 = q8_e4m3x2(ba, bb);
                         const float2 v1 = q8_e4m3x2_values(c1);
                         const uint32_t c2 = q8_e4m3x2((ba - v1.x) * 16.f, (bb - v1.y) * 16.f);
-                        const int offa = q8_swz(m, bcol);
-                        hb[offa] = (uint8_t)c0;
-                        hb[kQBBytes + offa] = (uint8_t)c1;
-                        hb[2 * kQBBytes + offa] = (uint8_t)c2;
-                        const bool second = m + 1 < nt;
-                        if (second) {
-                            const int offb = q8_swz(m + 1, bcol);
-                            hb[offb] = (uint8_t)(c0 >> 8);
-                            hb[kQBBytes + offb] = (uint8_t)(c1 >> 8);
-                            hb[2 * kQBBytes + offb] = (uint8_t)(c2 >> 8);
+                        uint8_t *pa = hrow + t * 128 + sw[t & 7];
+                        pa[0] = (uint8_t)c0;
+                        pa[kQBBytes] = (uint8_t)c1;
+                        pa[2 * kQBBytes] = (uint8_t)c2;
+                        if (m + 1 < nt) {
+                            uint8_t *pb = hrow + (t + 1) * 128 + sw[(t + 1) & 7];
+                            pb[0] = (uint8_t)(c0 >> 8);
+                            pb[kQBBytes] = (uint8_t)(c1 >> 8);
+                            pb[2 * kQBBytes] = (uint8_t)(c2 >> 8);
                         }
                         Eown = lane == t ? Ea : (lane == t + 1 ? Eb : Eown);
                     }
