@@ -270,8 +270,9 @@ __device__ __forceinline__ bool q8_warp_wait(uint64_t *bar, uint32_t parity, vol
 // per token so that small token counts still fill the GPU): lane j < k finds
 // where slot j goes, every lane keeps each slot's tile row offset for its own
 // 4 bytes, then per stage the warp reads x[t] once (lane l: values 4l .. 4l+3,
-// a 32-block being eight lanes), encodes, and writes every slot's two terms;
-// lane j writes slot j's four block scales of both terms as one word each.
+// a 32-block being eight lanes; the loads of NL stages issued together),
+// encodes, and writes every slot's two terms; lane j writes slot j's four
+// block scales of both terms as one word each.
 constexpr int kQMaxK = 32;
 
 template <int KMAX>
@@ -321,44 +322,55 @@ __global__ void __launch_bounds__(256) x8_terms_kernel(const uint16_t *__restric
         }
         const int64_t sbase = my_pass >= 0 ? my_pass * nkb * 2 * (int64_t)kQSfBytes + q8_sf_byte(my_row, 0) : -1;
         const uint2 *src = reinterpret_cast<const uint2 *>(x + (int64_t)t * H);
-        for (int kb = kb0; kb < kb1; ++kb) {
-            const uint2 raw = __ldg(src + kb * 32 + lane);
-            float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                          __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
-            uint32_t m = 0;
+        constexpr int NL = KMAX > 8 ? 2 : 4;  // stages whose x loads are in flight together
+        for (int kq = kb0; kq < kb1; kq += NL) {
+            uint2 raws[NL];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                m = max(m, __float_as_uint(v[j]) & 0x7FFFFFFFu);
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-            const int Eb = max((int)(m >> 23) - 127, -116);
-            const float inv0 = q8_pow2(7 - Eb), inv1 = q8_pow2(11 - Eb), sc0 = q8_pow2(Eb - 7);
-            uint32_t w0 = 0, w1 = 0;
+            for (int i = 0; i < NL; ++i)
+                raws[i] = kq + i < kb1 ? __ldg(src + (kq + i) * 32 + lane) : make_uint2(0u, 0u);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t c0 = q8_e4m3(v[j] * inv0);
-                const float rem = v[j] - q8_e4m3_value(c0) * sc0;  // exact
-                const uint32_t c1 = q8_e4m3(rem * inv1);
-                w0 |= c0 << (8 * j);
-                w1 |= c1 << (8 * j);
-            }
-            // the stage's four block scale bytes of term 0 (E - 7 + 127); term 1's are 4 less (E - 11 + 127)
-            const uint32_t s0 = (uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 0) + 120) |
-                                ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 8) + 120) << 8) |
-                                ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 16) + 120) << 16) |
-                                ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 24) + 120) << 24);
-            const int64_t koff = (int64_t)kb * 2 * kQBBytes;
+            for (int i = 0; i < NL; ++i) {
+                const int kb = kq + i;
+                if (kb >= kb1)
+                    break;
+                const uint2 raw = raws[i];
+                float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                              __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+                uint32_t m = 0;
 #pragma unroll
-            for (int j = 0; j < KMAX; ++j)
-                if (tb[j] >= 0) {
-                    *reinterpret_cast<uint32_t *>(terms + tb[j] + koff) = w0;
-                    *reinterpret_cast<uint32_t *>(terms + tb[j] + koff + kQBBytes) = w1;
+                for (int j = 0; j < 4; ++j)
+                    m = max(m, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+                const int Eb = max((int)(m >> 23) - 127, -116);
+                const float inv0 = q8_pow2(7 - Eb), inv1 = q8_pow2(11 - Eb), sc0 = q8_pow2(Eb - 7);
+                uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t c0 = q8_e4m3(v[j] * inv0);
+                    const float rem = v[j] - q8_e4m3_value(c0) * sc0;  // exact
+                    const uint32_t c1 = q8_e4m3(rem * inv1);
+                    w0 |= c0 << (8 * j);
+                    w1 |= c1 << (8 * j);
                 }
-            if (sbase >= 0) {
-                uint8_t *s = sf + sbase + (int64_t)kb * 2 * kQSfBytes;
-                *reinterpret_cast<uint32_t *>(s) = s0;
-                *reinterpret_cast<uint32_t *>(s + kQSfBytes) = s0 - 0x04040404u;
+                // the stage's four block scale bytes of term 0 (E - 7 + 127); term 1's are 4 less (E - 11 + 127)
+                const uint32_t s0 = (uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 0) + 120) |
+                                    ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 8) + 120) << 8) |
+                                    ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 16) + 120) << 16) |
+                                    ((uint32_t)(__shfl_sync(0xFFFFFFFFu, Eb, 24) + 120) << 24);
+                const int64_t koff = (int64_t)kb * 2 * kQBBytes;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j)
+                    if (tb[j] >= 0) {
+                        *reinterpret_cast<uint32_t *>(terms + tb[j] + koff) = w0;
+                        *reinterpret_cast<uint32_t *>(terms + tb[j] + koff + kQBBytes) = w1;
+                    }
+                if (sbase >= 0) {
+                    uint8_t *s = sf + sbase + (int64_t)kb * 2 * kQSfBytes;
+                    *reinterpret_cast<uint32_t *>(s) = s0;
+                    *reinterpret_cast<uint32_t *>(s + kQSfBytes) = s0 - 0x04040404u;
+                }
             }
         }
     }
