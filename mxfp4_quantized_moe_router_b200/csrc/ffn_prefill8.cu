@@ -198,6 +198,17 @@ __device__ __forceinline__ float2 q8_e4m3x2_values(uint32_t codes)
     return __half22float2(*reinterpret_cast<const __half2 *>(&h2));
 }
 
+// Byte transpose in groups of 4 lanes: lane 4j + r holds bytes k = 0..3 (its
+// values for 4 items k); afterwards it holds item r's bytes of lanes 4j .. 4j+3
+// (sel1 = r & 1 ? 0x3715 : 0x6240, sel2 = r & 2 ? 0x3276 : 0x5410).
+__device__ __forceinline__ uint32_t q8_t4(uint32_t w, uint32_t sel1, uint32_t sel2)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(__shfl_xor_sync(0xFFFFFFFFu, w, 1)), "r"(sel1));
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(w) : "r"(d), "r"(__shfl_xor_sync(0xFFFFFFFFu, d, 2)), "r"(sel2));
+    return w;
+}
+
 // Instruction descriptor of kind::mxf8f6f4.block_scale: A = E2M1 (the
 // weights, one per byte), B = E4M3 (the activation terms), UE8M0 scales, both
 // K-major, M = 128, N = n, scale byte sf_id (the 32-block of a 4-block column)
@@ -622,48 +633,57 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 const int nkb_d = p.I / kQK;
                 uint8_t *hb = p.h_terms + ((it.pass * nkb_d + it.box) * 3) * (int64_t)kQBBytes;
                 uint8_t *hs = p.h_sf + ((it.pass * nkb_d + it.box) * 3) * (int64_t)kQSfBytes;
-                const int bcol = 32 * q + lane;
-                // the lane's byte in a row of swizzle phase c (16-byte chunk bcol / 16 at chunk (bcol / 16) ^ c)
-                int sw[8];
+                // Codes are made with lane = h column 32q + lane, four tokens per step; a byte transpose in
+                // groups of 4 lanes leaves lane 4j + r with token r's codes of columns 32q + 4j .. 4j+3, one
+                // word per term. off[s]: that word in the rows of the step's token r, by swizzle phase 4s + r
+                // (chunks start at multiples of 32 tokens, so the phase is fixed by the step).
+                const int r = lane & 3, c4 = 32 * q + 4 * (lane >> 2);
+                const uint32_t sel1 = (r & 1) ? 0x3715u : 0x6240u, sel2 = (r & 2) ? 0x3276u : 0x5410u;
+                int off[2];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    sw[c] = (((bcol >> 4) ^ c) << 4) + (bcol & 15);
+                for (int s2 = 0; s2 < 2; ++s2)
+                    off[s2] = r * 128 + (((c4 >> 4) ^ (4 * s2 + r)) << 4) + (c4 & 15);
                 for (int n0 = 32 * half; n0 < nt && !aborted; n0 += 64) {
-                    uint8_t *hrow = hb + (int64_t)n0 * 128;  // row n0 of the tiles; n0 % 8 == 0, so row n0 + t has phase t % 8
+                    uint8_t *hrow = hb + (int64_t)n0 * 128;  // row n0 of the tiles
                     float g[32], u[32];
                     tc::ld_32x32b_x32(acc0 + (uint32_t)n0, g);
                     tc::ld_32x32b_x32(acc1 + (uint32_t)n0, u);
                     int Eown = 0;  // the block exponent of token n0 + lane, for the scale bytes written below
-                    // two tokens (rows m, m + 1 of the pass) per step, their codes converted together
 #pragma unroll
-                    for (int t = 0; t < 32; t += 2) {
-                        const int m = n0 + t;
-                        if (m >= nt)
+                    for (int t = 0; t < 32; t += 4) {
+                        if (n0 + t >= nt)
                             break;
-                        const float ha = q8_silu(g[t]) * u[t], hb2 = q8_silu(g[t + 1]) * u[t + 1];
-                        const uint32_t ma = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(ha) & 0x7FFFFFFFu);
-                        const uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hb2) & 0x7FFFFFFFu);
-                        const int Ea = max((int)(ma >> 23) - 127, -112), Eb = max((int)(mb >> 23) - 127, -112);
-                        // on the scale of term 0 (h / 2^(E-7), below 256 in magnitude); each remainder is exact
-                        // and times 16 is the next term's scale (2^(E-11), then 2^(E-15))
-                        const float aa = ha * q8_pow2(7 - Ea), ab = hb2 * q8_pow2(7 - Eb);
-                        const uint32_t c0 = q8_e4m3x2(aa, ab);
-                        const float2 v0 = q8_e4m3x2_values(c0);
-                        const float ba = (aa - v0.x) * 16.f, bb = (ab - v0.y) * 16.f;
-                        const uint32_t c1 = q8_e4m3x2(ba, bb);
-                        const float2 v1 = q8_e4m3x2_values(c1);
-                        const uint32_t c2 = q8_e4m3x2((ba - v1.x) * 16.f, (bb - v1.y) * 16.f);
-                        uint8_t *pa = hrow + t * 128 + sw[t & 7];
-                        pa[0] = (uint8_t)c0;
-                        pa[kQBBytes] = (uint8_t)c1;
-                        pa[2 * kQBBytes] = (uint8_t)c2;
-                        if (m + 1 < nt) {
-                            uint8_t *pb = hrow + (t + 1) * 128 + sw[(t + 1) & 7];
-                            pb[0] = (uint8_t)(c0 >> 8);
-                            pb[kQBBytes] = (uint8_t)(c1 >> 8);
-                            pb[2 * kQBBytes] = (uint8_t)(c2 >> 8);
+                        uint32_t w[3] = {0u, 0u, 0u};  // byte k of term i's word: the code of token t + k
+#pragma unroll
+                        for (int pr = 0; pr < 2; ++pr) {  // tokens t + 2pr, t + 2pr + 1, converted together
+                            const int ta = t + 2 * pr;
+                            const float ha = q8_silu(g[ta]) * u[ta], hb2 = q8_silu(g[ta + 1]) * u[ta + 1];
+                            const uint32_t ma = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(ha) & 0x7FFFFFFFu);
+                            const uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hb2) & 0x7FFFFFFFu);
+                            const int Ea = max((int)(ma >> 23) - 127, -112), Eb = max((int)(mb >> 23) - 127, -112);
+                            // on the scale of term 0 (h / 2^(E-7), below 256 in magnitude); each remainder is
+                            // exact and times 16 is the next term's scale (2^(E-11), then 2^(E-15))
+                            const float aa = ha * q8_pow2(7 - Ea), ab = hb2 * q8_pow2(7 - Eb);
+                            const uint32_t c0 = q8_e4m3x2(aa, ab);
+                            const float2 v0 = q8_e4m3x2_values(c0);
+                            const float ba = (aa - v0.x) * 16.f, bb = (ab - v0.y) * 16.f;
+                            const uint32_t c1 = q8_e4m3x2(ba, bb);
+                            const float2 v1 = q8_e4m3x2_values(c1);
+                            const uint32_t c2 = q8_e4m3x2((ba - v1.x) * 16.f, (bb - v1.y) * 16.f);
+                            w[0] |= c0 << (16 * pr);
+                            w[1] |= c1 << (16 * pr);
+                            w[2] |= c2 << (16 * pr);
+                            Eown = lane == ta ? Ea : (lane == ta + 1 ? Eb : Eown);
                         }
-                        Eown = lane == t ? Ea : (lane == t + 1 ? Eb : Eown);
+#pragma unroll
+                        for (int i = 0; i < 3; ++i)
+                            w[i] = q8_t4(w[i], sel1, sel2);
+                        if (n0 + t + r < nt) {
+                            uint32_t *pw = reinterpret_cast<uint32_t *>(hrow + t * 128 + off[(t >> 2) & 1]);
+                            pw[0] = w[0];
+                            pw[kQBBytes / 4] = w[1];
+                            pw[2 * kQBBytes / 4] = w[2];
+                        }
                     }
                     // scale bytes of the three terms: lane j those of token n0 + j, 32-block q of the stage
                     if (n0 + lane < nt) {
