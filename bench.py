@@ -44,7 +44,7 @@ import datagen  # noqa: E402
 
 METRIC = "MXFP4 MoE-layer tokens/s; expert-weight HBM GB/s as % of peak (1×B200)"
 UNIT = "tokens/s"
-BF16_PATH_ROWS = 16384  # grouped rows (tokens x top-k) from which both FFN stages run on bf16 tensor cores
+LARGE_PATH_ROWS = 16384  # grouped rows (tokens x top-k) from which both FFN stages run on the large-token kernel
 PERSISTENT_MAX_TOKENS = 0  # mxmoe_layer_forward runs one persistent kernel up to this many tokens
 
 
@@ -52,16 +52,16 @@ def kernels_per_step(T: int, k: int, E: int, H: int) -> int:
     """Kernels one layer step launches, following the library's dispatch:
     router GEMM (one kernel either way), route, grouping (one kernel, or three
     above 4096 pairs with E <= 1024), then the FFN -- E2M1-term path:
-    x_terms + two stages; bf16 path: passes + slot rows + x_tile + two stages;
-    both from 128 tokens below 16384 grouped rows -- then combine."""
+    x_terms + two stages; large-token path: passes + slot rows + x8_terms + two
+    stages; both from 128 tokens below 16384 grouped rows -- then combine."""
     rows = T * k
     n = 3 if (rows > 4096 and E <= 1024) else 1
     n += 2  # router GEMM, route
-    bf16_all = rows >= BF16_PATH_ROWS
-    hybrid = not bf16_all and T >= 128
-    if not bf16_all:
+    large_all = rows >= LARGE_PATH_ROWS
+    hybrid = not large_all and T >= 128
+    if not large_all:
         n += 3
-    if bf16_all or hybrid:
+    if large_all or hybrid:
         n += 5
     return n + 1  # combine
 
@@ -601,7 +601,7 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
                     else "fallback 6.65 TB/s", "traffic": None, "unit_ms": unit_ms_mean,
                     "algorithmic_bytes_per_launch": unit_bytes}
         dtype = "e2m1 digit terms x e4m3 -> f32"
-    elif T * k >= BF16_PATH_ROWS:
+    elif T * k >= LARGE_PATH_ROWS:
         # dominant unit: mxmoe_ffn_gate_up on block-scaled tensor cores (passes, slot rows, x8_terms +
         # ffn_f8_kernel<gate_up>); algorithmic work = the dense gate/up contraction of every grouped row,
         # 2 * rows * 2I * H flops, against the bf16 peak: x enters as two E4M3 terms on the fp8 kind,

@@ -196,10 +196,12 @@ MXMOE_API int64_t mxmoe_ffn_workspace_size(int T, int k, int E, int H, int I);
  * its own scale per 32 values. That represents every bf16 x within 2^-15 of
  * its block maximum exactly and any other value (smaller x, fp32 h) to within
  * 2^-23 of the block maximum. From 16384 grouped rows (and, from 128 tokens,
- * for experts with at least 128 rows) both stages run on bf16 tensor cores
- * instead: the weights dequantised exactly (an E2M1 value times its
- * power-of-two scale is a bf16 value), x as is, h as bf16 hi + lo (within
- * 2^-15 of h).
+ * for experts with at least 128 rows) both stages run on the large-token
+ * kernel instead (tcgen05 kind::mxf8f6f4 block-scaled MMAs): the E2M1 weight
+ * codes and their scales as stored, x as two E4M3 terms per value (exact for
+ * every bf16 x within 2^-13 of its 32-block maximum, smaller ones within
+ * 2^-21 of it), h as three E4M3 terms on scales 2^(E-7), 2^(E-11), 2^(E-15)
+ * of its 32-block maximum 2^E (within about 2^-16 of the block maximum).
  * Errors: H or I not a multiple of 128 or above 32768, k > 32, E > 1024,
  * T*k > 2^22, E*I*H >= 2^38 -> INVALID_SHAPE; workspace
  * too small -> WORKSPACE; x, y_perm not 16-byte or prepacked not 32-byte
@@ -211,9 +213,10 @@ MXMOE_API int mxmoe_expert_ffn(const void *x, const int32_t *offsets, const int3
 /* Stage 1 of mxmoe_expert_ffn on its own: for every grouped position r,
  * h[r] = silu(W_gate[e] x_t) * (W_up[e] x_t), written into the workspace for
  * mxmoe_ffn_down: as 8 E2M1 digit terms per value with their scale images,
- * or, for experts that the bf16 tensor-core kernel takes (every expert from
- * 16384 grouped rows; from 128 tokens, experts with at least 128 rows), as
- * bf16 hi + lo (within 2^-15 of h) in the tiled layout that kernel reads.
+ * or, for experts that the large-token kernel takes (every expert from 16384
+ * grouped rows; from 128 tokens, experts with at least 128 rows), as three
+ * E4M3 terms per value with their scale images, tiled per 224-token pass in
+ * the layout that kernel reads.
  * Arguments, layout and errors as for mxmoe_expert_ffn (workspace from
  * mxmoe_ffn_workspace_size, 256-byte aligned). */
 MXMOE_API int mxmoe_ffn_gate_up(const void *x, const int32_t *offsets, const int32_t *src_row, const void *prepacked,

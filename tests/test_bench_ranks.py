@@ -97,7 +97,7 @@ def test_bench_parses_its_arguments():
 
 def test_launch_count_follows_the_dispatch():
     # verify8: one grouping kernel, E2M1-term FFN; verify256: hybrid; zipf1024: hybrid + multi-block grouping;
-    # prefill8192: bf16 FFN + multi-block grouping
+    # prefill8192: large-token FFN + multi-block grouping
     assert [bench.kernels_per_step(T, 8, 384, 6144) for T in (8, 256, 1024, 8192)] == [7, 12, 14, 11]
 
 
