@@ -48,12 +48,22 @@ LARGE_PATH_ROWS = 16384  # grouped rows (tokens x top-k) from which both FFN sta
 PERSISTENT_MAX_TOKENS = 0  # mxmoe_layer_forward runs one persistent kernel up to this many tokens
 
 
+def front_path(T: int, k: int, E: int) -> bool:
+    """Whether mxmoe_layer_forward (MXFP4 weights) takes its front path: router,
+    routing, grouping and activation terms in one cooperative kernel, below
+    128 tokens with T*k <= 4096 and k <= E <= 384."""
+    return 1 <= T < 128 and T * k < LARGE_PATH_ROWS and T * k <= 4096 and k <= E <= 384
+
+
 def kernels_per_step(T: int, k: int, E: int, H: int) -> int:
-    """Kernels one layer step launches, following the library's dispatch:
-    router GEMM (one kernel either way), route, grouping (one kernel, or three
-    above 4096 pairs with E <= 1024), then the FFN -- E2M1-term path:
+    """Kernels one layer step launches, following the library's dispatch: on
+    the front path the front kernel, the two FFN stages and the combine;
+    otherwise router GEMM (one kernel either way), route, grouping (one kernel,
+    or three above 4096 pairs with E <= 1024), then the FFN -- E2M1-term path:
     x_terms + two stages; large-token path: passes + slot rows + x8_terms + two
     stages; both from 128 tokens below 16384 grouped rows -- then combine."""
+    if front_path(T, k, E):
+        return 4
     rows = T * k
     n = 3 if (rows > 4096 and E <= 1024) else 1
     n += 2  # router GEMM, route
@@ -644,7 +654,8 @@ def measure_layer(mx, cfg, wg, prepacked, args, steps, warmup, world, rank, dev,
     if fp8:
         out["weight_format"] = "fp8 (E4M3, one E8M0 scale per 32)"
     persistent = path == "persistent" or (path == "auto" and not fp8 and T <= PERSISTENT_MAX_TOKENS and E <= 384)
-    out["layer_path"] = "persistent kernel" if persistent else "chained launches"
+    out["layer_path"] = ("persistent kernel" if persistent else
+                         "front kernel + chained launches" if not fp8 and front_path(T, k, E) else "chained launches")
     if persistent:  # one cooperative launch per step (plus the status clear)
         out["gpu_launches"] = steps
     if ms_e2e is not None:

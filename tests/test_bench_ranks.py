@@ -96,9 +96,13 @@ def test_bench_parses_its_arguments():
 
 
 def test_launch_count_follows_the_dispatch():
-    # verify8: one grouping kernel, E2M1-term FFN; verify256: hybrid; zipf1024: hybrid + multi-block grouping;
-    # prefill8192: large-token FFN + multi-block grouping
-    assert [bench.kernels_per_step(T, 8, 384, 6144) for T in (8, 256, 1024, 8192)] == [7, 12, 14, 11]
+    # verify8: front kernel, two E2M1-term stages, combine; verify256: hybrid; zipf1024: hybrid + multi-block
+    # grouping; prefill8192: large-token FFN + multi-block grouping
+    assert [bench.kernels_per_step(T, 8, 384, 6144) for T in (8, 256, 1024, 8192)] == [4, 12, 14, 11]
+    # below 128 tokens with more than 384 experts: the chained launches
+    assert bench.kernels_per_step(8, 8, 512, 6144) == 1 + 2 + 3 + 1
+    assert bench.kernels_per_step(127, 32, 384, 6144) == 4  # 4064 pairs: still the front path
+    assert bench.kernels_per_step(4, 2, 16, 256) == 4  # tiny
 
 
 def test_verify_workload_reference_arm_prints_the_contract_line():
